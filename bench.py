@@ -1,0 +1,394 @@
+"""Throughput of the sparse paged attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole path over one resident batch: KV-set build,
+FP8 page decode (mixed cache only) and sparse sink attention. The default
+workload is the ratio-4 CSA prefill (2 x 8192 tokens, 128 heads, d = 128,
+W = 128, top-k 512, page 64): the configuration whose tensor-core target the
+method states; its inputs (Q and O are 537 MB each) exceed the 126 MB L2, so
+no flush is needed between steps. Decode workloads (c4, c5) write a 256 MB
+buffer (more than the L2) between timed steps, outside the timed intervals.
+
+Under torchrun every rank runs its own batch (independent requests, no
+collective on the data path; weak scaling); rank 0 prints one JSON line.
+``--impl reference`` times the CPU oracle (the only reference this path
+has) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("attended query·head·KV pairs/s and TFLOP/s (prefill); decode tok/s, HBM GB/s")
+UNIT = "query·head·KV pairs/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 - 0.15 <= t <= t1 + 0.15] or \
+               [s for (_, s) in self.samples[-3:]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4)
+                          if len(r) > 4 + k and r[4 + k].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def physical_gpu(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    parts = [x for x in vis.split(",") if x.strip()]
+    if parts and all(x.strip().isdigit() for x in parts) and local_rank < len(parts):
+        return int(parts[local_rank])
+    return local_rank
+
+
+def algorithmic(w, nnz):
+    """Per-step algorithmic work of the attention launch: FLOPs = 4 d per
+    (query, head, key) triple (2d for QK^T, 2d for PV); HBM bytes = Q + O +
+    LSE + each distinct K/V row once + the CSR indices."""
+    triples = nnz * w.H
+    flops = 4.0 * w.d * triples
+    return triples, flops
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on a bounded sample of the workload."""
+    if rank != 0:
+        return 0
+    import oracle
+    from sparse_paged_attention_build_b200 import workloads
+    w = workloads.make(args.workload)
+    ip, idx = oracle.build_kv_sets(w.pos, w.W, w.ratio, w.topk)
+    k_cmp, v_cmp = w.k_cmp, w.v_cmp
+    if w.k_cmp_fp8 is not None:
+        k_cmp = oracle.dequant_fp8_pages(w.k_cmp_fp8, w.k_cmp_scale, w.cmp_page_ids)
+        v_cmp = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids)
+    threads = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    rows_per_step = args.ref_rows or max(threads, 16)
+    times, triples = [], []
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(w.N, size=min(w.N, rows_per_step), replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, w.sink, w.scale,
+                                k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            triples.append(int((ip[rows + 1] - ip[rows]).sum()) * w.H)
+    value = float(sum(triples) / sum(times))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(times)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, world, None),
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": threads,
+                         "sample": f"{rows_per_step} random query tokens per step (of {w.N}), all heads, "
+                                   f"FP64 C oracle with {threads} threads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, world, nnz):
+    from sparse_paged_attention_build_b200 import workloads
+    c = {"workload": f"{w.name}: {workloads.DESCRIPTIONS[w.name]}", "n_queries": w.N, "heads": w.H,
+         "head_dim": w.d, "window": w.W, "ratio": w.ratio, "topk": w.K,
+         "page_size": w.raw_page_size, "parallelism": f"dp{world}",
+         "l2": "inputs larger than L2 (no flush)" if w.kind == "prefill"
+               else "256 MB buffer written between timed steps (L2 flush)"}
+    if nnz is not None:
+        c["kv_pairs_per_step"] = nnz
+        c["mean_set_size"] = nnz / w.N
+    return c
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank, local_rank, world = env_rank()
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from sparse_paged_attention_build_b200 import workloads
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    import sparse_paged_attention_build_b200 as spa
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = workloads.make(args.workload, seed_offset=rank)
+    decode = w.kind == "decode"
+    b0 = DeviceBatch(w, num_splits=args.splits)
+    stream = torch.cuda.current_stream()
+    b0.step()
+    torch.cuda.synchronize()
+    nnz = b0.nnz()
+    triples, flops = algorithmic(w, nnz)
+    # a decode batch fits in L2: write a buffer larger than L2 between
+    # timed steps (outside the timed intervals)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if decode else None
+
+    for s in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        b0.step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(physical_gpu(local_rank))
+    sampler.start()
+    time.sleep(0.3)
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record(stream)
+    for s in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev[s][0].record(stream)
+        b0.build_sets()
+        b0.dequant()
+        ev[s][1].record(stream)
+        b0.attend()
+        ev[s][2].record(stream)
+    stop.record(stream)
+    stop.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    time.sleep(0.25)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    if decode:   # the sum of the steps, without the flushes between them
+        elapsed_ms = float(sum(e0.elapsed_time(e2) for e0, _, e2 in ev))
+    else:
+        elapsed_ms = start.elapsed_time(stop)
+    attn_ms = float(np.mean([e1.elapsed_time(e2) for _, e1, e2 in ev]))
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = b0.status_word()
+
+    total_triples = triples * args.steps * world
+    value = total_triples / (elapsed_ms / 1e3)
+    pk, pk_kind = peaks()
+    timed_s = elapsed_ms / 1e3
+    peak_tf = pk["bf16_tflops"] if timed_s < 2.0 else pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    achieved_tf = flops / (attn_ms / 1e3) / 1e12
+    kernels_per_step = b0.kernels_per_step()
+
+    # end to end through the public API: pinned host inputs -> device ->
+    # the three calls -> O and LSE back to the host, every step
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(w, b0, args, stream, world, barrier, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, world, nnz),
+            "tflops": flops * args.steps * world / (elapsed_ms / 1e3) / 1e12,
+            "roofline": {"kernel": "sparse_sink_attn_kernel<128>", "bound": "tensor",
+                         "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved_tf / peak_tf, "traffic": None,
+                         "peak_source": f"{pk_kind} {'burst' if timed_s < 2.0 else 'sustained'} bf16",
+                         "attn_ms_per_launch": attn_ms},
+            "clocks": clocks, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
+            "device_status": status,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_e2e(w, b0, args, stream, world, barrier, dist):
+    import torch
+    import sparse_paged_attention_build_b200 as spa
+
+    def pinned(a, dtype=None):
+        if a is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if dtype is not None:
+            t = t.view(dtype)
+        return t.pin_memory()
+
+    bf = torch.bfloat16
+    host = {
+        "q": pinned(w.q.view(np.int16), bf), "pos": pinned(w.pos), "req": pinned(w.req),
+        "topk": pinned(w.topk), "pt_raw": pinned(w.pt_raw), "pt_cmp": pinned(w.pt_cmp),
+        "sink": pinned(w.sink),
+    }
+    if w.kind == "prefill":
+        host["k_raw"] = pinned(w.k_raw.view(np.int16), bf)
+        host["v_raw"] = pinned(w.v_raw.view(np.int16), bf)
+        if w.k_cmp is not None:
+            host["k_cmp"] = pinned(w.k_cmp.view(np.int16), bf)
+            host["v_cmp"] = pinned(w.v_cmp.view(np.int16), bf)
+    if w.k_cmp_fp8 is not None:
+        for k in ("k_cmp_fp8", "v_cmp_fp8", "k_cmp_scale", "v_cmp_scale", "cmp_page_ids"):
+            host[k] = pinned(getattr(w, k))
+    dev = {k: getattr(b0, k) for k in host}
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    out_h = torch.empty(b0.out.shape, dtype=bf).pin_memory()
+    lse_h = torch.empty(b0.lse.shape, dtype=torch.float32).pin_memory()
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        for k, t in host.items():
+            if t is not None:
+                dev[k].copy_(t, non_blocking=True)
+        b0.step()
+        out_h.copy_(b0.out, non_blocking=True)
+        lse_h.copy_(b0.lse, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    e.synchronize()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    triples = b0.nnz() * w.H
+    return {"value": triples * steps * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms / steps, "steps": steps}
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """The FP64 oracle on a bounded sample of the same workload."""
+    import oracle
+    threads = os.cpu_count() or 1
+    ip, idx = oracle.build_kv_sets(w.pos, w.W, w.ratio, w.topk)
+    k_cmp, v_cmp = w.k_cmp, w.v_cmp
+    if w.k_cmp_fp8 is not None:
+        k_cmp = oracle.dequant_fp8_pages(w.k_cmp_fp8, w.k_cmp_scale, w.cmp_page_ids)
+        v_cmp = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids)
+    rng = np.random.default_rng(1)
+
+    def run(n):
+        rows = np.sort(rng.choice(w.N, size=min(n, w.N), replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, w.sink, w.scale,
+                                k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp, rows=rows, threads=threads)
+        return time.perf_counter() - t0, int((ip[rows + 1] - ip[rows]).sum()) * w.H, rows.size
+
+    dt, _, n = run(threads)
+    n2 = int(max(threads, min(w.N, n * budget_s / max(dt, 1e-3))))
+    dt, tri, n2 = run(n2)
+    return {"kind": "oracle", "value": tri / dt, "unit": UNIT, "cores": threads,
+            "sample": f"{n2} random query tokens of {w.N} (all {w.H} heads), FP64 C oracle, "
+                      f"{threads} threads, {dt:.1f} s"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,204 @@
+/*
+ * spa.h -- C ABI of libspa.so: the forward of sparse paged attention with an
+ * attention sink, for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "Roadmap item 24 - joint compressed/window attention with
+ * sink", RL-Kernel PR #628, section "Reuse and arithmetic"): for each query
+ * token a KV set is gathered through a page table -- the complete recent
+ * window of raw tokens plus compressed-KV entries -- and all heads share it.
+ * Compressed KV, window and a per-head sink logit share one softmax
+ * denominator; the sink has no V. O is BF16 and LSE is the FP32 natural log
+ * of the denominator.
+ *
+ * Conventions shared by every call
+ *  - Pointers are DEVICE pointers unless a comment says otherwise. The
+ *    caller owns every buffer; the library never allocates, frees or
+ *    synchronises, and never reads device data on the host, so every call
+ *    can be captured in a CUDA graph. Work is enqueued on `stream`
+ *    (NULL = the legacy default stream).
+ *  - BF16 tensors are passed as `uint16_t*` holding the bit patterns.
+ *  - Host-side validation is synchronous: a call that returns anything but
+ *    SPA_OK has enqueued nothing. `spa_last_error_detail()` names the
+ *    failing clause.
+ *  - Faults that only the device can see (a page id outside the pool, a
+ *    logical index past the page table, a malformed key, an overflow of the
+ *    output capacity, a wait that ran out of time) never trap: the kernel
+ *    skips the offending entry and ORs a SPA_DEV_* bit into `*dev_status`
+ *    (may be NULL, then the bit is dropped). After any fault the call's
+ *    outputs are undefined ("poisoned"); do not reuse them.
+ *  - Workspaces are caller-provided device memory of at least the size the
+ *    matching *_workspace_size() returns; their contents need not be
+ *    initialised and are clobbered. One workspace must not be shared by
+ *    calls that may run at the same time.
+ */
+#ifndef SPA_H_
+#define SPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                     /* == cudaStream_t */
+typedef struct CUstream_st* spa_stream_t;
+
+#define SPA_ABI_VERSION 1
+
+typedef enum {
+    SPA_OK = 0,
+    SPA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad ratio/window ...   */
+    SPA_ERR_UNSUPPORTED = 2,   /* valid, but not a shape/format this build handles    */
+    SPA_ERR_CAPACITY = 3,      /* an output buffer is smaller than the bound          */
+    SPA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required          */
+    SPA_ERR_ALIGNMENT = 5,     /* a pointer or stride breaks the 16-byte rule         */
+    SPA_ERR_CUDA = 6,          /* a CUDA runtime call failed (e.g. launch)            */
+} spa_status;
+
+/* Bits of the device status word. */
+#define SPA_DEV_BAD_PAGE  1u   /* page id outside [0, num_pages)                      */
+#define SPA_DEV_BAD_INDEX 2u   /* key/position/request outside its table              */
+#define SPA_DEV_CAPACITY  4u   /* the key sets overflowed `capacity`                  */
+#define SPA_DEV_TIMEOUT   8u   /* a bounded wait inside a kernel ran out              */
+
+/* A key is a compressed-group index g (0 <= g < 2^30) or
+ * SPA_WINDOW_TAG | t for raw token t (0 <= t < 2^30). Ascending key order is
+ * the canonical order of a set: compressed groups first, then the window. */
+#define SPA_WINDOW_TAG (1 << 30)
+
+int spa_abi_version(void);
+const char* spa_status_string(int status);
+/* Host-thread-local text naming the clause that made the last call on this
+ * thread fail ("" after a success). */
+const char* spa_last_error_detail(void);
+
+/* ------------------------------------------------------------------------
+ * 1. spa_build_kv_sets -- per-token KV sets as CSR, canonical order.
+ *
+ * Defined by "Roadmap item 24", section "Contracts and lifetime" (logical
+ * request/position/kind keys, complete windows, C4/C128 group boundaries,
+ * canonical KV ordering), and "test: add block-level DeepSeek-V4 attention
+ * test" (ROCm/ATOM PR #1723), opening section (layer types: compress ratio
+ * 0 = dense, 4 = CSA, 128 = HCA) and "Validation" (top-k truncates only once
+ * the complete groups outnumber it).
+ *
+ * For query i at position p = pos[i]:
+ *   window  = { SPA_WINDOW_TAG | t : max(0, p-W+1) <= t <= p }
+ *   groups  = none                                  (ratio 0)
+ *           = { g : 0 <= g < floor((p+1)/ratio) }   (topk == NULL)
+ *           = { topk[i][j] : 0 <= topk[i][j] < floor((p+1)/ratio) } (else),
+ *             repeats removed (a group is complete once all `ratio` of its
+ *             tokens are at or before p)
+ *   set_i   = ascending(groups U window)
+ *   indptr[0] = 0, indptr[i+1] = indptr[i] + |set_i|,
+ *   indices[indptr[i] .. indptr[i+1]) = set_i.
+ *
+ * pos      int32 [n_queries], 0 <= pos < 2^30 (else SPA_DEV_BAD_INDEX and an
+ *          empty set for that query)
+ * window   W >= 1
+ * ratio    0, 4 or 128
+ * topk     int32 [n_queries, topk_width] row-major, or NULL; entries < 0
+ *          are padding. topk_width <= 2048.
+ * indptr   int32 [n_queries + 1] (output)
+ * indices  int32 [capacity] (output); capacity >= spa_kv_sets_capacity(..)
+ *          of the true maximum position is enough. Keys past `capacity`
+ *          are dropped and SPA_DEV_CAPACITY is set.
+ * workspace >= spa_build_kv_sets_workspace_size(n_queries) bytes.
+ * ---------------------------------------------------------------------- */
+int64_t spa_kv_sets_capacity(int32_t n_queries, int32_t window, int32_t ratio,
+                             int32_t topk_width, int32_t has_topk, int32_t max_pos);
+size_t spa_build_kv_sets_workspace_size(int32_t n_queries);
+int spa_build_kv_sets(const int32_t* pos, int32_t n_queries, int32_t window, int32_t ratio,
+                      const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                      int32_t* indices, int64_t capacity, void* workspace,
+                      size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * 2. spa_dequant_fp8_pages -- mixed FP8/BF16 cache: FP8 pages to BF16.
+ *
+ * Defined by "Roadmap item 24", section "Reuse and arithmetic" (a mixed
+ * FP8/BF16 cache decoder with an explicit OCP/FNUZ format and 64/128-token
+ * pages). Format: OCP E4M3 (bias 7, subnormals, S.1111.111 = NaN, max 448),
+ * one FP32 scale per 64 consecutive elements of a token row.
+ *
+ * For every listed page pg and every element e of its rows:
+ *   dst[pg][s][e] = bf16_rne( float(e4m3(src[pg][s][e])) * scales[pg][s][e/64] )
+ * (one binary32 multiply, then round-to-nearest-even to BF16). Unlisted
+ * pages of dst are not written.
+ *
+ * src       uint8 [num_pages, page_size, head_dim], 16-byte aligned
+ * scales    float [num_pages, page_size, head_dim/64]
+ * page_ids  int32 [n_page_ids]; ids outside [0, num_pages) set
+ *           SPA_DEV_BAD_PAGE and are skipped
+ * fp8_format 0 = OCP E4M3 (FNUZ is SPA_ERR_UNSUPPORTED)
+ * dst       BF16 bits [num_pages, page_size, head_dim], 16-byte aligned
+ * head_dim  a multiple of 64
+ * ---------------------------------------------------------------------- */
+int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
+                          int32_t page_size, int32_t head_dim, const int32_t* page_ids,
+                          int32_t n_page_ids, int32_t fp8_format, uint16_t* dst,
+                          uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * 3. spa_sparse_sink_attn_fwd -- attention over the per-token sets.
+ *
+ * Defined by "Roadmap item 24", section "Reuse and arithmetic" (compressed
+ * KV + full recent window + sink share the denominator; the sink has no V;
+ * BF16 P/O and FP32 natural-log LSE), and "test: add block-level
+ * DeepSeek-V4 attention test", "What this test actually drives" (sparse
+ * decode over KV splits followed by a reduce: here an exact LSE merge).
+ *
+ * For query i (request b = req[i]) and head h, over the keys of set i:
+ *   s_j   = scale * dot(q[i][h], k_j)
+ *   LSE   = ln( e^{sink[h]} + sum_j e^{s_j} )
+ *   O     = sum_j e^{s_j - LSE} v_j        (the sink contributes no V)
+ * A window key (SPA_WINDOW_TAG | t) reads row t of request b through
+ * pt_raw: page = pt_raw[b][t / raw_page_size], slot = t % raw_page_size;
+ * a compressed key g reads row g through pt_cmp the same way. P is rounded
+ * to BF16 before the PV product, as on the page; accumulation is FP32.
+ * sink == NULL means no sink (plain softmax); an empty set gives O = 0 and
+ * LSE = sink[h] (or -inf without a sink).
+ *
+ * q          BF16 [n_queries, num_heads, head_dim]; element (i,h,e) at
+ *            q + i*q_stride_tok + h*q_stride_head + e. Base and both
+ *            strides (in bytes) must be multiples of 16.
+ * head_dim   64 or 128 (d_qk = d_v)
+ * num_heads  1..128, or a multiple of 128
+ * k_raw, v_raw   BF16 [raw_num_pages, raw_page_size, head_dim], 16-B aligned
+ * pt_raw     int32 [n_requests, pt_raw_cols]
+ * k_cmp, v_cmp, pt_cmp   the compressed pool, laid out the same way; may be
+ *            NULL when no set holds a compressed key (ratio 0)
+ * page sizes powers of two, 1 .. 1024
+ * req        int32 [n_queries]
+ * indptr, indices   CSR key sets (as built by spa_build_kv_sets; any order
+ *            within a set is accepted)
+ * sink       float [num_heads] natural-log logits, or NULL
+ * scale      > 0
+ * out        BF16 [n_queries, num_heads, head_dim] contiguous, 16-B aligned
+ * lse        float [n_queries, num_heads]
+ * num_splits 0 = automatic, 1 = one CTA per query, S in 2..16 = the set of
+ *            each query is cut into S slices of 64-key tiles whose partial
+ *            results are merged exactly (O_s, LSE_s weighted by e^{LSE_s-LSE}).
+ * workspace  >= spa_sparse_sink_attn_workspace_size(...) bytes for the same
+ *            arguments (0 bytes when the call runs unsplit).
+ * ---------------------------------------------------------------------- */
+size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads,
+                                           int32_t head_dim, int32_t num_splits);
+int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads,
+                                       int32_t max_set_size);
+int spa_sparse_sink_attn_fwd(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+    int32_t num_heads, int32_t head_dim,
+    const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+    const int32_t* pt_raw, int32_t pt_raw_cols,
+    const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages, int32_t cmp_page_size,
+    const int32_t* pt_cmp, int32_t pt_cmp_cols,
+    const int32_t* req, int32_t n_requests, const int32_t* indptr, const int32_t* indices,
+    const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
+    void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPA_H_ */

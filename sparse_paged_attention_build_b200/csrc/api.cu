@@ -1,0 +1,251 @@
+// The C ABI of libspa.so (declared in include/spa.h): host-side argument
+// validation, workspace sizing and launch. Every failing clause returns
+// before anything is enqueued and leaves a message for
+// spa_last_error_detail(). No call allocates, frees or synchronises.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "spa.h"
+#include "spa_internal.h"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+int ok() {
+  g_detail[0] = '\0';
+  return SPA_OK;
+}
+
+int cuda_status(cudaError_t err, const char* what) {
+  if (err == cudaSuccess) return ok();
+  return fail(SPA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool pow2_in(int32_t v, int32_t lo, int32_t hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+int sm_count() {
+  static int cached = 0;
+  if (cached == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+      cached = n;
+    else
+      cached = 148;
+  }
+  return cached;
+}
+
+int32_t resolve_splits(int32_t n_queries, int32_t num_heads, int32_t requested) {
+  if (requested > 0) return requested;
+  return spa_sparse_sink_attn_choose_splits(n_queries, num_heads, 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+int spa_abi_version(void) { return SPA_ABI_VERSION; }
+
+const char* spa_status_string(int status) {
+  switch (status) {
+    case SPA_OK: return "ok";
+    case SPA_ERR_INVALID_ARG: return "invalid argument";
+    case SPA_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case SPA_ERR_CAPACITY: return "output capacity too small";
+    case SPA_ERR_WORKSPACE: return "workspace missing or too small";
+    case SPA_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case SPA_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+const char* spa_last_error_detail(void) { return g_detail; }
+
+// ---------------------------------------------------------------- sets
+int64_t spa_kv_sets_capacity(int32_t n_queries, int32_t window, int32_t ratio, int32_t topk_width,
+                             int32_t has_topk, int32_t max_pos) {
+  if (n_queries <= 0 || window < 1 || max_pos < 0) return 0;
+  const int64_t win = std::min<int64_t>(window, static_cast<int64_t>(max_pos) + 1);
+  int64_t groups = 0;
+  if (ratio > 0) {
+    groups = (static_cast<int64_t>(max_pos) + 1) / ratio;
+    if (has_topk) groups = std::min<int64_t>(groups, topk_width);
+  }
+  return static_cast<int64_t>(n_queries) * (win + groups);
+}
+
+size_t spa_build_kv_sets_workspace_size(int32_t n_queries) {
+  return n_queries < 0 ? 0 : spa::build_kv_sets_workspace_bytes(n_queries);
+}
+
+int spa_build_kv_sets(const int32_t* pos, int32_t n_queries, int32_t window, int32_t ratio,
+                      const int32_t* topk, int32_t topk_width, int32_t* indptr, int32_t* indices,
+                      int64_t capacity, void* workspace, size_t workspace_bytes,
+                      uint32_t* dev_status, spa_stream_t stream) {
+  if (n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
+  if (window < 1) return fail(SPA_ERR_INVALID_ARG, "window < 1");
+  if (ratio != 0 && ratio != 4 && ratio != 128) return fail(SPA_ERR_INVALID_ARG, "ratio must be 0, 4 or 128");
+  if (topk_width < 0) return fail(SPA_ERR_INVALID_ARG, "topk_width < 0");
+  if (capacity < 0) return fail(SPA_ERR_INVALID_ARG, "capacity < 0");
+  if (indptr == nullptr) return fail(SPA_ERR_INVALID_ARG, "indptr is NULL");
+  if (n_queries > 0 && pos == nullptr) return fail(SPA_ERR_INVALID_ARG, "pos is NULL");
+  if (n_queries > 0 && capacity > 0 && indices == nullptr) return fail(SPA_ERR_INVALID_ARG, "indices is NULL");
+  if (ratio > 0 && topk != nullptr && topk_width > spa::kMaxTopkWidth)
+    return fail(SPA_ERR_UNSUPPORTED, "topk_width > %d", spa::kMaxTopkWidth);
+  if (!aligned(pos, 4) || !aligned(topk, 4) || !aligned(indptr, 4) || !aligned(indices, 4))
+    return fail(SPA_ERR_ALIGNMENT, "int32 arrays must be 4-byte aligned");
+  if (n_queries > 0) {
+    const size_t need = spa::build_kv_sets_workspace_bytes(n_queries);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(SPA_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+    if (!aligned(workspace, 16)) return fail(SPA_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  }
+  return cuda_status(spa::launch_build_kv_sets(pos, n_queries, window, ratio, topk, topk_width, indptr,
+                                               indices, capacity, workspace, dev_status,
+                                               reinterpret_cast<cudaStream_t>(stream)),
+                     "build_kv_sets launch");
+}
+
+// ---------------------------------------------------------------- dequant
+int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages, int32_t page_size,
+                          int32_t head_dim, const int32_t* page_ids, int32_t n_page_ids,
+                          int32_t fp8_format, uint16_t* dst, uint32_t* dev_status, spa_stream_t stream) {
+  if (num_pages < 0) return fail(SPA_ERR_INVALID_ARG, "num_pages < 0");
+  if (page_size < 1) return fail(SPA_ERR_INVALID_ARG, "page_size < 1");
+  if (head_dim < 1) return fail(SPA_ERR_INVALID_ARG, "head_dim < 1");
+  if (n_page_ids < 0) return fail(SPA_ERR_INVALID_ARG, "n_page_ids < 0");
+  if (fp8_format == 1) return fail(SPA_ERR_UNSUPPORTED, "FNUZ E4M3 is not supported");
+  if (fp8_format != 0) return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3)");
+  if (head_dim % 64 != 0) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be a multiple of 64");
+  if (static_cast<int64_t>(page_size) * head_dim > (1 << 24))
+    return fail(SPA_ERR_UNSUPPORTED, "page_size * head_dim too large");
+  if (n_page_ids > 0 && (src == nullptr || scales == nullptr || page_ids == nullptr || dst == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "src, scales, page_ids and dst must be non-NULL");
+  if (!aligned(src, 16) || !aligned(dst, 16)) return fail(SPA_ERR_ALIGNMENT, "src and dst must be 16-byte aligned");
+  if (!aligned(scales, 4) || !aligned(page_ids, 4)) return fail(SPA_ERR_ALIGNMENT, "scales/page_ids misaligned");
+  return cuda_status(spa::launch_dequant_fp8_pages(src, scales, num_pages, page_size, head_dim, page_ids,
+                                                   n_page_ids, dst, dev_status,
+                                                   reinterpret_cast<cudaStream_t>(stream)),
+                     "dequant_fp8_pages launch");
+}
+
+// ---------------------------------------------------------------- attention
+int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int32_t max_set_size) {
+  if (n_queries <= 0 || num_heads <= 0) return 1;
+  const int64_t head_tiles = (num_heads + 127) / 128;
+  const int64_t units = static_cast<int64_t>(n_queries) * head_tiles;
+  const int64_t target = 2 * static_cast<int64_t>(sm_count());   // two CTAs per SM
+  int64_t s = (target + units - 1) / units;
+  if (max_set_size > 0) s = std::min<int64_t>(s, (max_set_size + spa::kAttnKeysPerTile - 1) / spa::kAttnKeysPerTile);
+  s = std::max<int64_t>(1, std::min<int64_t>(s, spa::kAttnMaxSplits));
+  return static_cast<int>(s);
+}
+
+size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads, int32_t head_dim,
+                                           int32_t num_splits) {
+  if (n_queries <= 0 || num_heads <= 0 || head_dim <= 0 || num_splits < 0) return 0;
+  return spa::attn_workspace_bytes(n_queries, num_heads, head_dim,
+                                   resolve_splits(n_queries, num_heads, num_splits));
+}
+
+int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+                             int32_t num_heads, int32_t head_dim, const uint16_t* k_raw, const uint16_t* v_raw,
+                             int64_t raw_num_pages, int32_t raw_page_size, const int32_t* pt_raw,
+                             int32_t pt_raw_cols, const uint16_t* k_cmp, const uint16_t* v_cmp,
+                             int64_t cmp_num_pages, int32_t cmp_page_size, const int32_t* pt_cmp,
+                             int32_t pt_cmp_cols, const int32_t* req, int32_t n_requests,
+                             const int32_t* indptr, const int32_t* indices, const float* sink, float scale,
+                             uint16_t* out, float* lse, int32_t num_splits, void* workspace,
+                             size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
+  if (n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
+  if (num_heads < 1) return fail(SPA_ERR_INVALID_ARG, "num_heads < 1");
+  if (n_requests < 1) return fail(SPA_ERR_INVALID_ARG, "n_requests < 1");
+  if (head_dim != 64 && head_dim != 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (num_heads > 128 && num_heads % 128 != 0)
+    return fail(SPA_ERR_UNSUPPORTED, "num_heads above 128 must be a multiple of 128");
+  if (raw_num_pages < 0 || pt_raw_cols < 0) return fail(SPA_ERR_INVALID_ARG, "raw pool sizes < 0");
+  if (raw_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "raw_page_size < 1");
+  if (!pow2_in(raw_page_size, 1, 1024)) return fail(SPA_ERR_UNSUPPORTED, "raw_page_size must be a power of two <= 1024");
+  if (pt_cmp != nullptr) {
+    if (cmp_num_pages < 0 || pt_cmp_cols < 0) return fail(SPA_ERR_INVALID_ARG, "compressed pool sizes < 0");
+    if (cmp_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "cmp_page_size < 1");
+    if (!pow2_in(cmp_page_size, 1, 1024))
+      return fail(SPA_ERR_UNSUPPORTED, "cmp_page_size must be a power of two <= 1024");
+    if (k_cmp == nullptr || v_cmp == nullptr) return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
+  }
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(SPA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (num_splits < 0 || num_splits > spa::kAttnMaxSplits)
+    return fail(SPA_ERR_INVALID_ARG, "num_splits must be in [0, %d]", spa::kAttnMaxSplits);
+  if (q_stride_tok < 0 || q_stride_head < 0) return fail(SPA_ERR_INVALID_ARG, "negative q stride");
+  if (n_queries == 0) return ok();
+  if (q == nullptr || out == nullptr || lse == nullptr) return fail(SPA_ERR_INVALID_ARG, "q, out and lse must be non-NULL");
+  if (k_raw == nullptr || v_raw == nullptr || pt_raw == nullptr)
+    return fail(SPA_ERR_INVALID_ARG, "k_raw, v_raw and pt_raw must be non-NULL");
+  if (req == nullptr || indptr == nullptr || indices == nullptr)
+    return fail(SPA_ERR_INVALID_ARG, "req, indptr and indices must be non-NULL");
+  if (!aligned(q, 16) || (q_stride_tok * 2) % 16 != 0 || (q_stride_head * 2) % 16 != 0)
+    return fail(SPA_ERR_ALIGNMENT, "q base and strides must be 16-byte multiples");
+  if (!aligned(k_raw, 16) || !aligned(v_raw, 16) || !aligned(k_cmp, 16) || !aligned(v_cmp, 16))
+    return fail(SPA_ERR_ALIGNMENT, "K/V pools must be 16-byte aligned");
+  if (!aligned(out, 16)) return fail(SPA_ERR_ALIGNMENT, "out must be 16-byte aligned");
+  if (!aligned(lse, 4) || !aligned(sink, 4) || !aligned(req, 4) || !aligned(indptr, 4) || !aligned(indices, 4) ||
+      !aligned(pt_raw, 4) || !aligned(pt_cmp, 4))
+    return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
+  const int32_t splits = resolve_splits(n_queries, num_heads, num_splits);
+  if (static_cast<int64_t>(n_queries) * splits > 0x7fffffffLL)
+    return fail(SPA_ERR_UNSUPPORTED, "n_queries * num_splits exceeds the grid");
+  const size_t need = spa::attn_workspace_bytes(n_queries, num_heads, head_dim, splits);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(SPA_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+    if (!aligned(workspace, 256)) return fail(SPA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  }
+  spa::AttnArgs a;
+  a.q = q;
+  a.q_stride_tok = q_stride_tok;
+  a.q_stride_head = q_stride_head;
+  a.n_queries = n_queries;
+  a.num_heads = num_heads;
+  a.head_dim = head_dim;
+  a.k_raw = k_raw;
+  a.v_raw = v_raw;
+  a.raw_num_pages = raw_num_pages;
+  a.raw_page_size = raw_page_size;
+  a.pt_raw = pt_raw;
+  a.pt_raw_cols = pt_raw_cols;
+  a.k_cmp = k_cmp;
+  a.v_cmp = v_cmp;
+  a.cmp_num_pages = cmp_num_pages;
+  a.cmp_page_size = cmp_page_size;
+  a.pt_cmp = pt_cmp;
+  a.pt_cmp_cols = pt_cmp_cols;
+  a.req = req;
+  a.n_requests = n_requests;
+  a.indptr = indptr;
+  a.indices = indices;
+  a.sink = sink;
+  a.scale = scale;
+  a.out = out;
+  a.lse = lse;
+  a.num_splits = splits;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  return cuda_status(spa::launch_sparse_sink_attn(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "sparse_sink_attn launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,247 @@
+// Per-token KV sets as CSR in canonical (ascending key) order.
+//
+// Page "Roadmap item 24 - joint compressed/window attention with sink",
+// section "Contracts and lifetime": logical request/position/kind keys,
+// complete windows, C4/C128 group boundaries, canonical KV ordering. Page
+// "test: add block-level DeepSeek-V4 attention test", opening section and
+// "Validation": ratio 0 / 4 / 128 layers; top-k truncates only once the
+// complete groups outnumber it.
+//
+// One pass over the queries. A CTA owns 8 consecutive queries, one warp
+// each. A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio)),
+// sorts it in shared memory with a bitonic network and counts the distinct
+// survivors; the window adds min(p+1, W) keys. The CTA publishes its total
+// and obtains its offset by a decoupled look-back over the CTAs before it
+// (CTA order taken from an atomic ticket, so every predecessor is already
+// running), then every warp writes its indptr entry and its keys: the
+// distinct groups ascending, then the window tokens ascending with the
+// window tag. Integer only; no floating point anywhere.
+#include <climits>
+
+#include "spa_device.cuh"
+#include "spa_internal.h"
+
+namespace spa {
+namespace {
+
+constexpr uint64_t kFlagAggregate = 1ull << 62;
+constexpr uint64_t kFlagInclusive = 2ull << 62;
+constexpr uint64_t kValueMask = (1ull << 62) - 1;
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Ascending bitonic sort of buf[0, n) (n a power of two) by one warp.
+__device__ void warp_bitonic_sort(int32_t* buf, int n, int lane) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = lane; t < (n >> 1); t += 32) {
+        const int lo = ((t & ~(j - 1)) << 1) | (t & (j - 1));
+        const int hi = lo | j;
+        const bool up = (lo & k) == 0;
+        const int32_t a = buf[lo], b = buf[hi];
+        if ((a > b) == up) {
+          buf[lo] = b;
+          buf[hi] = a;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+struct SetsParams {
+  const int32_t* pos;
+  int32_t n;
+  int32_t window;
+  int32_t ratio;
+  const int32_t* topk;
+  int32_t topk_width;
+  int32_t sort_width;  // topk_width rounded up to a power of two (>= 32)
+  int32_t* indptr;
+  int32_t* indices;
+  int64_t capacity;
+  uint64_t* tile_status;
+  uint32_t* tile_ticket;
+  uint32_t* dev_status;
+};
+
+__global__ void __launch_bounds__(kSetsQueriesPerCta * 32)
+build_kv_sets_kernel(const SetsParams P) {
+  extern __shared__ int32_t sort_buf[];  // [kSetsQueriesPerCta][sort_width]
+  __shared__ int64_t s_count[kSetsQueriesPerCta];
+  __shared__ int64_t s_tile_offset;
+  __shared__ uint32_t s_tile;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) s_tile = atomicAdd(P.tile_ticket, 1u);
+  __syncthreads();
+  const uint32_t tile = s_tile;
+  const int64_t i = static_cast<int64_t>(tile) * kSetsQueriesPerCta + warp;
+  const bool active = i < P.n;
+
+  int32_t p = 0, n_window = 0, n_complete = 0;
+  int64_t n_groups = 0;
+  int32_t* buf = sort_buf + warp * P.sort_width;
+  const bool sorted_list = P.ratio > 0 && P.topk != nullptr;
+  if (active) {
+    p = P.pos[i];
+    if (p < 0 || p >= SPA_WINDOW_TAG) {
+      if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
+      p = -1;  // empty set
+    } else {
+      n_window = min(p + 1, P.window);
+      n_complete = P.ratio > 0 ? (p + 1) / P.ratio : 0;
+    }
+    if (p >= 0 && P.ratio > 0) {
+      if (!sorted_list) {
+        n_groups = n_complete;
+      } else {
+        const int32_t* row = P.topk + i * P.topk_width;
+        for (int j = lane; j < P.sort_width; j += 32) {
+          int32_t g = j < P.topk_width ? row[j] : -1;
+          buf[j] = (g >= 0 && g < n_complete) ? g : INT_MAX;
+        }
+        __syncwarp();
+        warp_bitonic_sort(buf, P.sort_width, lane);
+        int64_t distinct = 0;
+        for (int j0 = 0; j0 < P.sort_width; j0 += 32) {
+          const int j = j0 + lane;
+          const int32_t v = buf[j];
+          const bool first = v != INT_MAX && (j == 0 || buf[j - 1] != v);
+          distinct += __popc(__ballot_sync(0xffffffffu, first));
+        }
+        n_groups = distinct;
+      }
+    }
+  }
+  const int64_t count = active && p >= 0 ? n_groups + n_window : 0;
+  if (lane == 0) s_count[warp] = count;
+  __syncthreads();
+
+  // Offset of this CTA's first key: decoupled look-back.
+  if (threadIdx.x == 0) {
+    int64_t aggregate = 0;
+    for (int w = 0; w < kSetsQueriesPerCta; ++w) aggregate += s_count[w];
+    int64_t exclusive = 0;
+    if (tile == 0) {
+      st_relaxed_u64(P.tile_status, kFlagInclusive | static_cast<uint64_t>(aggregate));
+    } else {
+      st_relaxed_u64(P.tile_status + tile, kFlagAggregate | static_cast<uint64_t>(aggregate));
+      int64_t pred = static_cast<int64_t>(tile) - 1;
+      const uint64_t t0 = global_timer_ns();
+      uint32_t spins = 0;
+      while (pred >= 0) {
+        const uint64_t s = ld_relaxed_u64(P.tile_status + pred);
+        if ((s & ~kValueMask) == 0) {
+          if ((++spins & 63u) == 0 && global_timer_ns() - t0 > kWaitTimeoutNs) {
+            report(P.dev_status, SPA_DEV_TIMEOUT);
+            break;
+          }
+          continue;
+        }
+        exclusive += static_cast<int64_t>(s & kValueMask);
+        if ((s & ~kValueMask) == kFlagInclusive) break;
+        --pred;
+      }
+      st_relaxed_u64(P.tile_status + tile,
+                     kFlagInclusive | static_cast<uint64_t>(exclusive + aggregate));
+    }
+    s_tile_offset = exclusive;
+  }
+  __syncthreads();
+  if (!active) return;
+
+  int64_t start = s_tile_offset;
+  for (int w = 0; w < warp; ++w) start += s_count[w];
+  const int64_t end = start + count;
+  if (lane == 0) {
+    if (end > P.capacity || end > INT_MAX) report(P.dev_status, SPA_DEV_CAPACITY);
+    P.indptr[i] = static_cast<int32_t>(start < INT_MAX ? start : INT_MAX);
+    if (i == P.n - 1) P.indptr[P.n] = static_cast<int32_t>(end < INT_MAX ? end : INT_MAX);
+  }
+  if (count == 0) return;
+  const int64_t limit = P.capacity < INT_MAX ? P.capacity : INT_MAX;
+
+  // compressed groups, ascending
+  if (sorted_list) {
+    int64_t written = 0;
+    for (int j0 = 0; j0 < P.sort_width; j0 += 32) {
+      if (buf[j0] == INT_MAX) break;  // sentinels sort last
+      const int j = j0 + lane;
+      const int32_t v = buf[j];
+      const bool first = v != INT_MAX && (j == 0 || buf[j - 1] != v);
+      const uint32_t m = __ballot_sync(0xffffffffu, first);
+      const int64_t dst = start + written + __popc(m & ((1u << lane) - 1u));
+      if (first && dst < limit) P.indices[dst] = v;
+      written += __popc(m);
+    }
+  } else {
+    for (int64_t g = lane; g < n_groups; g += 32) {
+      const int64_t dst = start + g;
+      if (dst < limit) P.indices[dst] = static_cast<int32_t>(g);
+    }
+  }
+  // window tokens, ascending
+  const int32_t t0 = p - n_window + 1;
+  for (int t = lane; t < n_window; t += 32) {
+    const int64_t dst = start + n_groups + t;
+    if (dst < limit) P.indices[dst] = SPA_WINDOW_TAG | (t0 + t);
+  }
+}
+
+int sort_width_for(int32_t topk_width) {
+  int w = 32;
+  while (w < topk_width) w <<= 1;
+  return w;
+}
+
+}  // namespace
+
+size_t build_kv_sets_workspace_bytes(int32_t n_queries) {
+  const int64_t tiles = (static_cast<int64_t>(n_queries) + kSetsQueriesPerCta - 1) / kSetsQueriesPerCta;
+  return static_cast<size_t>(tiles) * sizeof(uint64_t) + 16;
+}
+
+cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
+                                 const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                                 int32_t* indices, int64_t capacity, void* ws,
+                                 uint32_t* dev_status, cudaStream_t stream) {
+  if (n == 0) return cudaMemsetAsync(indptr, 0, sizeof(int32_t), stream);
+  const int64_t tiles = (static_cast<int64_t>(n) + kSetsQueriesPerCta - 1) / kSetsQueriesPerCta;
+  cudaError_t err = cudaMemsetAsync(ws, 0, build_kv_sets_workspace_bytes(n), stream);
+  if (err != cudaSuccess) return err;
+  SetsParams P;
+  P.pos = pos;
+  P.n = n;
+  P.window = window;
+  P.ratio = ratio;
+  P.topk = (ratio > 0) ? topk : nullptr;
+  P.topk_width = topk_width;
+  P.sort_width = (P.topk != nullptr) ? sort_width_for(topk_width) : 32;
+  P.indptr = indptr;
+  P.indices = indices;
+  P.capacity = capacity;
+  P.tile_status = static_cast<uint64_t*>(ws);
+  P.tile_ticket = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + tiles * sizeof(uint64_t));
+  P.dev_status = dev_status;
+  const size_t smem = (P.topk != nullptr)
+                          ? static_cast<size_t>(kSetsQueriesPerCta) * P.sort_width * sizeof(int32_t)
+                          : 0;
+  if (smem > 48 * 1024) {
+    err = cudaFuncSetAttribute(build_kv_sets_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  build_kv_sets_kernel<<<static_cast<unsigned>(tiles), kSetsQueriesPerCta * 32, smem, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace spa

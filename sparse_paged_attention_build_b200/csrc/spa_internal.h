@@ -1,0 +1,58 @@
+// Launchers shared between the C ABI (api.cu) and the kernel files. Host
+// validation happens in api.cu; these only enqueue work.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace spa {
+
+constexpr int kSetsQueriesPerCta = 8;      // one warp per query
+constexpr int kMaxTopkWidth = 2048;
+
+size_t build_kv_sets_workspace_bytes(int32_t n_queries);
+cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
+                                 const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                                 int32_t* indices, int64_t capacity, void* ws,
+                                 uint32_t* dev_status, cudaStream_t stream);
+
+cudaError_t launch_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
+                                     int32_t page_size, int32_t head_dim, const int32_t* page_ids,
+                                     int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status,
+                                     cudaStream_t stream);
+
+struct AttnArgs {
+  const uint16_t* q;
+  int64_t q_stride_tok, q_stride_head;  // elements
+  int32_t n_queries, num_heads, head_dim;
+  const uint16_t *k_raw, *v_raw;
+  int64_t raw_num_pages;
+  int32_t raw_page_size;
+  const int32_t* pt_raw;
+  int32_t pt_raw_cols;
+  const uint16_t *k_cmp, *v_cmp;
+  int64_t cmp_num_pages;
+  int32_t cmp_page_size;
+  const int32_t* pt_cmp;
+  int32_t pt_cmp_cols;
+  const int32_t* req;
+  int32_t n_requests;
+  const int32_t* indptr;
+  const int32_t* indices;
+  const float* sink;
+  float scale;
+  uint16_t* out;
+  float* lse;
+  int32_t num_splits;  // >= 1, resolved
+  void* workspace;
+  uint32_t* dev_status;
+};
+
+constexpr int kAttnKeysPerTile = 64;
+constexpr int kAttnMaxSplits = 16;
+size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_dim,
+                            int32_t num_splits);
+cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace spa

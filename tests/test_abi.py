@@ -1,0 +1,154 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/spa.h declares, sizes workspaces, and rejects each bad argument
+with its own validation clause before touching the device (the guard
+matrix asks that each fault hit a distinct clause: page "Roadmap item 24 -
+joint compressed/window attention with sink", review of the ROCm guard
+test)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_paged_attention_build_b200 import build
+    build.build()
+    import sparse_paged_attention_build_b200 as spa
+    return spa.lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(spa_\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 10, names
+    so = ctypes.CDLL(os.path.join(ROOT, "sparse_paged_attention_build_b200", "libspa.so"))
+    for n in names:
+        assert hasattr(so, n), n
+
+
+def test_host_helpers(L):
+    assert L.spa_abi_version() == 1
+    assert L.spa_status_string(0) == b"ok"
+    assert L.spa_status_string(4) == b"workspace missing or too small"
+    # capacity bound: N * (min(W, p+1) + min(K, (p+1)/r))
+    assert L.spa_kv_sets_capacity(16384, 128, 4, 512, 1, 8191) == 16384 * 640
+    assert L.spa_kv_sets_capacity(64, 128, 128, 0, 0, 65535) == 64 * (128 + 512)
+    assert L.spa_kv_sets_capacity(10, 128, 0, 0, 0, 5) == 60
+    assert L.spa_build_kv_sets_workspace_size(17) == 3 * 8 + 16
+    assert L.spa_sparse_sink_attn_workspace_size(100, 128, 128, 1) == 0
+    w2 = L.spa_sparse_sink_attn_workspace_size(10, 128, 128, 2)
+    assert w2 >= 10 * 2 * 128 * 128 * 4 + 10 * 2 * 128 * 8 + 10 * 4
+    assert L.spa_sparse_sink_attn_choose_splits(100000, 128, 0) == 1
+    assert 1 <= L.spa_sparse_sink_attn_choose_splits(64, 128, 0) <= 16
+    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 100) == 2
+
+
+FAKE = 0x10000  # a 16-byte aligned non-NULL address; never dereferenced on these paths
+
+
+def sets_call(L, **kw):
+    a = dict(pos=FAKE, n=8, W=128, ratio=4, topk=FAKE, K=16, indptr=FAKE, indices=FAKE, cap=1000,
+             ws=FAKE, ws_bytes=1 << 20)
+    a.update(kw)
+    return L.spa_build_kv_sets(a["pos"], a["n"], a["W"], a["ratio"], a["topk"], a["K"], a["indptr"],
+                               a["indices"], a["cap"], a["ws"], a["ws_bytes"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(n=-1), 1, "n_queries < 0"),
+    (dict(W=0), 1, "window < 1"),
+    (dict(ratio=3), 1, "ratio must be"),
+    (dict(K=-1), 1, "topk_width < 0"),
+    (dict(cap=-1), 1, "capacity < 0"),
+    (dict(indptr=None), 1, "indptr is NULL"),
+    (dict(pos=None), 1, "pos is NULL"),
+    (dict(indices=None), 1, "indices is NULL"),
+    (dict(K=4096), 2, "topk_width >"),
+    (dict(pos=FAKE + 2), 5, "int32 arrays"),
+    (dict(ws=None), 4, "workspace needs"),
+    (dict(ws_bytes=8), 4, "workspace needs"),
+    (dict(ws=FAKE + 8), 5, "workspace must be 16-byte"),
+])
+def test_guard_matrix_build_kv_sets(L, kw, status, clause):
+    assert sets_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def dq_call(L, **kw):
+    a = dict(src=FAKE, scales=FAKE, P=4, ps=64, d=128, ids=FAKE, n=2, fmt=0, dst=FAKE)
+    a.update(kw)
+    return L.spa_dequant_fp8_pages(a["src"], a["scales"], a["P"], a["ps"], a["d"], a["ids"], a["n"],
+                                   a["fmt"], a["dst"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(P=-1), 1, "num_pages < 0"),
+    (dict(ps=0), 1, "page_size < 1"),
+    (dict(d=0), 1, "head_dim < 1"),
+    (dict(n=-1), 1, "n_page_ids < 0"),
+    (dict(fmt=1), 2, "FNUZ"),
+    (dict(fmt=7), 1, "fp8_format must be 0"),
+    (dict(d=96), 2, "multiple of 64"),
+    (dict(src=None), 1, "must be non-NULL"),
+    (dict(dst=FAKE + 4), 5, "src and dst must be 16-byte"),
+    (dict(scales=FAKE + 1), 5, "scales/page_ids"),
+])
+def test_guard_matrix_dequant(L, kw, status, clause):
+    assert dq_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def attn_call(L, **kw):
+    a = dict(q=FAKE, sq=16384, sh=128, n=4, H=128, d=128, kr=FAKE, vr=FAKE, rp=10, rps=64, ptr=FAKE,
+             ptrc=4, kc=FAKE, vc=FAKE, cp=10, cps=64, ptc=FAKE, ptcc=4, req=FAKE, B=1, ip=FAKE,
+             idx=FAKE, sink=FAKE, scale=0.088, out=FAKE, lse=FAKE, splits=1, ws=None, wsb=0)
+    a.update(kw)
+    return L.spa_sparse_sink_attn_fwd(
+        a["q"], a["sq"], a["sh"], a["n"], a["H"], a["d"], a["kr"], a["vr"], a["rp"], a["rps"], a["ptr"],
+        a["ptrc"], a["kc"], a["vc"], a["cp"], a["cps"], a["ptc"], a["ptcc"], a["req"], a["B"], a["ip"],
+        a["idx"], a["sink"], a["scale"], a["out"], a["lse"], a["splits"], a["ws"], a["wsb"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(n=-1), 1, "n_queries < 0"),
+    (dict(H=0), 1, "num_heads < 1"),
+    (dict(B=0), 1, "n_requests < 1"),
+    (dict(d=96), 2, "head_dim must be 64 or 128"),
+    (dict(H=192), 2, "multiple of 128"),
+    (dict(rp=-1), 1, "raw pool sizes"),
+    (dict(rps=0), 1, "raw_page_size < 1"),
+    (dict(rps=48), 2, "raw_page_size must be a power of two"),
+    (dict(cp=-1), 1, "compressed pool sizes"),
+    (dict(cps=0), 1, "cmp_page_size < 1"),
+    (dict(cps=2048), 2, "cmp_page_size must be a power of two"),
+    (dict(kc=None), 1, "k_cmp/v_cmp NULL"),
+    (dict(scale=0.0), 1, "scale must be finite"),
+    (dict(scale=float("inf")), 1, "scale must be finite"),
+    (dict(splits=17), 1, "num_splits must be"),
+    (dict(sq=-8), 1, "negative q stride"),
+    (dict(q=None), 1, "q, out and lse"),
+    (dict(vr=None), 1, "k_raw, v_raw and pt_raw"),
+    (dict(idx=None), 1, "req, indptr and indices"),
+    (dict(sh=129), 5, "q base and strides"),
+    (dict(kr=FAKE + 8), 5, "K/V pools"),
+    (dict(out=FAKE + 2), 5, "out must be"),
+    (dict(lse=FAKE + 2), 5, "32-bit arrays"),
+    (dict(splits=2), 4, "workspace needs"),
+    (dict(splits=2, ws=FAKE + 16, wsb=1 << 30), 5, "workspace must be 256-byte"),
+])
+def test_guard_matrix_attention(L, kw, status, clause):
+    assert attn_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def test_attention_zero_queries_is_a_no_op(L):
+    assert attn_call(L, n=0, q=None, out=None, lse=None) == 0

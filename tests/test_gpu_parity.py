@@ -1,0 +1,320 @@
+"""GPU parity: the CUDA path against the FP64 oracle on identical seeded inputs.
+
+Bar (stated by the method's tolerance for this path):
+  * CSR key sets: bit-exact (indptr and indices);
+  * FP8 page decode: bit-exact BF16;
+  * O: |O - ref| <= 1e-2 * (1 + |ref|) for every element, zero failures;
+  * LSE: |LSE - ref| <= 2e-3 for every (query, head).
+The oracle builds its own key sets and decodes its own pages: nothing it
+consumes comes from the CUDA path.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+O_RTOL = 1e-2
+LSE_ATOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def spa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_paged_attention_build_b200 as m
+    return m
+
+
+@functools.lru_cache(maxsize=None)
+def workload(name, shrink=1):
+    from sparse_paged_attention_build_b200 import workloads
+    return workloads.make(name, shrink=shrink)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_sets(name, shrink=1):
+    import oracle
+    w = workload(name, shrink)
+    return oracle.build_kv_sets(w.pos, w.W, w.ratio, w.topk)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_cmp_pools(name, shrink=1):
+    import oracle
+    w = workload(name, shrink)
+    if w.k_cmp_fp8 is None:
+        return w.k_cmp, w.v_cmp
+    k = oracle.dequant_fp8_pages(w.k_cmp_fp8, w.k_cmp_scale, w.cmp_page_ids)
+    v = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids)
+    return k, v
+
+
+def oracle_attn(name, shrink, rows):
+    import oracle
+    w = workload(name, shrink)
+    ip, idx = oracle_sets(name, shrink)
+    k_cmp, v_cmp = oracle_cmp_pools(name, shrink)
+    return oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, w.sink, w.scale,
+                                   k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp,
+                                   rows=None if rows is None else np.asarray(rows, dtype=np.int32))
+
+
+def check_attn(out, lse, O_ref, L_ref, what):
+    o = out.float().cpu().double().numpy()
+    l_ = lse.cpu().double().numpy()
+    err = np.abs(o - O_ref)
+    bad = err > O_RTOL * (1.0 + np.abs(O_ref))
+    assert not bad.any(), f"{what}: {bad.sum()} O elements out of tolerance, max err {err.max():.3g}"
+    lerr = np.abs(l_ - L_ref)
+    assert (lerr <= LSE_ATOL).all(), f"{what}: LSE max err {lerr.max():.3g}"
+    return float(err.max()), float(lerr.max())
+
+
+def batch(spa, name, shrink=1, num_splits=0):
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    return DeviceBatch(workload(name, shrink), num_splits=num_splits)
+
+
+def sample_rows(w, n_random=48, seed=0):
+    rng = np.random.default_rng(seed)
+    N = w.N
+    rows = {0, 1, N - 1, N - 2}
+    for p in (w.W - 1, w.W, 4 * 64 - 1, 2047, 2048, 2051, 2559):   # window fill, truncation start
+        hits = np.nonzero(w.pos == p)[0]
+        rows.update(hits[:2].tolist())
+    rows.update(rng.choice(N, size=min(N, n_random), replace=False).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < N), dtype=np.int32)
+
+
+# ------------------------------------------------------------------ sets
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
+def test_kv_sets_bit_exact_full_size(spa, name):
+    b = batch(spa, name)
+    b.build_sets()
+    torch.cuda.synchronize()
+    ip, idx = oracle_sets(name)
+    got_ip = b.indptr.cpu().numpy()
+    assert np.array_equal(got_ip, ip)
+    assert np.array_equal(b.indices[: ip[-1]].cpu().numpy(), idx)
+    assert b.status_word() == 0
+
+
+def test_kv_sets_edge_cases(spa):
+    import oracle
+    rng = np.random.default_rng(5)
+    pos = np.concatenate([[0, 1, 2, 3, 4, 127, 128, 129, 4095], rng.integers(0, 9000, 300)]).astype(np.int32)
+    for K in (1, 5, 32, 33, 512, 2048):
+        topk = rng.integers(-3, 2300, size=(pos.size, K)).astype(np.int32)
+        topk[:, : K // 2] = topk[:, :1]           # many repeats
+        for ratio, W in ((4, 128), (4, 1), (128, 7), (0, 64)):
+            t = torch.from_numpy(topk).cuda() if ratio == 4 else None
+            st = spa.new_status()
+            ip_g, idx_g = spa.build_kv_sets(torch.from_numpy(pos).cuda(), W, ratio, t,
+                                            max_pos=int(pos.max()), dev_status=st)
+            ip, idx = oracle.build_kv_sets(pos, W, ratio, topk if ratio == 4 else None)
+            assert np.array_equal(ip_g.cpu().numpy(), ip), (K, ratio, W)
+            assert np.array_equal(idx_g[: ip[-1]].cpu().numpy(), idx), (K, ratio, W)
+            assert spa.read_status(st) == 0
+
+
+def test_kv_sets_empty_and_faults(spa):
+    ip, idx = spa.build_kv_sets(torch.zeros(0, dtype=torch.int32, device="cuda"), 8, 4, None, capacity=0)
+    assert ip.cpu().tolist() == [0]
+    # a negative position is reported and gets an empty set
+    st = spa.new_status()
+    pos = torch.tensor([5, -1, 7], dtype=torch.int32, device="cuda")
+    ip, idx = spa.build_kv_sets(pos, 4, 0, None, capacity=100, dev_status=st)
+    assert spa.read_status(st) & spa.DEV_BAD_INDEX
+    assert ip.cpu().tolist() == [0, 4, 4, 8]
+    # capacity overflow is reported, nothing is written past it
+    st = spa.new_status()
+    idx = torch.full((10,), -7, dtype=torch.int32, device="cuda")
+    pos = torch.tensor([50, 60, 70], dtype=torch.int32, device="cuda")
+    spa.build_kv_sets(pos, 8, 0, None, capacity=9, indices=idx, dev_status=st)
+    assert spa.read_status(st) & spa.DEV_CAPACITY
+    assert idx[9].item() == -7
+
+
+# ------------------------------------------------------------------ dequant
+@pytest.mark.parametrize("shrink", [16, 1])
+def test_dequant_bit_exact(spa, shrink):
+    b = batch(spa, "c5", shrink)
+    b.dequant()
+    torch.cuda.synchronize()
+    k_ref, v_ref = oracle_cmp_pools("c5", shrink)
+    got_k = b.k_cmp.view(torch.int16).cpu().numpy().view(np.uint16)
+    got_v = b.v_cmp.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got_k, k_ref)
+    assert np.array_equal(got_v, v_ref)
+    assert b.status_word() == 0
+
+
+def test_dequant_every_code_and_bad_page(spa):
+    import oracle
+    P, ps, d = 4, 16, 128
+    src = np.arange(P * ps * d, dtype=np.int64).reshape(P, ps, d) % 256
+    src = src.astype(np.uint8)
+    rng = np.random.default_rng(2)
+    scales = (rng.random((P, ps, d // 64)) * 4).astype(np.float32)
+    scales[0, 0, 0] = 1e-40    # subnormal products
+    scales[0, 0, 1] = 3e38     # overflow to inf
+    ids = np.array([0, 2, 3], dtype=np.int32)
+    ref = oracle.dequant_fp8_pages(src, scales, ids)
+    dst = torch.zeros((P, ps, d), dtype=torch.bfloat16, device="cuda")
+    st = spa.new_status()
+    spa.dequant_fp8_pages(torch.from_numpy(src).cuda(), torch.from_numpy(scales).cuda(),
+                          torch.from_numpy(ids).cuda(), dst, dev_status=st)
+    got = dst.view(torch.int16).cpu().numpy().view(np.uint16)
+    nan_ref = (ref & 0x7fff) > 0x7f80
+    nan_got = (got & 0x7fff) > 0x7f80
+    assert np.array_equal(nan_ref, nan_got)
+    assert np.array_equal(got[~nan_ref], ref[~nan_ref])
+    assert spa.read_status(st) == 0
+    bad = torch.tensor([1, 99], dtype=torch.int32, device="cuda")
+    spa.dequant_fp8_pages(torch.from_numpy(src).cuda(), torch.from_numpy(scales).cuda(), bad, dst, dev_status=st)
+    assert spa.read_status(st) & spa.DEV_BAD_PAGE
+
+
+# ------------------------------------------------------------------ attention
+@pytest.mark.parametrize("name,shrink", [("c1", 1), ("c2", 8), ("c3", 16), ("c4", 16), ("c5", 16)])
+def test_attention_every_element_small(spa, name, shrink):
+    b = batch(spa, name, shrink)
+    b.step()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+    O, L = oracle_attn(name, shrink, None)
+    check_attn(b.out, b.lse, O, L, f"{name}/{shrink}")
+
+
+@pytest.mark.parametrize("name", ["c2", "c3", "c4", "c5"])
+def test_attention_full_size_sampled(spa, name):
+    """Full-size inputs in the launch configuration the benchmark times
+    (automatic split count); sampled rows against the oracle."""
+    b = batch(spa, name)
+    b.step()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+    w = workload(name)
+    rows = np.arange(w.N, dtype=np.int32) if w.kind == "decode" else sample_rows(w)
+    O, L = oracle_attn(name, 1, rows)
+    check_attn(b.out[torch.from_numpy(rows).long().cuda()], b.lse[torch.from_numpy(rows).long().cuda()],
+               O, L, name)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 5, 16])
+def test_attention_split_counts(spa, splits):
+    b = batch(spa, "c4", 8, num_splits=splits)
+    b.step()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+    O, L = oracle_attn("c4", 8, None)
+    check_attn(b.out, b.lse, O, L, f"splits={splits}")
+
+
+def test_attention_no_sink_and_empty_sets(spa):
+    import oracle
+    w = workload("c1")
+    b = batch(spa, "c1")
+    b.build_sets()
+    ip, idx = oracle_sets("c1")
+    # empty every third set: indptr with repeated entries, keys dropped
+    keep = np.ones(w.N, dtype=bool)
+    keep[::3] = False
+    sizes = np.diff(ip) * keep
+    ip2 = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    idx2 = np.concatenate([idx[ip[i]:ip[i + 1]] for i in range(w.N) if keep[i]]).astype(np.int32)
+    for sink in (w.sink, None):
+        st = spa.new_status()
+        out, lse = spa.sparse_sink_attn_fwd(
+            b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, torch.from_numpy(ip2).cuda(),
+            torch.from_numpy(idx2).cuda(), None if sink is None else b.sink, w.scale,
+            k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp, dev_status=st)
+        torch.cuda.synchronize()
+        assert spa.read_status(st) == 0
+        s = np.full(w.H, -np.inf, dtype=np.float32) if sink is None else w.sink
+        O, L = oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip2, idx2, s, w.scale,
+                                       k_cmp=w.k_cmp, v_cmp=w.v_cmp, pt_cmp=w.pt_cmp)
+        o = out.float().cpu().double().numpy()
+        l_ = lse.cpu().double().numpy()
+        empty = ~keep
+        assert np.all(o[empty] == 0)
+        if sink is None:
+            assert np.all(np.isneginf(l_[empty]))
+            check_attn(out[torch.from_numpy(keep).cuda()], lse[torch.from_numpy(keep).cuda()],
+                       O[keep], L[keep], "no sink")
+        else:
+            check_attn(out, lse, O, L, "empty sets")
+
+
+def test_attention_bad_page_is_reported_not_trapped(spa):
+    w = workload("c1")
+    b = batch(spa, "c1")
+    b.build_sets()
+    pt = b.pt_raw.clone()
+    pt[0, 0] = 10 ** 7
+    st = spa.new_status()
+    spa.sparse_sink_attn_fwd(b.q, b.k_raw, b.v_raw, pt, b.req, b.indptr, b.indices, b.sink, w.scale,
+                             k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp, dev_status=st)
+    torch.cuda.synchronize()
+    assert spa.read_status(st) & spa.DEV_BAD_PAGE
+    # the context is still usable
+    b.step()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+
+
+def test_pool_beyond_2GiB_uses_64bit_addressing(spa):
+    """Rows placed past byte 2^31 of a >2 GiB pool are read correctly."""
+    import oracle
+    w = workload("c1")
+    ps, d = w.k_raw.shape[1], w.k_raw.shape[2]
+    page_bytes = ps * d * 2
+    big_pages = (2 ** 31 + 2 ** 26) // page_bytes + w.k_raw.shape[0]
+    shift = big_pages - w.k_raw.shape[0]
+    k_big = torch.zeros((big_pages, ps, d), dtype=torch.bfloat16, device="cuda")
+    v_big = torch.zeros_like(k_big)
+    b = batch(spa, "c1")
+    k_big[shift:] = b.k_raw
+    v_big[shift:] = b.v_raw
+    pt = (b.pt_raw + shift).contiguous()
+    b.build_sets()
+    st = spa.new_status()
+    out, lse = spa.sparse_sink_attn_fwd(b.q, k_big, v_big, pt, b.req, b.indptr, b.indices, b.sink,
+                                        w.scale, k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp,
+                                        dev_status=st)
+    torch.cuda.synchronize()
+    assert spa.read_status(st) == 0
+    O, L = oracle_attn("c1", 1, None)
+    check_attn(out, lse, O, L, ">2GiB pool")
+    del k_big, v_big
+
+
+def test_graph_capture_and_two_streams(spa):
+    """The three calls capture into a CUDA graph; replays and a second
+    stream give bit-identical results."""
+    b = batch(spa, "c5", 16)
+    b.step()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = b.out.clone(), b.lse.clone()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            b.step(stream=s)
+    b.out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(b.out, ref_out) and torch.equal(b.lse, ref_lse)
+    b2 = batch(spa, "c5", 16)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(s1):
+        b.step(stream=s1)
+    with torch.cuda.stream(s2):
+        b2.step(stream=s2)
+    torch.cuda.synchronize()
+    assert torch.equal(b.out, ref_out) and torch.equal(b2.out, ref_out)
+    assert torch.equal(b2.lse, ref_lse)
