@@ -183,6 +183,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=0)
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="divide requests/tokens (profiling cases only; not a bench line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, local_rank, world = env_rank()
@@ -204,7 +206,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    w = workloads.make(args.workload, seed_offset=rank)
+    w = workloads.make(args.workload, shrink=args.shrink, seed_offset=rank)
     decode = w.kind == "decode"
     b0 = DeviceBatch(w, num_splits=args.splits)
     stream = torch.cuda.current_stream()
