@@ -115,6 +115,37 @@ int spa_build_kv_sets(const int32_t* pos, int32_t n_queries, int32_t window, int
                       size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * 1b. spa_build_kv_sets_noalloc -- spa_build_kv_sets with no workspace.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory at the point where the sets are built: code
+ * that runs inside a host framework which reserves all device memory up
+ * front and hands out no scratch (a serving engine's fixed arena, a plugin
+ * interface without a workspace argument), or code called while a CUDA
+ * graph is being captured, where a fresh allocation would either fail or be
+ * baked into the graph.
+ *
+ * Same arguments, results and device-status bits as spa_build_kv_sets,
+ * minus `workspace` / `workspace_bytes`. The scan scratch is a fixed array
+ * of 1 MiB + 16 bytes inside the library (every GPU that loads the library
+ * keeps it until the process exits), so n_queries is limited to
+ * 1,048,576; larger calls return SPA_ERR_UNSUPPORTED without enqueueing
+ * anything. The call allocates nothing (no cudaMalloc, no allocating
+ * library routine); it clears the part of the scratch it uses, on `stream`,
+ * before its kernel runs.
+ *
+ * The first call on each device looks up the scratch array's device address
+ * (with that device current) and caches it; make that first call before any
+ * stream capture on the device. All calls share the one array: calls that
+ * may overlap on the GPU (different streams, or graph replays running
+ * concurrently) race on it and must be serialised by the caller.
+ * ---------------------------------------------------------------------- */
+int spa_build_kv_sets_noalloc(const int32_t* pos, int32_t n_queries, int32_t window, int32_t ratio,
+                              const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                              int32_t* indices, int64_t capacity, uint32_t* dev_status,
+                              spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * 2. spa_dequant_fp8_pages -- mixed FP8/BF16 cache: FP8 pages to BF16.
  *
  * Defined by "Roadmap item 24", section "Reuse and arithmetic" (a mixed

@@ -120,6 +120,35 @@ int spa_build_kv_sets(const int32_t* pos, int32_t n_queries, int32_t window, int
                      "build_kv_sets launch");
 }
 
+// For callers that cannot allocate device memory: the same sets as
+// spa_build_kv_sets, with the scan scratch taken from a fixed array inside
+// the library instead of a caller workspace.
+int spa_build_kv_sets_noalloc(const int32_t* pos, int32_t n_queries, int32_t window, int32_t ratio,
+                              const int32_t* topk, int32_t topk_width, int32_t* indptr, int32_t* indices,
+                              int64_t capacity, uint32_t* dev_status, spa_stream_t stream) {
+  if (n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
+  if (n_queries > spa::kNoAllocMaxQueries)
+    return fail(SPA_ERR_UNSUPPORTED,
+                "n_queries %d exceeds the fixed scratch of spa_build_kv_sets_noalloc (%d queries); "
+                "call spa_build_kv_sets with a workspace instead",
+                n_queries, spa::kNoAllocMaxQueries);
+  if (window < 1) return fail(SPA_ERR_INVALID_ARG, "window < 1");
+  if (ratio != 0 && ratio != 4 && ratio != 128) return fail(SPA_ERR_INVALID_ARG, "ratio must be 0, 4 or 128");
+  if (topk_width < 0) return fail(SPA_ERR_INVALID_ARG, "topk_width < 0");
+  if (capacity < 0) return fail(SPA_ERR_INVALID_ARG, "capacity < 0");
+  if (indptr == nullptr) return fail(SPA_ERR_INVALID_ARG, "indptr is NULL");
+  if (n_queries > 0 && pos == nullptr) return fail(SPA_ERR_INVALID_ARG, "pos is NULL");
+  if (n_queries > 0 && capacity > 0 && indices == nullptr) return fail(SPA_ERR_INVALID_ARG, "indices is NULL");
+  if (ratio > 0 && topk != nullptr && topk_width > spa::kMaxTopkWidth)
+    return fail(SPA_ERR_UNSUPPORTED, "topk_width > %d", spa::kMaxTopkWidth);
+  if (!aligned(pos, 4) || !aligned(topk, 4) || !aligned(indptr, 4) || !aligned(indices, 4))
+    return fail(SPA_ERR_ALIGNMENT, "int32 arrays must be 4-byte aligned");
+  return cuda_status(spa::launch_build_kv_sets_no_alloc(pos, n_queries, window, ratio, topk, topk_width,
+                                                        indptr, indices, capacity, dev_status,
+                                                        reinterpret_cast<cudaStream_t>(stream)),
+                     "build_kv_sets_noalloc launch");
+}
+
 // ---------------------------------------------------------------- dequant
 int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages, int32_t page_size,
                           int32_t head_dim, const int32_t* page_ids, int32_t n_page_ids,

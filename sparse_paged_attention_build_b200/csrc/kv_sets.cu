@@ -17,6 +17,7 @@
 // distinct groups ascending, then the window tokens ascending with the
 // window tag. Integer only; no floating point anywhere.
 #include <climits>
+#include <mutex>
 
 #include "spa_device.cuh"
 #include "spa_internal.h"
@@ -242,6 +243,60 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
   }
   build_kv_sets_kernel<<<static_cast<unsigned>(tiles), kSetsQueriesPerCta * 32, smem, stream>>>(P);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Variant without caller workspace, for callers that cannot allocate device
+// memory. The look-back status words and the CTA ticket live in a fixed
+// array that every GPU loading this library keeps for the life of the
+// process (kNoAllocScratchBytes, about 1 MiB).
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNoAllocMaxTiles = (kNoAllocMaxQueries + kSetsQueriesPerCta - 1) / kSetsQueriesPerCta;
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(kNoAllocMaxTiles) * sizeof(uint64_t) + 16;
+static_assert(kNoAllocScratchBytes == 1048576 + 16, "the documented limit");
+
+static __device__ __align__(256) uint64_t g_sets_scratch[kNoAllocScratchBytes / sizeof(uint64_t)];
+
+// Host code cannot pass &g_sets_scratch to a kernel: on the host that name
+// is only a stand-in. Its device address is looked up once per device, with
+// that device current, and cached.
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+cudaError_t scratch_for_current_device(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_sets_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t no_alloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_build_kv_sets_no_alloc(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
+                                          const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                                          int32_t* indices, int64_t capacity, uint32_t* dev_status,
+                                          cudaStream_t stream) {
+  void* scratch = nullptr;
+  cudaError_t err = scratch_for_current_device(&scratch);
+  if (err != cudaSuccess) return err;
+  // the same kernel as the workspace entry point; the launcher clears the
+  // part of the scratch this call uses before the kernel runs
+  return launch_build_kv_sets(pos, n, window, ratio, topk, topk_width, indptr, indices, capacity,
+                              scratch, dev_status, stream);
 }
 
 }  // namespace spa

@@ -17,6 +17,14 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
                                  int32_t* indices, int64_t capacity, void* ws,
                                  uint32_t* dev_status, cudaStream_t stream);
 
+// Fixed-scratch variant of the set builder (no caller workspace).
+constexpr int32_t kNoAllocMaxQueries = 1 << 20;
+size_t no_alloc_scratch_bytes();
+cudaError_t launch_build_kv_sets_no_alloc(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
+                                          const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                                          int32_t* indices, int64_t capacity, uint32_t* dev_status,
+                                          cudaStream_t stream);
+
 cudaError_t launch_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
                                      int32_t page_size, int32_t head_dim, const int32_t* page_ids,
                                      int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status,

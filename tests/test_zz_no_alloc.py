@@ -1,0 +1,78 @@
+"""spa_build_kv_sets_noalloc against spa_build_kv_sets, through the C ABI.
+
+The no-allocation entry point is for callers that cannot allocate device
+memory where they build the key sets: code inside a host framework that
+reserves all device memory up front and hands out no scratch, or code that
+runs while a CUDA graph is being captured. It keeps its scan scratch in a
+fixed array inside the library instead of a caller workspace, so it must
+give exactly the sets the workspace entry point gives -- on every call, since
+the array keeps the previous call's contents and each call must clear what
+it uses. This file is collected last on purpose.
+"""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "sparse_paged_attention_build_b200", "libspa.so")
+MAX_QUERIES = 1 << 20
+
+
+def _abi():
+    so = ctypes.CDLL(LIB)
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    so.spa_build_kv_sets_noalloc.argtypes = [P, i32, i32, i32, P, i32, P, P, i64, P, P]
+    so.spa_build_kv_sets_noalloc.restype = ctypes.c_int
+    so.spa_last_error_detail.restype = ctypes.c_char_p
+    return so
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def test_noalloc_rejects_more_queries_than_its_scratch():
+    so = _abi()
+    rc = so.spa_build_kv_sets_noalloc(ctypes.c_void_p(0x10000), MAX_QUERIES + 1, 128, 0, None, 0,
+                                      ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1 << 30,
+                                      None, None)
+    assert rc == 2    # SPA_ERR_UNSUPPORTED, nothing enqueued
+    assert b"fixed scratch" in so.spa_last_error_detail()
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_paged_attention_build_b200 as spa
+    from sparse_paged_attention_build_b200 import workloads
+
+    so = _abi()
+    # largest case first, so the second and third calls run over scratch
+    # that still holds the previous call's look-back words
+    cases = [workloads.make("c3", shrink=2), workloads.make("c2", shrink=8), workloads.make("c4")]
+    for w in cases:
+        pos = torch.from_numpy(w.pos).cuda()
+        topk = None if w.topk is None else torch.from_numpy(w.topk).cuda()
+        max_pos = int(w.pos.max())
+        cap = spa.kv_sets_capacity(w.N, w.W, w.ratio, w.K, topk is not None, max_pos)
+        ref_ip, ref_idx = spa.build_kv_sets(pos, w.W, w.ratio, topk, capacity=cap)
+        torch.cuda.synchronize()
+        ref_ip = ref_ip.cpu().numpy()
+        ref_idx = ref_idx[: ref_ip[-1]].cpu().numpy()
+        for call in range(2):
+            indptr = torch.full((w.N + 1,), -1, dtype=torch.int32, device="cuda")
+            indices = torch.full((max(cap, 1),), -1, dtype=torch.int32, device="cuda")
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            rc = so.spa_build_kv_sets_noalloc(
+                _ptr(pos), w.N, w.W, w.ratio, _ptr(topk), w.K if topk is not None else 0,
+                _ptr(indptr), _ptr(indices), cap, _ptr(status),
+                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+            assert rc == 0, so.spa_last_error_detail()
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0, (w.name, call)
+            assert np.array_equal(indptr.cpu().numpy(), ref_ip), (w.name, call)
+            assert np.array_equal(indices[: ref_ip[-1]].cpu().numpy(), ref_idx), (w.name, call)
