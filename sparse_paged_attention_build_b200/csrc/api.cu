@@ -177,8 +177,10 @@ int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int
   if (n_queries <= 0 || num_heads <= 0) return 1;
   const int64_t head_tiles = (num_heads + 127) / 128;
   const int64_t units = static_cast<int64_t>(n_queries) * head_tiles;
-  const int64_t target = 2 * static_cast<int64_t>(sm_count());   // two CTAs per SM
-  int64_t s = (target + units - 1) / units;
+  // enough slices to give every persistent CTA (two per SM) a unit, without
+  // exceeding one wave of units
+  const int64_t target = 2 * static_cast<int64_t>(sm_count());
+  int64_t s = target / units;
   if (max_set_size > 0) s = std::min<int64_t>(s, (max_set_size + spa::kAttnKeysPerTile - 1) / spa::kAttnKeysPerTile);
   s = std::max<int64_t>(1, std::min<int64_t>(s, spa::kAttnMaxSplits));
   return static_cast<int>(s);
@@ -209,11 +211,15 @@ int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
   if (raw_num_pages < 0 || pt_raw_cols < 0) return fail(SPA_ERR_INVALID_ARG, "raw pool sizes < 0");
   if (raw_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "raw_page_size < 1");
   if (!pow2_in(raw_page_size, 1, 1024)) return fail(SPA_ERR_UNSUPPORTED, "raw_page_size must be a power of two <= 1024");
+  if (raw_num_pages * raw_page_size >= 0x7fffffffLL)
+    return fail(SPA_ERR_UNSUPPORTED, "raw pool holds 2^31 - 1 rows or more");
   if (pt_cmp != nullptr) {
     if (cmp_num_pages < 0 || pt_cmp_cols < 0) return fail(SPA_ERR_INVALID_ARG, "compressed pool sizes < 0");
     if (cmp_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "cmp_page_size < 1");
     if (!pow2_in(cmp_page_size, 1, 1024))
       return fail(SPA_ERR_UNSUPPORTED, "cmp_page_size must be a power of two <= 1024");
+    if (cmp_num_pages * cmp_page_size >= 0x7fffffffLL)
+      return fail(SPA_ERR_UNSUPPORTED, "compressed pool holds 2^31 - 1 rows or more");
     if (k_cmp == nullptr || v_cmp == nullptr) return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
   }
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(SPA_ERR_INVALID_ARG, "scale must be finite and > 0");

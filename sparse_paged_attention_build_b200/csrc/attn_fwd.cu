@@ -18,18 +18,31 @@
 // The sink seeds the running max and the denominator (m = sink*log2e,
 // l = 1), so it is counted exactly once and never multiplies a V row.
 //
-// Warp roles (224 threads):
+// Persistent CTAs (two per SM) walk their units in a fixed stride. Warp
+// roles (256 threads):
 //   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t
 //   warp  4    TMEM allocation; lane 0 issues every UMMA and commit
-//   warps 5-6  paged gather: key -> page table -> 64-bit row address ->
-//              16-byte cp.async of K and V rows into a 2-stage ring,
-//              written in the 128-byte-swizzled K-major layout the UMMA
-//              descriptors describe
+//   warp  5    K (and Q) gather: TMA tile::gather4 loads (four rows of one
+//              pool per instruction, one instruction per lane per tile) into
+//              a 2-stage ring, 128-byte swizzled by the tensor map into the
+//              K-major layout of the UMMA descriptors; rows outside the pool
+//              (padding, faulty keys) are zero-filled by the TMA
+//   warp  6    V gather, into its own 2-stage ring
+//   warp  7    resolver: for a chunk of up to 1024 keys of a unit it loads
+//              the keys, looks their pages up and writes the physical row
+//              of every key (bit 31 = raw pool) to a double-buffered table,
+//              plus a chunk descriptor that every other role follows. All
+//              dependent global loads of the gather happen here, ahead of
+//              the copies.
 // TMEM columns: S/P buffer 0 [0,64), buffer 1 [64,128), O [128,128+d).
-// The running max is only moved when a tile's max exceeds it by more than
-// 8 (log2 units), so P <= 256 and O is rescaled rarely; the final O/l and
-// LSE use the same max, so the result is exact in exact arithmetic.
+// The running max only moves when a tile's max exceeds it by more than 8
+// (log2 units), so P <= 256 and O is rescaled rarely; O/l and LSE use the
+// same max, so the result is exact in exact arithmetic.
+#include <algorithm>
 #include <cmath>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "spa_device.cuh"
 #include "spa_internal.h"
@@ -38,20 +51,45 @@ namespace spa {
 namespace {
 
 constexpr int kT = kAttnKeysPerTile;   // keys per tile
-constexpr int kStages = 2;
+constexpr int kStagesK = 2;
+constexpr int kStagesV = 2;
 constexpr int kSoftThreads = 128;
 constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 5;
-constexpr int kProdThreads = 64;
-constexpr int kThreads = (kProdWarp0 * 32) + kProdThreads;   // 224
+constexpr int kKWarp = 5;
+constexpr int kVWarp = 6;
+constexpr int kResolverWarp = 7;
+constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
+constexpr int kChunkKeys = 1024;                 // keys resolved per chunk
+constexpr uint32_t kRawBit = 0x80000000u;
+constexpr uint32_t kInvalidRow = 0xFFFFFFFFu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
+// consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
+constexpr uint32_t kTabConsumers = 32 + 32 + 1 + kSoftThreads;
 
-static_assert(kT == kProdThreads, "one producer thread resolves one key of a tile");
+constexpr int kFlagFirst = 1;   // first chunk of its unit
+constexpr int kFlagLast = 2;    // last chunk of its unit
+constexpr int kFlagFinal = 4;   // last chunk of this CTA
+
+struct ChunkDesc {
+  int32_t i;          // query token
+  int32_t split;      // slice of the token's key set
+  int32_t key_base;   // CSR position of the chunk's first key
+  int32_t nkeys;      // keys in the chunk (tiles = ceil(nkeys / 64))
+  int32_t flags;
+  int32_t pad[3];
+};
 
 struct Params {
+  // TMA descriptors (passed as a __grid_constant__ parameter)
+  CUtensorMap tm_q;       // 3D {d, H, N}, box {64, q_box_rows, 1}
+  CUtensorMap tm_k_raw;   // 2D {d, rows}, box {64, 1}: gather4 / single rows
+  CUtensorMap tm_v_raw;
+  CUtensorMap tm_k_cmp;
+  CUtensorMap tm_v_cmp;
+  int32_t q_box_rows;     // min(128, num_heads)
   const uint16_t* q;
   int64_t q_stride_tok, q_stride_head;
   int32_t n_queries, num_heads;
@@ -84,109 +122,153 @@ template <int D>
 struct Layout {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kTileBytes = kT * D * 2;             // one K or V tile
-  static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQOff = 0;
-  static constexpr int kStageOff = kQBytes;
-  static constexpr int kRowPtrOff = kStageOff + kStages * kStageBytes;   // [stages][T][2] ptrs
-  static constexpr int kBarOff = kRowPtrOff + kStages * kT * 16;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2;
+  static constexpr int kKOff = kQBytes;
+  static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
+  static constexpr int kTabOff = kVOff + kStagesV * kTileBytes;       // [2][kChunkKeys] u32
+  static constexpr int kDescOff = kTabOff + 2 * kChunkKeys * 4;       // [2] ChunkDesc
+  static constexpr int kBarOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
+  // tab_full, tab_empty, q_full + q_empty, K ring, V ring, s_full, p_ready,
+  // o_done, o_free, mma_done
+  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 1 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kUsed = kMiscOff + 16;
-  // keep at most two CTAs per SM: TMEM holds two 256-column allocations
-  static constexpr int kBytes = (kUsed + 1024) < 96 * 1024 ? 96 * 1024 : (kUsed + 1024);
+  // + alignment slack; at least 80 KB so that no more than two CTAs share an
+  // SM (TMEM holds two 256-column allocations)
+  static constexpr int kBytes = (kUsed + 1024) < 80 * 1024 ? 80 * 1024 : (kUsed + 1024);
   static constexpr uint32_t kOCol = 2 * kT;
   static_assert(kOCol + D <= kTmemCols, "TMEM budget");
-  static_assert(kBytes * 2 <= 227 * 1024, "two CTAs per SM");
+  static_assert((kBytes + 1024) * 2 <= 228 * 1024, "two CTAs per SM");
 };
 
-// Resolve one key to its K and V row pointers (nullptr for padding or a
-// faulty key, which is zero-filled).
-__device__ __forceinline__ void resolve_key(const Params& P, int32_t b, int32_t key, int row_bytes,
-                                            const char*& kp, const char*& vp) {
-  kp = nullptr;
-  vp = nullptr;
-  if (key < 0) {
-    report(P.dev_status, SPA_DEV_BAD_INDEX);
-    return;
+struct Bars {
+  uint64_t* tab_full;   // [2]
+  uint64_t* tab_empty;  // [2]
+  uint64_t* q_full;
+  uint64_t* q_empty;
+  uint64_t* k_full;     // [kStagesK]
+  uint64_t* k_empty;
+  uint64_t* v_full;     // [kStagesV]
+  uint64_t* v_empty;
+  uint64_t* s_full;     // [2]
+  uint64_t* p_ready;    // [2]
+  // [2]: PV of tile g commits to o_done[g & 1]. One barrier per parity keeps
+  // a waiter two phases away from aliasing: when the softmax waits for PV(g)
+  // it has seen S(g) complete, so PV(g - 2) (issued before S(g)) is done.
+  uint64_t* o_done;
+  uint64_t* o_free;
+  uint64_t* mma_done;
+};
+
+__device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) / kT; }
+
+// ------------------------------------------------------------------ resolver
+// Keys -> physical rows for one chunk. Each lane handles keys lane, lane+32,
+// ...; the loads of each phase are issued together so the chunk costs two
+// round trips, not two per key.
+__device__ void resolve_chunk(const Params& P, int32_t b, int32_t key_base, int32_t nkeys,
+                              uint32_t* tab, int lane) {
+  constexpr int kPer = kChunkKeys / 32;
+  int32_t key[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int k = lane + 32 * e;
+    key[e] = k < nkeys ? __ldg(P.indices + key_base + k) : -2;
   }
-  const bool window = (key & SPA_WINDOW_TAG) != 0;
-  const int32_t t = key & (SPA_WINDOW_TAG - 1);
-  const int32_t* pt = window ? P.pt_raw : P.pt_cmp;
-  const int32_t cols = window ? P.pt_raw_cols : P.pt_cmp_cols;
-  const int32_t ps_log2 = window ? P.raw_ps_log2 : P.cmp_ps_log2;
-  const int64_t pages = window ? P.raw_pages : P.cmp_pages;
-  const int32_t lp = t >> ps_log2;
-  if (pt == nullptr || lp >= cols) {
-    report(P.dev_status, SPA_DEV_BAD_INDEX);
-    return;
+  int32_t page[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    page[e] = -1;
+    const int32_t kk = key[e];
+    if (kk == -2) continue;
+    if (kk < 0) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
+    const bool raw = (kk & SPA_WINDOW_TAG) != 0;
+    const int32_t t = kk & (SPA_WINDOW_TAG - 1);
+    const int32_t* pt = raw ? P.pt_raw : P.pt_cmp;
+    const int32_t cols = raw ? P.pt_raw_cols : P.pt_cmp_cols;
+    const int32_t lp = t >> (raw ? P.raw_ps_log2 : P.cmp_ps_log2);
+    if (pt == nullptr || lp >= cols) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
+    page[e] = __ldg(pt + static_cast<int64_t>(b) * cols + lp);
   }
-  const int64_t page = pt[static_cast<int64_t>(b) * cols + lp];
-  if (page < 0 || page >= pages) {
-    report(P.dev_status, SPA_DEV_BAD_PAGE);
-    return;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int k = lane + 32 * e;
+    if (k >= kChunkKeys) continue;
+    const int32_t kk = key[e];
+    uint32_t row = kInvalidRow;
+    if (kk >= 0) {
+      const bool raw = (kk & SPA_WINDOW_TAG) != 0;
+      const int32_t t = kk & (SPA_WINDOW_TAG - 1);
+      const int32_t ps_log2 = raw ? P.raw_ps_log2 : P.cmp_ps_log2;
+      const int64_t pages = raw ? P.raw_pages : P.cmp_pages;
+      const int64_t pg = page[e];
+      if (pg < 0 || pg >= pages) {
+        report(P.dev_status, SPA_DEV_BAD_PAGE);
+      } else {
+        row = static_cast<uint32_t>((pg << ps_log2) + (t & ((1 << ps_log2) - 1))) | (raw ? kRawBit : 0u);
+      }
+    }
+    if (k < nkeys) tab[k] = row;
   }
-  const int64_t row = (page << ps_log2) + (t & ((1 << ps_log2) - 1));
-  const int64_t off = row * row_bytes;
-  kp = (window ? P.k_raw : P.k_cmp) + off;
-  vp = (window ? P.v_raw : P.v_cmp) + off;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const Params P) {
+__global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __grid_constant__ Params P) {
   using L = Layout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + kStages;
-  uint64_t* s_full = bars + 1 + 2 * kStages;
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* o_done = p_ready + 2;
-  uint64_t* mma_done = o_done + 1;
+  uint64_t* bar0 = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  Bars B;
+  B.tab_full = bar0;
+  B.tab_empty = bar0 + 2;
+  B.q_full = bar0 + 4;
+  B.q_empty = bar0 + 5;
+  B.k_full = bar0 + 6;
+  B.k_empty = B.k_full + kStagesK;
+  B.v_full = B.k_empty + kStagesK;
+  B.v_empty = B.v_full + kStagesV;
+  B.s_full = B.v_empty + kStagesV;
+  B.p_ready = B.s_full + 2;
+  B.o_done = B.p_ready + 2;
+  B.o_free = B.o_done + 2;
+  B.mma_done = B.o_free + 1;
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
+  ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + L::kDescOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   uint32_t* ticket_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff + 8);
-  const char** rowptr = reinterpret_cast<const char**>(smem + L::kRowPtrOff);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int S = P.num_splits;
-  const int i = blockIdx.x / S;
-  const int split = blockIdx.x - i * S;
   const int head0 = blockIdx.y * 128;
   const int heads_here = min(128, P.num_heads - head0);
 
-  // ---- the unit's key range
-  int32_t set_begin = P.indptr[i];
-  int32_t set_len = P.indptr[i + 1] - set_begin;
-  const int32_t b = P.req[i];
-  if (set_len < 0 || b < 0 || b >= P.n_requests) {
-    if (tid == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
-    set_len = 0;
-  }
-  const int tiles_total = (set_len + kT - 1) / kT;
-  const int tile_lo = static_cast<int>((static_cast<int64_t>(tiles_total) * split) / S);
-  const int tile_hi = static_cast<int>((static_cast<int64_t>(tiles_total) * (split + 1)) / S);
-  const int ntiles = tile_hi - tile_lo;
-  const int32_t key_lo = tile_lo * kT;
-  const int32_t key_hi = min(tile_hi * kT, set_len);
-
   // ---- setup
   if (tid == 0) {
-    mbar_init(q_full, kProdThreads);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(kv_full + s, kProdThreads);
-      mbar_init(kv_empty + s, 1);
-    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full + s, 1);
-      mbar_init(p_ready + s, kSoftThreads);
+      mbar_init(B.tab_full + s, 32);
+      mbar_init(B.tab_empty + s, kTabConsumers);
+      mbar_init(B.s_full + s, 1);
+      mbar_init(B.p_ready + s, kSoftThreads);
     }
-    mbar_init(o_done, 1);
-    mbar_init(mma_done, 1);
+    mbar_init(B.q_full, 1);
+    mbar_init(B.q_empty, 1);
+    for (int s = 0; s < kStagesK; ++s) {
+      mbar_init(B.k_full + s, 1);
+      mbar_init(B.k_empty + s, 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
+      mbar_init(B.v_full + s, 1);
+      mbar_init(B.v_empty + s, 1);
+    }
+    mbar_init(B.o_done, 1);
+    mbar_init(B.o_done + 1, 1);
+    mbar_init(B.o_free, kSoftThreads);
+    mbar_init(B.mma_done, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -199,95 +281,192 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const Par
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kProdWarp0) {
-    // ================================================= producers
-    const int pt = tid - kProdWarp0 * 32;
-    if (ntiles > 0) {
-      // Q rows (zero rows past the unit's heads)
-      const char* qbase = reinterpret_cast<const char*>(P.q);
-      constexpr int kChunksPerRow = D / 8;   // 16-byte chunks
-      for (int c = pt; c < 128 * kChunksPerRow; c += kProdThreads) {
-        const int r = c / kChunksPerRow, ch = c % kChunksPerRow;
-        const int db = ch >> 3, u = ch & 7;
-        const uint32_t dst = sbase + L::kQOff + db * (128 * 128) + r * 128 + ((u ^ (r & 7)) << 4);
-        const bool ok = r < heads_here;
-        const char* src = ok ? qbase + 2 * (static_cast<int64_t>(i) * P.q_stride_tok +
-                                            static_cast<int64_t>(head0 + r) * P.q_stride_head) + ch * 16
-                             : qbase;
-        cp_async16(dst, src, ok ? 16u : 0u);
+  if (warp == kResolverWarp) {
+    // ================================================= resolver
+    int c = 0;
+    const int64_t n_units = static_cast<int64_t>(P.n_queries) * S;
+    for (int64_t u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
+      const int i = static_cast<int>(u / S);
+      const int split = static_cast<int>(u - static_cast<int64_t>(i) * S);
+      const int32_t set_begin = __ldg(P.indptr + i);
+      int32_t set_len = __ldg(P.indptr + i + 1) - set_begin;
+      const int32_t b = __ldg(P.req + i);
+      if (set_len < 0 || b < 0 || b >= P.n_requests) {
+        if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
+        set_len = 0;
       }
-      cp_async_arrive_noinc(q_full);
-
-      const char* dummy = P.k_raw;
-      for (int jt = 0; jt < ntiles; ++jt) {
-        const int stage = jt % kStages;
-        if (!mbar_wait(kv_empty + stage, ((jt / kStages) & 1) ^ 1, abort_flag, P.dev_status)) break;
-        // resolve this thread's key
-        const int32_t kpos = key_lo + jt * kT + pt;
-        const char* kp = nullptr;
-        const char* vp = nullptr;
-        if (kpos < key_hi) resolve_key(P, b, P.indices[set_begin + kpos], D * 2, kp, vp);
-        rowptr[(stage * kT + pt) * 2 + 0] = kp;
-        rowptr[(stage * kT + pt) * 2 + 1] = vp;
-        named_bar_sync(1, kProdThreads);
-        const uint32_t kdst = sbase + L::kStageOff + stage * L::kStageBytes;
-        const uint32_t vdst = kdst + L::kTileBytes;
-        for (int c = pt; c < kT * kChunksPerRow; c += kProdThreads) {
-          const int r = c / kChunksPerRow, ch = c % kChunksPerRow;
-          const int db = ch >> 3, u = ch & 7;
-          const uint32_t off = db * (kT * 128) + r * 128 + ((u ^ (r & 7)) << 4);
-          const char* ks = rowptr[(stage * kT + r) * 2 + 0];
-          const char* vs = rowptr[(stage * kT + r) * 2 + 1];
-          cp_async16(kdst + off, ks ? ks + ch * 16 : dummy, ks ? 16u : 0u);
-          cp_async16(vdst + off, vs ? vs + ch * 16 : dummy, vs ? 16u : 0u);
+      const int tiles_total = ceil_tiles(set_len);
+      const int tile_lo = static_cast<int>((static_cast<int64_t>(tiles_total) * split) / S);
+      const int tile_hi = static_cast<int>((static_cast<int64_t>(tiles_total) * (split + 1)) / S);
+      const int32_t key_lo = tile_lo * kT;
+      const int32_t key_hi = min(tile_hi * kT, set_len);
+      const bool final_unit = u + gridDim.x >= n_units;
+      int32_t k0 = key_lo;
+      do {
+        const int slot = c & 1;
+        if (!mbar_wait(B.tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status)) break;
+        const int32_t n = max(0, min(kChunkKeys, key_hi - k0));   // 0: an empty slice
+        resolve_chunk(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane);
+        if (lane == 0) {
+          ChunkDesc& d = desc[slot];
+          d.i = i;
+          d.split = split;
+          d.key_base = set_begin + k0;
+          d.nkeys = n;
+          const bool last = k0 + n >= key_hi;
+          d.flags = (k0 == key_lo ? kFlagFirst : 0) | (last ? kFlagLast : 0) |
+                    (last && final_unit ? kFlagFinal : 0);
         }
-        cp_async_arrive_noinc(kv_full + stage);
+        __syncwarp();
+        mbar_arrive(B.tab_full + slot);
+        ++c;
+        k0 += n;
+      } while (k0 < key_hi);
+    }
+  } else if (warp == kKWarp || warp == kVWarp) {
+    // ================================================= K / V gather (TMA)
+    // Each lane issues one gather4 per tile: rows 4*grp .. 4*grp+3 of the
+    // tile, one 64-column half of the row. A group whose four keys come from
+    // both pools (at most one per unit: the sets list compressed groups
+    // before window tokens) is loaded row by row instead.
+    const bool is_k = warp == kKWarp;
+    const int nst = is_k ? kStagesK : kStagesV;
+    uint64_t* full = is_k ? B.k_full : B.v_full;
+    uint64_t* empty = is_k ? B.k_empty : B.v_empty;
+    const CUtensorMap* map_raw = is_k ? &P.tm_k_raw : &P.tm_v_raw;
+    const CUtensorMap* map_cmp = is_k ? &P.tm_k_cmp : &P.tm_v_cmp;
+    const uint32_t ring = sbase + (is_k ? L::kKOff : L::kVOff);
+    constexpr int kHalves = D / 64;
+    constexpr int kGroups = kT / 4;
+    const int grp = lane % kGroups;
+    const int half = lane / kGroups;
+    const bool issuer = lane < kGroups * kHalves;
+    int c = 0, g = 0, qc = 0;
+    bool final_seen = false;
+    while (!final_seen) {
+      const int slot = c & 1;
+      if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status)) break;
+      const ChunkDesc d = desc[slot];
+      final_seen = (d.flags & kFlagFinal) != 0;
+      const uint32_t* t_rows = tab + slot * kChunkKeys;
+      const int ntiles = ceil_tiles(d.nkeys);
+      bool ok = true;
+      if (is_k && (d.flags & kFlagFirst) && ntiles > 0) {
+        // Q of the unit, once the previous unit's last QK^T has completed
+        ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status);
+        if (ok && lane == 0) {
+          mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
+          for (int hb = 0; hb < kHalves; ++hb)
+            tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0, d.i);
+        }
+        ++qc;
       }
-      cp_async_wait_all();
+      for (int t = 0; ok && t < ntiles; ++t, ++g) {
+        const int stage = g % nst;
+        if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
+        __syncwarp();
+        if (issuer) {
+          const int nv = min(kT, d.nkeys - t * kT);
+          uint32_t e[4];
+          bool any_raw = false, any_cmp = false;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = 4 * grp + k;
+            e[k] = r < nv ? t_rows[t * kT + r] : kInvalidRow;
+            if (e[k] != kInvalidRow) {
+              if (e[k] & kRawBit) any_raw = true;
+              else any_cmp = true;
+            }
+          }
+          int32_t y[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)   // rows outside the tensor are zero-filled
+            y[k] = e[k] == kInvalidRow ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
+          const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
+          if (!(any_raw && any_cmp)) {
+            tma_gather4(dst, any_cmp ? map_cmp : map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const bool cmp_row = e[k] != kInvalidRow && !(e[k] & kRawBit);
+              tma_load_2d(dst + k * 128, cmp_row ? map_cmp : map_raw, full + stage, half * 64, y[k]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      mbar_arrive(B.tab_empty + slot);
+      ++c;
+      if (!ok) break;
     }
   } else if (warp == kMmaWarp) {
     // ================================================= UMMA issuer
-    if ((tid & 31) == 0 && ntiles > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kT, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
       const uint32_t q_addr = sbase + L::kQOff;
-      bool ok = mbar_wait(q_full, 0, abort_flag, P.dev_status);
-      fence_proxy_async_smem();
-      auto issue_pv = [&](int j) -> bool {
-        const int sb = j & 1, st = j % kStages;
-        if (!mbar_wait(p_ready + sb, (j >> 1) & 1, abort_flag, P.dev_status)) return false;
+      int c = 0, g = 0, qc = 0;
+      bool ok = true, final_seen = false;
+      bool pv_pending = false, pv_first = false;
+      int pv_g = 0, pv_unit = 0;
+      auto issue_pv = [&]() -> bool {
+        const int sb = pv_g & 1, st = pv_g % kStagesV;
+        if (!mbar_wait(B.p_ready + sb, (pv_g >> 1) & 1, abort_flag, P.dev_status)) return false;
+        if (pv_first && !mbar_wait(B.o_free, (pv_unit & 1) ^ 1, abort_flag, P.dev_status)) return false;
+        if (!mbar_wait(B.v_full + st, (pv_g / kStagesV) & 1, abort_flag, P.dev_status)) return false;
         tc_fence_after_sync();
-        const uint32_t v_addr = sbase + L::kStageOff + st * L::kStageBytes + L::kTileBytes;
+        const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
 #pragma unroll
         for (int k = 0; k < kT / 16; ++k) {
           const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
           umma_ts(tmem + L::kOCol, tmem + sb * kT + k * 8, bdesc, idesc_o,
-                  (j > 0 || k > 0) ? 1u : 0u);
+                  (!pv_first || k > 0) ? 1u : 0u);
         }
-        tc_commit(kv_empty + st);
-        tc_commit(o_done);
+        tc_commit(B.v_empty + st);
+        tc_commit(B.o_done + (pv_g & 1));
+        pv_pending = false;
         return true;
       };
-      for (int jt = 0; ok && jt < ntiles; ++jt) {
-        const int stage = jt % kStages, sb = jt & 1;
-        if (!mbar_wait(kv_full + stage, (jt / kStages) & 1, abort_flag, P.dev_status)) { ok = false; break; }
-        fence_proxy_async_smem();
-        tc_fence_after_sync();
-        const uint32_t k_addr = sbase + L::kStageOff + stage * L::kStageBytes;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t koff = (k & 3) * 32;   // 16 elements = 32 bytes inside the swizzle atom
-          const uint64_t adesc = smem_desc_sw128(q_addr + (k >> 2) * (128 * 128) + koff, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + koff, 16, 1024);
-          umma_ss(tmem + sb * kT, adesc, bdesc, idesc_s, k > 0 ? 1u : 0u);
+      while (ok && !final_seen) {
+        const int slot = c & 1;
+        if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status)) { ok = false; break; }
+        const ChunkDesc d = desc[slot];
+        mbar_arrive(B.tab_empty + slot);
+        ++c;
+        final_seen = (d.flags & kFlagFinal) != 0;
+        const int ntiles = ceil_tiles(d.nkeys);
+        if (ntiles == 0) continue;
+        if (d.flags & kFlagFirst) {
+          if (!mbar_wait(B.q_full, qc & 1, abort_flag, P.dev_status)) { ok = false; break; }
+          ++qc;
         }
-        tc_commit(s_full + sb);
-        if (jt >= 1 && !issue_pv(jt - 1)) { ok = false; break; }
+        for (int t = 0; t < ntiles; ++t, ++g) {
+          const int stage = g % kStagesK, sb = g & 1;
+          if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status)) { ok = false; break; }
+            tc_fence_after_sync();
+          const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t koff = (k & 3) * 32;   // 16 elements = 32 bytes inside the atom
+            const uint64_t adesc = smem_desc_sw128(q_addr + (k >> 2) * (128 * 128) + koff, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + koff, 16, 1024);
+            umma_ss(tmem + sb * kT, adesc, bdesc, idesc_s, k > 0 ? 1u : 0u);
+          }
+          tc_commit(B.k_empty + stage);
+          tc_commit(B.s_full + sb);
+          if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.q_empty);
+          if (pv_pending && !issue_pv()) { ok = false; break; }
+          pv_pending = true;
+          pv_g = g;
+          pv_first = (d.flags & kFlagFirst) && t == 0;
+          pv_unit = qc - 1;
+        }
       }
-      if (ok) ok = issue_pv(ntiles - 1);
+      if (ok && pv_pending) ok = issue_pv();
       // every UMMA has completed before TMEM is released
-      tc_commit(mma_done);
-      mbar_wait(mma_done, 0, nullptr, P.dev_status);
+      tc_commit(B.mma_done);
+      mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
     }
   } else {
     // ================================================= softmax + epilogue
@@ -295,169 +474,211 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const Par
     const int h = head0 + row;
     const bool row_ok = row < heads_here;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sink2 = (P.sink != nullptr && row_ok) ? P.sink[h] * kLog2e : -INFINITY;
+    int c = 0, g = 0;
+    bool ok = true, final_seen = false;
     float m = -INFINITY, l = 0.f;
-    if (split == 0 && P.sink != nullptr && row_ok) {
-      m = P.sink[h] * kLog2e;
-      l = 1.f;
-      if (!(m > -INFINITY)) { m = -INFINITY; l = 0.f; }
-    }
-    bool ok = true;
-    for (int jt = 0; jt < ntiles; ++jt) {
-      const int sb = jt & 1;
-      // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full + sb, (jt >> 1) & 1, abort_flag, P.dev_status))) {
+    int unit_tiles = 0;
+    while (ok && !final_seen) {
+      const int slot = c & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status))) {
         ok = false;
         break;
       }
-      tc_fence_after_sync();
-      const int nv = min(kT, key_hi - (key_lo + jt * kT));
-      uint32_t s0[32], s1[32];
-      tmem_ld32(lane_addr + sb * kT, s0);
-      tmem_ld32(lane_addr + sb * kT + 32, s1);
-      tmem_ld_wait(s0);
-      tmem_ld_wait(s1);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        if (c < nv) mx = fmaxf(mx, __uint_as_float(s0[c]));
-        if (c + 32 < nv) mx = fmaxf(mx, __uint_as_float(s1[c]));
+      const ChunkDesc d = desc[slot];
+      mbar_arrive(B.tab_empty + slot);
+      ++c;
+      final_seen = (d.flags & kFlagFinal) != 0;
+      if (d.flags & kFlagFirst) {
+        unit_tiles = 0;
+        m = (d.split == 0 && sink2 > -INFINITY) ? sink2 : -INFINITY;
+        l = (d.split == 0 && sink2 > -INFINITY) ? 1.f : 0.f;
       }
-      const float tmax = mx * P.scale_log2;
-      const bool move = tmax > m + kRescaleThreshold || (m == -INFINITY && tmax > -INFINITY);
-      const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
-      l *= alpha;
-      if (move) m = tmax;
-      if (jt > 0 && __any_sync(0xffffffffu, move)) {
-        // rows whose max moved rescale their O row (alpha = 1 elsewhere);
-        // PV(jt-1) must have landed in TMEM first
-        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (jt - 1) & 1, abort_flag, P.dev_status))) {
+      const int ntiles = ceil_tiles(d.nkeys);
+      for (int t = 0; t < ntiles; ++t, ++g, ++unit_tiles) {
+        const int sb = g & 1;
+        // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
+        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full + sb, (g >> 1) & 1, abort_flag, P.dev_status))) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
+        const int nv = min(kT, d.nkeys - t * kT);
+        uint32_t s0[32], s1[32];
+        tmem_ld32(lane_addr + sb * kT, s0);
+        tmem_ld32(lane_addr + sb * kT + 32, s1);
+        tmem_ld_wait(s0);
+        tmem_ld_wait(s1);
+        if (nv < kT) {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
+            if (cc + 32 >= nv) s1[cc] = __float_as_uint(-INFINITY);
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc)
+          mx = fmaxf(mx, fmaxf(__uint_as_float(s0[cc]), __uint_as_float(s1[cc])));
+        const float tmax = mx * P.scale_log2;
+        const bool move = tmax > m + kRescaleThreshold || (m == -INFINITY && tmax > -INFINITY);
+        const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
+        l *= alpha;
+        if (move) m = tmax;
+        if (unit_tiles > 0 && __any_sync(0xffffffffu, move)) {
+          // rows whose max moved rescale their O row (alpha = 1 elsewhere);
+          // the previous PV must have landed in TMEM first
+          if (!__all_sync(0xffffffffu, mbar_wait(B.o_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag,
+                                                 P.dev_status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + L::kOCol + c0, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
+            tmem_st32(lane_addr + L::kOCol + c0, o);
+          }
+          tmem_st_wait();
+        }
+        const float neg_m = -m;
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
+          const float p2 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc]), P.scale_log2, neg_m));
+          const float p3 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc + 1]), P.scale_log2, neg_m));
+          sum0 += p0 + p1;
+          sum1 += p2 + p3;
+          pk[cc] = pack_bf16x2(p0, p1);
+          pk[cc + 16] = pack_bf16x2(p2, p3);
+        }
+        l += sum0 + sum1;
+        tmem_st32(lane_addr + sb * kT, pk);   // P overwrites the first 32 columns of S
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(B.p_ready + sb);
+      }
+      if (!ok || !(d.flags & kFlagLast)) continue;
+
+      // ---- epilogue of the unit
+      const bool have_o = unit_tiles > 0;
+      if (have_o) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.o_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag,
+                                               P.dev_status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+      }
+      const int i = d.i;
+      if (S == 1) {
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        uint16_t* orow = P.out + (static_cast<int64_t>(i) * P.num_heads + h) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_addr + L::kOCol + c0, o);
-          tmem_ld_wait(o);
+          if (have_o) {
+            tmem_ld32(lane_addr + L::kOCol + c0, o);
+            tmem_ld_wait(o);
+          } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(lane_addr + L::kOCol + c0, o);
+            for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc)
+            pk[cc] = pack_bf16x2(__uint_as_float(o[2 * cc]) * inv_l, __uint_as_float(o[2 * cc + 1]) * inv_l);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
-        tmem_st_wait();
-      }
-      const float neg_m = -m;
-      float sum = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float p0 = (2 * c < nv) ? exp2_approx(fmaf(__uint_as_float(s0[2 * c]), P.scale_log2, neg_m)) : 0.f;
-        const float p1 = (2 * c + 1 < nv) ? exp2_approx(fmaf(__uint_as_float(s0[2 * c + 1]), P.scale_log2, neg_m)) : 0.f;
-        const float p2 = (2 * c + 32 < nv) ? exp2_approx(fmaf(__uint_as_float(s1[2 * c]), P.scale_log2, neg_m)) : 0.f;
-        const float p3 = (2 * c + 33 < nv) ? exp2_approx(fmaf(__uint_as_float(s1[2 * c + 1]), P.scale_log2, neg_m)) : 0.f;
-        sum += (p0 + p1) + (p2 + p3);
-        pk[c] = pack_bf16x2(p0, p1);
-        pk[c + 16] = pack_bf16x2(p2, p3);
-      }
-      l += sum;
-      tmem_st32(lane_addr + sb * kT, pk);   // P overwrites the first 32 columns of S
-      tmem_st_wait();
-      tc_fence_before_sync();
-      mbar_arrive(p_ready + sb);
-    }
-    if (ok && ntiles > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(o_done, (ntiles - 1) & 1, abort_flag, P.dev_status));
-      tc_fence_after_sync();
-    }
-    const bool have_o = ok && ntiles > 0;
-    if (S == 1) {
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* orow = P.out + (static_cast<int64_t>(i) * P.num_heads + h) * D;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
         if (have_o) {
-          tmem_ld32(lane_addr + L::kOCol + c0, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0u;
+          tc_fence_before_sync();
+          mbar_arrive(B.o_free);   // O may be overwritten by the next unit
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-      }
-      if (row_ok) P.lse[static_cast<int64_t>(i) * P.num_heads + h] = l > 0.f ? (m + log2_approx(l)) * kLn2 : -INFINITY;
-    } else {
-      // partial result of this slice (no normalisation), then the last
-      // slice to finish merges all of them
-      const int64_t unit = static_cast<int64_t>(i) * S + split;
-      float* prow = P.part_o + (unit * P.num_heads + h) * D;
+        if (row_ok)
+          P.lse[static_cast<int64_t>(i) * P.num_heads + h] = l > 0.f ? (m + log2_approx(l)) * kLn2 : -INFINITY;
+      } else {
+        // partial result of this slice (no normalisation); the last slice
+        // of the query to finish merges all of them
+        const int64_t unit = static_cast<int64_t>(i) * S + d.split;
+        float* prow = P.part_o + (unit * P.num_heads + h) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          if (have_o) {
+            tmem_ld32(lane_addr + L::kOCol + c0, o);
+            tmem_ld_wait(o);
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
+          }
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(prow + c0);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                   __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          }
+        }
         if (have_o) {
-          tmem_ld32(lane_addr + L::kOCol + c0, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0u;
+          tc_fence_before_sync();
+          mbar_arrive(B.o_free);
         }
-        if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(prow + c0);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
-        }
-      }
-      if (row_ok) P.part_ml[unit * P.num_heads + h] = make_float2(m, l);
-      __threadfence();
-      named_bar_sync(2, kSoftThreads);
-      if (tid == 0) *ticket_slot = atomicAdd(P.tickets + static_cast<int64_t>(i) * gridDim.y + blockIdx.y, 1u);
-      named_bar_sync(2, kSoftThreads);
-      if (*ticket_slot == static_cast<uint32_t>(S - 1) && row_ok) {
+        if (row_ok) P.part_ml[unit * P.num_heads + h] = make_float2(m, l);
         __threadfence();
-        float M = -INFINITY;
-        for (int s = 0; s < S; ++s) {
-          const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
-          if (ml.y > 0.f) M = fmaxf(M, ml.x);
-        }
-        float Lsum = 0.f;
-        float w[kAttnMaxSplits];
-#pragma unroll
-        for (int s = 0; s < kAttnMaxSplits; ++s) {
-          w[s] = 0.f;
-          if (s < S) {
-            const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
-            w[s] = (ml.y > 0.f) ? exp2_approx(ml.x - M) : 0.f;
-            Lsum += w[s] * ml.y;
-          }
-        }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-        uint16_t* orow = P.out + (static_cast<int64_t>(i) * P.num_heads + h) * D;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 8) {
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        named_bar_sync(2, kSoftThreads);
+        if (tid == 0) *ticket_slot = atomicAdd(P.tickets + static_cast<int64_t>(i) * gridDim.y + blockIdx.y, 1u);
+        named_bar_sync(2, kSoftThreads);
+        const bool merge = *ticket_slot == static_cast<uint32_t>(S - 1);
+        named_bar_sync(2, kSoftThreads);   // ticket_slot is reused by the next unit
+        if (merge && row_ok) {
+          __threadfence();
+          float M = -INFINITY;
           for (int s = 0; s < S; ++s) {
-            if (w[s] == 0.f) continue;
-            const float4* src = reinterpret_cast<const float4*>(
-                P.part_o + (((static_cast<int64_t>(i) * S + s) * P.num_heads + h) * D + c0));
-            const float4 a = __ldcg(src), bq = __ldcg(src + 1);
-            acc[0] += w[s] * a.x; acc[1] += w[s] * a.y; acc[2] += w[s] * a.z; acc[3] += w[s] * a.w;
-            acc[4] += w[s] * bq.x; acc[5] += w[s] * bq.y; acc[6] += w[s] * bq.z; acc[7] += w[s] * bq.w;
+            const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
+            if (ml.y > 0.f) M = fmaxf(M, ml.x);
           }
-          *reinterpret_cast<uint4*>(orow + c0) =
-              make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                         pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+          float Lsum = 0.f;
+          float w[kAttnMaxSplits];
+#pragma unroll
+          for (int s = 0; s < kAttnMaxSplits; ++s) {
+            w[s] = 0.f;
+            if (s < S) {
+              const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
+              w[s] = (ml.y > 0.f) ? exp2_approx(ml.x - M) : 0.f;
+              Lsum += w[s] * ml.y;
+            }
+          }
+          const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+          uint16_t* orow = P.out + (static_cast<int64_t>(i) * P.num_heads + h) * D;
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 8) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int s = 0; s < S; ++s) {
+              if (w[s] == 0.f) continue;
+              const float4* src = reinterpret_cast<const float4*>(
+                  P.part_o + (((static_cast<int64_t>(i) * S + s) * P.num_heads + h) * D + c0));
+              const float4 a = __ldcg(src), bq = __ldcg(src + 1);
+              acc[0] += w[s] * a.x; acc[1] += w[s] * a.y; acc[2] += w[s] * a.z; acc[3] += w[s] * a.w;
+              acc[4] += w[s] * bq.x; acc[5] += w[s] * bq.y; acc[6] += w[s] * bq.z; acc[7] += w[s] * bq.w;
+            }
+            *reinterpret_cast<uint4*>(orow + c0) =
+                make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                           pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+          }
+          P.lse[static_cast<int64_t>(i) * P.num_heads + h] =
+              Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
         }
-        P.lse[static_cast<int64_t>(i) * P.num_heads + h] = Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
       }
     }
   }
@@ -470,6 +691,19 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const Par
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+int sm_count_cached() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+    else
+      n = 148;
+  }
+  return n;
+}
+
 template <int D>
 cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
   using L = Layout<D>;
@@ -480,7 +714,9 @@ cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     configured = true;
   }
-  dim3 grid(static_cast<unsigned>(P.n_queries) * P.num_splits, head_tiles);
+  const int64_t units = static_cast<int64_t>(P.n_queries) * P.num_splits;
+  const int64_t slots = std::max<int64_t>(1, (2 * static_cast<int64_t>(sm_count_cached())) / head_tiles);
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
   sparse_sink_attn_kernel<D><<<grid, kThreads, L::kBytes, stream>>>(P);
   return cudaGetLastError();
 }
@@ -489,6 +725,45 @@ int log2_exact(int32_t v) {
   int k = 0;
   while ((1 << k) < v) ++k;
   return k;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// A paged pool [rows, d] BF16 as a 2D tensor with a one-row, 64-column box,
+// 128-byte swizzle: the form tile::gather4 takes.
+bool encode_pool(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(std::max<int64_t>(rows, 1))};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t elem[2] = {1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                              box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q [N, H, d] with element strides (tok, head) as a 3D tensor {d, H, N}.
+bool encode_q(CUtensorMap* m, const void* base, int32_t n, int32_t h, int d, int64_t stride_tok,
+              int64_t stride_head, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(h),
+                              static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride_head) * 2, static_cast<cuuint64_t>(stride_tok) * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                              box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -507,6 +782,21 @@ size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_d
 cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
   if (a.n_queries == 0) return cudaSuccess;
   Params P;
+  memset(&P, 0, sizeof P);
+  if (tensor_map_encoder() == nullptr) return cudaErrorNotSupported;
+  P.q_box_rows = std::min(128, a.num_heads);
+  const int64_t raw_rows = a.raw_num_pages * a.raw_page_size;
+  if (!encode_q(&P.tm_q, a.q, a.n_queries, a.num_heads, a.head_dim, a.q_stride_tok, a.q_stride_head,
+                P.q_box_rows) ||
+      !encode_pool(&P.tm_k_raw, a.k_raw, raw_rows, a.head_dim) ||
+      !encode_pool(&P.tm_v_raw, a.v_raw, raw_rows, a.head_dim))
+    return cudaErrorInvalidValue;
+  if (a.pt_cmp != nullptr) {
+    const int64_t cmp_rows = a.cmp_num_pages * a.cmp_page_size;
+    if (!encode_pool(&P.tm_k_cmp, a.k_cmp, cmp_rows, a.head_dim) ||
+        !encode_pool(&P.tm_v_cmp, a.v_cmp, cmp_rows, a.head_dim))
+      return cudaErrorInvalidValue;
+  }
   P.q = a.q;
   P.q_stride_tok = a.q_stride_tok;
   P.q_stride_head = a.q_stride_head;

@@ -8,9 +8,12 @@
 // complete groups outnumber it.
 //
 // One pass over the queries. A CTA owns 8 consecutive queries, one warp
-// each. A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio)),
-// sorts it in shared memory with a bitonic network and counts the distinct
-// survivors; the window adds min(p+1, W) keys. The CTA publishes its total
+// each. A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio))
+// into a shared-memory bitmap over the complete groups -- setting a bit drops
+// repeats and reading the words in order yields the ascending list -- and
+// counts the set bits; when the complete groups outnumber the bitmap it
+// sorts the row with a bitonic network instead. The window adds min(p+1, W)
+// keys. The CTA publishes its total
 // and obtains its offset by a decoupled look-back over the CTAs before it
 // (CTA order taken from an atomic ticket, so every predecessor is already
 // running), then every warp writes its indptr entry and its keys: the
@@ -65,6 +68,7 @@ struct SetsParams {
   const int32_t* topk;
   int32_t topk_width;
   int32_t sort_width;  // topk_width rounded up to a power of two (>= 32)
+  int32_t buf_words;   // per-warp shared buffer (>= sort_width), also the bitmap size
   int32_t* indptr;
   int32_t* indices;
   int64_t capacity;
@@ -75,7 +79,7 @@ struct SetsParams {
 
 __global__ void __launch_bounds__(kSetsQueriesPerCta * 32)
 build_kv_sets_kernel(const SetsParams P) {
-  extern __shared__ int32_t sort_buf[];  // [kSetsQueriesPerCta][sort_width]
+  extern __shared__ int32_t sort_buf[];  // [kSetsQueriesPerCta][buf_words]
   __shared__ int64_t s_count[kSetsQueriesPerCta];
   __shared__ int64_t s_tile_offset;
   __shared__ uint32_t s_tile;
@@ -90,7 +94,7 @@ build_kv_sets_kernel(const SetsParams P) {
 
   int32_t p = 0, n_window = 0, n_complete = 0;
   int64_t n_groups = 0;
-  int32_t* buf = sort_buf + warp * P.sort_width;
+  int32_t* buf = sort_buf + warp * P.buf_words;
   const bool sorted_list = P.ratio > 0 && P.topk != nullptr;
   if (active) {
     p = P.pos[i];
@@ -104,6 +108,22 @@ build_kv_sets_kernel(const SetsParams P) {
     if (p >= 0 && P.ratio > 0) {
       if (!sorted_list) {
         n_groups = n_complete;
+      } else if (((n_complete + 31) >> 5) <= P.buf_words) {
+        // bitmap over the complete groups: marking a bit removes repeats,
+        // reading the words in order gives the ascending list
+        uint32_t* bm = reinterpret_cast<uint32_t*>(buf);
+        const int words = (n_complete + 31) >> 5;
+        for (int w = lane; w < words; w += 32) bm[w] = 0u;
+        __syncwarp();
+        const int32_t* row = P.topk + i * P.topk_width;
+        for (int j = lane; j < P.topk_width; j += 32) {
+          const int32_t g = row[j];
+          if (g >= 0 && g < n_complete) atomicOr(bm + (g >> 5), 1u << (g & 31));
+        }
+        __syncwarp();
+        int cnt = 0;
+        for (int w = lane; w < words; w += 32) cnt += __popc(bm[w]);
+        n_groups = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(cnt));
       } else {
         const int32_t* row = P.topk + i * P.topk_width;
         for (int j = lane; j < P.sort_width; j += 32) {
@@ -172,7 +192,30 @@ build_kv_sets_kernel(const SetsParams P) {
   const int64_t limit = P.capacity < INT_MAX ? P.capacity : INT_MAX;
 
   // compressed groups, ascending
-  if (sorted_list) {
+  if (sorted_list && ((n_complete + 31) >> 5) <= P.buf_words) {
+    const uint32_t* bm = reinterpret_cast<const uint32_t*>(buf);
+    const int words = (n_complete + 31) >> 5;
+    int64_t written = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t bits = w < words ? bm[w] : 0u;
+      const int cnt = __popc(bits);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int64_t dst = start + written + (incl - cnt);
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        if (dst < limit) P.indices[dst] = w * 32 + bit;
+        ++dst;
+        bits &= bits - 1u;
+      }
+      written += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  } else if (sorted_list) {
     int64_t written = 0;
     for (int j0 = 0; j0 < P.sort_width; j0 += 32) {
       if (buf[j0] == INT_MAX) break;  // sentinels sort last
@@ -227,6 +270,9 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
   P.topk = (ratio > 0) ? topk : nullptr;
   P.topk_width = topk_width;
   P.sort_width = (P.topk != nullptr) ? sort_width_for(topk_width) : 32;
+  // bitmap of at least 512 words (16384 groups) per warp; the sort handles
+  // queries with more complete groups than that
+  P.buf_words = P.sort_width > 512 ? P.sort_width : 512;
   P.indptr = indptr;
   P.indices = indices;
   P.capacity = capacity;
@@ -234,7 +280,7 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
   P.tile_ticket = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + tiles * sizeof(uint64_t));
   P.dev_status = dev_status;
   const size_t smem = (P.topk != nullptr)
-                          ? static_cast<size_t>(kSetsQueriesPerCta) * P.sort_width * sizeof(int32_t)
+                          ? static_cast<size_t>(kSetsQueriesPerCta) * P.buf_words * sizeof(int32_t)
                           : 0;
   if (smem > 48 * 1024) {
     err = cudaFuncSetAttribute(build_kv_sets_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

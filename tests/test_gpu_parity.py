@@ -105,9 +105,14 @@ def test_kv_sets_bit_exact_full_size(spa, name):
 def test_kv_sets_edge_cases(spa):
     import oracle
     rng = np.random.default_rng(5)
-    pos = np.concatenate([[0, 1, 2, 3, 4, 127, 128, 129, 4095], rng.integers(0, 9000, 300)]).astype(np.int32)
+    # positions past 65535 have more than 16384 complete ratio-4 groups: the
+    # builder's bitmap is too small for them and it sorts instead
+    pos = np.concatenate([[0, 1, 2, 3, 4, 127, 128, 129, 4095, 65535, 65536, 65539],
+                          rng.integers(0, 9000, 300), rng.integers(60000, 140000, 40)]).astype(np.int32)
     for K in (1, 5, 32, 33, 512, 2048):
         topk = rng.integers(-3, 2300, size=(pos.size, K)).astype(np.int32)
+        far = pos >= 60000
+        topk[far] = rng.integers(-3, 36000, size=(int(far.sum()), K))
         topk[:, : K // 2] = topk[:, :1]           # many repeats
         for ratio, W in ((4, 128), (4, 1), (128, 7), (0, 64)):
             t = torch.from_numpy(topk).cuda() if ratio == 4 else None
