@@ -19,21 +19,22 @@
 // l = 1), so it is counted exactly once and never multiplies a V row.
 //
 // Persistent CTAs (two per SM) walk their units in a fixed stride. Warp
-// roles (256 threads):
+// roles (384 threads):
 //   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t
 //   warp  4    TMEM allocation; lane 0 issues every UMMA and commit
-//   warp  5    K (and Q) gather: TMA tile::gather4 loads (four rows of one
-//              pool per instruction, one instruction per lane per tile) into
-//              a 2-stage ring, 128-byte swizzled by the tensor map into the
-//              K-major layout of the UMMA descriptors; rows outside the pool
-//              (padding, faulty keys) are zero-filled by the TMA
-//   warp  6    V gather, into its own 2-stage ring
-//   warp  7    resolver: for a chunk of up to 1024 keys of a unit it loads
+//   warp  5    resolver: for a chunk of up to 512 keys of a unit it loads
 //              the keys, looks their pages up and writes the physical row
 //              of every key (bit 31 = raw pool) to a double-buffered table,
 //              plus a chunk descriptor that every other role follows. All
 //              dependent global loads of the gather happen here, ahead of
 //              the copies.
+//   warps 6-8  K gather: 96 lanes copy the tile's rows in 16-byte cp.async
+//              pieces into a 2-stage ring, 128-byte swizzled in the K-major
+//              layout of the UMMA descriptors (random rows need many copies
+//              in flight: measured on B200, 16-byte copies from eight warps
+//              per CTA reach 14.7 TB/s of L2 gather, TMA gather4 from one or
+//              two warps 4-6 TB/s); lane 0 of warp 6 also loads Q (TMA box)
+//   warps 9-11 V gather, into its own 2-stage ring
 // TMEM columns: S/P buffer 0 [0,64), buffer 1 [64,128), O [128,128+d).
 // The running max only moves when a tile's max exceeds it by more than 8
 // (log2 units), so P <= 256 and O is rescaled rarely; O/l and LSE use the
@@ -55,19 +56,21 @@ constexpr int kStagesK = 2;
 constexpr int kStagesV = 2;
 constexpr int kSoftThreads = 128;
 constexpr int kMmaWarp = 4;
-constexpr int kKWarp = 5;
-constexpr int kVWarp = 6;
-constexpr int kResolverWarp = 7;
+constexpr int kResolverWarp = 5;
+constexpr int kKWarp0 = 6;                       // K producer: warp 6
+constexpr int kVWarp0 = 7;                       // V producer: warp 7
+constexpr int kProdWarps = 1;
+constexpr int kProdLanes = kProdWarps * 32;
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
-constexpr int kChunkKeys = 1024;                 // keys resolved per chunk
+constexpr int kChunkKeys = 768;                  // keys resolved per chunk (12 tiles)
 constexpr uint32_t kRawBit = 0x80000000u;
 constexpr uint32_t kInvalidRow = 0xFFFFFFFFu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 // consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
-constexpr uint32_t kTabConsumers = 32 + 32 + 1 + kSoftThreads;
+constexpr uint32_t kTabConsumers = 2 * kProdLanes + 1 + kSoftThreads;
 
 constexpr int kFlagFirst = 1;   // first chunk of its unit
 constexpr int kFlagLast = 2;    // last chunk of its unit
@@ -127,7 +130,8 @@ struct Layout {
   static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
   static constexpr int kTabOff = kVOff + kStagesV * kTileBytes;       // [2][kChunkKeys] u32
   static constexpr int kDescOff = kTabOff + 2 * kChunkKeys * 4;       // [2] ChunkDesc
-  static constexpr int kBarOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
+  static constexpr int kMergeOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));  // [16][128] f32
+  static constexpr int kBarOff = kMergeOff + kAttnMaxSplits * 128 * 4;
   // tab_full, tab_empty, q_full + q_empty, K ring, V ring, s_full, p_ready,
   // o_done, o_free, mma_done
   static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 1 + 1;
@@ -258,11 +262,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     mbar_init(B.q_full, 1);
     mbar_init(B.q_empty, 1);
     for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(B.k_full + s, 1);
+      mbar_init(B.k_full + s, kProdWarps);   // one expect_tx arrival per producer warp
       mbar_init(B.k_empty + s, 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(B.v_full + s, 1);
+      mbar_init(B.v_full + s, kProdWarps);
       mbar_init(B.v_empty + s, 1);
     }
     mbar_init(B.o_done, 1);
@@ -323,13 +327,20 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         k0 += n;
       } while (k0 < key_hi);
     }
-  } else if (warp == kKWarp || warp == kVWarp) {
+  } else if (warp >= kKWarp0) {
     // ================================================= K / V gather (TMA)
-    // Each lane issues one gather4 per tile: rows 4*grp .. 4*grp+3 of the
-    // tile, one 64-column half of the row. A group whose four keys come from
-    // both pools (at most one per unit: the sets list compressed groups
-    // before window tokens) is loaded row by row instead.
-    const bool is_k = warp == kKWarp;
+    // Two warps stream K tiles and two stream V tiles. Each tile is 16
+    // four-row groups x D/64 column halves = "jobs"; a warp's lanes issue one
+    // TMA tile::gather4 per job of its share (four rows of one pool, 512
+    // bytes, 128-byte swizzled by the tensor map into the K-major layout of
+    // the UMMA descriptors). Measured on B200, gather4 throughput scales with
+    // the number of issuing warps, hence two per operand. A group whose four
+    // keys come from both pools (at most one per unit: compressed groups
+    // precede window tokens) is loaded row by row. Rows past the chunk's keys
+    // and rows of faulty keys are outside the tensor and zero-filled. Lane 0
+    // of the first K warp also loads Q, as TMA boxes.
+    const bool is_k = warp < kVWarp0;
+    const int wsub = warp - (is_k ? kKWarp0 : kVWarp0);   // 0 or 1
     const int nst = is_k ? kStagesK : kStagesV;
     uint64_t* full = is_k ? B.k_full : B.v_full;
     uint64_t* empty = is_k ? B.k_empty : B.v_empty;
@@ -338,9 +349,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     const uint32_t ring = sbase + (is_k ? L::kKOff : L::kVOff);
     constexpr int kHalves = D / 64;
     constexpr int kGroups = kT / 4;
-    const int grp = lane % kGroups;
-    const int half = lane / kGroups;
-    const bool issuer = lane < kGroups * kHalves;
+    constexpr int kJobsPerWarp = kGroups * kHalves / kProdWarps;
+    const int job = wsub * kJobsPerWarp + lane;
+    const int grp = job % kGroups, half = job / kGroups;
+    const bool issuer = lane < kJobsPerWarp;
+    const bool q_loader = warp == kKWarp0;
     int c = 0, g = 0, qc = 0;
     bool final_seen = false;
     while (!final_seen) {
@@ -351,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const uint32_t* t_rows = tab + slot * kChunkKeys;
       const int ntiles = ceil_tiles(d.nkeys);
       bool ok = true;
-      if (is_k && (d.flags & kFlagFirst) && ntiles > 0) {
+      if (q_loader && (d.flags & kFlagFirst) && ntiles > 0) {
         // Q of the unit, once the previous unit's last QK^T has completed
         ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status);
         if (ok && lane == 0) {
@@ -364,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       for (int t = 0; ok && t < ntiles; ++t, ++g) {
         const int stage = g % nst;
         if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
+        if (lane == 0) mbar_arrive_expect_tx(full + stage, kJobsPerWarp * 512);
         __syncwarp();
         if (issuer) {
           const int nv = min(kT, d.nkeys - t * kT);
@@ -395,7 +408,6 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           }
         }
       }
-      __syncwarp();
       mbar_arrive(B.tab_empty + slot);
       ++c;
       if (!ok) break;
@@ -509,17 +521,23 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         tmem_ld32(lane_addr + sb * kT + 32, s1);
         tmem_ld_wait(s0);
         tmem_ld_wait(s1);
-        if (nv < kT) {
+        if (nv < kT) {   // columns past the set: -inf, so they add nothing
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) {
             if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
             if (cc + 32 >= nv) s1[cc] = __float_as_uint(-INFINITY);
           }
         }
-        float mx = -INFINITY;
+        // row max as eight independent chains and a tree (a single chain
+        // of 64 dependent max operations would dominate the tile's latency)
+        float mx8[8];
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc)
-          mx = fmaxf(mx, fmaxf(__uint_as_float(s0[cc]), __uint_as_float(s1[cc])));
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(__uint_as_float(s0[k]), __uint_as_float(s1[k]));
+#pragma unroll
+        for (int k = 8; k < 32; ++k)
+          mx8[k & 7] = fmaxf(mx8[k & 7], fmaxf(__uint_as_float(s0[k]), __uint_as_float(s1[k])));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float tmax = mx * P.scale_log2;
         const bool move = tmax > m + kRescaleThreshold || (m == -INFINITY && tmax > -INFINITY);
         const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
@@ -546,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           tmem_st_wait();
         }
         const float neg_m = -m;
-        float sum0 = 0.f, sum1 = 0.f;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[32];
 #pragma unroll
         for (int cc = 0; cc < 16; ++cc) {
@@ -554,12 +572,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
           const float p2 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc]), P.scale_log2, neg_m));
           const float p3 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc + 1]), P.scale_log2, neg_m));
-          sum0 += p0 + p1;
-          sum1 += p2 + p3;
+          sum4[cc & 3] += (p0 + p1) + (p2 + p3);
           pk[cc] = pack_bf16x2(p0, p1);
           pk[cc + 16] = pack_bf16x2(p2, p3);
         }
-        l += sum0 + sum1;
+        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         tmem_st32(lane_addr + sb * kT, pk);   // P overwrites the first 32 columns of S
         tmem_st_wait();
         tc_fence_before_sync();
@@ -641,43 +658,66 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         named_bar_sync(2, kSoftThreads);
         const bool merge = *ticket_slot == static_cast<uint32_t>(S - 1);
         named_bar_sync(2, kSoftThreads);   // ticket_slot is reused by the next unit
-        if (merge && row_ok) {
+        if (merge) {
+          // exact merge of the S slices: LSE = M + log2(L), O = sum_s w_s O_s
+          // with w_s = 2^(m_s - M) / L. Thread h first turns its head's
+          // (m_s, l_s) into the weights (in shared memory), then the 128
+          // threads sum the partial rows column-wise: each warp covers
+          // whole 512-byte rows with float4 loads, coalesced.
           __threadfence();
-          float M = -INFINITY;
-          for (int s = 0; s < S; ++s) {
-            const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
-            if (ml.y > 0.f) M = fmaxf(M, ml.x);
-          }
-          float Lsum = 0.f;
-          float w[kAttnMaxSplits];
-#pragma unroll
-          for (int s = 0; s < kAttnMaxSplits; ++s) {
-            w[s] = 0.f;
-            if (s < S) {
-              const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
-              w[s] = (ml.y > 0.f) ? exp2_approx(ml.x - M) : 0.f;
-              Lsum += w[s] * ml.y;
-            }
-          }
-          const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-          uint16_t* orow = P.out + (static_cast<int64_t>(i) * P.num_heads + h) * D;
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 8) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float* wl = reinterpret_cast<float*>(smem + L::kMergeOff);   // [kAttnMaxSplits][128]
+          if (row_ok) {
+            float M = -INFINITY;
             for (int s = 0; s < S; ++s) {
-              if (w[s] == 0.f) continue;
-              const float4* src = reinterpret_cast<const float4*>(
-                  P.part_o + (((static_cast<int64_t>(i) * S + s) * P.num_heads + h) * D + c0));
-              const float4 a = __ldcg(src), bq = __ldcg(src + 1);
-              acc[0] += w[s] * a.x; acc[1] += w[s] * a.y; acc[2] += w[s] * a.z; acc[3] += w[s] * a.w;
-              acc[4] += w[s] * bq.x; acc[5] += w[s] * bq.y; acc[6] += w[s] * bq.z; acc[7] += w[s] * bq.w;
+              const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
+              if (ml.y > 0.f) M = fmaxf(M, ml.x);
             }
-            *reinterpret_cast<uint4*>(orow + c0) =
-                make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                           pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+            float Lsum = 0.f;
+            for (int s = 0; s < S; ++s) {
+              const float2 ml = __ldcg(P.part_ml + (static_cast<int64_t>(i) * S + s) * P.num_heads + h);
+              const float w = (ml.y > 0.f) ? exp2_approx(ml.x - M) : 0.f;
+              wl[s * 128 + row] = w;
+              Lsum += w * ml.y;
+            }
+            const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+            for (int s = 0; s < S; ++s) wl[s * 128 + row] *= inv;
+            P.lse[static_cast<int64_t>(i) * P.num_heads + h] =
+                Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
           }
-          P.lse[static_cast<int64_t>(i) * P.num_heads + h] =
-              Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
+          named_bar_sync(2, kSoftThreads);
+          constexpr int kF4 = D / 4;                   // float4 per row
+          constexpr int kRowsPerPass = kSoftThreads / kF4;
+          constexpr int kBatch = 4;                    // row passes whose loads are in flight together
+          const int rsub = tid / kF4, c4 = tid % kF4;
+          const float4* part4 = reinterpret_cast<const float4*>(P.part_o);
+#pragma unroll 1
+          for (int r0 = 0; r0 < heads_here; r0 += kRowsPerPass * kBatch) {
+            float4 acc[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // all loads of the batch first (no store in between)
+            for (int s = 0; s < S; ++s) {
+#pragma unroll
+              for (int q = 0; q < kBatch; ++q) {
+                const int hr = r0 + q * kRowsPerPass + rsub;
+                if (hr >= heads_here) continue;
+                const float w = wl[s * 128 + hr];
+                const float4 v = __ldcg(part4 + ((static_cast<int64_t>(i) * S + s) * P.num_heads + head0 + hr) * kF4 + c4);
+                acc[q].x = fmaf(w, v.x, acc[q].x);
+                acc[q].y = fmaf(w, v.y, acc[q].y);
+                acc[q].z = fmaf(w, v.z, acc[q].z);
+                acc[q].w = fmaf(w, v.w, acc[q].w);
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+              const int hr = r0 + q * kRowsPerPass + rsub;
+              if (hr >= heads_here) continue;
+              *reinterpret_cast<uint2*>(P.out + (static_cast<int64_t>(i) * P.num_heads + head0 + hr) * D + 4 * c4) =
+                  make_uint2(pack_bf16x2(acc[q].x, acc[q].y), pack_bf16x2(acc[q].z, acc[q].w));
+            }
+          }
+          named_bar_sync(2, kSoftThreads);   // wl is reused by the next merge
         }
       }
     }
