@@ -7,18 +7,18 @@
 // "Validation": ratio 0 / 4 / 128 layers; top-k truncates only once the
 // complete groups outnumber it.
 //
-// One pass over the queries. A CTA owns 8 consecutive queries, one warp
-// each. A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio))
+// A CTA owns a block of consecutive queries, one warp per query at a time.
+// A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio))
 // into a shared-memory bitmap over the complete groups -- setting a bit drops
 // repeats and reading the words in order yields the ascending list -- and
 // counts the set bits; when the complete groups outnumber the bitmap it
 // sorts the row with a bitonic network instead. The window adds min(p+1, W)
-// keys. The CTA publishes its total
-// and obtains its offset by a decoupled look-back over the CTAs before it
-// (CTA order taken from an atomic ticket, so every predecessor is already
-// running), then every warp writes its indptr entry and its keys: the
-// distinct groups ascending, then the window tokens ascending with the
-// window tag. Integer only; no floating point anywhere.
+// keys. The CTA scans its counts, publishes its total and obtains its offset
+// by a decoupled look-back over the CTAs before it (CTA order taken from an
+// atomic ticket, so every predecessor is already running; one warp reads 32
+// predecessors per step), then recomputes every set and writes its indptr
+// entry and its keys: the distinct groups ascending, then the window tokens
+// ascending with the window tag. Integer only; no floating point anywhere.
 #include <climits>
 #include <mutex>
 
@@ -69,6 +69,7 @@ struct SetsParams {
   int32_t topk_width;
   int32_t sort_width;  // topk_width rounded up to a power of two (>= 32)
   int32_t buf_words;   // per-warp shared buffer (>= sort_width), also the bitmap size
+  int32_t per_cta;     // consecutive queries owned by one CTA
   int32_t* indptr;
   int32_t* indices;
   int64_t capacity;
@@ -77,124 +78,48 @@ struct SetsParams {
   uint32_t* dev_status;
 };
 
-__global__ void __launch_bounds__(kSetsQueriesPerCta * 32)
-build_kv_sets_kernel(const SetsParams P) {
-  extern __shared__ int32_t sort_buf[];  // [kSetsQueriesPerCta][buf_words]
-  __shared__ int64_t s_count[kSetsQueriesPerCta];
-  __shared__ int64_t s_tile_offset;
-  __shared__ uint32_t s_tile;
+constexpr int kSetsWarps = kSetsQueriesPerCta;   // warps per CTA
+constexpr int kMaxPerCta = 2048;
 
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) s_tile = atomicAdd(P.tile_ticket, 1u);
-  __syncthreads();
-  const uint32_t tile = s_tile;
-  const int64_t i = static_cast<int64_t>(tile) * kSetsQueriesPerCta + warp;
-  const bool active = i < P.n;
+__device__ __forceinline__ int64_t warp_sum64(int64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
 
-  int32_t p = 0, n_window = 0, n_complete = 0;
+// The key set of query i, by one warp (all lanes call together). Returns
+// the number of keys; when `write` is set, stores them at
+// indices[start ..) ascending (entries at or past `limit` are dropped).
+__device__ int64_t one_query(const SetsParams& P, int64_t i, int32_t* buf, int lane, bool write,
+                             int64_t start, int64_t limit) {
+  const int32_t p = P.pos[i];
+  if (p < 0 || p >= SPA_WINDOW_TAG) {
+    if (lane == 0 && !write) report(P.dev_status, SPA_DEV_BAD_INDEX);
+    return 0;
+  }
+  const int32_t n_window = min(p + 1, P.window);
+  const int32_t n_complete = P.ratio > 0 ? (p + 1) / P.ratio : 0;
+  const bool listed = P.ratio > 0 && P.topk != nullptr;
+  const int words = (n_complete + 31) >> 5;
+  const bool use_bitmap = listed && words <= P.buf_words;
   int64_t n_groups = 0;
-  int32_t* buf = sort_buf + warp * P.buf_words;
-  const bool sorted_list = P.ratio > 0 && P.topk != nullptr;
-  if (active) {
-    p = P.pos[i];
-    if (p < 0 || p >= SPA_WINDOW_TAG) {
-      if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
-      p = -1;  // empty set
-    } else {
-      n_window = min(p + 1, P.window);
-      n_complete = P.ratio > 0 ? (p + 1) / P.ratio : 0;
+  if (P.ratio > 0 && !listed) {
+    n_groups = n_complete;
+    if (write)
+      for (int64_t g = lane; g < n_groups; g += 32)
+        if (start + g < limit) P.indices[start + g] = static_cast<int32_t>(g);
+  } else if (use_bitmap) {
+    // bitmap over the complete groups: marking a bit removes repeats,
+    // reading the words in order gives the ascending list
+    uint32_t* bm = reinterpret_cast<uint32_t*>(buf);
+    for (int w = lane; w < words; w += 32) bm[w] = 0u;
+    __syncwarp();
+    const int32_t* row = P.topk + i * P.topk_width;
+    for (int j = lane; j < P.topk_width; j += 32) {
+      const int32_t g = row[j];
+      if (g >= 0 && g < n_complete) atomicOr(bm + (g >> 5), 1u << (g & 31));
     }
-    if (p >= 0 && P.ratio > 0) {
-      if (!sorted_list) {
-        n_groups = n_complete;
-      } else if (((n_complete + 31) >> 5) <= P.buf_words) {
-        // bitmap over the complete groups: marking a bit removes repeats,
-        // reading the words in order gives the ascending list
-        uint32_t* bm = reinterpret_cast<uint32_t*>(buf);
-        const int words = (n_complete + 31) >> 5;
-        for (int w = lane; w < words; w += 32) bm[w] = 0u;
-        __syncwarp();
-        const int32_t* row = P.topk + i * P.topk_width;
-        for (int j = lane; j < P.topk_width; j += 32) {
-          const int32_t g = row[j];
-          if (g >= 0 && g < n_complete) atomicOr(bm + (g >> 5), 1u << (g & 31));
-        }
-        __syncwarp();
-        int cnt = 0;
-        for (int w = lane; w < words; w += 32) cnt += __popc(bm[w]);
-        n_groups = __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(cnt));
-      } else {
-        const int32_t* row = P.topk + i * P.topk_width;
-        for (int j = lane; j < P.sort_width; j += 32) {
-          int32_t g = j < P.topk_width ? row[j] : -1;
-          buf[j] = (g >= 0 && g < n_complete) ? g : INT_MAX;
-        }
-        __syncwarp();
-        warp_bitonic_sort(buf, P.sort_width, lane);
-        int64_t distinct = 0;
-        for (int j0 = 0; j0 < P.sort_width; j0 += 32) {
-          const int j = j0 + lane;
-          const int32_t v = buf[j];
-          const bool first = v != INT_MAX && (j == 0 || buf[j - 1] != v);
-          distinct += __popc(__ballot_sync(0xffffffffu, first));
-        }
-        n_groups = distinct;
-      }
-    }
-  }
-  const int64_t count = active && p >= 0 ? n_groups + n_window : 0;
-  if (lane == 0) s_count[warp] = count;
-  __syncthreads();
-
-  // Offset of this CTA's first key: decoupled look-back.
-  if (threadIdx.x == 0) {
-    int64_t aggregate = 0;
-    for (int w = 0; w < kSetsQueriesPerCta; ++w) aggregate += s_count[w];
-    int64_t exclusive = 0;
-    if (tile == 0) {
-      st_relaxed_u64(P.tile_status, kFlagInclusive | static_cast<uint64_t>(aggregate));
-    } else {
-      st_relaxed_u64(P.tile_status + tile, kFlagAggregate | static_cast<uint64_t>(aggregate));
-      int64_t pred = static_cast<int64_t>(tile) - 1;
-      const uint64_t t0 = global_timer_ns();
-      uint32_t spins = 0;
-      while (pred >= 0) {
-        const uint64_t s = ld_relaxed_u64(P.tile_status + pred);
-        if ((s & ~kValueMask) == 0) {
-          if ((++spins & 63u) == 0 && global_timer_ns() - t0 > kWaitTimeoutNs) {
-            report(P.dev_status, SPA_DEV_TIMEOUT);
-            break;
-          }
-          continue;
-        }
-        exclusive += static_cast<int64_t>(s & kValueMask);
-        if ((s & ~kValueMask) == kFlagInclusive) break;
-        --pred;
-      }
-      st_relaxed_u64(P.tile_status + tile,
-                     kFlagInclusive | static_cast<uint64_t>(exclusive + aggregate));
-    }
-    s_tile_offset = exclusive;
-  }
-  __syncthreads();
-  if (!active) return;
-
-  int64_t start = s_tile_offset;
-  for (int w = 0; w < warp; ++w) start += s_count[w];
-  const int64_t end = start + count;
-  if (lane == 0) {
-    if (end > P.capacity || end > INT_MAX) report(P.dev_status, SPA_DEV_CAPACITY);
-    P.indptr[i] = static_cast<int32_t>(start < INT_MAX ? start : INT_MAX);
-    if (i == P.n - 1) P.indptr[P.n] = static_cast<int32_t>(end < INT_MAX ? end : INT_MAX);
-  }
-  if (count == 0) return;
-  const int64_t limit = P.capacity < INT_MAX ? P.capacity : INT_MAX;
-
-  // compressed groups, ascending
-  if (sorted_list && ((n_complete + 31) >> 5) <= P.buf_words) {
-    const uint32_t* bm = reinterpret_cast<const uint32_t*>(buf);
-    const int words = (n_complete + 31) >> 5;
+    __syncwarp();
     int64_t written = 0;
     for (int w0 = 0; w0 < words; w0 += 32) {
       const int w = w0 + lane;
@@ -206,38 +131,142 @@ build_kv_sets_kernel(const SetsParams P) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
-      int64_t dst = start + written + (incl - cnt);
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        if (dst < limit) P.indices[dst] = w * 32 + bit;
-        ++dst;
-        bits &= bits - 1u;
+      if (write) {
+        int64_t dst = start + written + (incl - cnt);
+        while (bits) {
+          const int bit = __ffs(bits) - 1;
+          if (dst < limit) P.indices[dst] = w * 32 + bit;
+          ++dst;
+          bits &= bits - 1u;
+        }
       }
       written += __shfl_sync(0xffffffffu, incl, 31);
     }
-  } else if (sorted_list) {
+    n_groups = written;
+    __syncwarp();   // the bitmap is rebuilt by the next query
+  } else if (listed) {
+    const int32_t* row = P.topk + i * P.topk_width;
+    for (int j = lane; j < P.sort_width; j += 32) {
+      const int32_t g = j < P.topk_width ? row[j] : -1;
+      buf[j] = (g >= 0 && g < n_complete) ? g : INT_MAX;
+    }
+    __syncwarp();
+    warp_bitonic_sort(buf, P.sort_width, lane);
     int64_t written = 0;
     for (int j0 = 0; j0 < P.sort_width; j0 += 32) {
-      if (buf[j0] == INT_MAX) break;  // sentinels sort last
+      if (buf[j0] == INT_MAX) break;   // sentinels sort last
       const int j = j0 + lane;
       const int32_t v = buf[j];
       const bool first = v != INT_MAX && (j == 0 || buf[j - 1] != v);
       const uint32_t m = __ballot_sync(0xffffffffu, first);
-      const int64_t dst = start + written + __popc(m & ((1u << lane) - 1u));
-      if (first && dst < limit) P.indices[dst] = v;
+      if (write) {
+        const int64_t dst = start + written + __popc(m & ((1u << lane) - 1u));
+        if (first && dst < limit) P.indices[dst] = v;
+      }
       written += __popc(m);
     }
-  } else {
-    for (int64_t g = lane; g < n_groups; g += 32) {
-      const int64_t dst = start + g;
-      if (dst < limit) P.indices[dst] = static_cast<int32_t>(g);
+    n_groups = written;
+    __syncwarp();
+  }
+  if (write) {
+    const int32_t t0 = p - n_window + 1;
+    for (int t = lane; t < n_window; t += 32) {
+      const int64_t dst = start + n_groups + t;
+      if (dst < limit) P.indices[dst] = SPA_WINDOW_TAG | (t0 + t);
     }
   }
-  // window tokens, ascending
-  const int32_t t0 = p - n_window + 1;
-  for (int t = lane; t < n_window; t += 32) {
-    const int64_t dst = start + n_groups + t;
-    if (dst < limit) P.indices[dst] = SPA_WINDOW_TAG | (t0 + t);
+  return n_groups + n_window;
+}
+
+// Persistent layout: CTA k (in the order of an atomic ticket, so that every
+// CTA before it is already running) owns queries [k * per_cta, ...). It
+// counts every owned set, scans the counts, publishes its total and finds
+// its offset by a decoupled look-back whose warp reads 32 predecessors per
+// step, then recomputes each set and writes it with its indptr entry.
+__global__ void __launch_bounds__(kSetsWarps * 32) build_kv_sets_kernel(const SetsParams P) {
+  extern __shared__ int32_t sets_smem[];   // [kSetsWarps][buf_words] | int64 prefix[per_cta]
+  __shared__ int64_t s_base;
+  __shared__ uint32_t s_tile;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  int32_t* buf = sets_smem + warp * P.buf_words;
+  int64_t* prefix = reinterpret_cast<int64_t*>(sets_smem + kSetsWarps * P.buf_words);
+  if (threadIdx.x == 0) s_tile = atomicAdd(P.tile_ticket, 1u);
+  __syncthreads();
+  const uint32_t tile = s_tile;
+  const int64_t q0 = static_cast<int64_t>(tile) * P.per_cta;
+  const int nq = static_cast<int>(min(static_cast<int64_t>(P.per_cta), static_cast<int64_t>(P.n) - q0));
+
+  for (int q = warp; q < nq; q += kSetsWarps) {
+    const int64_t c = one_query(P, q0 + q, buf, lane, false, 0, 0);
+    if (lane == 0) prefix[q] = c;
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // exclusive scan of the counts: a block of them per lane, then the lanes
+    const int per = (nq + 31) / 32;
+    const int lo = min(lane * per, nq), hi = min(lo + per, nq);
+    int64_t own = 0;
+    for (int q = lo; q < hi; ++q) own += prefix[q];
+    int64_t incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int64_t run = incl - own;
+    for (int q = lo; q < hi; ++q) {
+      const int64_t v = prefix[q];
+      prefix[q] = run;
+      run += v;
+    }
+    const int64_t total = __shfl_sync(0xffffffffu, incl, 31);
+
+    // offset of this CTA: decoupled look-back, 32 predecessors per step
+    int64_t excl = 0;
+    if (tile == 0) {
+      if (lane == 0) st_relaxed_u64(P.tile_status, kFlagInclusive | static_cast<uint64_t>(total));
+    } else {
+      if (lane == 0) st_relaxed_u64(P.tile_status + tile, kFlagAggregate | static_cast<uint64_t>(total));
+      int64_t top = static_cast<int64_t>(tile) - 1;
+      const uint64_t t0 = global_timer_ns();
+      uint32_t spins = 0;
+      while (true) {
+        const int64_t idx = top - lane;
+        const uint64_t s = idx >= 0 ? ld_relaxed_u64(P.tile_status + idx) : kFlagInclusive;
+        if (__any_sync(0xffffffffu, (s & ~kValueMask) == 0)) {   // a predecessor has not published yet
+          if ((++spins & 63u) == 0 && global_timer_ns() - t0 > kWaitTimeoutNs) {
+            if (lane == 0) report(P.dev_status, SPA_DEV_TIMEOUT);
+            break;
+          }
+          continue;
+        }
+        const uint32_t inc = __ballot_sync(0xffffffffu, (s & ~kValueMask) == kFlagInclusive);
+        const int last = inc ? __ffs(inc) - 1 : 31;   // nearest inclusive predecessor
+        excl += warp_sum64(lane <= last ? static_cast<int64_t>(s & kValueMask) : 0);
+        if (inc) break;
+        top -= 32;
+      }
+      if (lane == 0)
+        st_relaxed_u64(P.tile_status + tile, kFlagInclusive | static_cast<uint64_t>(excl + total));
+    }
+    if (lane == 0) s_base = excl;
+  }
+  __syncthreads();
+
+  const int64_t base = s_base;
+  const int64_t limit = P.capacity < INT_MAX ? P.capacity : INT_MAX;
+  for (int q = warp; q < nq; q += kSetsWarps) {
+    const int64_t i = q0 + q;
+    const int64_t start = base + prefix[q];
+    const int64_t c = one_query(P, i, buf, lane, true, start, limit);
+    if (lane == 0) {
+      const int64_t end = start + c;
+      if (end > P.capacity || end > INT_MAX) report(P.dev_status, SPA_DEV_CAPACITY);
+      P.indptr[i] = static_cast<int32_t>(start < INT_MAX ? start : INT_MAX);
+      if (i == P.n - 1) P.indptr[P.n] = static_cast<int32_t>(end < INT_MAX ? end : INT_MAX);
+    }
   }
 }
 
@@ -247,8 +276,23 @@ int sort_width_for(int32_t topk_width) {
   return w;
 }
 
+int sm_count_for_sets() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+    else
+      n = 148;
+  }
+  return n;
+}
+
 }  // namespace
 
+// An upper bound of the scratch the launcher uses (it uses fewer status
+// words when a CTA owns more than kSetsQueriesPerCta queries).
 size_t build_kv_sets_workspace_bytes(int32_t n_queries) {
   const int64_t tiles = (static_cast<int64_t>(n_queries) + kSetsQueriesPerCta - 1) / kSetsQueriesPerCta;
   return static_cast<size_t>(tiles) * sizeof(uint64_t) + 16;
@@ -259,8 +303,13 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
                                  int32_t* indices, int64_t capacity, void* ws,
                                  uint32_t* dev_status, cudaStream_t stream) {
   if (n == 0) return cudaMemsetAsync(indptr, 0, sizeof(int32_t), stream);
-  const int64_t tiles = (static_cast<int64_t>(n) + kSetsQueriesPerCta - 1) / kSetsQueriesPerCta;
-  cudaError_t err = cudaMemsetAsync(ws, 0, build_kv_sets_workspace_bytes(n), stream);
+  // about two CTAs per SM, each with a contiguous block of queries
+  const int64_t slots = 2 * static_cast<int64_t>(sm_count_for_sets());
+  int64_t per_cta = (static_cast<int64_t>(n) + slots - 1) / slots;
+  per_cta = per_cta < kSetsQueriesPerCta ? kSetsQueriesPerCta : (per_cta > kMaxPerCta ? kMaxPerCta : per_cta);
+  const int64_t tiles = (static_cast<int64_t>(n) + per_cta - 1) / per_cta;
+  const size_t ws_used = static_cast<size_t>(tiles) * sizeof(uint64_t) + 16;
+  cudaError_t err = cudaMemsetAsync(ws, 0, ws_used, stream);
   if (err != cudaSuccess) return err;
   SetsParams P;
   P.pos = pos;
@@ -272,22 +321,22 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
   P.sort_width = (P.topk != nullptr) ? sort_width_for(topk_width) : 32;
   // bitmap of at least 512 words (16384 groups) per warp; the sort handles
   // queries with more complete groups than that
-  P.buf_words = P.sort_width > 512 ? P.sort_width : 512;
+  P.buf_words = (P.topk != nullptr) ? (P.sort_width > 512 ? P.sort_width : 512) : 0;
+  P.per_cta = static_cast<int32_t>(per_cta);
   P.indptr = indptr;
   P.indices = indices;
   P.capacity = capacity;
   P.tile_status = static_cast<uint64_t*>(ws);
   P.tile_ticket = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + tiles * sizeof(uint64_t));
   P.dev_status = dev_status;
-  const size_t smem = (P.topk != nullptr)
-                          ? static_cast<size_t>(kSetsQueriesPerCta) * P.buf_words * sizeof(int32_t)
-                          : 0;
+  const size_t smem = static_cast<size_t>(kSetsWarps) * P.buf_words * sizeof(int32_t) +
+                      static_cast<size_t>(per_cta) * sizeof(int64_t);
   if (smem > 48 * 1024) {
     err = cudaFuncSetAttribute(build_kv_sets_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  build_kv_sets_kernel<<<static_cast<unsigned>(tiles), kSetsQueriesPerCta * 32, smem, stream>>>(P);
+  build_kv_sets_kernel<<<static_cast<unsigned>(tiles), kSetsWarps * 32, smem, stream>>>(P);
   return cudaGetLastError();
 }
 
