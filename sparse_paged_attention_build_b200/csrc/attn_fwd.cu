@@ -68,7 +68,11 @@ constexpr uint32_t kRawBit = 0x80000000u;
 constexpr uint32_t kInvalidRow = 0xFFFFFFFFu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;
+// A tile whose row sum of P, taken with the running max as it stands,
+// exceeds 2^16 (or is not a number) is recomputed with its exact max. P
+// therefore stays below 2^16: harmless in BF16 and in the FP32 sums, whose
+// relative precision does not depend on magnitude.
+constexpr float kSpecBound = 65536.0f;
 // consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
 constexpr uint32_t kTabConsumers = 2 * kProdLanes + 1 + kSoftThreads;
 
@@ -130,11 +134,13 @@ struct Layout {
   static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
   static constexpr int kTabOff = kVOff + kStagesV * kTileBytes;       // [2][kChunkKeys] u32
   static constexpr int kDescOff = kTabOff + 2 * kChunkKeys * 4;       // [2] ChunkDesc
-  static constexpr int kMergeOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));  // [16][128] f32
+  // [16][128] f32 merge weights; between merges, a 2 KB output staging area
+  // per softmax warp
+  static constexpr int kMergeOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
   static constexpr int kBarOff = kMergeOff + kAttnMaxSplits * 128 * 4;
   // tab_full, tab_empty, q_full + q_empty, K ring, V ring, s_full, p_ready,
-  // o_done, o_free, mma_done
-  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 1 + 1;
+  // o_done, o_free, mma_done, soft_sync
+  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 1 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kUsed = kMiscOff + 16;
   // + alignment slack; at least 80 KB so that no more than two CTAs share an
@@ -162,6 +168,10 @@ struct Bars {
   uint64_t* o_done;
   uint64_t* o_free;
   uint64_t* mma_done;
+  // [2]: barrier of the softmax threads, the two used in turn. An mbarrier
+  // rather than a named barrier so that the wait is bounded: a thread that
+  // gave up elsewhere cannot leave the others stuck.
+  uint64_t* soft_sync;
 };
 
 __device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) / kT; }
@@ -238,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   B.o_done = B.p_ready + 2;
   B.o_free = B.o_done + 2;
   B.mma_done = B.o_free + 1;
+  B.soft_sync = B.mma_done + 1;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + L::kDescOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
@@ -273,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     mbar_init(B.o_done + 1, 1);
     mbar_init(B.o_free, kSoftThreads);
     mbar_init(B.mma_done, 1);
+    mbar_init(B.soft_sync, kSoftThreads);
+    mbar_init(B.soft_sync + 1, kSoftThreads);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -447,6 +460,9 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         mbar_arrive(B.tab_empty + slot);
         ++c;
         final_seen = (d.flags & kFlagFinal) != 0;
+        // the previous unit's last PV goes first: its epilogue must not wait
+        // for this unit's Q and first K tile
+        if ((d.flags & kFlagFirst) && pv_pending && !issue_pv()) { ok = false; break; }
         const int ntiles = ceil_tiles(d.nkeys);
         if (ntiles == 0) continue;
         if (d.flags & kFlagFirst) {
@@ -456,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         for (int t = 0; t < ntiles; ++t, ++g) {
           const int stage = g % kStagesK, sb = g & 1;
           if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status)) { ok = false; break; }
-            tc_fence_after_sync();
+          tc_fence_after_sync();
           const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
@@ -487,6 +503,39 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     const bool row_ok = row < heads_here;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sink2 = (P.sink != nullptr && row_ok) ? P.sink[h] * kLog2e : -INFINITY;
+    uint32_t nsync = 0;
+    // barrier of the softmax threads (bounded: false once a wait gave up)
+    auto gsync = [&]() -> bool {
+      uint64_t* bar = B.soft_sync + (nsync & 1);
+      const uint32_t parity = (nsync >> 1) & 1;
+      ++nsync;
+      mbar_arrive(bar);
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, P.dev_status));
+    };
+    // Output rows leave through a per-warp staging area so that the global
+    // stores are coalesced: each thread holds one head row, but a warp-wide
+    // store of one 16-byte piece per row would touch 32 rows at once. A
+    // pass stages 64 bytes of each of the warp's 32 rows (16-byte pieces
+    // XOR-swizzled by row pair, conflict-free both ways), then every
+    // instruction writes 8 rows x 64 contiguous bytes.
+    uint8_t* stage = smem + L::kMergeOff + warp * 2048;
+    const int st_swz = (lane >> 1) & 3;
+    auto stage_put = [&](uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4, uint32_t a5, uint32_t a6,
+                         uint32_t a7, uint32_t a8, uint32_t a9, uint32_t a10, uint32_t a11, uint32_t a12,
+                         uint32_t a13, uint32_t a14, uint32_t a15) {
+      uint4* r = reinterpret_cast<uint4*>(stage + lane * 64);
+      r[0 ^ st_swz] = make_uint4(a0, a1, a2, a3);
+      r[1 ^ st_swz] = make_uint4(a4, a5, a6, a7);
+      r[2 ^ st_swz] = make_uint4(a8, a9, a10, a11);
+      r[3 ^ st_swz] = make_uint4(a12, a13, a14, a15);
+      __syncwarp();
+    };
+    // piece k of the coalesced write-out: row 8k + lane/4, 16-byte piece lane%4
+    auto stage_get = [&](int k, int& r, int& piece) -> uint4 {
+      r = 8 * k + (lane >> 2);
+      piece = lane & 3;
+      return reinterpret_cast<const uint4*>(stage + r * 64)[piece ^ ((r >> 1) & 3)];
+    };
     int c = 0, g = 0;
     bool ok = true, final_seen = false;
     float m = -INFINITY, l = 0.f;
@@ -503,7 +552,10 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       final_seen = (d.flags & kFlagFinal) != 0;
       if (d.flags & kFlagFirst) {
         unit_tiles = 0;
-        m = (d.split == 0 && sink2 > -INFINITY) ? sink2 : -INFINITY;
+        // the sink logit seeds the max of every slice (any reference point
+        // is exact; this one is usually within the bound of the scores) but
+        // joins the denominator only once, in slice 0
+        m = sink2;
         l = (d.split == 0 && sink2 > -INFINITY) ? 1.f : 0.f;
       }
       const int ntiles = ceil_tiles(d.nkeys);
@@ -517,66 +569,89 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         tc_fence_after_sync();
         const int nv = min(kT, d.nkeys - t * kT);
         uint32_t s0[32], s1[32];
-        tmem_ld32(lane_addr + sb * kT, s0);
-        tmem_ld32(lane_addr + sb * kT + 32, s1);
-        tmem_ld_wait(s0);
-        tmem_ld_wait(s1);
-        if (nv < kT) {   // columns past the set: -inf, so they add nothing
+        // Speculative pass: P with the running max as it stands. Only when
+        // some row's tile sum leaves the bound (NaN and +inf, from a max
+        // still at -inf, included) is the exact tile max taken and P
+        // recomputed, so the max reduction stays off the common path. S is
+        // still intact in TMEM for that second pass.
+        auto load_s = [&]() {
+          tmem_ld32(lane_addr + sb * kT, s0);
+          tmem_ld32(lane_addr + sb * kT + 32, s1);
+          tmem_ld_wait(s0);
+          tmem_ld_wait(s1);
+          if (nv < kT) {   // columns past the set: -inf, so they add nothing
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) {
-            if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
-            if (cc + 32 >= nv) s1[cc] = __float_as_uint(-INFINITY);
+            for (int cc = 0; cc < 32; ++cc) {
+              if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
+              if (cc + 32 >= nv) s1[cc] = __float_as_uint(-INFINITY);
+            }
           }
-        }
-        // row max as eight independent chains and a tree (a single chain
-        // of 64 dependent max operations would dominate the tile's latency)
-        float mx8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(__uint_as_float(s0[k]), __uint_as_float(s1[k]));
-#pragma unroll
-        for (int k = 8; k < 32; ++k)
-          mx8[k & 7] = fmaxf(mx8[k & 7], fmaxf(__uint_as_float(s0[k]), __uint_as_float(s1[k])));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float tmax = mx * P.scale_log2;
-        const bool move = tmax > m + kRescaleThreshold || (m == -INFINITY && tmax > -INFINITY);
-        const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
-        l *= alpha;
-        if (move) m = tmax;
-        if (unit_tiles > 0 && __any_sync(0xffffffffu, move)) {
-          // rows whose max moved rescale their O row (alpha = 1 elsewhere);
-          // the previous PV must have landed in TMEM first
-          if (!__all_sync(0xffffffffu, mbar_wait(B.o_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag,
-                                                 P.dev_status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + L::kOCol + c0, o);
-            tmem_ld_wait(o);
-#pragma unroll
-            for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
-            tmem_st32(lane_addr + L::kOCol + c0, o);
-          }
-          tmem_st_wait();
-        }
-        const float neg_m = -m;
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        };
         uint32_t pk[32];
+        auto exp_pass = [&]() -> float {
+          const float neg_m = -m;
+          float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
-          const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
-          const float p2 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc]), P.scale_log2, neg_m));
-          const float p3 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc + 1]), P.scale_log2, neg_m));
-          sum4[cc & 3] += (p0 + p1) + (p2 + p3);
-          pk[cc] = pack_bf16x2(p0, p1);
-          pk[cc + 16] = pack_bf16x2(p2, p3);
+          for (int cc = 0; cc < 16; ++cc) {
+            const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
+            const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
+            const float p2 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc]), P.scale_log2, neg_m));
+            const float p3 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc + 1]), P.scale_log2, neg_m));
+            sum4[cc & 3] += (p0 + p1) + (p2 + p3);
+            pk[cc] = pack_bf16x2(p0, p1);
+            pk[cc + 16] = pack_bf16x2(p2, p3);
+          }
+          return (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        };
+        load_s();
+        float lsum = exp_pass();
+        const bool flag = row_ok && !(lsum <= kSpecBound);
+        if (__any_sync(0xffffffffu, flag)) {
+          load_s();
+          // row max: eight independent chains of 3-input max and a tree
+          float mx8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(__uint_as_float(s0[k]), __uint_as_float(s1[k]), __uint_as_float(s0[k + 8]));
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(mx8[k], __uint_as_float(s1[k + 8]), __uint_as_float(s0[k + 16]));
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(mx8[k], __uint_as_float(s1[k + 16]), __uint_as_float(s0[k + 24]));
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s1[k + 24]));
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float tmax = mx * P.scale_log2;
+          // a flagged row's tile max lies above its running max
+          const bool move = flag && (tmax > m || m == -INFINITY);
+          const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
+          l *= alpha;
+          if (move) m = tmax;
+          if (unit_tiles > 0 && __any_sync(0xffffffffu, move)) {
+            // rows whose max moved rescale their O row (alpha = 1
+            // elsewhere); the previous PV must have landed in TMEM first
+            if (!__all_sync(0xffffffffu, mbar_wait(B.o_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag,
+                                                   P.dev_status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + L::kOCol + c0, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
+              tmem_st32(lane_addr + L::kOCol + c0, o);
+            }
+            tmem_st_wait();
+          }
+          lsum = exp_pass();
         }
-        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        l += lsum;
         tmem_st32(lane_addr + sb * kT, pk);   // P overwrites the first 32 columns of S
         tmem_st_wait();
         tc_fence_before_sync();
@@ -597,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const int i = d.i;
       if (S == 1) {
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        uint16_t* orow = P.out + (static_cast<int64_t>(i) * P.num_heads + h) * D;
+        uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -612,11 +687,16 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc)
             pk[cc] = pack_bf16x2(__uint_as_float(o[2 * cc]) * inv_l, __uint_as_float(o[2 * cc + 1]) * inv_l);
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+          stage_put(pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7], pk[8], pk[9], pk[10], pk[11], pk[12],
+                    pk[13], pk[14], pk[15]);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int k = 0; k < 4; ++k) {
+            int r, piece;
+            const uint4 v = stage_get(k, r, piece);
+            if (warp * 32 + r < heads_here)
+              *reinterpret_cast<uint4*>(obase + static_cast<int64_t>(warp * 32 + r) * D + c0 + piece * 8) = v;
           }
+          __syncwarp();   // the stage is rewritten by the next pass
         }
         if (have_o) {
           tc_fence_before_sync();
@@ -628,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         // partial result of this slice (no normalisation); the last slice
         // of the query to finish merges all of them
         const int64_t unit = static_cast<int64_t>(i) * S + d.split;
-        float* prow = P.part_o + (unit * P.num_heads + h) * D;
+        float* pbase = P.part_o + (unit * P.num_heads + head0) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -639,12 +719,19 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
 #pragma unroll
             for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
           }
-          if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(prow + c0);
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                   __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          for (int hf = 0; hf < 2; ++hf) {   // 16 fp32 columns (64 bytes) per pass
+            stage_put(o[16 * hf], o[16 * hf + 1], o[16 * hf + 2], o[16 * hf + 3], o[16 * hf + 4], o[16 * hf + 5],
+                      o[16 * hf + 6], o[16 * hf + 7], o[16 * hf + 8], o[16 * hf + 9], o[16 * hf + 10],
+                      o[16 * hf + 11], o[16 * hf + 12], o[16 * hf + 13], o[16 * hf + 14], o[16 * hf + 15]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              int r, piece;
+              const uint4 v = stage_get(k, r, piece);
+              if (warp * 32 + r < heads_here)
+                *reinterpret_cast<uint4*>(pbase + static_cast<int64_t>(warp * 32 + r) * D + c0 + 16 * hf + piece * 4) = v;
+            }
+            __syncwarp();
           }
         }
         if (have_o) {
@@ -653,11 +740,20 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         }
         if (row_ok) P.part_ml[unit * P.num_heads + h] = make_float2(m, l);
         __threadfence();
-        named_bar_sync(2, kSoftThreads);
+        if (!gsync()) {
+          ok = false;
+          break;
+        }
         if (tid == 0) *ticket_slot = atomicAdd(P.tickets + static_cast<int64_t>(i) * gridDim.y + blockIdx.y, 1u);
-        named_bar_sync(2, kSoftThreads);
+        if (!gsync()) {
+          ok = false;
+          break;
+        }
         const bool merge = *ticket_slot == static_cast<uint32_t>(S - 1);
-        named_bar_sync(2, kSoftThreads);   // ticket_slot is reused by the next unit
+        if (!gsync()) {   // ticket_slot is reused by the next unit
+          ok = false;
+          break;
+        }
         if (merge) {
           // exact merge of the S slices: LSE = M + log2(L), O = sum_s w_s O_s
           // with w_s = 2^(m_s - M) / L. Thread h first turns its head's
@@ -684,7 +780,10 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
             P.lse[static_cast<int64_t>(i) * P.num_heads + h] =
                 Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
           }
-          named_bar_sync(2, kSoftThreads);
+          if (!gsync()) {
+            ok = false;
+            break;
+          }
           constexpr int kF4 = D / 4;                   // float4 per row
           constexpr int kRowsPerPass = kSoftThreads / kF4;
           constexpr int kBatch = 4;                    // row passes whose loads are in flight together
@@ -717,7 +816,10 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
                   make_uint2(pack_bf16x2(acc[q].x, acc[q].y), pack_bf16x2(acc[q].z, acc[q].w));
             }
           }
-          named_bar_sync(2, kSoftThreads);   // wl is reused by the next merge
+          if (!gsync()) {   // wl and the staging areas are reused next
+            ok = false;
+            break;
+          }
         }
       }
     }
