@@ -12,35 +12,44 @@
 // Work unit = (query token i, slice s of its key set, 128-head tile). All
 // heads of the unit share every K/V row, so the unit is a dense MQA problem
 // with M = 128 heads:
-//   S  = Q[128 x d] . K_tile[64 x d]^T       tcgen05.mma, SMEM x SMEM -> TMEM
-//   P  = exp2(S*scale*log2e - m)  (BF16)     softmax warps, TMEM -> regs -> TMEM
-//   O += P[128 x 64] . V_tile[64 x d]         tcgen05.mma, TMEM x SMEM -> TMEM
-// The sink seeds the running max and the denominator (m = sink*log2e,
-// l = 1), so it is counted exactly once and never multiplies a V row.
+//   S  = Q[128 x d] . K_tile[64 x d]^T      tcgen05.mma, Q in TMEM, K in SMEM
+//   P  = exp2(S*scale*log2e - m)  (BF16)    softmax warps, TMEM -> regs -> TMEM
+//   O += P[128 x 64] . V_tile[64 x d]        tcgen05.mma, P in TMEM, V in SMEM
+// Both products take their A operand from TMEM: measured on B200, an
+// M = 128, N = 64 product with both operands in shared memory is bound by
+// shared-memory bandwidth at two thirds of the tensor rate, while with A in
+// TMEM it runs at the full rate. The sink seeds the running max and the
+// denominator (m = sink*log2e, l = 1), so it is counted exactly once and
+// never multiplies a V row.
 //
-// Persistent CTAs (two per SM) walk their units in a fixed stride. Warp
-// roles (384 threads):
-//   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t
+// Persistent CTAs (two per SM) walk their units in a fixed stride; the two
+// CTAs of an SM interleave on the tensor core and on the exp unit. Warp
+// roles (256 threads):
+//   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t.
+//              They also move each unit's Q from shared memory into TMEM.
 //   warp  4    TMEM allocation; lane 0 issues every UMMA and commit
-//   warp  5    resolver: for a chunk of up to 512 keys of a unit it loads
+//   warp  5    resolver: for a chunk of up to 768 keys of a unit it loads
 //              the keys, looks their pages up and writes the physical row
 //              of every key (bit 31 = raw pool) to a double-buffered table,
 //              plus a chunk descriptor that every other role follows. All
 //              dependent global loads of the gather happen here, ahead of
 //              the copies.
-//   warps 6-8  K gather: 96 lanes copy the tile's rows in 16-byte cp.async
-//              pieces into a 2-stage ring, 128-byte swizzled in the K-major
-//              layout of the UMMA descriptors (random rows need many copies
-//              in flight: measured on B200, 16-byte copies from eight warps
-//              per CTA reach 14.7 TB/s of L2 gather, TMA gather4 from one or
-//              two warps 4-6 TB/s); lane 0 of warp 6 also loads Q (TMA box)
-//   warps 9-11 V gather, into its own 2-stage ring
-// TMEM columns: S/P buffer 0 [0,64), buffer 1 [64,128), O [128,128+d).
-// The running max only moves when a tile's max exceeds it by more than 8
-// (log2 units), so P <= 256 and O is rescaled rarely; O/l and LSE use the
-// same max, so the result is exact in exact arithmetic.
+//   warp  6    K gather (and Q): TMA tile::gather4 loads, four rows of one
+//              pool per instruction, into a 2-stage ring, 128-byte swizzled
+//              by the tensor map into the K-major layout of the UMMA
+//              descriptors; rows outside a pool (padding, faulty keys) are
+//              zero-filled by the TMA. Q arrives as TMA boxes.
+//   warp  7    V gather, into its own 2-stage ring
+// TMEM columns: S/P [0,64), Q [64, 64 + d/2) as packed BF16 pairs, O after.
+// S is single-buffered: QK^T of tile g+1 is issued after PV of tile g, and
+// the UMMAs of a CTA run in issue order, so P(g) is read before S(g+1)
+// overwrites it; the other CTA on the SM fills the tensor core meanwhile.
+// The softmax first takes P with the running max as it stands and only
+// recomputes a tile whose row sum leaves a fixed bound (see kSpecBound);
+// O/l and LSE use the same max, so the result is exact in exact arithmetic.
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -57,10 +66,8 @@ constexpr int kStagesV = 2;
 constexpr int kSoftThreads = 128;
 constexpr int kMmaWarp = 4;
 constexpr int kResolverWarp = 5;
-constexpr int kKWarp0 = 6;                       // K producer: warp 6
-constexpr int kVWarp0 = 7;                       // V producer: warp 7
-constexpr int kProdWarps = 1;
-constexpr int kProdLanes = kProdWarps * 32;
+constexpr int kKWarp0 = 6;                       // K (and Q) producer
+constexpr int kVWarp0 = 7;                       // V producer
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kChunkKeys = 768;                  // keys resolved per chunk (12 tiles)
@@ -74,7 +81,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 // relative precision does not depend on magnitude.
 constexpr float kSpecBound = 65536.0f;
 // consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
-constexpr uint32_t kTabConsumers = 2 * kProdLanes + 1 + kSoftThreads;
+constexpr uint32_t kTabConsumers = 32 + 32 + 1 + kSoftThreads;
 
 constexpr int kFlagFirst = 1;   // first chunk of its unit
 constexpr int kFlagLast = 2;    // last chunk of its unit
@@ -97,16 +104,10 @@ struct Params {
   CUtensorMap tm_k_cmp;
   CUtensorMap tm_v_cmp;
   int32_t q_box_rows;     // min(128, num_heads)
-  const uint16_t* q;
-  int64_t q_stride_tok, q_stride_head;
   int32_t n_queries, num_heads;
-  const char* k_raw;
-  const char* v_raw;
   int64_t raw_pages;
   int32_t raw_ps_log2, pt_raw_cols;
   const int32_t* pt_raw;
-  const char* k_cmp;
-  const char* v_cmp;
   int64_t cmp_pages;
   int32_t cmp_ps_log2, pt_cmp_cols;
   const int32_t* pt_cmp;
@@ -129,7 +130,7 @@ template <int D>
 struct Layout {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kTileBytes = kT * D * 2;             // one K or V tile
-  static constexpr int kQOff = 0;
+  static constexpr int kQOff = 0;                           // TMA landing area of Q
   static constexpr int kKOff = kQBytes;
   static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
   static constexpr int kTabOff = kVOff + kStagesV * kTileBytes;       // [2][kChunkKeys] u32
@@ -138,35 +139,35 @@ struct Layout {
   // per softmax warp
   static constexpr int kMergeOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
   static constexpr int kBarOff = kMergeOff + kAttnMaxSplits * 128 * 4;
-  // tab_full, tab_empty, q_full + q_empty, K ring, V ring, s_full, p_ready,
-  // o_done, o_free, mma_done, soft_sync
-  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 1 + 1 + 2;
+  // tab_full[2], tab_empty[2], q_full, q_empty, q_ready, K ring, V ring,
+  // s_full, p_ready, o_done, mma_done, soft_sync[2]
+  static constexpr int kNumBars = 2 + 2 + 3 + 2 * kStagesK + 2 * kStagesV + 1 + 1 + 1 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kUsed = kMiscOff + 16;
   // + alignment slack; at least 80 KB so that no more than two CTAs share an
   // SM (TMEM holds two 256-column allocations)
   static constexpr int kBytes = (kUsed + 1024) < 80 * 1024 ? 80 * 1024 : (kUsed + 1024);
-  static constexpr uint32_t kOCol = 2 * kT;
+  static constexpr uint32_t kSCol = 0;
+  static constexpr uint32_t kQCol = kT;
+  static constexpr uint32_t kOCol = kT + D / 2;
   static_assert(kOCol + D <= kTmemCols, "TMEM budget");
   static_assert((kBytes + 1024) * 2 <= 228 * 1024, "two CTAs per SM");
+  static_assert(kMergeOff % 16 == 0, "staging alignment");
 };
 
 struct Bars {
   uint64_t* tab_full;   // [2]
   uint64_t* tab_empty;  // [2]
-  uint64_t* q_full;
-  uint64_t* q_empty;
+  uint64_t* q_full;     // Q of the next unit landed in shared memory
+  uint64_t* q_empty;    // ... and has been moved on to TMEM
+  uint64_t* q_ready;    // Q of the next unit is in TMEM
   uint64_t* k_full;     // [kStagesK]
   uint64_t* k_empty;
   uint64_t* v_full;     // [kStagesV]
   uint64_t* v_empty;
-  uint64_t* s_full;     // [2]
-  uint64_t* p_ready;    // [2]
-  // [2]: PV of tile g commits to o_done[g & 1]. One barrier per parity keeps
-  // a waiter two phases away from aliasing: when the softmax waits for PV(g)
-  // it has seen S(g) complete, so PV(g - 2) (issued before S(g)) is done.
-  uint64_t* o_done;
-  uint64_t* o_free;
+  uint64_t* s_full;     // S of the current tile (also: every earlier UMMA done)
+  uint64_t* p_ready;    // P of the current tile in TMEM
+  uint64_t* o_done;     // last PV of a unit complete
   uint64_t* mma_done;
   // [2]: barrier of the softmax threads, the two used in turn. An mbarrier
   // rather than a named barrier so that the wait is bounded: a thread that
@@ -207,7 +208,6 @@ __device__ void resolve_chunk(const Params& P, int32_t b, int32_t key_base, int3
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int k = lane + 32 * e;
-    if (k >= kChunkKeys) continue;
     const int32_t kk = key[e];
     uint32_t row = kInvalidRow;
     if (kk >= 0) {
@@ -239,15 +239,15 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   B.tab_empty = bar0 + 2;
   B.q_full = bar0 + 4;
   B.q_empty = bar0 + 5;
-  B.k_full = bar0 + 6;
+  B.q_ready = bar0 + 6;
+  B.k_full = bar0 + 7;
   B.k_empty = B.k_full + kStagesK;
   B.v_full = B.k_empty + kStagesK;
   B.v_empty = B.v_full + kStagesV;
   B.s_full = B.v_empty + kStagesV;
-  B.p_ready = B.s_full + 2;
-  B.o_done = B.p_ready + 2;
-  B.o_free = B.o_done + 2;
-  B.mma_done = B.o_free + 1;
+  B.p_ready = B.s_full + 1;
+  B.o_done = B.p_ready + 1;
+  B.mma_done = B.o_done + 1;
   B.soft_sync = B.mma_done + 1;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + L::kDescOff);
@@ -267,25 +267,23 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     for (int s = 0; s < 2; ++s) {
       mbar_init(B.tab_full + s, 32);
       mbar_init(B.tab_empty + s, kTabConsumers);
-      mbar_init(B.s_full + s, 1);
-      mbar_init(B.p_ready + s, kSoftThreads);
+      mbar_init(B.soft_sync + s, kSoftThreads);
     }
     mbar_init(B.q_full, 1);
-    mbar_init(B.q_empty, 1);
+    mbar_init(B.q_empty, kSoftThreads);
+    mbar_init(B.q_ready, kSoftThreads);
     for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(B.k_full + s, kProdWarps);   // one expect_tx arrival per producer warp
+      mbar_init(B.k_full + s, 1);
       mbar_init(B.k_empty + s, 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(B.v_full + s, kProdWarps);
+      mbar_init(B.v_full + s, 1);
       mbar_init(B.v_empty + s, 1);
     }
+    mbar_init(B.s_full, 1);
+    mbar_init(B.p_ready, kSoftThreads);
     mbar_init(B.o_done, 1);
-    mbar_init(B.o_done + 1, 1);
-    mbar_init(B.o_free, kSoftThreads);
     mbar_init(B.mma_done, 1);
-    mbar_init(B.soft_sync, kSoftThreads);
-    mbar_init(B.soft_sync + 1, kSoftThreads);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -340,20 +338,17 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         k0 += n;
       } while (k0 < key_hi);
     }
-  } else if (warp >= kKWarp0) {
+  } else if (warp == kKWarp0 || warp == kVWarp0) {
     // ================================================= K / V gather (TMA)
-    // Two warps stream K tiles and two stream V tiles. Each tile is 16
-    // four-row groups x D/64 column halves = "jobs"; a warp's lanes issue one
-    // TMA tile::gather4 per job of its share (four rows of one pool, 512
-    // bytes, 128-byte swizzled by the tensor map into the K-major layout of
-    // the UMMA descriptors). Measured on B200, gather4 throughput scales with
-    // the number of issuing warps, hence two per operand. A group whose four
-    // keys come from both pools (at most one per unit: compressed groups
-    // precede window tokens) is loaded row by row. Rows past the chunk's keys
-    // and rows of faulty keys are outside the tensor and zero-filled. Lane 0
-    // of the first K warp also loads Q, as TMA boxes.
-    const bool is_k = warp < kVWarp0;
-    const int wsub = warp - (is_k ? kKWarp0 : kVWarp0);   // 0 or 1
+    // A tile is 16 four-row groups x D/64 column halves = "jobs"; lane j
+    // issues one TMA tile::gather4 for job j (four rows of one pool, 512
+    // bytes). A group whose four keys come from both pools (at most one per
+    // unit: compressed groups precede window tokens) is loaded row by row.
+    // Rows past the chunk's keys and rows of faulty keys are outside the
+    // tensor and zero-filled. Lane 0 of the K warp also loads each unit's Q
+    // (every unit, empty ones included, so that the Q phases of all roles
+    // stay in step).
+    const bool is_k = warp == kKWarp0;
     const int nst = is_k ? kStagesK : kStagesV;
     uint64_t* full = is_k ? B.k_full : B.v_full;
     uint64_t* empty = is_k ? B.k_empty : B.v_empty;
@@ -362,11 +357,9 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     const uint32_t ring = sbase + (is_k ? L::kKOff : L::kVOff);
     constexpr int kHalves = D / 64;
     constexpr int kGroups = kT / 4;
-    constexpr int kJobsPerWarp = kGroups * kHalves / kProdWarps;
-    const int job = wsub * kJobsPerWarp + lane;
-    const int grp = job % kGroups, half = job / kGroups;
-    const bool issuer = lane < kJobsPerWarp;
-    const bool q_loader = warp == kKWarp0;
+    constexpr int kJobs = kGroups * kHalves;
+    const int grp = lane % kGroups, half = lane / kGroups;
+    const bool issuer = lane < kJobs;
     int c = 0, g = 0, qc = 0;
     bool final_seen = false;
     while (!final_seen) {
@@ -377,8 +370,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const uint32_t* t_rows = tab + slot * kChunkKeys;
       const int ntiles = ceil_tiles(d.nkeys);
       bool ok = true;
-      if (q_loader && (d.flags & kFlagFirst) && ntiles > 0) {
-        // Q of the unit, once the previous unit's last QK^T has completed
+      if (is_k && (d.flags & kFlagFirst)) {
+        // the landing area is free once the previous Q has moved to TMEM
         ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status);
         if (ok && lane == 0) {
           mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
@@ -390,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       for (int t = 0; ok && t < ntiles; ++t, ++g) {
         const int stage = g % nst;
         if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(full + stage, kJobsPerWarp * 512);
+        if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
         __syncwarp();
         if (issuer) {
           const int nv = min(kT, d.nkeys - t * kT);
@@ -427,32 +420,15 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     }
   } else if (warp == kMmaWarp) {
     // ================================================= UMMA issuer
+    // Per tile: S = Q K^T (A = Q from TMEM), then, once P is in TMEM,
+    // O += P V (A = P from TMEM). s_full is committed after the QK^T of a
+    // tile, so its arrival also means every earlier UMMA (the previous PV)
+    // has completed.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kT, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
-      const uint32_t q_addr = sbase + L::kQOff;
-      int c = 0, g = 0, qc = 0;
+      int c = 0, g = 0, u = 0;
       bool ok = true, final_seen = false;
-      bool pv_pending = false, pv_first = false;
-      int pv_g = 0, pv_unit = 0;
-      auto issue_pv = [&]() -> bool {
-        const int sb = pv_g & 1, st = pv_g % kStagesV;
-        if (!mbar_wait(B.p_ready + sb, (pv_g >> 1) & 1, abort_flag, P.dev_status)) return false;
-        if (pv_first && !mbar_wait(B.o_free, (pv_unit & 1) ^ 1, abort_flag, P.dev_status)) return false;
-        if (!mbar_wait(B.v_full + st, (pv_g / kStagesV) & 1, abort_flag, P.dev_status)) return false;
-        tc_fence_after_sync();
-        const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
-#pragma unroll
-        for (int k = 0; k < kT / 16; ++k) {
-          const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
-          umma_ts(tmem + L::kOCol, tmem + sb * kT + k * 8, bdesc, idesc_o,
-                  (!pv_first || k > 0) ? 1u : 0u);
-        }
-        tc_commit(B.v_empty + st);
-        tc_commit(B.o_done + (pv_g & 1));
-        pv_pending = false;
-        return true;
-      };
       while (ok && !final_seen) {
         const int slot = c & 1;
         if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status)) { ok = false; break; }
@@ -460,38 +436,38 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         mbar_arrive(B.tab_empty + slot);
         ++c;
         final_seen = (d.flags & kFlagFinal) != 0;
-        // the previous unit's last PV goes first: its epilogue must not wait
-        // for this unit's Q and first K tile
-        if ((d.flags & kFlagFirst) && pv_pending && !issue_pv()) { ok = false; break; }
-        const int ntiles = ceil_tiles(d.nkeys);
-        if (ntiles == 0) continue;
-        if (d.flags & kFlagFirst) {
-          if (!mbar_wait(B.q_full, qc & 1, abort_flag, P.dev_status)) { ok = false; break; }
-          ++qc;
+        if (d.flags & kFlagFirst) {   // this unit's Q is in TMEM
+          if (!mbar_wait(B.q_ready, u & 1, abort_flag, P.dev_status)) { ok = false; break; }
+          ++u;
+          tc_fence_after_sync();
         }
+        const int ntiles = ceil_tiles(d.nkeys);
         for (int t = 0; t < ntiles; ++t, ++g) {
-          const int stage = g % kStagesK, sb = g & 1;
+          const int stage = g % kStagesK, st = g % kStagesV;
           if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status)) { ok = false; break; }
           tc_fence_after_sync();
           const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t koff = (k & 3) * 32;   // 16 elements = 32 bytes inside the atom
-            const uint64_t adesc = smem_desc_sw128(q_addr + (k >> 2) * (128 * 128) + koff, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + koff, 16, 1024);
-            umma_ss(tmem + sb * kT, adesc, bdesc, idesc_s, k > 0 ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + (k & 3) * 32, 16, 1024);
+            umma_ts(tmem + L::kSCol, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
           }
           tc_commit(B.k_empty + stage);
-          tc_commit(B.s_full + sb);
-          if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.q_empty);
-          if (pv_pending && !issue_pv()) { ok = false; break; }
-          pv_pending = true;
-          pv_g = g;
-          pv_first = (d.flags & kFlagFirst) && t == 0;
-          pv_unit = qc - 1;
+          tc_commit(B.s_full);
+          if (!mbar_wait(B.p_ready, g & 1, abort_flag, P.dev_status)) { ok = false; break; }
+          if (!mbar_wait(B.v_full + st, (g / kStagesV) & 1, abort_flag, P.dev_status)) { ok = false; break; }
+          tc_fence_after_sync();
+          const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
+          const bool first = (d.flags & kFlagFirst) && t == 0;
+#pragma unroll
+          for (int k = 0; k < kT / 16; ++k) {
+            const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
+            umma_ts(tmem + L::kOCol, tmem + L::kSCol + k * 8, bdesc, idesc_o, (!first || k > 0) ? 1u : 0u);
+          }
+          tc_commit(B.v_empty + st);
+          if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.o_done);
         }
       }
-      if (ok && pv_pending) ok = issue_pv();
       // every UMMA has completed before TMEM is released
       tc_commit(B.mma_done);
       mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
@@ -512,6 +488,34 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       mbar_arrive(bar);
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, P.dev_status));
     };
+    // Q of the next unit: shared memory (TMA, 128-byte swizzled rows) ->
+    // registers -> this thread's TMEM lane, as the packed BF16 pairs the
+    // UMMA takes for a K-major A operand. Only called once every UMMA that
+    // reads the previous Q has completed.
+    int qc = 0;
+    auto copy_q = [&]() -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(B.q_full, qc & 1, abort_flag, P.dev_status))) return false;
+      ++qc;
+      const uint8_t* qrow = smem + L::kQOff + row * 128;
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a) {
+        uint32_t v[32];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 x = *reinterpret_cast<const uint4*>(qrow + a * (128 * 128) + ((ch ^ (row & 7)) * 16));
+          v[4 * ch] = x.x;
+          v[4 * ch + 1] = x.y;
+          v[4 * ch + 2] = x.z;
+          v[4 * ch + 3] = x.w;
+        }
+        tmem_st32(lane_addr + L::kQCol + a * 32, v);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(B.q_ready);
+      mbar_arrive(B.q_empty);
+      return true;
+    };
     // Output rows leave through a per-warp staging area so that the global
     // stores are coalesced: each thread holds one head row, but a warp-wide
     // store of one 16-byte piece per row would touch 32 rows at once. A
@@ -520,14 +524,10 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     // instruction writes 8 rows x 64 contiguous bytes.
     uint8_t* stage = smem + L::kMergeOff + warp * 2048;
     const int st_swz = (lane >> 1) & 3;
-    auto stage_put = [&](uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4, uint32_t a5, uint32_t a6,
-                         uint32_t a7, uint32_t a8, uint32_t a9, uint32_t a10, uint32_t a11, uint32_t a12,
-                         uint32_t a13, uint32_t a14, uint32_t a15) {
+    auto stage_put = [&](const uint32_t* a) {
       uint4* r = reinterpret_cast<uint4*>(stage + lane * 64);
-      r[0 ^ st_swz] = make_uint4(a0, a1, a2, a3);
-      r[1 ^ st_swz] = make_uint4(a4, a5, a6, a7);
-      r[2 ^ st_swz] = make_uint4(a8, a9, a10, a11);
-      r[3 ^ st_swz] = make_uint4(a12, a13, a14, a15);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) r[v ^ st_swz] = make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
       __syncwarp();
     };
     // piece k of the coalesced write-out: row 8k + lane/4, 16-byte piece lane%4
@@ -536,10 +536,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       piece = lane & 3;
       return reinterpret_cast<const uint4*>(stage + r * 64)[piece ^ ((r >> 1) & 3)];
     };
-    int c = 0, g = 0;
-    bool ok = true, final_seen = false;
+    int c = 0, g = 0, n_o = 0;
+    bool ok = copy_q(), final_seen = false;
     float m = -INFINITY, l = 0.f;
     int unit_tiles = 0;
+    uint32_t s0[32], s1[32];
     while (ok && !final_seen) {
       const int slot = c & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status))) {
@@ -560,23 +561,21 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       }
       const int ntiles = ceil_tiles(d.nkeys);
       for (int t = 0; t < ntiles; ++t, ++g, ++unit_tiles) {
-        const int sb = g & 1;
         // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
-        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full + sb, (g >> 1) & 1, abort_flag, P.dev_status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full, g & 1, abort_flag, P.dev_status))) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
         const int nv = min(kT, d.nkeys - t * kT);
-        uint32_t s0[32], s1[32];
         // Speculative pass: P with the running max as it stands. Only when
         // some row's tile sum leaves the bound (NaN and +inf, from a max
         // still at -inf, included) is the exact tile max taken and P
         // recomputed, so the max reduction stays off the common path. S is
         // still intact in TMEM for that second pass.
         auto load_s = [&]() {
-          tmem_ld32(lane_addr + sb * kT, s0);
-          tmem_ld32(lane_addr + sb * kT + 32, s1);
+          tmem_ld32(lane_addr + L::kSCol, s0);
+          tmem_ld32(lane_addr + L::kSCol + 32, s1);
           tmem_ld_wait(s0);
           tmem_ld_wait(s1);
           if (nv < kT) {   // columns past the set: -inf, so they add nothing
@@ -631,13 +630,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           if (move) m = tmax;
           if (unit_tiles > 0 && __any_sync(0xffffffffu, move)) {
             // rows whose max moved rescale their O row (alpha = 1
-            // elsewhere); the previous PV must have landed in TMEM first
-            if (!__all_sync(0xffffffffu, mbar_wait(B.o_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag,
-                                                   P.dev_status))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after_sync();
+            // elsewhere); the previous PV has completed (s_full)
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
               uint32_t o[32];
@@ -647,26 +640,31 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
               for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
               tmem_st32(lane_addr + L::kOCol + c0, o);
             }
-            tmem_st_wait();
           }
           lsum = exp_pass();
         }
         l += lsum;
-        tmem_st32(lane_addr + sb * kT, pk);   // P overwrites the first 32 columns of S
+        tmem_st32(lane_addr + L::kSCol, pk);   // P overwrites the first 32 columns of S
         tmem_st_wait();
         tc_fence_before_sync();
-        mbar_arrive(B.p_ready + sb);
+        mbar_arrive(B.p_ready);
       }
       if (!ok || !(d.flags & kFlagLast)) continue;
+      // The next unit's Q goes to TMEM first (every QK^T of this unit has
+      // completed: its S was seen), so its first QK^T overlaps this epilogue.
+      if (!final_seen && !copy_q()) {
+        ok = false;
+        break;
+      }
 
       // ---- epilogue of the unit
       const bool have_o = unit_tiles > 0;
       if (have_o) {
-        if (!__all_sync(0xffffffffu, mbar_wait(B.o_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag,
-                                               P.dev_status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.o_done, n_o & 1, abort_flag, P.dev_status))) {
           ok = false;
           break;
         }
+        ++n_o;
         tc_fence_after_sync();
       }
       const int i = d.i;
@@ -687,8 +685,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc)
             pk[cc] = pack_bf16x2(__uint_as_float(o[2 * cc]) * inv_l, __uint_as_float(o[2 * cc + 1]) * inv_l);
-          stage_put(pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7], pk[8], pk[9], pk[10], pk[11], pk[12],
-                    pk[13], pk[14], pk[15]);
+          stage_put(pk);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             int r, piece;
@@ -697,10 +694,6 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
               *reinterpret_cast<uint4*>(obase + static_cast<int64_t>(warp * 32 + r) * D + c0 + piece * 8) = v;
           }
           __syncwarp();   // the stage is rewritten by the next pass
-        }
-        if (have_o) {
-          tc_fence_before_sync();
-          mbar_arrive(B.o_free);   // O may be overwritten by the next unit
         }
         if (row_ok)
           P.lse[static_cast<int64_t>(i) * P.num_heads + h] = l > 0.f ? (m + log2_approx(l)) * kLn2 : -INFINITY;
@@ -721,9 +714,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {   // 16 fp32 columns (64 bytes) per pass
-            stage_put(o[16 * hf], o[16 * hf + 1], o[16 * hf + 2], o[16 * hf + 3], o[16 * hf + 4], o[16 * hf + 5],
-                      o[16 * hf + 6], o[16 * hf + 7], o[16 * hf + 8], o[16 * hf + 9], o[16 * hf + 10],
-                      o[16 * hf + 11], o[16 * hf + 12], o[16 * hf + 13], o[16 * hf + 14], o[16 * hf + 15]);
+            stage_put(o + 16 * hf);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               int r, piece;
@@ -733,10 +724,6 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
             }
             __syncwarp();
           }
-        }
-        if (have_o) {
-          tc_fence_before_sync();
-          mbar_arrive(B.o_free);
         }
         if (row_ok) P.part_ml[unit * P.num_heads + h] = make_float2(m, l);
         __threadfence();
@@ -758,8 +745,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           // exact merge of the S slices: LSE = M + log2(L), O = sum_s w_s O_s
           // with w_s = 2^(m_s - M) / L. Thread h first turns its head's
           // (m_s, l_s) into the weights (in shared memory), then the 128
-          // threads sum the partial rows column-wise: each warp covers
-          // whole 512-byte rows with float4 loads, coalesced.
+          // threads sum the partial rows column-wise with coalesced float4
+          // loads, all loads of a batch issued before its stores.
           __threadfence();
           float* wl = reinterpret_cast<float*>(smem + L::kMergeOff);   // [kAttnMaxSplits][128]
           if (row_ok) {
@@ -794,7 +781,6 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
             float4 acc[kBatch];
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            // all loads of the batch first (no store in between)
             for (int s = 0; s < S; ++s) {
 #pragma unroll
               for (int q = 0; q < kBatch; ++q) {
@@ -939,19 +925,12 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
         !encode_pool(&P.tm_v_cmp, a.v_cmp, cmp_rows, a.head_dim))
       return cudaErrorInvalidValue;
   }
-  P.q = a.q;
-  P.q_stride_tok = a.q_stride_tok;
-  P.q_stride_head = a.q_stride_head;
   P.n_queries = a.n_queries;
   P.num_heads = a.num_heads;
-  P.k_raw = reinterpret_cast<const char*>(a.k_raw);
-  P.v_raw = reinterpret_cast<const char*>(a.v_raw);
   P.raw_pages = a.raw_num_pages;
   P.raw_ps_log2 = log2_exact(a.raw_page_size);
   P.pt_raw = a.pt_raw;
   P.pt_raw_cols = a.pt_raw_cols;
-  P.k_cmp = reinterpret_cast<const char*>(a.k_cmp);
-  P.v_cmp = reinterpret_cast<const char*>(a.v_cmp);
   P.cmp_pages = a.pt_cmp ? a.cmp_num_pages : 0;
   P.cmp_ps_log2 = a.pt_cmp ? log2_exact(a.cmp_page_size) : 0;
   P.pt_cmp = a.pt_cmp;
