@@ -208,9 +208,13 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
  * scale      > 0
  * out        BF16 [n_queries, num_heads, head_dim] contiguous, 16-B aligned
  * lse        float [n_queries, num_heads]
- * num_splits 0 = automatic, 1 = one CTA per query, S in 2..16 = the set of
- *            each query is cut into S slices of 64-key tiles whose partial
- *            results are merged exactly (O_s, LSE_s weighted by e^{LSE_s-LSE}).
+ * num_splits 0 = automatic (one slice: the size of the sets is not known
+ *            here), 1 = one CTA per query, S in 2..16 = the set of each query
+ *            is cut into S slices of 64-key tiles whose partial results are
+ *            merged exactly (O_s, LSE_s weighted by e^{LSE_s-LSE}).
+ *            spa_sparse_sink_attn_choose_splits(n, H, max_set_size) picks S
+ *            for a known largest set: slices of at least 1024 keys, no more
+ *            slices than fill the GPU, and 1 when max_set_size <= 0.
  * workspace  >= spa_sparse_sink_attn_workspace_size(...) bytes for the same
  *            arguments (0 bytes when the call runs unsplit).
  * ---------------------------------------------------------------------- */

@@ -174,14 +174,16 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
 
 // ---------------------------------------------------------------- attention
 int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int32_t max_set_size) {
-  if (n_queries <= 0 || num_heads <= 0) return 1;
+  if (n_queries <= 0 || num_heads <= 0 || max_set_size <= 0) return 1;
   const int64_t head_tiles = (num_heads + 127) / 128;
   const int64_t units = static_cast<int64_t>(n_queries) * head_tiles;
-  // enough slices to give every persistent CTA (two per SM) a unit, without
-  // exceeding one wave of units
-  const int64_t target = 2 * static_cast<int64_t>(sm_count());
-  int64_t s = target / units;
-  if (max_set_size > 0) s = std::min<int64_t>(s, (max_set_size + spa::kAttnKeysPerTile - 1) / spa::kAttnKeysPerTile);
+  // Slicing pays only when each slice keeps a long run of tiles: measured on
+  // B200, with sets of up to 640 keys (decode of 64 or 128 queries) one
+  // slice per query is fastest, because the partial results and their merge
+  // cost more than the shorter chain saves. So: slices of at least 16 tiles
+  // (1024 keys), no more than fill the persistent CTAs (two per SM).
+  const int64_t tiles = (max_set_size + spa::kAttnKeysPerTile - 1) / spa::kAttnKeysPerTile;
+  int64_t s = std::min<int64_t>(2 * static_cast<int64_t>(sm_count()) / units, tiles / 16);
   s = std::max<int64_t>(1, std::min<int64_t>(s, spa::kAttnMaxSplits));
   return static_cast<int>(s);
 }

@@ -48,8 +48,11 @@ def test_host_helpers(L):
     w2 = L.spa_sparse_sink_attn_workspace_size(10, 128, 128, 2)
     assert w2 >= 10 * 2 * 128 * 128 * 4 + 10 * 2 * 128 * 8 + 10 * 4
     assert L.spa_sparse_sink_attn_choose_splits(100000, 128, 0) == 1
-    assert 1 <= L.spa_sparse_sink_attn_choose_splits(64, 128, 0) <= 16
-    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 100) == 2
+    assert L.spa_sparse_sink_attn_choose_splits(64, 128, 0) == 1        # set size unknown
+    assert L.spa_sparse_sink_attn_choose_splits(64, 128, 640) == 1      # short sets: one slice
+    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 100) == 1
+    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 65536) == 16    # long set, few queries
+    assert 1 < L.spa_sparse_sink_attn_choose_splits(64, 128, 8192) <= 8
 
 
 FAKE = 0x10000  # a 16-byte aligned non-NULL address; never dereferenced on these paths
