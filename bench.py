@@ -135,13 +135,20 @@ def measured_traffic(w, args):
     return entry["dram_bytes_per_launch"]
 
 
-def algorithmic_bytes(w, indptr, indices):
+def algorithmic_bytes(w, indptr, indices, fused_fp8=False):
     """HBM bytes the attention launch must move at least once: Q, O, LSE,
-    the CSR sets, the page tables and every distinct (request, key) K/V row."""
+    the CSR sets, the page tables and every distinct (request, key) K/V row
+    (a compressed row read as FP8 codes and scales when the decode is fused
+    into the gather)."""
     req_of_key = np.repeat(w.req.astype(np.int64), np.diff(indptr))
-    distinct = np.unique(req_of_key * (1 << 31) + indices.astype(np.int64)).size
+    keys = np.unique(req_of_key * (1 << 31) + indices.astype(np.int64))
+    distinct = keys.size
     qo = 2 * w.N * w.H * w.d * 2
-    kv = distinct * 2 * w.d * 2
+    if fused_fp8:
+        n_cmp = int(((keys & ((1 << 31) - 1)) < (1 << 30)).sum())
+        kv = (distinct - n_cmp) * 2 * w.d * 2 + n_cmp * 2 * (w.d + 4 * (w.d // 64))
+    else:
+        kv = distinct * 2 * w.d * 2
     other = w.N * w.H * 4 + indptr.nbytes + indices.nbytes + w.pt_raw.nbytes + \
         (0 if w.pt_cmp is None else w.pt_cmp.nbytes)
     return qo + kv + other, distinct
@@ -187,7 +194,7 @@ def run_reference(args, rank, world):
     return 0
 
 
-def config_of(w, world, nnz):
+def config_of(w, world, nnz, fp8_path=None):
     from sparse_paged_attention_build_b200 import workloads
     c = {"workload": f"{w.name}: {workloads.DESCRIPTIONS[w.name]}", "n_queries": w.N, "heads": w.H,
          "head_dim": w.d, "window": w.W, "ratio": w.ratio, "topk": w.K,
@@ -197,6 +204,8 @@ def config_of(w, world, nnz):
     if nnz is not None:
         c["kv_pairs_per_step"] = nnz
         c["mean_set_size"] = nnz / w.N
+    if w.k_cmp_fp8 is not None:
+        c["fp8_path"] = fp8_path
     return c
 
 
@@ -208,6 +217,8 @@ def main():
     ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
+                    help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=0)
@@ -236,14 +247,14 @@ def main():
 
     w = workloads.make(args.workload, shrink=args.shrink, seed_offset=rank)
     decode = w.kind == "decode"
-    b0 = DeviceBatch(w, num_splits=args.splits)
+    b0 = DeviceBatch(w, num_splits=args.splits, fp8_path=args.fp8_path)
     stream = torch.cuda.current_stream()
     b0.step()
     torch.cuda.synchronize()
     nnz = b0.nnz()
     triples, flops = algorithmic(w, nnz)
     hbm_bytes, distinct_rows = algorithmic_bytes(w, b0.indptr.cpu().numpy(),
-                                                 b0.indices[:nnz].cpu().numpy())
+                                                 b0.indices[:nnz].cpu().numpy(), fused_fp8=b0.fused)
     # a decode batch fits in L2: write a buffer larger than L2 between
     # timed steps (outside the timed intervals)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if decode else None
@@ -326,7 +337,8 @@ def main():
     else:
         roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peak_gbs, "unit": "GB/s",
                     "frac": achieved_gbs / peak_gbs, "peak_source": f"{pk_kind} HBM copy"}
-    roofline.update({"kernel": f"sparse_sink_attn_kernel<{w.d}>", "traffic": traffic,
+    roofline.update({"kernel": f"sparse_sink_attn_kernel<{w.d}, {'true' if b0.fused else 'false'}>",
+                     "traffic": traffic,
                      "algorithmic_bytes": hbm_bytes, "algorithmic_flops": flops,
                      "distinct_kv_rows": int(distinct_rows), "tflops": achieved_tf,
                      "hbm_gbs": achieved_gbs, "attn_ms_per_launch": attn_ms})
@@ -347,7 +359,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_of(w, world, nnz),
+            "config": config_of(w, world, nnz, args.fp8_path),
             "tflops": flops * args.steps * world / (elapsed_ms / 1e3) / 1e12,
             "roofline": roofline,
             "clocks": clocks, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
@@ -386,7 +398,8 @@ def measure_e2e(w, b0, args, stream, world, barrier, dist):
             host["k_cmp"] = pinned(w.k_cmp.view(np.int16), bf)
             host["v_cmp"] = pinned(w.v_cmp.view(np.int16), bf)
     if w.k_cmp_fp8 is not None:
-        for k in ("k_cmp_fp8", "v_cmp_fp8", "k_cmp_scale", "v_cmp_scale", "cmp_page_ids"):
+        names = ("k_cmp_fp8", "v_cmp_fp8", "k_cmp_scale", "v_cmp_scale")
+        for k in names + (() if b0.fused else ("cmp_page_ids",)):
             host[k] = pinned(getattr(w, k))
     dev = {k: getattr(b0, k) for k in host}
     h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)

@@ -233,6 +233,38 @@ int spa_sparse_sink_attn_fwd(
     const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * 3b. spa_sparse_sink_attn_fwd_fp8 -- the same attention over a mixed
+ * cache whose compressed pool is stored in FP8, decoded inside the gather.
+ *
+ * Defined by "Roadmap item 24", section "Reuse and arithmetic" (the mixed
+ * FP8/BF16 cache, an explicit OCP format, FP32 scales, decoded to BF16
+ * before the BF16 attention). Every compressed element enters the products
+ * as bf16_rne(float(e4m3) * scale), the value spa_dequant_fp8_pages writes,
+ * so the result is bit-identical to decoding the pages first and calling
+ * spa_sparse_sink_attn_fwd on the decoded pool.
+ *
+ * Arguments as for spa_sparse_sink_attn_fwd, except the compressed pool:
+ * k_cmp_fp8, v_cmp_fp8    E4M3 codes [cmp_num_pages, cmp_page_size,
+ *                         head_dim] bytes, 16-B aligned
+ * k_cmp_scale, v_cmp_scale FP32 [cmp_num_pages, cmp_page_size,
+ *                         head_dim / 64]: one scale per 64 elements
+ * pt_cmp                  required (non-NULL)
+ * fp8_format              0 = OCP E4M3 (1 = FNUZ: SPA_ERR_UNSUPPORTED)
+ * The window (raw) pool stays BF16.
+ * ---------------------------------------------------------------------- */
+int spa_sparse_sink_attn_fwd_fp8(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+    int32_t num_heads, int32_t head_dim,
+    const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+    const int32_t* pt_raw, int32_t pt_raw_cols,
+    const uint8_t* k_cmp_fp8, const uint8_t* v_cmp_fp8, const float* k_cmp_scale,
+    const float* v_cmp_scale, int64_t cmp_num_pages, int32_t cmp_page_size,
+    const int32_t* pt_cmp, int32_t pt_cmp_cols, int32_t fp8_format,
+    const int32_t* req, int32_t n_requests, const int32_t* indptr, const int32_t* indices,
+    const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
+    void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,12 @@ def _load():
         P, P, i64, i32, P, i32,
         P, i32, P, P, P, ctypes.c_float, P, P, i32, P, sz, P, P]
     L.spa_sparse_sink_attn_fwd.restype = ctypes.c_int
+    L.spa_sparse_sink_attn_fwd_fp8.argtypes = [
+        P, i64, i64, i32, i32, i32,
+        P, P, i64, i32, P, i32,
+        P, P, P, P, i64, i32, P, i32, i32,
+        P, i32, P, P, P, ctypes.c_float, P, P, i32, P, sz, P, P]
+    L.spa_sparse_sink_attn_fwd_fp8.restype = ctypes.c_int
     return L
 
 
@@ -212,6 +218,50 @@ def sparse_sink_attn_fwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
         _p(k_cmp), _p(v_cmp), 0 if k_cmp is None else k_cmp.shape[0],
         1 if k_cmp is None else k_cmp.shape[1],
         _p(None if pt_cmp is None else pt_cmp.contiguous()), 0 if pt_cmp is None else pt_cmp.shape[1],
+        _p(req.contiguous()), pt_raw.shape[0], _p(indptr.contiguous()), _p(indices.contiguous()),
+        _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
+        _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
+    return out, lse
+
+
+def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale,
+                             k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale, pt_cmp, out=None, lse=None,
+                             num_splits=0, workspace=None, dev_status=None, stream=None):
+    """Like sparse_sink_attn_fwd, with the compressed pool in FP8 (OCP E4M3
+    codes uint8 [pages, page_size, d], FP32 scales [pages, page_size, d/64])
+    decoded inside the attention gather; bit-identical to decoding the pages
+    with dequant_fp8_pages first."""
+    _need(q, "q", torch.bfloat16)
+    for name, t in (("k_raw", k_raw), ("v_raw", v_raw)):
+        _need(t, name, torch.bfloat16)
+        assert t.is_contiguous(), name
+    for name, t in (("pt_raw", pt_raw), ("req", req), ("indptr", indptr), ("indices", indices),
+                    ("pt_cmp", pt_cmp)):
+        _need(t, name, torch.int32)
+    for name, t in (("k_cmp_fp8", k_cmp_fp8), ("v_cmp_fp8", v_cmp_fp8)):
+        _need(t, name, torch.uint8)
+        assert t.is_contiguous(), name
+    for name, t in (("k_cmp_scale", k_cmp_scale), ("v_cmp_scale", v_cmp_scale)):
+        _need(t, name, torch.float32)
+        assert t.is_contiguous(), name
+    N, H, d = q.shape
+    if q.stride(2) != 1:
+        raise ValueError("q's last dimension must be contiguous")
+    if sink is not None:
+        _need(sink, "sink", torch.float32)
+    if out is None:
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((N, H), dtype=torch.float32, device=q.device)
+    ws_bytes = attn_workspace_size(N, H, d, num_splits)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    pt_raw = pt_raw.contiguous()
+    _check("spa_sparse_sink_attn_fwd_fp8", lib.spa_sparse_sink_attn_fwd_fp8(
+        _p(q), q.stride(0), q.stride(1), N, H, d,
+        _p(k_raw), _p(v_raw), k_raw.shape[0], k_raw.shape[1], _p(pt_raw), pt_raw.shape[1],
+        _p(k_cmp_fp8), _p(v_cmp_fp8), _p(k_cmp_scale), _p(v_cmp_scale), k_cmp_fp8.shape[0], k_cmp_fp8.shape[1],
+        _p(pt_cmp.contiguous()), pt_cmp.shape[1], 0,
         _p(req.contiguous()), pt_raw.shape[0], _p(indptr.contiguous()), _p(indices.contiguous()),
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))

@@ -195,62 +195,74 @@ size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads,
                                    resolve_splits(n_queries, num_heads, num_splits));
 }
 
-int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
-                             int32_t num_heads, int32_t head_dim, const uint16_t* k_raw, const uint16_t* v_raw,
-                             int64_t raw_num_pages, int32_t raw_page_size, const int32_t* pt_raw,
-                             int32_t pt_raw_cols, const uint16_t* k_cmp, const uint16_t* v_cmp,
-                             int64_t cmp_num_pages, int32_t cmp_page_size, const int32_t* pt_cmp,
-                             int32_t pt_cmp_cols, const int32_t* req, int32_t n_requests,
-                             const int32_t* indptr, const int32_t* indices, const float* sink, float scale,
-                             uint16_t* out, float* lse, int32_t num_splits, void* workspace,
-                             size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
-  if (n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
-  if (num_heads < 1) return fail(SPA_ERR_INVALID_ARG, "num_heads < 1");
-  if (n_requests < 1) return fail(SPA_ERR_INVALID_ARG, "n_requests < 1");
-  if (head_dim != 64 && head_dim != 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
-  if (num_heads > 128 && num_heads % 128 != 0)
+}  // extern "C"
+
+namespace {
+
+// Checks shared by both attention entry points (everything except the
+// compressed pool's storage), then the launch.
+int attn_run(spa::AttnArgs a, int32_t requested_splits, size_t workspace_bytes, cudaStream_t stream) {
+  if (a.n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
+  if (a.num_heads < 1) return fail(SPA_ERR_INVALID_ARG, "num_heads < 1");
+  if (a.n_requests < 1) return fail(SPA_ERR_INVALID_ARG, "n_requests < 1");
+  if (a.head_dim != 64 && a.head_dim != 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (a.num_heads > 128 && a.num_heads % 128 != 0)
     return fail(SPA_ERR_UNSUPPORTED, "num_heads above 128 must be a multiple of 128");
-  if (raw_num_pages < 0 || pt_raw_cols < 0) return fail(SPA_ERR_INVALID_ARG, "raw pool sizes < 0");
-  if (raw_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "raw_page_size < 1");
-  if (!pow2_in(raw_page_size, 1, 1024)) return fail(SPA_ERR_UNSUPPORTED, "raw_page_size must be a power of two <= 1024");
-  if (raw_num_pages * raw_page_size >= 0x7fffffffLL)
+  if (a.raw_num_pages < 0 || a.pt_raw_cols < 0) return fail(SPA_ERR_INVALID_ARG, "raw pool sizes < 0");
+  if (a.raw_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "raw_page_size < 1");
+  if (!pow2_in(a.raw_page_size, 1, 1024))
+    return fail(SPA_ERR_UNSUPPORTED, "raw_page_size must be a power of two <= 1024");
+  if (a.raw_num_pages * a.raw_page_size >= 0x7fffffffLL)
     return fail(SPA_ERR_UNSUPPORTED, "raw pool holds 2^31 - 1 rows or more");
-  if (pt_cmp != nullptr) {
-    if (cmp_num_pages < 0 || pt_cmp_cols < 0) return fail(SPA_ERR_INVALID_ARG, "compressed pool sizes < 0");
-    if (cmp_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "cmp_page_size < 1");
-    if (!pow2_in(cmp_page_size, 1, 1024))
+  if (a.pt_cmp != nullptr) {
+    if (a.cmp_num_pages < 0 || a.pt_cmp_cols < 0) return fail(SPA_ERR_INVALID_ARG, "compressed pool sizes < 0");
+    if (a.cmp_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "cmp_page_size < 1");
+    if (!pow2_in(a.cmp_page_size, 1, 1024))
       return fail(SPA_ERR_UNSUPPORTED, "cmp_page_size must be a power of two <= 1024");
-    if (cmp_num_pages * cmp_page_size >= 0x7fffffffLL)
+    if (a.cmp_num_pages * a.cmp_page_size >= 0x7fffffffLL)
       return fail(SPA_ERR_UNSUPPORTED, "compressed pool holds 2^31 - 1 rows or more");
-    if (k_cmp == nullptr || v_cmp == nullptr) return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
   }
-  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(SPA_ERR_INVALID_ARG, "scale must be finite and > 0");
-  if (num_splits < 0 || num_splits > spa::kAttnMaxSplits)
+  if (!(a.scale > 0.f) || !std::isfinite(a.scale)) return fail(SPA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (requested_splits < 0 || requested_splits > spa::kAttnMaxSplits)
     return fail(SPA_ERR_INVALID_ARG, "num_splits must be in [0, %d]", spa::kAttnMaxSplits);
-  if (q_stride_tok < 0 || q_stride_head < 0) return fail(SPA_ERR_INVALID_ARG, "negative q stride");
-  if (n_queries == 0) return ok();
-  if (q == nullptr || out == nullptr || lse == nullptr) return fail(SPA_ERR_INVALID_ARG, "q, out and lse must be non-NULL");
-  if (k_raw == nullptr || v_raw == nullptr || pt_raw == nullptr)
+  if (a.q_stride_tok < 0 || a.q_stride_head < 0) return fail(SPA_ERR_INVALID_ARG, "negative q stride");
+  if (a.n_queries == 0) return ok();
+  if (a.q == nullptr || a.out == nullptr || a.lse == nullptr)
+    return fail(SPA_ERR_INVALID_ARG, "q, out and lse must be non-NULL");
+  if (a.k_raw == nullptr || a.v_raw == nullptr || a.pt_raw == nullptr)
     return fail(SPA_ERR_INVALID_ARG, "k_raw, v_raw and pt_raw must be non-NULL");
-  if (req == nullptr || indptr == nullptr || indices == nullptr)
+  if (a.req == nullptr || a.indptr == nullptr || a.indices == nullptr)
     return fail(SPA_ERR_INVALID_ARG, "req, indptr and indices must be non-NULL");
-  if (!aligned(q, 16) || (q_stride_tok * 2) % 16 != 0 || (q_stride_head * 2) % 16 != 0)
+  if (!aligned(a.q, 16) || (a.q_stride_tok * 2) % 16 != 0 || (a.q_stride_head * 2) % 16 != 0)
     return fail(SPA_ERR_ALIGNMENT, "q base and strides must be 16-byte multiples");
-  if (!aligned(k_raw, 16) || !aligned(v_raw, 16) || !aligned(k_cmp, 16) || !aligned(v_cmp, 16))
+  if (!aligned(a.k_raw, 16) || !aligned(a.v_raw, 16) || !aligned(a.k_cmp, 16) || !aligned(a.v_cmp, 16) ||
+      !aligned(a.k_cmp_fp8, 16) || !aligned(a.v_cmp_fp8, 16))
     return fail(SPA_ERR_ALIGNMENT, "K/V pools must be 16-byte aligned");
-  if (!aligned(out, 16)) return fail(SPA_ERR_ALIGNMENT, "out must be 16-byte aligned");
-  if (!aligned(lse, 4) || !aligned(sink, 4) || !aligned(req, 4) || !aligned(indptr, 4) || !aligned(indices, 4) ||
-      !aligned(pt_raw, 4) || !aligned(pt_cmp, 4))
+  if (!aligned(a.out, 16)) return fail(SPA_ERR_ALIGNMENT, "out must be 16-byte aligned");
+  if (!aligned(a.lse, 4) || !aligned(a.sink, 4) || !aligned(a.req, 4) || !aligned(a.indptr, 4) ||
+      !aligned(a.indices, 4) || !aligned(a.pt_raw, 4) || !aligned(a.pt_cmp, 4) || !aligned(a.k_cmp_scale, 4) ||
+      !aligned(a.v_cmp_scale, 4))
     return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
-  const int32_t splits = resolve_splits(n_queries, num_heads, num_splits);
-  if (static_cast<int64_t>(n_queries) * splits > 0x7fffffffLL)
+  const int32_t splits = resolve_splits(a.n_queries, a.num_heads, requested_splits);
+  if (static_cast<int64_t>(a.n_queries) * splits > 0x7fffffffLL)
     return fail(SPA_ERR_UNSUPPORTED, "n_queries * num_splits exceeds the grid");
-  const size_t need = spa::attn_workspace_bytes(n_queries, num_heads, head_dim, splits);
+  const size_t need = spa::attn_workspace_bytes(a.n_queries, a.num_heads, a.head_dim, splits);
   if (need > 0) {
-    if (workspace == nullptr || workspace_bytes < need)
+    if (a.workspace == nullptr || workspace_bytes < need)
       return fail(SPA_ERR_WORKSPACE, "workspace needs %zu bytes", need);
-    if (!aligned(workspace, 256)) return fail(SPA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    if (!aligned(a.workspace, 256)) return fail(SPA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
   }
+  a.num_splits = splits;
+  return cuda_status(spa::launch_sparse_sink_attn(a, stream), "sparse_sink_attn launch");
+}
+
+spa::AttnArgs attn_args(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+                        int32_t num_heads, int32_t head_dim, const uint16_t* k_raw, const uint16_t* v_raw,
+                        int64_t raw_num_pages, int32_t raw_page_size, const int32_t* pt_raw, int32_t pt_raw_cols,
+                        int64_t cmp_num_pages, int32_t cmp_page_size, const int32_t* pt_cmp, int32_t pt_cmp_cols,
+                        const int32_t* req, int32_t n_requests, const int32_t* indptr, const int32_t* indices,
+                        const float* sink, float scale, uint16_t* out, float* lse, void* workspace,
+                        uint32_t* dev_status) {
   spa::AttnArgs a;
   a.q = q;
   a.q_stride_tok = q_stride_tok;
@@ -264,8 +276,8 @@ int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
   a.raw_page_size = raw_page_size;
   a.pt_raw = pt_raw;
   a.pt_raw_cols = pt_raw_cols;
-  a.k_cmp = k_cmp;
-  a.v_cmp = v_cmp;
+  a.k_cmp = nullptr;
+  a.v_cmp = nullptr;
   a.cmp_num_pages = cmp_num_pages;
   a.cmp_page_size = cmp_page_size;
   a.pt_cmp = pt_cmp;
@@ -278,11 +290,61 @@ int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
   a.scale = scale;
   a.out = out;
   a.lse = lse;
-  a.num_splits = splits;
+  a.num_splits = 0;
   a.workspace = workspace;
   a.dev_status = dev_status;
-  return cuda_status(spa::launch_sparse_sink_attn(a, reinterpret_cast<cudaStream_t>(stream)),
-                     "sparse_sink_attn launch");
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+                             int32_t num_heads, int32_t head_dim, const uint16_t* k_raw, const uint16_t* v_raw,
+                             int64_t raw_num_pages, int32_t raw_page_size, const int32_t* pt_raw,
+                             int32_t pt_raw_cols, const uint16_t* k_cmp, const uint16_t* v_cmp,
+                             int64_t cmp_num_pages, int32_t cmp_page_size, const int32_t* pt_cmp,
+                             int32_t pt_cmp_cols, const int32_t* req, int32_t n_requests,
+                             const int32_t* indptr, const int32_t* indices, const float* sink, float scale,
+                             uint16_t* out, float* lse, int32_t num_splits, void* workspace,
+                             size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
+  if (pt_cmp != nullptr && n_queries > 0 && (k_cmp == nullptr || v_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
+  spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
+                              raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
+                              pt_cmp_cols, req, n_requests, indptr, indices, sink, scale, out, lse, workspace,
+                              dev_status);
+  a.k_cmp = k_cmp;
+  a.v_cmp = v_cmp;
+  return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spa_sparse_sink_attn_fwd_fp8(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head,
+                                 int32_t n_queries, int32_t num_heads, int32_t head_dim, const uint16_t* k_raw,
+                                 const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+                                 const int32_t* pt_raw, int32_t pt_raw_cols, const uint8_t* k_cmp_fp8,
+                                 const uint8_t* v_cmp_fp8, const float* k_cmp_scale, const float* v_cmp_scale,
+                                 int64_t cmp_num_pages, int32_t cmp_page_size, const int32_t* pt_cmp,
+                                 int32_t pt_cmp_cols, int32_t fp8_format, const int32_t* req, int32_t n_requests,
+                                 const int32_t* indptr, const int32_t* indices, const float* sink, float scale,
+                                 uint16_t* out, float* lse, int32_t num_splits, void* workspace,
+                                 size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
+  if (fp8_format == 1) return fail(SPA_ERR_UNSUPPORTED, "FNUZ E4M3 is not supported");
+  if (fp8_format != 0) return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3)");
+  if (pt_cmp == nullptr) return fail(SPA_ERR_INVALID_ARG, "pt_cmp must be non-NULL on the FP8 path");
+  if (n_queries > 0 &&
+      (k_cmp_fp8 == nullptr || v_cmp_fp8 == nullptr || k_cmp_scale == nullptr || v_cmp_scale == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "FP8 codes and scales must be non-NULL");
+  spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
+                              raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
+                              pt_cmp_cols, req, n_requests, indptr, indices, sink, scale, out, lse, workspace,
+                              dev_status);
+  a.k_cmp_fp8 = k_cmp_fp8;
+  a.v_cmp_fp8 = v_cmp_fp8;
+  a.k_cmp_scale = k_cmp_scale;
+  a.v_cmp_scale = v_cmp_scale;
+  return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

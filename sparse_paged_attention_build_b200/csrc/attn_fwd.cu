@@ -111,6 +111,12 @@ struct Params {
   int64_t cmp_pages;
   int32_t cmp_ps_log2, pt_cmp_cols;
   const int32_t* pt_cmp;
+  // compressed pool in FP8 (OCP E4M3, one FP32 scale per 64 elements), for
+  // the fused decode; NULL on the BF16 path
+  const uint8_t* k_cmp8;
+  const uint8_t* v_cmp8;
+  const float* k_cmp_sc;
+  const float* v_cmp_sc;
   const int32_t* req;
   int32_t n_requests;
   const int32_t* indptr;
@@ -226,7 +232,7 @@ __device__ void resolve_chunk(const Params& P, int32_t b, int32_t key_base, int3
   }
 }
 
-template <int D>
+template <int D, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __grid_constant__ Params P) {
   using L = Layout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -380,38 +386,119 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         }
         ++qc;
       }
-      for (int t = 0; ok && t < ntiles; ++t, ++g) {
-        const int stage = g % nst;
-        if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
-        __syncwarp();
-        if (issuer) {
-          const int nv = min(kT, d.nkeys - t * kT);
-          uint32_t e[4];
-          bool any_raw = false, any_cmp = false;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int r = 4 * grp + k;
-            e[k] = r < nv ? t_rows[t * kT + r] : kInvalidRow;
-            if (e[k] != kInvalidRow) {
-              if (e[k] & kRawBit) any_raw = true;
-              else any_cmp = true;
+      if constexpr (!kFp8) {
+        for (int t = 0; ok && t < ntiles; ++t, ++g) {
+          const int stage = g % nst;
+          if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
+          if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
+          __syncwarp();
+          if (issuer) {
+            const int nv = min(kT, d.nkeys - t * kT);
+            uint32_t e[4];
+            bool any_raw = false, any_cmp = false;
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 4 * grp + k;
+              e[k] = r < nv ? t_rows[t * kT + r] : kInvalidRow;
+              if (e[k] != kInvalidRow) {
+                if (e[k] & kRawBit) any_raw = true;
+                else any_cmp = true;
+              }
+            }
+            int32_t y[4];
+  #pragma unroll
+            for (int k = 0; k < 4; ++k)   // rows outside the tensor are zero-filled
+              y[k] = e[k] == kInvalidRow ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
+            const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
+            if (!(any_raw && any_cmp)) {
+              tma_gather4(dst, any_cmp ? map_cmp : map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
+            } else {
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const bool cmp_row = e[k] != kInvalidRow && !(e[k] & kRawBit);
+                tma_load_2d(dst + k * 128, cmp_row ? map_cmp : map_raw, full + stage, half * 64, y[k]);
+              }
             }
           }
-          int32_t y[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k)   // rows outside the tensor are zero-filled
-            y[k] = e[k] == kInvalidRow ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
-          const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
-          if (!(any_raw && any_cmp)) {
-            tma_gather4(dst, any_cmp ? map_cmp : map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
-          } else {
+        }
+      } else {
+        // Fused FP8 decode. Raw (window) rows and zero rows (past the set,
+        // faulty keys) still come by TMA; compressed rows are read as E4M3
+        // codes and scales with plain loads (all of a tile's loads in flight
+        // together), decoded exactly as the page decode does, and written
+        // into the same 128-byte swizzled BF16 layout. The tile is complete
+        // once the TMA bytes have landed and lane 0 has arrived after every
+        // lane's shared-memory writes. (Staging the codes through cp.async
+        // to overlap the next tile's fetch measured slower on B200.)
+        constexpr int kPieces = D / 16;   // 16 codes per piece
+        constexpr int kPerLane = kT * kPieces / 32;
+        const uint8_t* pool8 = is_k ? P.k_cmp8 : P.v_cmp8;
+        const float* psc = is_k ? P.k_cmp_sc : P.v_cmp_sc;
+        for (int t = 0; ok && t < ntiles; ++t, ++g) {
+          const int stage = g % nst;
+          if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
+          const int nv = min(kT, d.nkeys - t * kT);
+          const uint32_t* trow = t_rows + t * kT;
+          uint32_t tx = 0;
+          uint32_t e[4];
+          bool fp8_row[4] = {false, false, false, false};
+          if (issuer) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const bool cmp_row = e[k] != kInvalidRow && !(e[k] & kRawBit);
-              tma_load_2d(dst + k * 128, cmp_row ? map_cmp : map_raw, full + stage, half * 64, y[k]);
+              const int r = 4 * grp + k;
+              e[k] = r < nv ? trow[r] : kInvalidRow;
+              fp8_row[k] = e[k] != kInvalidRow && !(e[k] & kRawBit);
+              if (!fp8_row[k]) tx += 128;
             }
           }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) tx += __shfl_xor_sync(0xffffffffu, tx, off);
+          if (lane == 0) mbar_expect_tx(full + stage, tx);
+          __syncwarp();
+          if (issuer) {
+            int32_t y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              y[k] = (e[k] == kInvalidRow || fp8_row[k]) ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
+            const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
+            if (!(fp8_row[0] || fp8_row[1] || fp8_row[2] || fp8_row[3])) {
+              tma_gather4(dst, map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (!fp8_row[k]) tma_load_2d(dst + k * 128, map_raw, full + stage, half * 64, y[k]);
+            }
+          }
+          uint8_t* tile = smem + (is_k ? L::kKOff : L::kVOff) + stage * L::kTileBytes;
+          uint4 raw[kPerLane];
+          float sc[kPerLane];
+#pragma unroll
+          for (int j = 0; j < kPerLane; ++j) {   // every load first
+            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
+            const uint32_t er = r < nv ? trow[r] : kInvalidRow;
+            raw[j] = make_uint4(0u, 0u, 0u, 0u);
+            sc[j] = 0.f;
+            if (er != kInvalidRow && !(er & kRawBit)) {
+              const int64_t row8 = er;
+              raw[j] = __ldg(reinterpret_cast<const uint4*>(pool8 + row8 * D + piece * 16));
+              sc[j] = __ldg(psc + row8 * (D / 64) + (piece * 16) / 64);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < kPerLane; ++j) {
+            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
+            const uint32_t er = r < nv ? trow[r] : kInvalidRow;
+            if (er == kInvalidRow || (er & kRawBit)) continue;
+            uint32_t o[8];
+            decode_e4m3x16(raw[j], sc[j], o);
+            const int hf = (piece * 16) / 64, ch0 = ((piece * 16) % 64) / 8;
+            uint8_t* row_ptr = tile + hf * (kT * 128) + r * 128;
+            *reinterpret_cast<uint4*>(row_ptr + ((ch0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(row_ptr + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+          fence_proxy_async_smem();   // generic-proxy writes -> the UMMA's reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full + stage);
         }
       }
       mbar_arrive(B.tab_empty + slot);
@@ -832,12 +919,12 @@ int sm_count_cached() {
   return n;
 }
 
-template <int D>
+template <int D, bool kFp8>
 cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
   using L = Layout<D>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t err = cudaFuncSetAttribute(sparse_sink_attn_kernel<D>,
+    cudaError_t err = cudaFuncSetAttribute(sparse_sink_attn_kernel<D, kFp8>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (err != cudaSuccess) return err;
     configured = true;
@@ -845,7 +932,7 @@ cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
   const int64_t units = static_cast<int64_t>(P.n_queries) * P.num_splits;
   const int64_t slots = std::max<int64_t>(1, (2 * static_cast<int64_t>(sm_count_cached())) / head_tiles);
   dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
-  sparse_sink_attn_kernel<D><<<grid, kThreads, L::kBytes, stream>>>(P);
+  sparse_sink_attn_kernel<D, kFp8><<<grid, kThreads, L::kBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
@@ -919,7 +1006,7 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
       !encode_pool(&P.tm_k_raw, a.k_raw, raw_rows, a.head_dim) ||
       !encode_pool(&P.tm_v_raw, a.v_raw, raw_rows, a.head_dim))
     return cudaErrorInvalidValue;
-  if (a.pt_cmp != nullptr) {
+  if (a.pt_cmp != nullptr && a.k_cmp_fp8 == nullptr) {
     const int64_t cmp_rows = a.cmp_num_pages * a.cmp_page_size;
     if (!encode_pool(&P.tm_k_cmp, a.k_cmp, cmp_rows, a.head_dim) ||
         !encode_pool(&P.tm_v_cmp, a.v_cmp, cmp_rows, a.head_dim))
@@ -935,6 +1022,10 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
   P.cmp_ps_log2 = a.pt_cmp ? log2_exact(a.cmp_page_size) : 0;
   P.pt_cmp = a.pt_cmp;
   P.pt_cmp_cols = a.pt_cmp ? a.pt_cmp_cols : 0;
+  P.k_cmp8 = a.k_cmp_fp8;
+  P.v_cmp8 = a.v_cmp_fp8;
+  P.k_cmp_sc = a.k_cmp_scale;
+  P.v_cmp_sc = a.v_cmp_scale;
   P.req = a.req;
   P.n_requests = a.n_requests;
   P.indptr = a.indptr;
@@ -961,7 +1052,10 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
                                       static_cast<size_t>(a.n_queries) * head_tiles * sizeof(uint32_t), stream);
     if (err != cudaSuccess) return err;
   }
-  return a.head_dim == 128 ? launch_d<128>(P, head_tiles, stream) : launch_d<64>(P, head_tiles, stream);
+  const bool fp8 = a.k_cmp_fp8 != nullptr;
+  if (a.head_dim == 128)
+    return fp8 ? launch_d<128, true>(P, head_tiles, stream) : launch_d<128, false>(P, head_tiles, stream);
+  return fp8 ? launch_d<64, true>(P, head_tiles, stream) : launch_d<64, false>(P, head_tiles, stream);
 }
 
 }  // namespace spa

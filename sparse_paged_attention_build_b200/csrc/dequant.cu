@@ -10,19 +10,11 @@
 // One CTA per listed page; each thread moves 16 source bytes (one 16-byte
 // load) to 32 destination bytes (two 16-byte stores). HBM-bound: 3 bytes of
 // traffic per element plus 4 bytes of scale per 64 elements.
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
-
 #include "spa_device.cuh"
 #include "spa_internal.h"
 
 namespace spa {
 namespace {
-
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
-}
 
 __global__ void __launch_bounds__(256)
 dequant_fp8_pages_kernel(const uint8_t* __restrict__ src, const float* __restrict__ scales,
@@ -39,15 +31,8 @@ dequant_fp8_pages_kernel(const uint8_t* __restrict__ src, const float* __restric
     const int64_t e0 = page_elem0 + static_cast<int64_t>(c) * 16;
     const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + e0));
     const float s = __ldg(scales + (e0 >> 6));  // rows are whole multiples of 64
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     uint32_t o[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
-      const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
-      o[2 * k] = pack_bf16x2(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
-      o[2 * k + 1] = pack_bf16x2(__fmul_rn(b.x, s), __fmul_rn(b.y, s));
-    }
+    decode_e4m3x16(raw, s, o);
     uint4* out = reinterpret_cast<uint4*>(dst + e0);
     out[0] = make_uint4(o[0], o[1], o[2], o[3]);
     out[1] = make_uint4(o[4], o[5], o[6], o[7]);

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "spa.h"
 
@@ -110,6 +112,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
+               : "memory");
+}
+
+// Add `bytes` to the transaction count of the current phase without
+// arriving (the arrival comes later, once other writes are done too).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
 
@@ -293,6 +302,29 @@ __device__ __forceinline__ float log2_approx(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------- FP8
+// Two OCP E4M3 codes -> two floats, exactly: every E4M3 value is a half
+// value and half -> float is exact.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// 16 E4M3 codes (one 16-byte load) with their group scale -> 16 BF16 values
+// packed in pairs: bf16_rne(float(e4m3) * scale), one binary32 multiply and
+// one rounding. The FP8 page decode and the fused attention gather both use
+// this, so their BF16 values are identical.
+__device__ __forceinline__ void decode_e4m3x16(const uint4 raw, float s, uint32_t (&o)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
+    const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
+    o[2 * k] = pack_bf16x2(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
+    o[2 * k + 1] = pack_bf16x2(__fmul_rn(b.x, s), __fmul_rn(b.y, s));
+  }
 }
 
 }  // namespace spa

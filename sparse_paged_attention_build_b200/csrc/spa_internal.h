@@ -40,6 +40,10 @@ struct AttnArgs {
   const int32_t* pt_raw;
   int32_t pt_raw_cols;
   const uint16_t *k_cmp, *v_cmp;
+  // FP8 compressed pool (fused decode): codes [pages, page_size, d] and
+  // FP32 scales [pages, page_size, d / 64]; when set, k_cmp/v_cmp are unused
+  const uint8_t *k_cmp_fp8 = nullptr, *v_cmp_fp8 = nullptr;
+  const float *k_cmp_scale = nullptr, *v_cmp_scale = nullptr;
   int64_t cmp_num_pages;
   int32_t cmp_page_size;
   const int32_t* pt_cmp;

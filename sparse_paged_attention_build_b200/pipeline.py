@@ -11,7 +11,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (build_kv_sets, dequant_fp8_pages, kv_sets_capacity, sparse_sink_attn_fwd,
+from . import (build_kv_sets, dequant_fp8_pages, kv_sets_capacity, sparse_sink_attn_fwd, sparse_sink_attn_fwd_fp8,
                attn_workspace_size, new_status, read_status)
 from . import lib
 
@@ -28,7 +28,7 @@ def _dev(a, dtype=None, device="cuda"):
 class DeviceBatch:
     """A workload resident in device memory, with its outputs."""
 
-    def __init__(self, w, device="cuda", num_splits=0):
+    def __init__(self, w, device="cuda", num_splits=0, fp8_path="decode"):
         self.w = w
         self.device = device
         bf16 = torch.bfloat16
@@ -42,14 +42,20 @@ class DeviceBatch:
         self.pt_cmp = _dev(w.pt_cmp, None, device)
         self.sink = _dev(w.sink, None, device)
         self.fp8 = w.k_cmp_fp8 is not None
+        if fp8_path not in ("fused", "decode"):
+            raise ValueError("fp8_path is 'fused' or 'decode'")
+        # mixed cache: decode inside the attention gather ("fused"), or decode
+        # the pages to a BF16 pool first ("decode")
+        self.fused = self.fp8 and fp8_path == "fused"
         if self.fp8:
             self.k_cmp_fp8 = _dev(w.k_cmp_fp8, None, device)
             self.v_cmp_fp8 = _dev(w.v_cmp_fp8, None, device)
             self.k_cmp_scale = _dev(w.k_cmp_scale, None, device)
             self.v_cmp_scale = _dev(w.v_cmp_scale, None, device)
             self.cmp_page_ids = _dev(w.cmp_page_ids, None, device)
-            self.k_cmp = torch.zeros(w.k_cmp_fp8.shape, dtype=bf16, device=device)
-            self.v_cmp = torch.zeros(w.v_cmp_fp8.shape, dtype=bf16, device=device)
+            if not self.fused:
+                self.k_cmp = torch.zeros(w.k_cmp_fp8.shape, dtype=bf16, device=device)
+                self.v_cmp = torch.zeros(w.v_cmp_fp8.shape, dtype=bf16, device=device)
         else:
             self.k_cmp = _dev(None if w.k_cmp is None else w.k_cmp.view(np.int16), bf16, device)
             self.v_cmp = _dev(None if w.v_cmp is None else w.v_cmp.view(np.int16), bf16, device)
@@ -74,7 +80,7 @@ class DeviceBatch:
                       stream=stream)
 
     def dequant(self, stream=None):
-        if self.fp8:
+        if self.fp8 and not self.fused:
             dequant_fp8_pages(self.k_cmp_fp8, self.k_cmp_scale, self.cmp_page_ids, self.k_cmp,
                               dev_status=self.status, stream=stream)
             dequant_fp8_pages(self.v_cmp_fp8, self.v_cmp_scale, self.cmp_page_ids, self.v_cmp,
@@ -82,6 +88,13 @@ class DeviceBatch:
 
     def attend(self, stream=None):
         w = self.w
+        if self.fused:
+            sparse_sink_attn_fwd_fp8(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.indptr,
+                                     self.indices, self.sink, w.scale, self.k_cmp_fp8, self.v_cmp_fp8,
+                                     self.k_cmp_scale, self.v_cmp_scale, self.pt_cmp, out=self.out,
+                                     lse=self.lse, num_splits=self.num_splits, workspace=self.attn_ws,
+                                     dev_status=self.status, stream=stream)
+            return
         sparse_sink_attn_fwd(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.indptr,
                              self.indices, self.sink, w.scale, k_cmp=self.k_cmp, v_cmp=self.v_cmp,
                              pt_cmp=self.pt_cmp, out=self.out, lse=self.lse,
@@ -95,7 +108,7 @@ class DeviceBatch:
         self.attend(stream)
 
     def kernels_per_step(self) -> int:
-        return 1 + (2 if self.fp8 else 0) + 1
+        return 1 + (2 if self.fp8 and not self.fused else 0) + 1
 
     def nnz(self) -> int:
         return int(self.indptr[-1].item())

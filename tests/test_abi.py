@@ -155,3 +155,37 @@ def test_guard_matrix_attention(L, kw, status, clause):
 
 def test_attention_zero_queries_is_a_no_op(L):
     assert attn_call(L, n=0, q=None, out=None, lse=None) == 0
+
+
+def attn8_call(L, **kw):
+    a = dict(q=FAKE, sq=16384, sh=128, n=4, H=128, d=128, kr=FAKE, vr=FAKE, rp=10, rps=64, ptr=FAKE,
+             ptrc=4, k8=FAKE, v8=FAKE, ks=FAKE, vs=FAKE, cp=10, cps=128, ptc=FAKE, ptcc=4, fmt=0,
+             req=FAKE, B=1, ip=FAKE, idx=FAKE, sink=FAKE, scale=0.088, out=FAKE, lse=FAKE, splits=1,
+             ws=None, wsb=0)
+    a.update(kw)
+    return L.spa_sparse_sink_attn_fwd_fp8(
+        a["q"], a["sq"], a["sh"], a["n"], a["H"], a["d"], a["kr"], a["vr"], a["rp"], a["rps"], a["ptr"],
+        a["ptrc"], a["k8"], a["v8"], a["ks"], a["vs"], a["cp"], a["cps"], a["ptc"], a["ptcc"], a["fmt"],
+        a["req"], a["B"], a["ip"], a["idx"], a["sink"], a["scale"], a["out"], a["lse"], a["splits"],
+        a["ws"], a["wsb"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(fmt=1), 2, "FNUZ"),
+    (dict(fmt=3), 1, "fp8_format must be 0"),
+    (dict(ptc=None), 1, "pt_cmp must be non-NULL"),
+    (dict(ks=None), 1, "codes and scales"),
+    (dict(v8=None), 1, "codes and scales"),
+    (dict(n=-1), 1, "n_queries < 0"),
+    (dict(cps=96), 2, "cmp_page_size must be a power of two"),
+    (dict(k8=FAKE + 8), 5, "K/V pools"),
+    (dict(vs=FAKE + 2), 5, "32-bit arrays"),
+    (dict(splits=2), 4, "workspace needs"),
+])
+def test_guard_matrix_attention_fp8(L, kw, status, clause):
+    assert attn8_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def test_attention_fp8_zero_queries_is_a_no_op(L):
+    assert attn8_call(L, n=0, q=None, out=None, lse=None, k8=None, v8=None, ks=None, vs=None) == 0

@@ -297,6 +297,88 @@ def test_pool_beyond_2GiB_uses_64bit_addressing(spa):
     del k_big, v_big
 
 
+# ------------------------------------------------------------------ fused FP8
+def fp8_batches(name, shrink, num_splits=0):
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    w = workload(name, shrink)
+    return (w, DeviceBatch(w, num_splits=num_splits, fp8_path="decode"),
+            DeviceBatch(w, num_splits=num_splits, fp8_path="fused"))
+
+
+def assert_bit_identical(a_out, a_lse, b_out, b_lse, what):
+    assert torch.equal(a_out.view(torch.int16), b_out.view(torch.int16)), f"{what}: O differs"
+    assert torch.equal(a_lse.view(torch.int32), b_lse.view(torch.int32)), f"{what}: LSE differs"
+
+
+@pytest.mark.parametrize("shrink,splits", [(32, 0), (8, 0), (8, 3)])
+def test_fused_fp8_gather_bit_identical_to_page_decode(spa, shrink, splits):
+    """Decoding the compressed rows inside the gather gives exactly the
+    result of decoding the pages first (same BF16 operands, same kernel)."""
+    w, dec, fus = fp8_batches("c5", shrink, splits)
+    dec.step()
+    fus.step()
+    torch.cuda.synchronize()
+    assert dec.status_word() == 0 and fus.status_word() == 0
+    assert fus.kernels_per_step() == 2
+    assert_bit_identical(dec.out, dec.lse, fus.out, fus.lse, f"c5/{shrink} splits={splits}")
+    O, L = oracle_attn("c5", shrink, None)
+    check_attn(fus.out, fus.lse, O, L, f"fused c5/{shrink}")
+
+
+def test_fused_fp8_full_size_against_oracle(spa):
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    w = workload("c5")
+    b = DeviceBatch(w, fp8_path="fused")
+    b.step()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+    O, L = oracle_attn("c5", 1, None)
+    check_attn(b.out, b.lse, O, L, "fused c5 full size")
+
+
+def test_fused_fp8_mixed_groups_and_faults(spa):
+    """Sets whose four-row groups straddle the two pools (one compressed key
+    dropped per query), and a faulty compressed page, on the fused path."""
+    w, dec, fus = fp8_batches("c5", 16)
+    dec.build_sets()
+    dec.dequant()
+    fus.build_sets()
+    ip = dec.indptr.cpu().numpy()
+    idx = dec.indices[: int(ip[-1])].cpu().numpy()
+    keep = np.ones(idx.size, dtype=bool)
+    keep[ip[:-1]] = False                     # drop each set's first (compressed) key
+    idx2 = idx[keep].astype(np.int32)
+    ip2 = (ip - np.arange(ip.size)).astype(np.int32)
+    ip2_t, idx2_t = torch.from_numpy(ip2).cuda(), torch.from_numpy(idx2).cuda()
+    st1, st2 = spa.new_status(), spa.new_status()
+    o1, l1 = spa.sparse_sink_attn_fwd(dec.q, dec.k_raw, dec.v_raw, dec.pt_raw, dec.req, ip2_t, idx2_t,
+                                      dec.sink, w.scale, k_cmp=dec.k_cmp, v_cmp=dec.v_cmp,
+                                      pt_cmp=dec.pt_cmp, dev_status=st1)
+    o2, l2 = spa.sparse_sink_attn_fwd_fp8(fus.q, fus.k_raw, fus.v_raw, fus.pt_raw, fus.req, ip2_t, idx2_t,
+                                          fus.sink, w.scale, fus.k_cmp_fp8, fus.v_cmp_fp8, fus.k_cmp_scale,
+                                          fus.v_cmp_scale, fus.pt_cmp, dev_status=st2)
+    torch.cuda.synchronize()
+    assert spa.read_status(st1) == 0 and spa.read_status(st2) == 0
+    assert_bit_identical(o1, l1, o2, l2, "straddling groups")
+    import oracle
+    k_cmp, v_cmp = oracle_cmp_pools("c5", 16)
+    O, L = oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip2, idx2, w.sink, w.scale,
+                                   k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp)
+    check_attn(o2, l2, O, L, "fused, straddling groups")
+    # a compressed page id outside the pool: reported, skipped, no trap
+    pt = fus.pt_cmp.clone()
+    pt[0, 0] = 10 ** 7
+    st = spa.new_status()
+    spa.sparse_sink_attn_fwd_fp8(fus.q, fus.k_raw, fus.v_raw, fus.pt_raw, fus.req, fus.indptr, fus.indices,
+                                 fus.sink, w.scale, fus.k_cmp_fp8, fus.v_cmp_fp8, fus.k_cmp_scale,
+                                 fus.v_cmp_scale, pt, dev_status=st)
+    torch.cuda.synchronize()
+    assert spa.read_status(st) & spa.DEV_BAD_PAGE
+    fus.step()
+    torch.cuda.synchronize()
+    assert fus.status_word() == 0
+
+
 def test_graph_capture_and_two_streams(spa):
     """The three calls capture into a CUDA graph; replays and a second
     stream give bit-identical results."""
