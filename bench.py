@@ -49,6 +49,21 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
+def job_totals(local_units, local_ms, world, device):
+    """Whole-job figures over the ranks: the units every rank processed
+    (ranks draw their own inputs, so their counts may differ) and the time
+    of the slowest rank. Every rank makes the same two collective calls."""
+    if world == 1:
+        return float(local_units), float(local_ms)
+    import torch
+    import torch.distributed as dist
+    u = torch.tensor([float(local_units)], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(u.item()), float(t.item())
+
+
 class ClockSampler:
     """nvidia-smi samples of the SM clock and throttle reasons."""
 
@@ -312,13 +327,10 @@ def main():
     else:
         elapsed_ms = start.elapsed_time(stop)
     attn_ms = float(np.mean([e1.elapsed_time(e2) for _, e1, e2 in ev]))
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    total_triples, elapsed_ms = job_totals(triples * args.steps, elapsed_ms, world, "cuda")
+    total_flops = total_triples * 4.0 * w.d
     status = b0.status_word()
 
-    total_triples = triples * args.steps * world
     value = total_triples / (elapsed_ms / 1e3)
     pk, pk_kind = peaks()
     timed_s = elapsed_ms / 1e3
@@ -360,7 +372,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_of(w, world, nnz, args.fp8_path),
-            "tflops": flops * args.steps * world / (elapsed_ms / 1e3) / 1e12,
+            "tflops": total_flops / (elapsed_ms / 1e3) / 1e12,
             "roofline": roofline,
             "clocks": clocks, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
             "device_status": status,
@@ -427,12 +439,8 @@ def measure_e2e(w, b0, args, stream, world, barrier, dist):
     e.record(stream)
     e.synchronize()
     ms = s.elapsed_time(e)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    triples = b0.nnz() * w.H
-    return {"value": triples * steps * world / (ms / 1e3), "unit": UNIT,
+    total, ms = job_totals(b0.nnz() * w.H * steps, ms, world, "cuda")
+    return {"value": total / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": ms / steps, "steps": steps}
 
