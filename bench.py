@@ -144,7 +144,8 @@ def measured_traffic(w, args):
     h = hashlib.sha256()
     for f in ("attn_fwd.cu", "spa_device.cuh"):
         h.update(open(os.path.join(ROOT, "sparse_paged_attention_build_b200", "csrc", f), "rb").read())
-    entry = rec.get(w.name)
+    fused = w.k_cmp_fp8 is not None and args.fp8_path == "fused"
+    entry = rec.get(w.name + (":fused" if fused else ""))
     if entry is None or rec.get("kernel_sha256") != h.hexdigest() or args.shrink != 1:
         return None
     return entry["dram_bytes_per_launch"]
