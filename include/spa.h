@@ -208,15 +208,18 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
  * scale      > 0
  * out        BF16 [n_queries, num_heads, head_dim] contiguous, 16-B aligned
  * lse        float [n_queries, num_heads]
- * num_splits 0 = automatic (one slice: the size of the sets is not known
- *            here), 1 = one CTA per query, S in 2..16 = the set of each query
- *            is cut into S slices of 64-key tiles whose partial results are
+ * num_splits 0 = automatic (spa_sparse_sink_attn_choose_splits(n, H, 0)),
+ *            1 = one CTA per query, S in 2..16 = the set of each query is
+ *            cut into S slices of 64-key tiles whose partial results are
  *            merged exactly (O_s, LSE_s weighted by e^{LSE_s-LSE}).
- *            spa_sparse_sink_attn_choose_splits(n, H, max_set_size) picks S
- *            for a known largest set: slices of at least 1024 keys, no more
- *            slices than fill the GPU, and 1 when max_set_size <= 0.
+ *            choose_splits: 1 for batches that fill the GPU; for small
+ *            batches (decode) up to 4 slices, no more than fill one wave of
+ *            CTAs; for a known long largest set, slices of >= 1024 keys.
  * workspace  >= spa_sparse_sink_attn_workspace_size(...) bytes for the same
- *            arguments (0 bytes when the call runs unsplit).
+ *            arguments: 0 bytes unsplit or with at most 8 slices (the slices
+ *            of a query then run as one thread-block cluster and merge
+ *            through distributed shared memory); 9..16 slices write FP32
+ *            partial results there, merged by the last slice to finish.
  * ---------------------------------------------------------------------- */
 size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads,
                                            int32_t head_dim, int32_t num_splits);

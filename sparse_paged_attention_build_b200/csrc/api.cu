@@ -174,16 +174,25 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
 
 // ---------------------------------------------------------------- attention
 int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int32_t max_set_size) {
-  if (n_queries <= 0 || num_heads <= 0 || max_set_size <= 0) return 1;
+  if (n_queries <= 0 || num_heads <= 0) return 1;
   const int64_t head_tiles = (num_heads + 127) / 128;
   const int64_t units = static_cast<int64_t>(n_queries) * head_tiles;
-  // Slicing pays only when each slice keeps a long run of tiles: measured on
-  // B200, with sets of up to 640 keys (decode of 64 or 128 queries) one
-  // slice per query is fastest, because the partial results and their merge
-  // cost more than the shorter chain saves. So: slices of at least 16 tiles
-  // (1024 keys), no more than fill the persistent CTAs (two per SM).
-  const int64_t tiles = (max_set_size + spa::kAttnKeysPerTile - 1) / spa::kAttnKeysPerTile;
-  int64_t s = std::min<int64_t>(2 * static_cast<int64_t>(sm_count()) / units, tiles / 16);
+  const int64_t slots = 2 * static_cast<int64_t>(sm_count());   // persistent CTAs, two per SM
+  int64_t s = 1;
+  if (units <= slots / 2) {
+    // A small batch (decode) leaves CTAs idle: cut each set into slices
+    // that merge inside one cluster. Measured on B200 with sets of up to
+    // 640 keys: 64 queries -> 4 slices and 128 queries -> 2 slices are
+    // 6 % and 15 % faster than one, while more slices than fill one wave
+    // of CTAs are slower.
+    s = std::min<int64_t>(slots / units, 4);
+  }
+  if (max_set_size > 0) {
+    // long sets: slices of at least 16 tiles (1024 keys), within one wave
+    const int64_t tiles = (max_set_size + spa::kAttnKeysPerTile - 1) / spa::kAttnKeysPerTile;
+    s = std::max<int64_t>(s, std::min<int64_t>(slots / units, tiles / 16));
+    s = std::min<int64_t>(s, std::max<int64_t>(1, tiles));   // no empty slices
+  }
   s = std::max<int64_t>(1, std::min<int64_t>(s, spa::kAttnMaxSplits));
   return static_cast<int>(s);
 }

@@ -126,6 +126,10 @@ struct Params {
   uint16_t* out;
   float* lse;
   int32_t num_splits;
+  // 1: the slices of a query are the CTAs of one cluster (one unit per
+  // CTA) and merge through distributed shared memory; 0: FP32 partials in
+  // the workspace, merged by the last slice to finish
+  int32_t cluster_merge;
   float* part_o;       // [n_queries * num_splits][num_heads][d]  (split runs only)
   float2* part_ml;     // [n_queries * num_splits][num_heads]
   uint32_t* tickets;   // [n_queries * head_tiles]
@@ -784,6 +788,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         }
         if (row_ok)
           P.lse[static_cast<int64_t>(i) * P.num_heads + h] = l > 0.f ? (m + log2_approx(l)) * kLn2 : -INFINITY;
+      } else if (P.cluster_merge) {
+        // this CTA's (m, l) rows for the cluster merge at the end; O stays
+        // in TMEM
+        reinterpret_cast<float2*>(smem + L::kMergeOff)[row] = make_float2(m, l);
+        if (tid == 0) *reinterpret_cast<int*>(smem + L::kMiscOff + 12) = have_o ? 1 : 0;
       } else {
         // partial result of this slice (no normalisation); the last slice
         // of the query to finish merges all of them
@@ -903,6 +912,108 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  if (P.cluster_merge) {
+    // Exact merge of the S slices of query i, CTA `rank` holding slice
+    // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
+    // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
+    // Summary: the deterministic (out, lse) merge). Each CTA scales its own
+    // O rows by its weight into shared memory (the K/V rings are idle now);
+    // then CTA `rank` sums its share of the rows over the cluster's shared
+    // memory and writes them. Every thread of every CTA reaches the three
+    // cluster barriers: every earlier wait in the kernel is bounded.
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int i = static_cast<int>(blockIdx.x / S);
+    const uint32_t ml_addr = sbase + L::kMergeOff;
+    const uint32_t wo_addr = sbase + L::kKOff;               // [128][D] FP32, 16-byte chunks swizzled by row
+    constexpr int kChunks = D / 4;                           // 16-byte chunks per row
+    __syncwarp();
+    cluster_sync_all();                                      // every slice's (m, l) is in place
+    if (tid < kSoftThreads) {
+      const int row = tid;
+      // all slices' (m, l) of this row, the loads in flight together
+      float2 ml[kAttnMaxClusterSplits];
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+        ml[s] = s < S ? ld_dsmem_f2(dsmem_addr(ml_addr + row * 8, s)) : make_float2(-INFINITY, 0.f);
+      float M = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+        if (ml[s].y > 0.f) M = fmaxf(M, ml[s].x);
+      float Lsum = 0.f, w_own = 0.f;
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
+        const float w = (ml[s].y > 0.f) ? exp2_approx(ml[s].x - M) : 0.f;
+        Lsum += w * ml[s].y;
+        if (s == rank) w_own = w;
+      }
+      const float scale_own = Lsum > 0.f ? w_own / Lsum : 0.f;
+      if (rank == 0 && row < heads_here)
+        P.lse[static_cast<int64_t>(i) * P.num_heads + head0 + row] =
+            Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
+      const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
+      const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
+      float* wo = reinterpret_cast<float*>(smem + L::kKOff);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {   // warp-uniform: one flag per CTA
+          tmem_ld32(o_lane + c0, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const int chunk = (c0 >> 2) + v;
+          const int phys = chunk ^ (row & (kChunks - 1));
+          *reinterpret_cast<float4*>(wo + row * D + phys * 4) =
+              make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
+                          __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own);
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();                                      // every slice's weighted rows are in place
+    if (tid < kSoftThreads) {
+      const int per = (heads_here + S - 1) / S;
+      const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
+      uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
+      // two 16-byte pieces per thread per pass, every slice's copy of both
+      // loaded before any is added
+      const int n_items = (r1 - r0) * kChunks;
+      for (int base = tid; base < n_items; base += 2 * kSoftThreads) {
+        float4 v[2][kAttnMaxClusterSplits];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int idx = base + k * kSoftThreads;
+          const int r = r0 + idx / kChunks, c = idx % kChunks;
+          const uint32_t off = wo_addr + static_cast<uint32_t>((r * D + (c ^ (r & (kChunks - 1))) * 4) * 4);
+#pragma unroll
+          for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+            v[k][s] = (idx < n_items && s < S) ? ld_dsmem_f4(dsmem_addr(off, s)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int idx = base + k * kSoftThreads;
+          if (idx >= n_items) continue;
+          const int r = r0 + idx / kChunks, c = idx % kChunks;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
+            acc.x += v[k][s].x;
+            acc.y += v[k][s].y;
+            acc.z += v[k][s].z;
+            acc.w += v[k][s].w;
+          }
+          *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r) * D + 4 * c) =
+              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();                                      // no slice leaves while its memory is read
+  }
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
@@ -930,6 +1041,24 @@ cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
     configured = true;
   }
   const int64_t units = static_cast<int64_t>(P.n_queries) * P.num_splits;
+  if (P.cluster_merge) {
+    // one unit per CTA, the S slices of a query in one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units), head_tiles);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(P.num_splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, sparse_sink_attn_kernel<D, kFp8>, P);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+  }
   const int64_t slots = std::max<int64_t>(1, (2 * static_cast<int64_t>(sm_count_cached())) / head_tiles);
   dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
   sparse_sink_attn_kernel<D, kFp8><<<grid, kThreads, L::kBytes, stream>>>(P);
@@ -985,7 +1114,7 @@ bool encode_q(CUtensorMap* m, const void* base, int32_t n, int32_t h, int d, int
 
 size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                             int32_t num_splits) {
-  if (num_splits <= 1) return 0;
+  if (num_splits <= kAttnMaxClusterSplits) return 0;   // unsplit, or merged within a cluster
   const int64_t units = static_cast<int64_t>(n_queries) * num_splits;
   const int64_t head_tiles = (num_heads + 127) / 128;
   size_t bytes = static_cast<size_t>(units * num_heads * head_dim) * sizeof(float);   // part_o
@@ -1040,7 +1169,8 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
   P.part_o = nullptr;
   P.part_ml = nullptr;
   P.tickets = nullptr;
-  if (a.num_splits > 1) {
+  P.cluster_merge = (a.num_splits > 1 && a.num_splits <= kAttnMaxClusterSplits) ? 1 : 0;
+  if (a.num_splits > kAttnMaxClusterSplits) {
     const int64_t units = static_cast<int64_t>(a.n_queries) * a.num_splits;
     char* ws = static_cast<char*>(a.workspace);
     P.part_o = reinterpret_cast<float*>(ws);

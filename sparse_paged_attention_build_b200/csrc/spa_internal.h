@@ -63,6 +63,9 @@ struct AttnArgs {
 
 constexpr int kAttnKeysPerTile = 64;
 constexpr int kAttnMaxSplits = 16;
+// up to this many slices merge inside one thread-block cluster (portable
+// cluster size); more slices use FP32 partials in the workspace
+constexpr int kAttnMaxClusterSplits = 8;
 size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                             int32_t num_splits);
 cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream);

@@ -45,14 +45,20 @@ def test_host_helpers(L):
     assert L.spa_kv_sets_capacity(10, 128, 0, 0, 0, 5) == 60
     assert L.spa_build_kv_sets_workspace_size(17) == 3 * 8 + 16
     assert L.spa_sparse_sink_attn_workspace_size(100, 128, 128, 1) == 0
-    w2 = L.spa_sparse_sink_attn_workspace_size(10, 128, 128, 2)
-    assert w2 >= 10 * 2 * 128 * 128 * 4 + 10 * 2 * 128 * 8 + 10 * 4
-    assert L.spa_sparse_sink_attn_choose_splits(100000, 128, 0) == 1
-    assert L.spa_sparse_sink_attn_choose_splits(64, 128, 0) == 1        # set size unknown
-    assert L.spa_sparse_sink_attn_choose_splits(64, 128, 640) == 1      # short sets: one slice
-    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 100) == 1
-    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 65536) == 16    # long set, few queries
-    assert 1 < L.spa_sparse_sink_attn_choose_splits(64, 128, 8192) <= 8
+    # up to 8 slices merge inside a cluster: no workspace; more use FP32 partials
+    for s in (2, 5, 8):
+        assert L.spa_sparse_sink_attn_workspace_size(10, 128, 128, s) == 0
+    w12 = L.spa_sparse_sink_attn_workspace_size(10, 128, 128, 12)
+    assert w12 >= 10 * 12 * 128 * 128 * 4 + 10 * 12 * 128 * 8 + 10 * 4
+    # (no GPU here: 148 SMs assumed, 296 persistent CTAs)
+    assert L.spa_sparse_sink_attn_choose_splits(100000, 128, 0) == 1   # prefill fills the GPU
+    assert L.spa_sparse_sink_attn_choose_splits(512, 128, 0) == 1
+    assert L.spa_sparse_sink_attn_choose_splits(64, 128, 0) == 4       # decode: cluster slices
+    assert L.spa_sparse_sink_attn_choose_splits(128, 128, 0) == 2
+    assert L.spa_sparse_sink_attn_choose_splits(64, 128, 640) == 4
+    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 100) == 2      # no empty slices
+    assert L.spa_sparse_sink_attn_choose_splits(1, 128, 65536) == 16   # long set, few queries
+    assert 4 <= L.spa_sparse_sink_attn_choose_splits(64, 128, 8192) <= 8
 
 
 FAKE = 0x10000  # a 16-byte aligned non-NULL address; never dereferenced on these paths
@@ -145,8 +151,8 @@ def attn_call(L, **kw):
     (dict(kr=FAKE + 8), 5, "K/V pools"),
     (dict(out=FAKE + 2), 5, "out must be"),
     (dict(lse=FAKE + 2), 5, "32-bit arrays"),
-    (dict(splits=2), 4, "workspace needs"),
-    (dict(splits=2, ws=FAKE + 16, wsb=1 << 30), 5, "workspace must be 256-byte"),
+    (dict(splits=12), 4, "workspace needs"),
+    (dict(splits=12, ws=FAKE + 16, wsb=1 << 30), 5, "workspace must be 256-byte"),
 ])
 def test_guard_matrix_attention(L, kw, status, clause):
     assert attn_call(L, **kw) == status
@@ -180,7 +186,7 @@ def attn8_call(L, **kw):
     (dict(cps=96), 2, "cmp_page_size must be a power of two"),
     (dict(k8=FAKE + 8), 5, "K/V pools"),
     (dict(vs=FAKE + 2), 5, "32-bit arrays"),
-    (dict(splits=2), 4, "workspace needs"),
+    (dict(splits=12), 4, "workspace needs"),
 ])
 def test_guard_matrix_attention_fp8(L, kw, status, clause):
     assert attn8_call(L, **kw) == status
