@@ -79,6 +79,10 @@ def lib() -> ctypes.CDLL:
             L.oracle_build_kv_sets.restype = ctypes.c_int
             L.oracle_dequant_fp8_pages.argtypes = [P, P, i64, i32, i32, P, i32, P]
             L.oracle_dequant_fp8_pages.restype = ctypes.c_int
+            L.oracle_dequant_fp8_pages_fmt.argtypes = [P, P, i64, i32, i32, P, i32, i32, P]
+            L.oracle_dequant_fp8_pages_fmt.restype = ctypes.c_int
+            L.oracle_e4m3fnuz_to_double.argtypes = [ctypes.c_uint8]
+            L.oracle_e4m3fnuz_to_double.restype = dbl
             L.oracle_sparse_sink_attn.argtypes = [
                 P, i64, i64, i32, i32, i32,
                 P, P, i64, i32, P, i32,
@@ -125,6 +129,15 @@ def e4m3_table() -> np.ndarray:
     return np.array([e4m3_to_double(c) for c in range(256)], dtype=np.float64)
 
 
+def e4m3fnuz_to_double(code: int) -> float:
+    return lib().oracle_e4m3fnuz_to_double(int(code))
+
+
+def e4m3fnuz_table() -> np.ndarray:
+    """All 256 E4M3 FNUZ codes decoded to FP64."""
+    return np.array([e4m3fnuz_to_double(c) for c in range(256)], dtype=np.float64)
+
+
 # --------------------------------------------------------------------------
 # the three steps of the path
 # --------------------------------------------------------------------------
@@ -155,8 +168,9 @@ def build_kv_sets(pos, W: int, ratio: int, topk=None, K: int | None = None):
     return indptr, indices[: indptr[-1]].copy()
 
 
-def dequant_fp8_pages(src, scales, page_ids, dst=None):
-    """BF16 bits of the listed pages: bf16_rne(float(e4m3(byte)) * scale)."""
+def dequant_fp8_pages(src, scales, page_ids, dst=None, fmt=0):
+    """BF16 bits of the listed pages: bf16_rne(float(e4m3(byte)) * scale);
+    fmt 0 = OCP E4M3, 1 = E4M3 FNUZ."""
     src = _c(src, np.uint8)
     P, ps, d = src.shape
     scales = _c(scales, np.float32).reshape(P, ps, d // 64)
@@ -164,8 +178,8 @@ def dequant_fp8_pages(src, scales, page_ids, dst=None):
     if dst is None:
         dst = np.zeros((P, ps, d), dtype=np.uint16)
     assert dst.dtype == np.uint16 and dst.flags.c_contiguous and dst.shape == (P, ps, d)
-    _check(lib().oracle_dequant_fp8_pages(_ptr(src), _ptr(scales), P, ps, d, _ptr(page_ids),
-                                          page_ids.shape[0], _ptr(dst)))
+    _check(lib().oracle_dequant_fp8_pages_fmt(_ptr(src), _ptr(scales), P, ps, d, _ptr(page_ids),
+                                              page_ids.shape[0], int(fmt), _ptr(dst)))
     return dst
 
 

@@ -106,6 +106,25 @@ double oracle_e4m3_to_double(uint8_t code)
     return sign ? -mag : mag;
 }
 
+/* E4M3 "FNUZ" variant (finite, no negative zero): the same three fields,
+ * exponent bias 8; the code 1.0000.000 is the only NaN, every other code is
+ * finite, so there is no -0 and the largest magnitude is 1.875 * 2^7 = 240.
+ * Exponent field 0 encodes subnormals m * 2^-10. */
+double oracle_e4m3fnuz_to_double(uint8_t code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xf;
+    int m = code & 0x7;
+    double mag;
+    if (code == 0x80)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m, -10);           /* (m/8) * 2^(1-8) */
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 8);
+    return sign ? -mag : mag;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Per-token KV sets.                                                        */
 /* ------------------------------------------------------------------------ */
@@ -184,19 +203,21 @@ int oracle_build_kv_sets(const int32_t* pos, int32_t N, int32_t W, int32_t ratio
 
 /* src: [num_pages, page_size, d] bytes; scales: [num_pages, page_size, d/64]
  * FP32; the listed pages of dst ([num_pages, page_size, d] BF16 bits) get
- * bf16_rne(float(e4m3(byte)) * scale); other pages are left untouched. */
-int oracle_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
-                             int32_t page_size, int32_t d, const int32_t* page_ids,
-                             int32_t n, uint16_t* dst)
+ * bf16_rne(float(e4m3(byte)) * scale); other pages are left untouched.
+ * fmt 0 reads the bytes as OCP E4M3, fmt 1 as E4M3 FNUZ. */
+int oracle_dequant_fp8_pages_fmt(const uint8_t* src, const float* scales, int64_t num_pages,
+                                 int32_t page_size, int32_t d, const int32_t* page_ids,
+                                 int32_t n, int32_t fmt, uint16_t* dst)
 {
-    if (page_size < 1 || d < 64 || d % 64 != 0 || n < 0) return ORACLE_BAD_ARG;
+    if (page_size < 1 || d < 64 || d % 64 != 0 || n < 0 || (fmt != 0 && fmt != 1)) return ORACLE_BAD_ARG;
     for (int32_t k = 0; k < n; ++k) {
         int64_t pg = page_ids[k];
         if (pg < 0 || pg >= num_pages) return ORACLE_BAD_PAGE;
         for (int64_t s = 0; s < page_size; ++s) {
             int64_t row = pg * page_size + s;
             for (int32_t e = 0; e < d; ++e) {
-                float value = (float)oracle_e4m3_to_double(src[row * d + e]);
+                uint8_t code = src[row * d + e];
+                float value = (float)(fmt == 0 ? oracle_e4m3_to_double(code) : oracle_e4m3fnuz_to_double(code));
                 float scale = scales[row * (d / 64) + e / 64];
                 float product = value * scale; /* one binary32 multiply */
                 dst[row * d + e] = oracle_float_to_bf16_rne(product);
@@ -204,6 +225,13 @@ int oracle_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t nu
         }
     }
     return ORACLE_OK;
+}
+
+int oracle_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
+                             int32_t page_size, int32_t d, const int32_t* page_ids,
+                             int32_t n, uint16_t* dst)
+{
+    return oracle_dequant_fp8_pages_fmt(src, scales, num_pages, page_size, d, page_ids, n, 0, dst);
 }
 
 /* ------------------------------------------------------------------------ */

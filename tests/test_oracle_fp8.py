@@ -87,3 +87,58 @@ def test_dequant_generator_values_are_within_a_scale_of_n01():
     codes = torch.from_numpy(w.k_cmp_fp8).view(torch.float8_e4m3fn).to(torch.float32).numpy()
     assert np.nanmax(np.abs(codes)) <= 448.0
     assert not np.isnan(codes).any()
+
+
+# ---------------------------------------------------------------- E4M3 FNUZ
+# The page also names the FNUZ flavour of E4M3 (bias 8, no negative zero,
+# 0x80 the only NaN, largest magnitude 240).
+
+def test_e4m3fnuz_definition_points(oracle):
+    assert oracle.e4m3fnuz_to_double(0x7F) == 240.0        # largest finite: no NaN at S.1111.111
+    assert oracle.e4m3fnuz_to_double(0xFF) == -240.0
+    assert oracle.e4m3fnuz_to_double(0x08) == 2.0 ** -7    # smallest normal
+    assert oracle.e4m3fnuz_to_double(0x01) == 2.0 ** -10   # smallest subnormal
+    assert oracle.e4m3fnuz_to_double(0x40) == 1.0          # exponent field 8 = bias
+    assert oracle.e4m3fnuz_to_double(0x00) == 0.0
+    assert math.isnan(oracle.e4m3fnuz_to_double(0x80))     # no -0: the code is the NaN
+    # the same code is worth half its OCP value wherever both are finite
+    for c in range(256):
+        if c in (0x7F, 0xFF, 0x80):
+            continue
+        assert oracle.e4m3fnuz_to_double(c) == 0.5 * oracle.e4m3_to_double(c)
+
+
+def test_e4m3fnuz_all_codes_match_torch_float8(oracle):
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fnuz).to(torch.float64).numpy()
+    mine = oracle.e4m3fnuz_table()
+    nan = np.isnan(ref)
+    assert nan.sum() == 1
+    assert np.array_equal(nan, np.isnan(mine))
+    assert np.array_equal(ref[~nan], mine[~nan])
+
+
+def test_e4m3fnuz_encode_round_trip(oracle):
+    table = oracle.e4m3fnuz_table()
+    finite = np.where(~np.isnan(table))[0]
+    back = torch.from_numpy(table[finite].astype(np.float32)).to(torch.float8_e4m3fnuz) \
+        .view(torch.uint8).numpy()
+    assert np.array_equal(back.astype(np.int64), finite)
+
+
+def test_dequant_fnuz_matches_torch_route(oracle):
+    rng = np.random.default_rng(3)
+    P, ps, d = 4, 16, 128
+    src = rng.integers(0, 256, size=(P, ps, d), dtype=np.uint8)
+    src[src == 0x80] = 0x00
+    scales = (rng.random((P, ps, d // 64)) * 3.0 + 1e-3).astype(np.float32)
+    page_ids = np.array([3, 1], dtype=np.int32)
+    dst = oracle.dequant_fp8_pages(src, scales, page_ids, fmt=1)
+    x = torch.from_numpy(src).view(torch.float8_e4m3fnuz).to(torch.float32)
+    s = torch.from_numpy(scales).repeat_interleave(64, dim=2)
+    ref = (x * s).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for p in page_ids:
+        assert np.array_equal(dst[p], ref[p])
+    # the two formats differ on the same bytes
+    ocp = oracle.dequant_fp8_pages(src, scales, page_ids, fmt=0)
+    assert not np.array_equal(ocp[3], dst[3])
