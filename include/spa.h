@@ -162,7 +162,8 @@ int spa_build_kv_sets_noalloc(const int32_t* pos, int32_t n_queries, int32_t win
  * scales    float [num_pages, page_size, head_dim/64]
  * page_ids  int32 [n_page_ids]; ids outside [0, num_pages) set
  *           SPA_DEV_BAD_PAGE and are skipped
- * fp8_format 0 = OCP E4M3 (FNUZ is SPA_ERR_UNSUPPORTED)
+ * fp8_format 0 = OCP E4M3, 1 = E4M3 FNUZ (exponent bias 8, no -0, the
+ *            code 0x80 is the NaN, largest magnitude 240)
  * dst       BF16 bits [num_pages, page_size, head_dim], 16-byte aligned
  * head_dim  a multiple of 64
  * ---------------------------------------------------------------------- */
@@ -253,7 +254,7 @@ int spa_sparse_sink_attn_fwd(
  * k_cmp_scale, v_cmp_scale FP32 [cmp_num_pages, cmp_page_size,
  *                         head_dim / 64]: one scale per 64 elements
  * pt_cmp                  required (non-NULL)
- * fp8_format              0 = OCP E4M3 (1 = FNUZ: SPA_ERR_UNSUPPORTED)
+ * fp8_format              0 = OCP E4M3, 1 = E4M3 FNUZ
  * The window (raw) pool stays BF16.
  * ---------------------------------------------------------------------- */
 int spa_sparse_sink_attn_fwd_fp8(

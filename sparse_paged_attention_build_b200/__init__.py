@@ -157,7 +157,8 @@ def build_kv_sets(pos, window, ratio, topk=None, capacity=None, max_pos=None, in
 
 
 def dequant_fp8_pages(src, scales, page_ids, dst, fp8_format=0, dev_status=None, stream=None):
-    """dst[pg] = bf16(float(e4m3(src[pg])) * scale) for every listed page."""
+    """dst[pg] = bf16(float(e4m3(src[pg])) * scale) for every listed page;
+    fp8_format 0 = OCP E4M3, 1 = E4M3 FNUZ."""
     _need(src, "src", torch.uint8)
     _need(scales, "scales", torch.float32)
     _need(page_ids, "page_ids", torch.int32)
@@ -226,7 +227,7 @@ def sparse_sink_attn_fwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
 
 def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale,
                              k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale, pt_cmp, out=None, lse=None,
-                             num_splits=0, workspace=None, dev_status=None, stream=None):
+                             num_splits=0, workspace=None, dev_status=None, stream=None, fp8_format=0):
     """Like sparse_sink_attn_fwd, with the compressed pool in FP8 (OCP E4M3
     codes uint8 [pages, page_size, d], FP32 scales [pages, page_size, d/64])
     decoded inside the attention gather; bit-identical to decoding the pages
@@ -261,7 +262,7 @@ def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink
         _p(q), q.stride(0), q.stride(1), N, H, d,
         _p(k_raw), _p(v_raw), k_raw.shape[0], k_raw.shape[1], _p(pt_raw), pt_raw.shape[1],
         _p(k_cmp_fp8), _p(v_cmp_fp8), _p(k_cmp_scale), _p(v_cmp_scale), k_cmp_fp8.shape[0], k_cmp_fp8.shape[1],
-        _p(pt_cmp.contiguous()), pt_cmp.shape[1], 0,
+        _p(pt_cmp.contiguous()), pt_cmp.shape[1], int(fp8_format),
         _p(req.contiguous()), pt_raw.shape[0], _p(indptr.contiguous()), _p(indices.contiguous()),
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))

@@ -157,8 +157,8 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
   if (page_size < 1) return fail(SPA_ERR_INVALID_ARG, "page_size < 1");
   if (head_dim < 1) return fail(SPA_ERR_INVALID_ARG, "head_dim < 1");
   if (n_page_ids < 0) return fail(SPA_ERR_INVALID_ARG, "n_page_ids < 0");
-  if (fp8_format == 1) return fail(SPA_ERR_UNSUPPORTED, "FNUZ E4M3 is not supported");
-  if (fp8_format != 0) return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3)");
+  if (fp8_format != 0 && fp8_format != 1)
+    return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3) or 1 (E4M3 FNUZ)");
   if (head_dim % 64 != 0) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be a multiple of 64");
   if (static_cast<int64_t>(page_size) * head_dim > (1 << 24))
     return fail(SPA_ERR_UNSUPPORTED, "page_size * head_dim too large");
@@ -167,7 +167,7 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
   if (!aligned(src, 16) || !aligned(dst, 16)) return fail(SPA_ERR_ALIGNMENT, "src and dst must be 16-byte aligned");
   if (!aligned(scales, 4) || !aligned(page_ids, 4)) return fail(SPA_ERR_ALIGNMENT, "scales/page_ids misaligned");
   return cuda_status(spa::launch_dequant_fp8_pages(src, scales, num_pages, page_size, head_dim, page_ids,
-                                                   n_page_ids, dst, dev_status,
+                                                   n_page_ids, fp8_format == 1, dst, dev_status,
                                                    reinterpret_cast<cudaStream_t>(stream)),
                      "dequant_fp8_pages launch");
 }
@@ -339,8 +339,8 @@ int spa_sparse_sink_attn_fwd_fp8(const uint16_t* q, int64_t q_stride_tok, int64_
                                  const int32_t* indptr, const int32_t* indices, const float* sink, float scale,
                                  uint16_t* out, float* lse, int32_t num_splits, void* workspace,
                                  size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
-  if (fp8_format == 1) return fail(SPA_ERR_UNSUPPORTED, "FNUZ E4M3 is not supported");
-  if (fp8_format != 0) return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3)");
+  if (fp8_format != 0 && fp8_format != 1)
+    return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3) or 1 (E4M3 FNUZ)");
   if (pt_cmp == nullptr) return fail(SPA_ERR_INVALID_ARG, "pt_cmp must be non-NULL on the FP8 path");
   if (n_queries > 0 &&
       (k_cmp_fp8 == nullptr || v_cmp_fp8 == nullptr || k_cmp_scale == nullptr || v_cmp_scale == nullptr))
@@ -353,6 +353,7 @@ int spa_sparse_sink_attn_fwd_fp8(const uint16_t* q, int64_t q_stride_tok, int64_
   a.v_cmp_fp8 = v_cmp_fp8;
   a.k_cmp_scale = k_cmp_scale;
   a.v_cmp_scale = v_cmp_scale;
+  a.fp8_fnuz = fp8_format == 1;
   return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 

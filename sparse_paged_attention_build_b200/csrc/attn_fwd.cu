@@ -117,6 +117,7 @@ struct Params {
   const uint8_t* v_cmp8;
   const float* k_cmp_sc;
   const float* v_cmp_sc;
+  int32_t fp8_fnuz;    // the codes are E4M3 FNUZ (1) or OCP E4M3 (0)
   const int32_t* req;
   int32_t n_requests;
   const int32_t* indptr;
@@ -494,7 +495,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
             const uint32_t er = r < nv ? trow[r] : kInvalidRow;
             if (er == kInvalidRow || (er & kRawBit)) continue;
             uint32_t o[8];
-            decode_e4m3x16(raw[j], sc[j], o);
+            if (P.fp8_fnuz) decode_e4m3x16<true>(raw[j], sc[j], o);
+            else decode_e4m3x16<false>(raw[j], sc[j], o);
             const int hf = (piece * 16) / 64, ch0 = ((piece * 16) % 64) / 8;
             uint8_t* row_ptr = tile + hf * (kT * 128) + r * 128;
             *reinterpret_cast<uint4*>(row_ptr + ((ch0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -1155,6 +1157,7 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
   P.v_cmp8 = a.v_cmp_fp8;
   P.k_cmp_sc = a.k_cmp_scale;
   P.v_cmp_sc = a.v_cmp_scale;
+  P.fp8_fnuz = a.fp8_fnuz ? 1 : 0;
   P.req = a.req;
   P.n_requests = a.n_requests;
   P.indptr = a.indptr;

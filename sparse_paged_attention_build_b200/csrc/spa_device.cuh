@@ -347,16 +347,33 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
+// E4M3 FNUZ (exponent bias 8, no negative zero) from the OCP reading of
+// the same byte: every code but three is worth exactly half its OCP value;
+// S.1111.111 is +-240 (NaN in OCP) and 1.0000.000 is the NaN (-0 in OCP).
+__device__ __forceinline__ float fnuz_from_ocp(float ocp, uint32_t code) {
+  if ((code & 0x7fu) == 0x7fu) return (code & 0x80u) ? -240.f : 240.f;
+  if (code == 0x80u) return __int_as_float(0x7fffffff);
+  return ocp * 0.5f;   // exact: a power of two
+}
+
 // 16 E4M3 codes (one 16-byte load) with their group scale -> 16 BF16 values
 // packed in pairs: bf16_rne(float(e4m3) * scale), one binary32 multiply and
-// one rounding. The FP8 page decode and the fused attention gather both use
-// this, so their BF16 values are identical.
+// one rounding; kFnuz reads the codes as E4M3 FNUZ instead of OCP E4M3. The
+// FP8 page decode and the fused attention gather both use this, so their
+// BF16 values are identical.
+template <bool kFnuz = false>
 __device__ __forceinline__ void decode_e4m3x16(const uint4 raw, float s, uint32_t (&o)[8]) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
-    const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
+    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
+    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
+    if (kFnuz) {
+      a.x = fnuz_from_ocp(a.x, w[k] & 0xffu);
+      a.y = fnuz_from_ocp(a.y, (w[k] >> 8) & 0xffu);
+      b.x = fnuz_from_ocp(b.x, (w[k] >> 16) & 0xffu);
+      b.y = fnuz_from_ocp(b.y, w[k] >> 24);
+    }
     o[2 * k] = pack_bf16x2(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
     o[2 * k + 1] = pack_bf16x2(__fmul_rn(b.x, s), __fmul_rn(b.y, s));
   }

@@ -27,7 +27,7 @@ cudaError_t launch_build_kv_sets_no_alloc(const int32_t* pos, int32_t n, int32_t
 
 cudaError_t launch_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
                                      int32_t page_size, int32_t head_dim, const int32_t* page_ids,
-                                     int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status,
+                                     int32_t n_page_ids, bool fnuz, uint16_t* dst, uint32_t* dev_status,
                                      cudaStream_t stream);
 
 struct AttnArgs {
@@ -44,6 +44,7 @@ struct AttnArgs {
   // FP32 scales [pages, page_size, d / 64]; when set, k_cmp/v_cmp are unused
   const uint8_t *k_cmp_fp8 = nullptr, *v_cmp_fp8 = nullptr;
   const float *k_cmp_scale = nullptr, *v_cmp_scale = nullptr;
+  bool fp8_fnuz = false;   // the codes are E4M3 FNUZ rather than OCP E4M3
   int64_t cmp_num_pages;
   int32_t cmp_page_size;
   const int32_t* pt_cmp;

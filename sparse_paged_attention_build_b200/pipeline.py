@@ -82,9 +82,9 @@ class DeviceBatch:
     def dequant(self, stream=None):
         if self.fp8 and not self.fused:
             dequant_fp8_pages(self.k_cmp_fp8, self.k_cmp_scale, self.cmp_page_ids, self.k_cmp,
-                              dev_status=self.status, stream=stream)
+                              fp8_format=self.w.fp8_format, dev_status=self.status, stream=stream)
             dequant_fp8_pages(self.v_cmp_fp8, self.v_cmp_scale, self.cmp_page_ids, self.v_cmp,
-                              dev_status=self.status, stream=stream)
+                              fp8_format=self.w.fp8_format, dev_status=self.status, stream=stream)
 
     def attend(self, stream=None):
         w = self.w
@@ -93,7 +93,7 @@ class DeviceBatch:
                                      self.indices, self.sink, w.scale, self.k_cmp_fp8, self.v_cmp_fp8,
                                      self.k_cmp_scale, self.v_cmp_scale, self.pt_cmp, out=self.out,
                                      lse=self.lse, num_splits=self.num_splits, workspace=self.attn_ws,
-                                     dev_status=self.status, stream=stream)
+                                     dev_status=self.status, stream=stream, fp8_format=self.w.fp8_format)
             return
         sparse_sink_attn_fwd(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.indptr,
                              self.indices, self.sink, w.scale, k_cmp=self.k_cmp, v_cmp=self.v_cmp,

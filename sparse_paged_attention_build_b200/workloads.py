@@ -66,6 +66,7 @@ class Workload:
     v_cmp_scale: np.ndarray | None = None
     cmp_page_ids: np.ndarray | None = None  # int32: pages holding compressed entries
     meta: dict = field(default_factory=dict)
+    fp8_format: int = 0                       # 0 = OCP E4M3, 1 = E4M3 FNUZ
 
     @property
     def raw_page_size(self):
@@ -89,14 +90,16 @@ def _normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
     return _bf16_bits(rng.standard_normal(shape, dtype=np.float32))
 
 
-def _e4m3_with_scales(rng: np.random.Generator, shape):
-    """x ~ N(0,1); per 64-element group s = max|x| / 448; byte = e4m3(x / s)."""
+def _e4m3_with_scales(rng: np.random.Generator, shape, fmt: int = 0):
+    """x ~ N(0,1); per 64-element group s = max|x| / fmax; byte = e4m3(x / s)
+    with fmax = 448 for OCP E4M3 (fmt 0) or 240 for E4M3 FNUZ (fmt 1)."""
     P, ps, d = shape
+    fmax, dtype = (448.0, torch.float8_e4m3fn) if fmt == 0 else (240.0, torch.float8_e4m3fnuz)
     x = rng.standard_normal((P, ps, d // 64, 64), dtype=np.float32)
     amax = np.abs(x).max(axis=-1, keepdims=True)
-    s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
-    y = np.clip(x / s, -448.0, 448.0).astype(np.float32)
-    codes = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    s = np.where(amax > 0, amax / np.float32(fmax), np.float32(1.0)).astype(np.float32)
+    y = np.clip(x / s, -fmax, fmax).astype(np.float32)
+    codes = torch.from_numpy(y).to(dtype).view(torch.uint8).numpy()
     return codes.reshape(P, ps, d).copy(), s.reshape(P, ps, d // 64).copy()
 
 
@@ -155,7 +158,7 @@ def _zero_pool_with_pages(rng, P, ps, d, pages):
     return pool
 
 
-def _decode(name, seed, B, lengths, H, d, W, ratio, K, ps, fp8):
+def _decode(name, seed, B, lengths, H, d, W, ratio, K, ps, fp8, fmt=0):
     ss = np.random.SeedSequence(seed)
     r_q, r_kv, r_cmp, r_sink, r_pt, r_topk = [np.random.Generator(np.random.PCG64(s)) for s in ss.spawn(6)]
     lengths = np.asarray(lengths, dtype=np.int64)
@@ -195,8 +198,8 @@ def _decode(name, seed, B, lengths, H, d, W, ratio, K, ps, fp8):
     k_cmp = v_cmp = None
     kf8 = vf8 = ks = vs = None
     if fp8:
-        kf8, ks = _e4m3_with_scales(r_cmp, (p_cmp, ps, d))
-        vf8, vs = _e4m3_with_scales(r_cmp, (p_cmp, ps, d))
+        kf8, ks = _e4m3_with_scales(r_cmp, (p_cmp, ps, d), fmt)
+        vf8, vs = _e4m3_with_scales(r_cmp, (p_cmp, ps, d), fmt)
     else:
         k_cmp = _normal_bf16(r_cmp, (p_cmp, ps, d))
         v_cmp = _normal_bf16(r_cmp, (p_cmp, ps, d))
@@ -204,7 +207,7 @@ def _decode(name, seed, B, lengths, H, d, W, ratio, K, ps, fp8):
     sink = r_sink.standard_normal(H, dtype=np.float32)
     return Workload(name, "decode", N, H, d, W, ratio, K, B, q, pos, req, topk,
                     k_raw, v_raw, pt_raw, k_cmp, v_cmp, pt_cmp, sink, 1.0 / float(np.sqrt(d)),
-                    kf8, vf8, ks, vs, cmp_page_ids, {"lengths": lengths})
+                    kf8, vf8, ks, vs, cmp_page_ids, {"lengths": lengths}, fmt)
 
 
 DESCRIPTIONS = {
@@ -216,9 +219,11 @@ DESCRIPTIONS = {
 }
 
 
-def make(name: str, shrink: int = 1, seed_offset: int = 0) -> Workload:
+def make(name: str, shrink: int = 1, seed_offset: int = 0, fp8_format: int = 0) -> Workload:
     """The named workload. ``shrink`` > 1 divides the number of requests and
-    the tokens per request (prefill) or the context lengths (decode)."""
+    the tokens per request (prefill) or the context lengths (decode).
+    ``fp8_format`` picks the encoding of the mixed cache (c5): 0 = OCP
+    E4M3, 1 = E4M3 FNUZ."""
     idx = int(name[1:])
     seed = BASE_SEED + idx + 1000 * seed_offset
     if name == "c1":
@@ -237,5 +242,5 @@ def make(name: str, shrink: int = 1, seed_offset: int = 0) -> Workload:
     if name == "c5":
         B = max(1, 128 // shrink)
         L = max(1024, 32768 // shrink)
-        return _decode(name, seed, B, np.full(B, L), 128, 128, 128, 4, 512, 128, fp8=True)
+        return _decode(name, seed, B, np.full(B, L), 128, 128, 128, 4, 512, 128, fp8=True, fmt=fp8_format)
     raise KeyError(name)

@@ -104,7 +104,6 @@ def dq_call(L, **kw):
     (dict(ps=0), 1, "page_size < 1"),
     (dict(d=0), 1, "head_dim < 1"),
     (dict(n=-1), 1, "n_page_ids < 0"),
-    (dict(fmt=1), 2, "FNUZ"),
     (dict(fmt=7), 1, "fp8_format must be 0"),
     (dict(d=96), 2, "multiple of 64"),
     (dict(src=None), 1, "must be non-NULL"),
@@ -177,7 +176,6 @@ def attn8_call(L, **kw):
 
 
 @pytest.mark.parametrize("kw,status,clause", [
-    (dict(fmt=1), 2, "FNUZ"),
     (dict(fmt=3), 1, "fp8_format must be 0"),
     (dict(ptc=None), 1, "pt_cmp must be non-NULL"),
     (dict(ks=None), 1, "codes and scales"),

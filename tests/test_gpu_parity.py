@@ -29,9 +29,9 @@ def spa():
 
 
 @functools.lru_cache(maxsize=None)
-def workload(name, shrink=1):
+def workload(name, shrink=1, fp8_format=0):
     from sparse_paged_attention_build_b200 import workloads
-    return workloads.make(name, shrink=shrink)
+    return workloads.make(name, shrink=shrink, fp8_format=fp8_format)
 
 
 @functools.lru_cache(maxsize=None)
@@ -42,21 +42,21 @@ def oracle_sets(name, shrink=1):
 
 
 @functools.lru_cache(maxsize=None)
-def oracle_cmp_pools(name, shrink=1):
+def oracle_cmp_pools(name, shrink=1, fp8_format=0):
     import oracle
-    w = workload(name, shrink)
+    w = workload(name, shrink, fp8_format)
     if w.k_cmp_fp8 is None:
         return w.k_cmp, w.v_cmp
-    k = oracle.dequant_fp8_pages(w.k_cmp_fp8, w.k_cmp_scale, w.cmp_page_ids)
-    v = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids)
+    k = oracle.dequant_fp8_pages(w.k_cmp_fp8, w.k_cmp_scale, w.cmp_page_ids, fmt=fp8_format)
+    v = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids, fmt=fp8_format)
     return k, v
 
 
-def oracle_attn(name, shrink, rows):
+def oracle_attn(name, shrink, rows, fp8_format=0):
     import oracle
-    w = workload(name, shrink)
+    w = workload(name, shrink, fp8_format)
     ip, idx = oracle_sets(name, shrink)
-    k_cmp, v_cmp = oracle_cmp_pools(name, shrink)
+    k_cmp, v_cmp = oracle_cmp_pools(name, shrink, fp8_format)
     return oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, w.sink, w.scale,
                                    k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp,
                                    rows=None if rows is None else np.asarray(rows, dtype=np.int32))
@@ -377,6 +377,46 @@ def test_fused_fp8_mixed_groups_and_faults(spa):
     fus.step()
     torch.cuda.synchronize()
     assert fus.status_word() == 0
+
+
+def test_dequant_fnuz_every_code(spa):
+    import oracle
+    P, ps, d = 4, 16, 128
+    src = (np.arange(P * ps * d, dtype=np.int64).reshape(P, ps, d) % 256).astype(np.uint8)
+    rng = np.random.default_rng(5)
+    scales = (rng.random((P, ps, d // 64)) * 4).astype(np.float32)
+    ids = np.array([0, 1, 3], dtype=np.int32)
+    ref = oracle.dequant_fp8_pages(src, scales, ids, fmt=1)
+    dst = torch.zeros((P, ps, d), dtype=torch.bfloat16, device="cuda")
+    st = spa.new_status()
+    spa.dequant_fp8_pages(torch.from_numpy(src).cuda(), torch.from_numpy(scales).cuda(),
+                          torch.from_numpy(ids).cuda(), dst, fp8_format=1, dev_status=st)
+    got = dst.view(torch.int16).cpu().numpy().view(np.uint16)
+    nan_ref = (ref & 0x7fff) > 0x7f80
+    nan_got = (got & 0x7fff) > 0x7f80
+    assert np.array_equal(nan_ref, nan_got)
+    assert np.array_equal(got[~nan_ref], ref[~nan_ref])
+    assert spa.read_status(st) == 0
+
+
+def test_fused_fp8_fnuz_bit_identical_and_against_oracle(spa):
+    """The mixed cache encoded as E4M3 FNUZ: page decode and fused gather
+    give identical results, within tolerance of the oracle."""
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    w = workload("c5", 16, 1)
+    assert w.fp8_format == 1
+    dec = DeviceBatch(w, fp8_path="decode")
+    fus = DeviceBatch(w, fp8_path="fused")
+    dec.step()
+    fus.step()
+    torch.cuda.synchronize()
+    assert dec.status_word() == 0 and fus.status_word() == 0
+    k_ref, _ = oracle_cmp_pools("c5", 16, 1)
+    got = dec.k_cmp.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, k_ref)
+    assert_bit_identical(dec.out, dec.lse, fus.out, fus.lse, "FNUZ")
+    O, L = oracle_attn("c5", 16, None, 1)
+    check_attn(fus.out, fus.lse, O, L, "fused FNUZ")
 
 
 def test_graph_capture_and_two_streams(spa):
