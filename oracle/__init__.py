@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
             L.oracle_dequant_fp8_pages_fmt.restype = ctypes.c_int
             L.oracle_e4m3fnuz_to_double.argtypes = [ctypes.c_uint8]
             L.oracle_e4m3fnuz_to_double.restype = dbl
+            L.oracle_paged_kv_write.argtypes = [P, P, i32, i32, P, P, P, i32, i32, i32, i64, P, P]
+            L.oracle_paged_kv_write.restype = ctypes.c_int
             L.oracle_sparse_sink_attn.argtypes = [
                 P, i64, i64, i32, i32, i32,
                 P, P, i64, i32, P, i32,
@@ -226,3 +228,22 @@ def lse_merge(lse_parts, o_parts):
     lse = np.zeros(1, dtype=np.float64)
     lib().oracle_lse_merge(S, _ptr(lse_parts), _ptr(o_parts), d, _ptr(o), _ptr(lse))
     return o, float(lse[0])
+
+
+def paged_kv_write(k_new, v_new, req, pos, pt, k_pool, v_pool):
+    """Copies of the pools (uint16 BF16 bits [pages, page_size, d]) with token
+    j's rows written at pt[req[j]][pos[j] // ps] * ps + pos[j] % ps, and the
+    fault flags (2: bad request/position, 1: bad page; 0: none)."""
+    k_new = _c(k_new, np.uint16)
+    v_new = _c(v_new, np.uint16)
+    req = _c(req, np.int32)
+    pos = _c(pos, np.int32)
+    pt = _c(pt, np.int32)
+    k_out = np.array(k_pool, dtype=np.uint16, copy=True, order="C")
+    v_out = np.array(v_pool, dtype=np.uint16, copy=True, order="C")
+    P, ps, d = k_out.shape
+    n = k_new.shape[0]
+    flags = lib().oracle_paged_kv_write(_ptr(k_new), _ptr(v_new), n, d, _ptr(req), _ptr(pos), _ptr(pt),
+                                        pt.shape[1], pt.shape[0], ps, P, _ptr(k_out), _ptr(v_out))
+    return k_out, v_out, flags
+

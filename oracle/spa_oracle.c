@@ -235,6 +235,39 @@ int oracle_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t nu
 }
 
 /* ------------------------------------------------------------------------ */
+/* Paged KV write.                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Token j (request req[j], position pos[j]) copies its d-element K and V
+ * rows (BF16 bits) into row pt[req][pos / page_size] * page_size +
+ * pos % page_size of the pools. A token whose request, position or page is
+ * out of range is skipped; the return value ORs 2 (bad request/position)
+ * and 1 (bad page) for the skipped ones, 0 when none was. */
+int oracle_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n, int32_t d,
+                          const int32_t* req, const int32_t* pos, const int32_t* pt, int32_t pt_cols,
+                          int32_t n_requests, int32_t page_size, int64_t num_pages,
+                          uint16_t* k_pool, uint16_t* v_pool)
+{
+    int flags = 0;
+    for (int32_t j = 0; j < n; ++j) {
+        int32_t b = req[j], t = pos[j];
+        if (b < 0 || b >= n_requests || t < 0 || t / page_size >= pt_cols) {
+            flags |= 2;
+            continue;
+        }
+        int64_t page = pt[(int64_t)b * pt_cols + t / page_size];
+        if (page < 0 || page >= num_pages) {
+            flags |= 1;
+            continue;
+        }
+        int64_t row = page * page_size + t % page_size;
+        memcpy(k_pool + row * d, k_new + (int64_t)j * d, (size_t)d * sizeof(uint16_t));
+        memcpy(v_pool + row * d, v_new + (int64_t)j * d, (size_t)d * sizeof(uint16_t));
+    }
+    return flags;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Attention with an attention sink.                                         */
 /* ------------------------------------------------------------------------ */
 
