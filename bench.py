@@ -235,6 +235,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
                     help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
+    ap.add_argument("--op", default="path", choices=["path", "kv_write"],
+                    help="path: the attention hot path (the bench line); kv_write: the paged KV write alone")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=0)
@@ -246,6 +248,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.op == "kv_write":
+        return run_kv_write(args, rank, local_rank, world)
 
     import torch
     import torch.distributed as dist
@@ -381,6 +385,73 @@ def main():
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_kv_write(args, rank, local_rank, world):
+    """The paged KV write alone: the workload's new tokens (every token of a
+    prefill batch, the last token of each decode request) written into the
+    raw window pools through the page table; HBM GB/s against the copy peak.
+    The rows written are the ones the pools already hold, so the pools keep
+    their contents."""
+    import torch
+    import torch.distributed as dist
+    from sparse_paged_attention_build_b200 import workloads
+    import sparse_paged_attention_build_b200 as spa
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    w = workloads.make(args.workload, shrink=args.shrink, seed_offset=rank)
+    ps = w.raw_page_size
+    rows = w.pt_raw[w.req, w.pos // ps].astype(np.int64) * ps + w.pos % ps
+    k_new = w.k_raw.reshape(-1, w.d)[rows]
+    v_new = w.v_raw.reshape(-1, w.d)[rows]
+    dev = lambda a, dt=None: torch.from_numpy(np.ascontiguousarray(a)).cuda() if dt is None else \
+        torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(dt)
+    bf = torch.bfloat16
+    kn, vn = dev(k_new, bf), dev(v_new, bf)
+    kp, vp = dev(w.k_raw, bf), dev(w.v_raw, bf)
+    req, pos, pt = dev(w.req), dev(w.pos), dev(w.pt_raw)
+    st = spa.new_status()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            spa.paged_kv_write(kn, vn, req, pos, pt, kp, vp, dev_status=st)
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(args.warmup):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()   # new tokens and pools come from HBM
+        e0.record()
+        g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in evs]))
+    n = len(rows)
+    bytes_step = n * 2 * (2 * w.d * 2) + 2 * n * 4 + w.pt_raw.nbytes   # rows read + written, req/pos, table
+    total_bytes, ms = job_totals(bytes_step, ms, world, "cuda")
+    pk, pk_kind = peaks()
+    gbs = total_bytes / (ms / 1e3) / 1e9
+    ok = np.array_equal(kp.view(torch.int16).cpu().numpy().view(np.uint16), w.k_raw) and spa.read_status(st) == 0
+    if rank == 0:
+        print(json.dumps({
+            "metric": "paged KV write HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: {workloads.DESCRIPTIONS[w.name]}", "tokens_written": int(n),
+                       "l2": "256 MB buffer written between timed steps (L2 flush)"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_kind} HBM copy",
+                         "kernel": "paged_kv_write_kernel", "algorithmic_bytes": int(bytes_step)},
+            "gpu_launches": args.steps, "pools_unchanged": bool(ok)}))
     if world > 1:
         dist.destroy_process_group()
     return 0

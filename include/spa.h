@@ -238,6 +238,32 @@ int spa_sparse_sink_attn_fwd(
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * 4. spa_paged_kv_write -- new raw tokens into the paged window cache.
+ *
+ * Defined by "test: add block-level DeepSeek-V4 attention test", decode
+ * kernel timeline and notes (the paged KV write, "swa_write" / "kvw_paged",
+ * runs ahead of the sparse attention core); without the qk-norm and RoPE
+ * the model fuses into it. Token j, of request b = req[j] at position
+ * t = pos[j], is copied to row pt[b][t / page_size] * page_size +
+ * t % page_size of k_pool and of v_pool.
+ *
+ * k_new, v_new  BF16 [n_tokens, head_dim] contiguous, 16-B aligned
+ * head_dim      a multiple of 8
+ * req, pos      int32 [n_tokens]; a request outside [0, n_requests) or a
+ *               position outside the table sets SPA_DEV_BAD_INDEX, a page id
+ *               outside [0, num_pages) SPA_DEV_BAD_PAGE; the token is skipped
+ * pt            int32 [n_requests, pt_cols] (the raw page table)
+ * page_size     power of two, 1 .. 1024
+ * k_pool, v_pool BF16 [num_pages, page_size, head_dim], 16-B aligned
+ * Rows not named by a token are left as they are; two tokens naming the
+ * same row leave one of them there (which one is unspecified).
+ * ---------------------------------------------------------------------- */
+int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_tokens, int32_t head_dim,
+                       const int32_t* req, const int32_t* pos, const int32_t* pt, int32_t pt_cols,
+                       int32_t n_requests, int32_t page_size, int64_t num_pages, uint16_t* k_pool,
+                       uint16_t* v_pool, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * 3b. spa_sparse_sink_attn_fwd_fp8 -- the same attention over a mixed
  * cache whose compressed pool is stored in FP8, decoded inside the gather.
  *

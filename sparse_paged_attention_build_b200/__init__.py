@@ -71,6 +71,8 @@ def _load():
         P, P, P, P, i64, i32, P, i32, i32,
         P, i32, P, P, P, ctypes.c_float, P, P, i32, P, sz, P, P]
     L.spa_sparse_sink_attn_fwd_fp8.restype = ctypes.c_int
+    L.spa_paged_kv_write.argtypes = [P, P, i32, i32, P, P, P, i32, i32, i32, i64, P, P, P, P]
+    L.spa_paged_kv_write.restype = ctypes.c_int
     return L
 
 
@@ -267,3 +269,21 @@ def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
     return out, lse
+
+
+def paged_kv_write(k_new, v_new, req, pos, pt, k_pool, v_pool, dev_status=None, stream=None):
+    """Write token j's K and V rows (bf16 [n, d]) to row pt[req[j]][pos[j] //
+    page_size] * page_size + pos[j] % page_size of the pools (bf16
+    [pages, page_size, d])."""
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_pool", k_pool), ("v_pool", v_pool)):
+        _need(t, name, torch.bfloat16)
+        assert t.is_contiguous(), name
+    for name, t in (("req", req), ("pos", pos), ("pt", pt)):
+        _need(t, name, torch.int32)
+    n, d = k_new.shape
+    assert tuple(v_new.shape) == (n, d) and k_pool.shape == v_pool.shape and k_pool.shape[2] == d
+    pt = pt.contiguous()
+    _check("spa_paged_kv_write", lib.spa_paged_kv_write(
+        _p(k_new), _p(v_new), n, d, _p(req.contiguous()), _p(pos.contiguous()), _p(pt), pt.shape[1], pt.shape[0],
+        k_pool.shape[1], k_pool.shape[0], _p(k_pool), _p(v_pool), _p(dev_status), _stream(stream)))
+

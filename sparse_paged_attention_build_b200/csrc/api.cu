@@ -197,6 +197,29 @@ int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int
   return static_cast<int>(s);
 }
 
+int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_tokens, int32_t head_dim,
+                       const int32_t* req, const int32_t* pos, const int32_t* pt, int32_t pt_cols,
+                       int32_t n_requests, int32_t page_size, int64_t num_pages, uint16_t* k_pool,
+                       uint16_t* v_pool, uint32_t* dev_status, spa_stream_t stream) {
+  if (n_tokens < 0) return fail(SPA_ERR_INVALID_ARG, "n_tokens < 0");
+  if (head_dim < 8 || head_dim % 8 != 0) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
+  if (n_requests < 1 || pt_cols < 1) return fail(SPA_ERR_INVALID_ARG, "n_requests and pt_cols must be >= 1");
+  if (num_pages < 0) return fail(SPA_ERR_INVALID_ARG, "num_pages < 0");
+  if (!pow2_in(page_size, 1, 1024)) return fail(SPA_ERR_UNSUPPORTED, "page_size must be a power of two <= 1024");
+  if (n_tokens == 0) return ok();
+  if (k_new == nullptr || v_new == nullptr || req == nullptr || pos == nullptr || pt == nullptr ||
+      k_pool == nullptr || v_pool == nullptr)
+    return fail(SPA_ERR_INVALID_ARG, "k_new, v_new, req, pos, pt and the pools must be non-NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16))
+    return fail(SPA_ERR_ALIGNMENT, "rows and pools must be 16-byte aligned");
+  if (!aligned(req, 4) || !aligned(pos, 4) || !aligned(pt, 4))
+    return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
+  return cuda_status(spa::launch_paged_kv_write(k_new, v_new, n_tokens, head_dim, req, pos, pt, pt_cols, n_requests,
+                                                page_size, num_pages, k_pool, v_pool, dev_status,
+                                                reinterpret_cast<cudaStream_t>(stream)),
+                     "paged_kv_write launch");
+}
+
 size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                                            int32_t num_splits) {
   if (n_queries <= 0 || num_heads <= 0 || head_dim <= 0 || num_splits < 0) return 0;

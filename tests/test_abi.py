@@ -193,3 +193,30 @@ def test_guard_matrix_attention_fp8(L, kw, status, clause):
 
 def test_attention_fp8_zero_queries_is_a_no_op(L):
     assert attn8_call(L, n=0, q=None, out=None, lse=None, k8=None, v8=None, ks=None, vs=None) == 0
+
+
+def kvw_call(L, **kw):
+    a = dict(kn=FAKE, vn=FAKE, n=4, d=128, req=FAKE, pos=FAKE, pt=FAKE, cols=4, B=2, ps=64, P=10,
+             kp=FAKE, vp=FAKE)
+    a.update(kw)
+    return L.spa_paged_kv_write(a["kn"], a["vn"], a["n"], a["d"], a["req"], a["pos"], a["pt"], a["cols"], a["B"],
+                                a["ps"], a["P"], a["kp"], a["vp"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(n=-1), 1, "n_tokens < 0"),
+    (dict(d=12), 2, "multiple of 8"),
+    (dict(B=0), 1, "n_requests and pt_cols"),
+    (dict(P=-1), 1, "num_pages < 0"),
+    (dict(ps=48), 2, "page_size must be a power of two"),
+    (dict(pt=None), 1, "must be non-NULL"),
+    (dict(kp=FAKE + 4), 5, "16-byte aligned"),
+    (dict(pos=FAKE + 2), 5, "4-byte aligned"),
+])
+def test_guard_matrix_kv_write(L, kw, status, clause):
+    assert kvw_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def test_kv_write_zero_tokens_is_a_no_op(L):
+    assert kvw_call(L, n=0, kn=None, vn=None) == 0

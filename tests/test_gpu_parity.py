@@ -419,6 +419,36 @@ def test_fused_fp8_fnuz_bit_identical_and_against_oracle(spa):
     check_attn(fus.out, fus.lse, O, L, "fused FNUZ")
 
 
+# ------------------------------------------------------------------ paged KV write
+def test_paged_kv_write_bit_exact_and_faults(spa):
+    import oracle
+    rng = np.random.default_rng(11)
+    P, ps, d, B, cols = 40, 64, 128, 3, 8
+    pt = rng.permutation(P)[: B * cols].reshape(B, cols).astype(np.int32)
+    k_pool = rng.integers(0, 1 << 16, size=(P, ps, d), dtype=np.uint16)
+    v_pool = rng.integers(0, 1 << 16, size=(P, ps, d), dtype=np.uint16)
+    flat = rng.choice(B * cols * ps, size=500, replace=False)
+    req = (flat // (cols * ps)).astype(np.int32)
+    pos = (flat % (cols * ps)).astype(np.int32)
+    req[0] = 9                                   # faulty request
+    k_new = rng.integers(0, 1 << 16, size=(500, d), dtype=np.uint16)
+    v_new = rng.integers(0, 1 << 16, size=(500, d), dtype=np.uint16)
+    k_ref, v_ref, flags = oracle.paged_kv_write(k_new, v_new, req, pos, pt, k_pool, v_pool)
+    assert flags == 2
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+
+    kp, vp = dev_bf16(k_pool).clone(), dev_bf16(v_pool).clone()
+    st = spa.new_status()
+    spa.paged_kv_write(dev_bf16(k_new), dev_bf16(v_new), torch.from_numpy(req).cuda(),
+                       torch.from_numpy(pos).cuda(), torch.from_numpy(pt).cuda(), kp, vp, dev_status=st)
+    torch.cuda.synchronize()
+    assert spa.read_status(st) == spa.DEV_BAD_INDEX
+    assert np.array_equal(kp.view(torch.int16).cpu().numpy().view(np.uint16), k_ref)
+    assert np.array_equal(vp.view(torch.int16).cpu().numpy().view(np.uint16), v_ref)
+
+
 def test_graph_capture_and_two_streams(spa):
     """The three calls capture into a CUDA graph; replays and a second
     stream give bit-identical results."""
