@@ -17,6 +17,9 @@ What each function follows (page title, then section):
 * :func:`sparse_sink_attn` -- "Roadmap item 24", "Reuse and arithmetic"
   (one denominator for compressed KV, window and sink; the sink has no V;
   natural-log LSE) and "MI300X validation" (an FP64 O/LSE oracle).
+* :func:`sparse_sink_attn_bwd` -- "Roadmap item 24", the backward named as
+  its follow-on item (dQ, dK/dV, d_sink): the chain rule through the forward
+  above, with the sink's logit carrying no V.
 * :func:`lse_merge` -- "[WS2] Add CP-aware Attention contract and dispatch
   metadata", "Summary" (deterministic (out, lse) merge) and "docs: Block
   AttnRes model + ROCm-first plan", "Summary" (attn-with-stats +
@@ -91,6 +94,12 @@ def lib() -> ctypes.CDLL:
                 P, P, i64, i32, P, i32,
                 P, i32, P, P, P, dbl, i32, P, i32, P, P, i32]
             L.oracle_sparse_sink_attn.restype = ctypes.c_int
+            L.oracle_sparse_sink_attn_bwd.argtypes = [
+                P, i64, i64, i32, i32, i32,
+                P, P, i64, i32, P, i32,
+                P, P, i64, i32, P, i32,
+                P, i32, P, P, P, dbl, P, P, i32, P, P, P, P, P, P, i32]
+            L.oracle_sparse_sink_attn_bwd.restype = ctypes.c_int
             L.oracle_lse_merge.argtypes = [i32, P, P, i32, P, P]
             L.oracle_lse_merge.restype = None
             _lib = L
@@ -217,6 +226,48 @@ def sparse_sink_attn(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale,
         _ptr(req), pt_raw.shape[0], _ptr(indptr), _ptr(indices), _ptr(sink), float(scale),
         1 if include_sink else 0, _ptr(rows), n_rows, _ptr(out), _ptr(lse), int(threads)))
     return out, lse
+
+
+def sparse_sink_attn_bwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale, dout,
+                         k_cmp=None, v_cmp=None, pt_cmp=None, rows=None, threads=None):
+    """FP64 gradients of sum(dout * O) from the exact forward.
+
+    Returns (dq [n_rows, H, d], dk_raw, dv_raw, dk_cmp, dv_cmp, dsink [H]);
+    dk/dv are shaped like their pools ([pages, page_size, d]) and hold the
+    contributions of the given query tokens only (all of them when rows is
+    None); dk_cmp/dv_cmp are None without a compressed pool and dsink is
+    None without a sink. dout: BF16 bits [N, H, d].
+    """
+    q = np.asarray(q)
+    assert q.dtype == np.uint16 and q.ndim == 3 and q.strides[2] == 2
+    N, H, d = q.shape
+    k_raw, v_raw = _c(k_raw, np.uint16), _c(v_raw, np.uint16)
+    pt_raw = _c(pt_raw, np.int32)
+    if pt_cmp is not None:
+        k_cmp, v_cmp, pt_cmp = _c(k_cmp, np.uint16), _c(v_cmp, np.uint16), _c(pt_cmp, np.int32)
+    req, indptr, indices = _c(req, np.int32), _c(indptr, np.int32), _c(indices, np.int32)
+    sink = _c(sink, np.float32)
+    dout = _c(dout, np.uint16)
+    assert dout.shape == (N, H, d)
+    rows = None if rows is None else _c(rows, np.int32)
+    n_rows = N if rows is None else rows.shape[0]
+    dq = np.zeros((n_rows, H, d), dtype=np.float64)
+    dk_raw = np.zeros(k_raw.shape, dtype=np.float64)
+    dv_raw = np.zeros(v_raw.shape, dtype=np.float64)
+    dk_cmp = None if k_cmp is None else np.zeros(k_cmp.shape, dtype=np.float64)
+    dv_cmp = None if v_cmp is None else np.zeros(v_cmp.shape, dtype=np.float64)
+    dsink = None if sink is None else np.zeros(H, dtype=np.float64)
+    threads = threads or os.cpu_count() or 1
+    _check(lib().oracle_sparse_sink_attn_bwd(
+        _ptr(q), q.strides[0] // 2, q.strides[1] // 2, N, H, d,
+        _ptr(k_raw), _ptr(v_raw), k_raw.shape[0], k_raw.shape[1], _ptr(pt_raw), pt_raw.shape[1],
+        _ptr(k_cmp), _ptr(v_cmp), 0 if k_cmp is None else k_cmp.shape[0],
+        1 if k_cmp is None else k_cmp.shape[1], _ptr(pt_cmp),
+        0 if pt_cmp is None else pt_cmp.shape[1],
+        _ptr(req), pt_raw.shape[0], _ptr(indptr), _ptr(indices), _ptr(sink), float(scale),
+        _ptr(dout), _ptr(rows), n_rows, _ptr(dq), _ptr(dk_raw), _ptr(dv_raw), _ptr(dk_cmp),
+        _ptr(dv_cmp), _ptr(dsink), int(threads)))
+    return dq, dk_raw, dv_raw, dk_cmp, dv_cmp, dsink
 
 
 def lse_merge(lse_parts, o_parts):

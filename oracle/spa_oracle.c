@@ -446,3 +446,182 @@ void oracle_lse_merge(int32_t n_parts, const double* lse_parts, const double* o_
         for (int32_t e = 0; e < d; ++e) o[e] += w * o_parts[(int64_t)s * d + e];
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the attention with sink.                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Gradients of L = sum over (i, h, e) of dO[i,h,e] * O[i,h,e] for the query
+ * tokens rows[0..n_rows) (all N when rows is NULL), in FP64, from the exact
+ * forward of the same inputs. "Roadmap item 24 - joint compressed/window
+ * attention with sink" names the backward (dQ, dK/dV, d_sink) as its
+ * follow-on item; the formulas are the chain rule through the forward
+ * above. For one (i, h) with logits s_j = scale q.k_j and the sink c_h:
+ *   p_j = e^{s_j - LSE}, p_c = e^{c_h - LSE}, O = sum_j p_j v_j,
+ *   D = dO . O, dp_j = dO . v_j, ds_j = p_j (dp_j - D),
+ *   dq = scale sum_j ds_j k_j, dk_j += scale ds_j q, dv_j += p_j dO,
+ *   dsink_h += -p_c D (the sink's logit has no V, so its dp is 0).
+ * dq is written ([n_rows, H, d]); dk/dv are ADDED into arrays shaped like
+ * the pools ([pages * page_size, d]); dsink (may be NULL) is added into. */
+typedef struct {
+    attn_job A;
+    const uint16_t* dout;            /* BF16 bits [N, H, d], contiguous */
+    double *dq, *dk_raw, *dv_raw, *dk_cmp, *dv_cmp, *dsink;
+} bwd_job;
+
+static int one_query_bwd(bwd_job* G, int32_t r, double* kbuf, double* vbuf, double* s,
+                         double* dkb, double* dvb, int64_t* rowb, int* rawb, double* dsink_loc)
+{
+    const attn_job* J = &G->A;
+    int32_t i = J->rows ? J->rows[r] : r;
+    int32_t d = J->d, H = J->H;
+    if (i < 0 || i >= J->N) return ORACLE_BAD_INDEX;
+    int32_t b = J->req[i];
+    if (b < 0 || b >= J->B) return ORACLE_BAD_INDEX;
+    int32_t j0 = J->indptr[i], n = J->indptr[i + 1] - J->indptr[i];
+    for (int32_t j = 0; j < n; ++j) {
+        const uint16_t *kr, *vr;
+        int32_t key = J->indices[j0 + j];
+        int st = locate(J, b, key, &kr, &vr);
+        if (st) return st;
+        rawb[j] = (key & ORACLE_WINDOW_TAG) != 0;
+        rowb[j] = (kr - (rawb[j] ? J->k_raw : J->k_cmp)) / d;
+        for (int32_t e = 0; e < d; ++e) {
+            kbuf[(int64_t)j * d + e] = oracle_bf16_to_double(kr[e]);
+            vbuf[(int64_t)j * d + e] = oracle_bf16_to_double(vr[e]);
+            dkb[(int64_t)j * d + e] = 0.0;
+            dvb[(int64_t)j * d + e] = 0.0;
+        }
+    }
+    double* p = s + n;               /* [n] */
+    for (int32_t h = 0; h < H; ++h) {
+        const uint16_t* qh = J->q + (int64_t)i * J->q_stride_tok + (int64_t)h * J->q_stride_head;
+        const uint16_t* doh = G->dout + ((int64_t)i * H + h) * d;
+        double* dq = G->dq + ((int64_t)r * H + h) * d;
+        double sink = J->sink ? (double)J->sink[h] : -INFINITY;
+        for (int32_t e = 0; e < d; ++e) dq[e] = 0.0;
+        /* the forward: logits, max, denominator, LSE */
+        double m = sink;
+        for (int32_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int32_t e = 0; e < d; ++e)
+                acc += oracle_bf16_to_double(qh[e]) * kbuf[(int64_t)j * d + e];
+            s[j] = J->scale * acc;
+            if (s[j] > m) m = s[j];
+        }
+        if (m == -INFINITY) continue;            /* no keys, no sink: O = 0, no gradient */
+        double l = exp(sink - m);
+        for (int32_t j = 0; j < n; ++j) l += exp(s[j] - m);
+        double lse = m + log(l);
+        /* probabilities, O and D = dO . O */
+        double D = 0.0;
+        for (int32_t j = 0; j < n; ++j) p[j] = exp(s[j] - lse);
+        for (int32_t e = 0; e < d; ++e) {
+            double o = 0.0;
+            for (int32_t j = 0; j < n; ++j) o += p[j] * vbuf[(int64_t)j * d + e];
+            D += oracle_bf16_to_double(doh[e]) * o;
+        }
+        for (int32_t j = 0; j < n; ++j) {
+            double dp = 0.0;
+            for (int32_t e = 0; e < d; ++e)
+                dp += oracle_bf16_to_double(doh[e]) * vbuf[(int64_t)j * d + e];
+            double ds = p[j] * (dp - D);
+            for (int32_t e = 0; e < d; ++e) {
+                dq[e] += J->scale * ds * kbuf[(int64_t)j * d + e];
+                dkb[(int64_t)j * d + e] += J->scale * ds * oracle_bf16_to_double(qh[e]);
+                dvb[(int64_t)j * d + e] += p[j] * oracle_bf16_to_double(doh[e]);
+            }
+        }
+        if (J->sink) dsink_loc[h] += -exp(sink - lse) * D;
+    }
+    return ORACLE_OK;
+}
+
+static void* bwd_worker(void* arg)
+{
+    bwd_job* G = (bwd_job*)arg;
+    attn_job* J = &G->A;
+    int32_t cap = 0, d = J->d;
+    double *kbuf = NULL, *vbuf = NULL, *s = NULL, *dkb = NULL, *dvb = NULL;
+    int64_t* rowb = NULL; int* rawb = NULL;
+    double* dsink_loc = (double*)calloc((size_t)J->H, sizeof(double));
+    if (!dsink_loc) { pthread_mutex_lock(&J->lock); J->status = ORACLE_NO_MEMORY; pthread_mutex_unlock(&J->lock); return NULL; }
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int32_t r = J->status ? J->n_rows : J->next_row++;
+        pthread_mutex_unlock(&J->lock);
+        if (r >= J->n_rows) break;
+        int32_t i = J->rows ? J->rows[r] : r;
+        int32_t n = (i >= 0 && i < J->N) ? J->indptr[i + 1] - J->indptr[i] : 0;
+        if (n < 0) n = 0;
+        if (n + 1 > cap) {
+            cap = n + 1;
+            free(kbuf); free(vbuf); free(s); free(dkb); free(dvb); free(rowb); free(rawb);
+            kbuf = (double*)malloc((size_t)cap * d * sizeof(double));
+            vbuf = (double*)malloc((size_t)cap * d * sizeof(double));
+            dkb = (double*)malloc((size_t)cap * d * sizeof(double));
+            dvb = (double*)malloc((size_t)cap * d * sizeof(double));
+            s = (double*)malloc((size_t)cap * 2 * sizeof(double));
+            rowb = (int64_t*)malloc((size_t)cap * sizeof(int64_t));
+            rawb = (int*)malloc((size_t)cap * sizeof(int));
+            if (!kbuf || !vbuf || !s || !dkb || !dvb || !rowb || !rawb) {
+                pthread_mutex_lock(&J->lock); J->status = ORACLE_NO_MEMORY;
+                pthread_mutex_unlock(&J->lock); break;
+            }
+        }
+        int st = one_query_bwd(G, r, kbuf, vbuf, s, dkb, dvb, rowb, rawb, dsink_loc);
+        pthread_mutex_lock(&J->lock);
+        if (st) {
+            if (!J->status) J->status = st;
+        } else {
+            /* this query's key-row gradients into the pool-shaped sums */
+            for (int32_t j = 0; j < n; ++j) {
+                double* dk = (rawb[j] ? G->dk_raw : G->dk_cmp) + rowb[j] * d;
+                double* dv = (rawb[j] ? G->dv_raw : G->dv_cmp) + rowb[j] * d;
+                for (int32_t e = 0; e < d; ++e) {
+                    dk[e] += dkb[(int64_t)j * d + e];
+                    dv[e] += dvb[(int64_t)j * d + e];
+                }
+            }
+        }
+        pthread_mutex_unlock(&J->lock);
+    }
+    pthread_mutex_lock(&J->lock);
+    if (G->dsink)
+        for (int32_t h = 0; h < J->H; ++h) G->dsink[h] += dsink_loc[h];
+    pthread_mutex_unlock(&J->lock);
+    free(kbuf); free(vbuf); free(s); free(dkb); free(dvb); free(rowb); free(rawb); free(dsink_loc);
+    return NULL;
+}
+
+int oracle_sparse_sink_attn_bwd(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t N, int32_t H,
+    int32_t d, const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_pages,
+    int32_t raw_ps, const int32_t* pt_raw, int32_t pt_raw_cols, const uint16_t* k_cmp,
+    const uint16_t* v_cmp, int64_t cmp_pages, int32_t cmp_ps, const int32_t* pt_cmp,
+    int32_t pt_cmp_cols, const int32_t* req, int32_t B, const int32_t* indptr,
+    const int32_t* indices, const float* sink, double scale, const uint16_t* dout,
+    const int32_t* rows, int32_t n_rows, double* dq, double* dk_raw, double* dv_raw,
+    double* dk_cmp, double* dv_cmp, double* dsink, int32_t n_threads)
+{
+    if (N < 0 || H < 1 || d < 1 || raw_ps < 1 || (pt_cmp && cmp_ps < 1) || n_rows < 0 || !dout)
+        return ORACLE_BAD_ARG;
+    if (pt_cmp && (!dk_cmp || !dv_cmp)) return ORACLE_BAD_ARG;
+    bwd_job G;
+    attn_job A = {q, q_stride_tok, q_stride_head, N, H, d, k_raw, v_raw, raw_pages, raw_ps,
+                  pt_raw, pt_raw_cols, k_cmp, v_cmp, cmp_pages, cmp_ps, pt_cmp, pt_cmp_cols,
+                  req, B, indptr, indices, sink, scale, 1, rows, n_rows, NULL, NULL,
+                  0, PTHREAD_MUTEX_INITIALIZER, 0};
+    G.A = A;
+    G.dout = dout; G.dq = dq; G.dk_raw = dk_raw; G.dv_raw = dv_raw;
+    G.dk_cmp = dk_cmp; G.dv_cmp = dv_cmp; G.dsink = dsink;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    pthread_t tid[256];
+    int started = 0;
+    for (int t = 1; t < n_threads; ++t)
+        if (pthread_create(&tid[started], NULL, bwd_worker, &G) == 0) ++started;
+    bwd_worker(&G);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    return G.A.status;
+}
