@@ -98,7 +98,7 @@ def lib() -> ctypes.CDLL:
                 P, i64, i64, i32, i32, i32,
                 P, P, i64, i32, P, i32,
                 P, P, i64, i32, P, i32,
-                P, i32, P, P, P, dbl, P, P, i32, P, P, P, P, P, P, i32]
+                P, i32, P, P, P, dbl, P, P, P, P, i32, P, P, P, P, P, P, i32]
             L.oracle_sparse_sink_attn_bwd.restype = ctypes.c_int
             L.oracle_lse_merge.argtypes = [i32, P, P, i32, P, P]
             L.oracle_lse_merge.restype = None
@@ -229,8 +229,11 @@ def sparse_sink_attn(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale,
 
 
 def sparse_sink_attn_bwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale, dout,
-                         k_cmp=None, v_cmp=None, pt_cmp=None, rows=None, threads=None):
-    """FP64 gradients of sum(dout * O) from the exact forward.
+                         k_cmp=None, v_cmp=None, pt_cmp=None, rows=None, threads=None,
+                         o_saved=None, lse_saved=None):
+    """FP64 gradients of sum(dout * O) from the exact forward, or from saved
+    forward results: o_saved [N, H, d] (for D = dO . O) and lse_saved [N, H]
+    (for the probabilities), FP64 arrays, each optional.
 
     Returns (dq [n_rows, H, d], dk_raw, dv_raw, dk_cmp, dv_cmp, dsink [H]);
     dk/dv are shaped like their pools ([pages, page_size, d]) and hold the
@@ -249,6 +252,8 @@ def sparse_sink_attn_bwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
     sink = _c(sink, np.float32)
     dout = _c(dout, np.uint16)
     assert dout.shape == (N, H, d)
+    o_saved = None if o_saved is None else _c(o_saved, np.float64).reshape(N, H, d)
+    lse_saved = None if lse_saved is None else _c(lse_saved, np.float64).reshape(N, H)
     rows = None if rows is None else _c(rows, np.int32)
     n_rows = N if rows is None else rows.shape[0]
     dq = np.zeros((n_rows, H, d), dtype=np.float64)
@@ -265,7 +270,7 @@ def sparse_sink_attn_bwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
         1 if k_cmp is None else k_cmp.shape[1], _ptr(pt_cmp),
         0 if pt_cmp is None else pt_cmp.shape[1],
         _ptr(req), pt_raw.shape[0], _ptr(indptr), _ptr(indices), _ptr(sink), float(scale),
-        _ptr(dout), _ptr(rows), n_rows, _ptr(dq), _ptr(dk_raw), _ptr(dv_raw), _ptr(dk_cmp),
+        _ptr(dout), _ptr(o_saved), _ptr(lse_saved), _ptr(rows), n_rows, _ptr(dq), _ptr(dk_raw), _ptr(dv_raw), _ptr(dk_cmp),
         _ptr(dv_cmp), _ptr(dsink), int(threads)))
     return dq, dk_raw, dv_raw, dk_cmp, dv_cmp, dsink
 

@@ -453,7 +453,10 @@ void oracle_lse_merge(int32_t n_parts, const double* lse_parts, const double* o_
 
 /* Gradients of L = sum over (i, h, e) of dO[i,h,e] * O[i,h,e] for the query
  * tokens rows[0..n_rows) (all N when rows is NULL), in FP64, from the exact
- * forward of the same inputs. "Roadmap item 24 - joint compressed/window
+ * forward of the same inputs, or, when o_saved / lse_saved are given
+ * ([N, H, d] and [N, H], FP64), from those saved forward results: D then
+ * takes O from o_saved and the probabilities take LSE from lse_saved, as a
+ * backward that reads the forward's stored outputs does. "Roadmap item 24 - joint compressed/window
  * attention with sink" names the backward (dQ, dK/dV, d_sink) as its
  * follow-on item; the formulas are the chain rule through the forward
  * above. For one (i, h) with logits s_j = scale q.k_j and the sink c_h:
@@ -466,6 +469,8 @@ void oracle_lse_merge(int32_t n_parts, const double* lse_parts, const double* o_
 typedef struct {
     attn_job A;
     const uint16_t* dout;            /* BF16 bits [N, H, d], contiguous */
+    const double* o_saved;           /* [N, H, d] or NULL */
+    const double* lse_saved;         /* [N, H] or NULL */
     double *dq, *dk_raw, *dv_raw, *dk_cmp, *dv_cmp, *dsink;
 } bwd_job;
 
@@ -512,13 +517,17 @@ static int one_query_bwd(bwd_job* G, int32_t r, double* kbuf, double* vbuf, doub
         if (m == -INFINITY) continue;            /* no keys, no sink: O = 0, no gradient */
         double l = exp(sink - m);
         for (int32_t j = 0; j < n; ++j) l += exp(s[j] - m);
-        double lse = m + log(l);
+        double lse = G->lse_saved ? G->lse_saved[(int64_t)i * H + h] : m + log(l);
         /* probabilities, O and D = dO . O */
         double D = 0.0;
         for (int32_t j = 0; j < n; ++j) p[j] = exp(s[j] - lse);
         for (int32_t e = 0; e < d; ++e) {
             double o = 0.0;
-            for (int32_t j = 0; j < n; ++j) o += p[j] * vbuf[(int64_t)j * d + e];
+            if (G->o_saved) {
+                o = G->o_saved[((int64_t)i * H + h) * d + e];
+            } else {
+                for (int32_t j = 0; j < n; ++j) o += p[j] * vbuf[(int64_t)j * d + e];
+            }
             D += oracle_bf16_to_double(doh[e]) * o;
         }
         for (int32_t j = 0; j < n; ++j) {
@@ -601,6 +610,7 @@ int oracle_sparse_sink_attn_bwd(
     const uint16_t* v_cmp, int64_t cmp_pages, int32_t cmp_ps, const int32_t* pt_cmp,
     int32_t pt_cmp_cols, const int32_t* req, int32_t B, const int32_t* indptr,
     const int32_t* indices, const float* sink, double scale, const uint16_t* dout,
+    const double* o_saved, const double* lse_saved,
     const int32_t* rows, int32_t n_rows, double* dq, double* dk_raw, double* dv_raw,
     double* dk_cmp, double* dv_cmp, double* dsink, int32_t n_threads)
 {
@@ -613,7 +623,7 @@ int oracle_sparse_sink_attn_bwd(
                   req, B, indptr, indices, sink, scale, 1, rows, n_rows, NULL, NULL,
                   0, PTHREAD_MUTEX_INITIALIZER, 0};
     G.A = A;
-    G.dout = dout; G.dq = dq; G.dk_raw = dk_raw; G.dv_raw = dv_raw;
+    G.dout = dout; G.o_saved = o_saved; G.lse_saved = lse_saved; G.dq = dq; G.dk_raw = dk_raw; G.dv_raw = dv_raw;
     G.dk_cmp = dk_cmp; G.dv_cmp = dv_cmp; G.dsink = dsink;
     if (n_threads < 1) n_threads = 1;
     if (n_threads > 256) n_threads = 256;

@@ -233,3 +233,61 @@ def test_empty_set_has_no_gradient(oracle):
     ip0 = np.zeros(N + 1, dtype=np.int32)
     dq, dkr, dvr, dkc, dvc, ds = _bwd(oracle, pr, ip0, idx[:0], _dout(pr, 6))
     assert np.all(dq == 0) and np.all(dkr == 0) and np.all(dvr == 0) and np.all(ds == 0)
+
+
+def _fwd(oracle, pr, ip, idx, v_raw=None, v_cmp=None):
+    return oracle.sparse_sink_attn(pr.q, pr.k_raw, pr.v_raw if v_raw is None else v_raw, pr.pt_raw, pr.req,
+                                   ip, idx, pr.sink, pr.scale, k_cmp=pr.k_cmp,
+                                   v_cmp=pr.v_cmp if v_cmp is None else v_cmp, pt_cmp=pr.pt_cmp, threads=2)
+
+
+def test_saved_results_equal_to_the_exact_ones_change_nothing(oracle):
+    pr = small_problem(seed=15, S=40, H=4, d=16)
+    ip, idx = _sets(oracle, pr)
+    dout = _dout(pr, 7)
+    O, L = _fwd(oracle, pr, ip, idx)
+    exact = _bwd(oracle, pr, ip, idx, dout)
+    saved = oracle.sparse_sink_attn_bwd(pr.q, pr.k_raw, pr.v_raw, pr.pt_raw, pr.req, ip, idx, pr.sink, pr.scale,
+                                        dout, k_cmp=pr.k_cmp, v_cmp=pr.v_cmp, pt_cmp=pr.pt_cmp, threads=2,
+                                        o_saved=O, lse_saved=L)
+    for a, b in zip(exact, saved):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+def test_saved_o_enters_only_through_d(oracle):
+    """O_saved = O + delta moves D by dO . delta, so dq moves by
+    -scale (dO . delta) sum_j p_j k_j (that sum is the forward with V := K),
+    dsink by -sum_i p_sink (dO . delta), and dv not at all."""
+    pr = small_problem(seed=16, S=40, H=4, d=16)
+    ip, idx = _sets(oracle, pr)
+    dout = _dout(pr, 8)
+    O, L = _fwd(oracle, pr, ip, idx)
+    delta = 1e-2 * np.random.default_rng(3).standard_normal(O.shape)
+    base = oracle.sparse_sink_attn_bwd(pr.q, pr.k_raw, pr.v_raw, pr.pt_raw, pr.req, ip, idx, pr.sink, pr.scale,
+                                       dout, k_cmp=pr.k_cmp, v_cmp=pr.v_cmp, pt_cmp=pr.pt_cmp, threads=2,
+                                       o_saved=O, lse_saved=L)
+    moved = oracle.sparse_sink_attn_bwd(pr.q, pr.k_raw, pr.v_raw, pr.pt_raw, pr.req, ip, idx, pr.sink, pr.scale,
+                                        dout, k_cmp=pr.k_cmp, v_cmp=pr.v_cmp, pt_cmp=pr.pt_cmp, threads=2,
+                                        o_saved=O + delta, lse_saved=L)
+    dD = (bits_to_f64(dout) * delta).sum(axis=2)                                 # [N, H]
+    PK, _ = _fwd(oracle, pr, ip, idx, v_raw=pr.k_raw, v_cmp=pr.k_cmp)             # sum_j p_j k_j
+    np.testing.assert_allclose(moved[0] - base[0], -pr.scale * dD[:, :, None] * PK, rtol=1e-9, atol=1e-13)
+    p_sink = np.exp(pr.sink.astype(np.float64)[None, :] - L)
+    np.testing.assert_allclose(moved[5] - base[5], -(p_sink * dD).sum(axis=0), rtol=1e-9, atol=1e-13)
+    np.testing.assert_allclose(moved[2], base[2], rtol=0, atol=0)
+    np.testing.assert_allclose(moved[4], base[4], rtol=0, atol=0)
+
+
+def test_saved_lse_scales_every_gradient(oracle):
+    """With O_saved fixed, every gradient is linear in the probabilities, so
+    LSE_saved = LSE + c multiplies all of them by e^-c."""
+    pr = small_problem(seed=17, S=40, H=4, d=16)
+    ip, idx = _sets(oracle, pr)
+    dout = _dout(pr, 9)
+    O, L = _fwd(oracle, pr, ip, idx)
+    c = 0.3
+    base, shifted = [oracle.sparse_sink_attn_bwd(pr.q, pr.k_raw, pr.v_raw, pr.pt_raw, pr.req, ip, idx, pr.sink,
+                                                 pr.scale, dout, k_cmp=pr.k_cmp, v_cmp=pr.v_cmp, pt_cmp=pr.pt_cmp,
+                                                 threads=2, o_saved=O, lse_saved=L + sh) for sh in (0.0, c)]
+    for a, b in zip(base, shifted):
+        np.testing.assert_allclose(b, np.exp(-c) * a, rtol=1e-12, atol=1e-14)
