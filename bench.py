@@ -235,8 +235,9 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
                     help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
-    ap.add_argument("--op", default="path", choices=["path", "kv_write"],
-                    help="path: the attention hot path (the bench line); kv_write: the paged KV write alone")
+    ap.add_argument("--op", default="path", choices=["path", "kv_write", "bwd"],
+                    help="path: the attention hot path (the bench line); kv_write: the paged KV write alone; "
+                         "bwd: the backward of the attention alone")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=0)
@@ -250,6 +251,8 @@ def main():
         return run_reference(args, rank, world)
     if args.op == "kv_write":
         return run_kv_write(args, rank, local_rank, world)
+    if args.op == "bwd":
+        return run_bwd(args, rank, local_rank, world)
 
     import torch
     import torch.distributed as dist
@@ -452,6 +455,84 @@ def run_kv_write(args, rank, local_rank, world):
                          "frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_kind} HBM copy",
                          "kernel": "paged_kv_write_kernel", "algorithmic_bytes": int(bytes_step)},
             "gpu_launches": args.steps, "pools_unchanged": bool(ok)}))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_bwd(args, rank, local_rank, world):
+    """The backward of the attention alone (dq, dk/dv into the pool-shaped
+    gradients, dsink), from the forward's O and LSE and a seeded dO. The
+    sets and the forward run once, untimed; each timed step is one backward
+    launch, graph-replayed, after an L2 flush. The gradients are added into
+    (zeroing them is the caller's, once per accumulation, and is not timed).
+    Algorithmic FLOPs per query.head.key pair: 5 products x 2d."""
+    import torch
+    import torch.distributed as dist
+    from sparse_paged_attention_build_b200 import workloads
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    import sparse_paged_attention_build_b200 as spa
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    w = workloads.make(args.workload, shrink=args.shrink, seed_offset=rank)
+    if w.k_cmp_fp8 is not None:
+        raise SystemExit("the backward takes BF16 pools; the mixed FP8 workload has none")
+    b = DeviceBatch(w)
+    b.build_sets()
+    out, lse = spa.sparse_sink_attn_fwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, b.indptr, b.indices, b.sink,
+                                        w.scale, k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp)
+    dO = torch.from_numpy(workloads.make_dout(w).view(np.int16)).cuda().view(torch.bfloat16)
+    torch.cuda.synchronize()
+    pairs = int(b.indptr[-1].item()) * w.H
+    st = spa.new_status()
+    grads = spa.sparse_sink_attn_bwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, b.indptr, b.indices, b.sink,
+                                     w.scale, out, lse, dO, k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp,
+                                     num_splits=args.splits, dev_status=st)
+    torch.cuda.synchronize()
+    dq, dkr, dvr, dkc, dvc, dsk = grads
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            spa.sparse_sink_attn_bwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, b.indptr, b.indices, b.sink,
+                                     w.scale, out, lse, dO, k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp,
+                                     dq=dq, dk_raw=dkr, dv_raw=dvr, dk_cmp=dkc, dv_cmp=dvc, dsink=dsk,
+                                     num_splits=args.splits, dev_status=st)
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(args.warmup):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record()
+        g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    times = [e0.elapsed_time(e1) for e0, e1 in evs]
+    ms = float(np.median(times))
+    total_pairs, ms = job_totals(pairs, ms, world, "cuda")
+    flops = 10.0 * w.d * total_pairs
+    tflops = flops / (ms / 1e3) / 1e12
+    pk, pk_kind = peaks()
+    ok = spa.read_status(st) == 0 and all(bool(torch.isfinite(t).all()) for t in grads if t is not None)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "backward query.head.KV pairs/s", "value": total_pairs / (ms / 1e3),
+            "unit": "pairs/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "ms_min": float(np.min(times)), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: {workloads.DESCRIPTIONS[w.name]}", "pairs": int(pairs),
+                       "num_splits": args.splits, "l2": "256 MB buffer written between timed steps (L2 flush)",
+                       "gradient zeroing": "not timed (the call adds into the gradients)"},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / pk["bf16_tflops"], "peak_source": f"{pk_kind} BF16 burst",
+                         "kernel": "sparse_sink_attn_bwd_kernel", "algorithmic_flops": flops},
+            "gpu_launches": args.steps, "finite_and_status_ok": bool(ok)}))
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -295,6 +295,44 @@ int spa_sparse_sink_attn_fwd_fp8(
     const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * 5. spa_sparse_sink_attn_bwd -- gradients of the attention with sink.
+ *
+ * The follow-on item of "Roadmap item 24 - joint compressed/window attention
+ * with sink": dQ, dK/dV scattered to the pages, and d_sink, from the saved O
+ * and LSE. With p_j = exp(scale q.k_j - LSE) recomputed per (query, head),
+ * D = dO . O, ds_j = p_j (dO . v_j - D):
+ *   dq += scale sum_j ds_j k_j         dk[row(j)] += scale ds_j q  (all heads)
+ *   dv[row(j)] += p_j dO (all heads)   dsink[h] += -exp(sink_h - LSE) D
+ * P and dS enter the tensor-core products as BF16; every sum is FP32.
+ *
+ * Arguments as for spa_sparse_sink_attn_fwd (BF16 pools only), plus:
+ * out, lse   the forward's O (BF16 [n_queries, num_heads, head_dim],
+ *            contiguous, 16-B aligned) and LSE (FP32 [n_queries, num_heads])
+ * dout       dO, BF16 [n_queries, num_heads, head_dim], contiguous, 16-B aligned
+ * dq         FP32 [n_queries, num_heads, head_dim], 16-B aligned
+ * dk_raw, dv_raw  FP32 [raw_num_pages * raw_page_size, head_dim]: the raw
+ *            pools' gradient rows; dk_cmp, dv_cmp likewise for the
+ *            compressed pool (required when pt_cmp is set)
+ * dsink      FP32 [num_heads] or NULL (ignored when sink is NULL)
+ * Every gradient is ADDED into its array (zero them for a fresh gradient);
+ * the additions are FP32 atomics, so their order, and the last bits of a
+ * sum, vary from run to run. Rows of faulty keys receive nothing (the
+ * status word says why, as in the forward). num_splits as in the forward
+ * (0 = automatic); slices add their dq. No workspace.
+ * ---------------------------------------------------------------------- */
+int spa_sparse_sink_attn_bwd(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+    int32_t num_heads, int32_t head_dim,
+    const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+    const int32_t* pt_raw, int32_t pt_raw_cols,
+    const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages, int32_t cmp_page_size,
+    const int32_t* pt_cmp, int32_t pt_cmp_cols,
+    const int32_t* req, int32_t n_requests, const int32_t* indptr, const int32_t* indices,
+    const float* sink, float scale, const uint16_t* out, const float* lse, const uint16_t* dout,
+    float* dq, float* dk_raw, float* dv_raw, float* dk_cmp, float* dv_cmp, float* dsink,
+    int32_t num_splits, uint32_t* dev_status, spa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

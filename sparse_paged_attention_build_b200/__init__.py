@@ -73,6 +73,12 @@ def _load():
     L.spa_sparse_sink_attn_fwd_fp8.restype = ctypes.c_int
     L.spa_paged_kv_write.argtypes = [P, P, i32, i32, P, P, P, i32, i32, i32, i64, P, P, P, P]
     L.spa_paged_kv_write.restype = ctypes.c_int
+    L.spa_sparse_sink_attn_bwd.argtypes = [
+        P, i64, i64, i32, i32, i32,
+        P, P, i64, i32, P, i32,
+        P, P, i64, i32, P, i32,
+        P, i32, P, P, P, ctypes.c_float, P, P, P, P, P, P, P, P, P, i32, P, P]
+    L.spa_sparse_sink_attn_bwd.restype = ctypes.c_int
     return L
 
 
@@ -269,6 +275,63 @@ def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
     return out, lse
+
+
+def sparse_sink_attn_bwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale, out, lse, dout,
+                         k_cmp=None, v_cmp=None, pt_cmp=None, dq=None, dk_raw=None, dv_raw=None,
+                         dk_cmp=None, dv_cmp=None, dsink=None, num_splits=0, dev_status=None, stream=None):
+    """Gradients of sum(dout * O) for the attention of sparse_sink_attn_fwd.
+
+    out, lse: the forward's O (bf16 [N, H, d]) and LSE (fp32 [N, H]); dout:
+    bf16 [N, H, d]. Returns (dq fp32 [N, H, d], dk_raw, dv_raw fp32 shaped
+    like the raw pools, dk_cmp, dv_cmp (None without a compressed pool),
+    dsink fp32 [H] (None without a sink)). Gradients passed in are added
+    into; those not passed start from zeros.
+    """
+    _need(q, "q", torch.bfloat16)
+    for name, t in (("k_raw", k_raw), ("v_raw", v_raw), ("out", out), ("dout", dout)):
+        _need(t, name, torch.bfloat16)
+        assert t.is_contiguous(), name
+    for name, t in (("pt_raw", pt_raw), ("req", req), ("indptr", indptr), ("indices", indices)):
+        _need(t, name, torch.int32)
+    _need(lse, "lse", torch.float32)
+    N, H, d = q.shape
+    if q.stride(2) != 1:
+        raise ValueError("q's last dimension must be contiguous")
+    if pt_cmp is not None:
+        _need(pt_cmp, "pt_cmp", torch.int32)
+        _need(k_cmp, "k_cmp", torch.bfloat16)
+        _need(v_cmp, "v_cmp", torch.bfloat16)
+        assert k_cmp.is_contiguous() and v_cmp.is_contiguous()
+    if sink is not None:
+        _need(sink, "sink", torch.float32)
+
+    def grad(t, like, name):
+        if t is None:
+            return torch.zeros(like.shape, dtype=torch.float32, device=like.device)
+        _need(t, name, torch.float32)
+        assert t.is_contiguous() and t.shape == like.shape, name
+        return t
+
+    dq = grad(dq, q, "dq")
+    dk_raw, dv_raw = grad(dk_raw, k_raw, "dk_raw"), grad(dv_raw, v_raw, "dv_raw")
+    if pt_cmp is not None:
+        dk_cmp, dv_cmp = grad(dk_cmp, k_cmp, "dk_cmp"), grad(dv_cmp, v_cmp, "dv_cmp")
+    else:
+        dk_cmp = dv_cmp = None
+    dsink = None if sink is None else grad(dsink, sink, "dsink")
+    pt_raw = pt_raw.contiguous()
+    _check("spa_sparse_sink_attn_bwd", lib.spa_sparse_sink_attn_bwd(
+        _p(q), q.stride(0), q.stride(1), N, H, d,
+        _p(k_raw), _p(v_raw), k_raw.shape[0], k_raw.shape[1], _p(pt_raw), pt_raw.shape[1],
+        _p(k_cmp), _p(v_cmp), 0 if k_cmp is None else k_cmp.shape[0],
+        1 if k_cmp is None else k_cmp.shape[1],
+        _p(None if pt_cmp is None else pt_cmp.contiguous()), 0 if pt_cmp is None else pt_cmp.shape[1],
+        _p(req.contiguous()), pt_raw.shape[0], _p(indptr.contiguous()), _p(indices.contiguous()),
+        _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse.contiguous()),
+        _p(dout), _p(dq), _p(dk_raw), _p(dv_raw), _p(dk_cmp), _p(dv_cmp), _p(dsink), num_splits,
+        _p(dev_status), _stream(stream)))
+    return dq, dk_raw, dv_raw, dk_cmp, dv_cmp, dsink
 
 
 def paged_kv_write(k_new, v_new, req, pos, pt, k_pool, v_pool, dev_status=None, stream=None):

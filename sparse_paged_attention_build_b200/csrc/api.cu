@@ -231,9 +231,9 @@ size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads,
 
 namespace {
 
-// Checks shared by both attention entry points (everything except the
-// compressed pool's storage), then the launch.
-int attn_run(spa::AttnArgs a, int32_t requested_splits, size_t workspace_bytes, cudaStream_t stream) {
+// Checks shared by every attention entry point (shapes, pools, sets; not
+// the outputs nor the compressed pool's storage). SPA_OK or a failure.
+int attn_check(const spa::AttnArgs& a, int32_t requested_splits) {
   if (a.n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
   if (a.num_heads < 1) return fail(SPA_ERR_INVALID_ARG, "num_heads < 1");
   if (a.n_requests < 1) return fail(SPA_ERR_INVALID_ARG, "n_requests < 1");
@@ -259,8 +259,7 @@ int attn_run(spa::AttnArgs a, int32_t requested_splits, size_t workspace_bytes, 
     return fail(SPA_ERR_INVALID_ARG, "num_splits must be in [0, %d]", spa::kAttnMaxSplits);
   if (a.q_stride_tok < 0 || a.q_stride_head < 0) return fail(SPA_ERR_INVALID_ARG, "negative q stride");
   if (a.n_queries == 0) return ok();
-  if (a.q == nullptr || a.out == nullptr || a.lse == nullptr)
-    return fail(SPA_ERR_INVALID_ARG, "q, out and lse must be non-NULL");
+  if (a.q == nullptr) return fail(SPA_ERR_INVALID_ARG, "q must be non-NULL");
   if (a.k_raw == nullptr || a.v_raw == nullptr || a.pt_raw == nullptr)
     return fail(SPA_ERR_INVALID_ARG, "k_raw, v_raw and pt_raw must be non-NULL");
   if (a.req == nullptr || a.indptr == nullptr || a.indices == nullptr)
@@ -270,14 +269,24 @@ int attn_run(spa::AttnArgs a, int32_t requested_splits, size_t workspace_bytes, 
   if (!aligned(a.k_raw, 16) || !aligned(a.v_raw, 16) || !aligned(a.k_cmp, 16) || !aligned(a.v_cmp, 16) ||
       !aligned(a.k_cmp_fp8, 16) || !aligned(a.v_cmp_fp8, 16))
     return fail(SPA_ERR_ALIGNMENT, "K/V pools must be 16-byte aligned");
-  if (!aligned(a.out, 16)) return fail(SPA_ERR_ALIGNMENT, "out must be 16-byte aligned");
-  if (!aligned(a.lse, 4) || !aligned(a.sink, 4) || !aligned(a.req, 4) || !aligned(a.indptr, 4) ||
+  if (!aligned(a.sink, 4) || !aligned(a.req, 4) || !aligned(a.indptr, 4) ||
       !aligned(a.indices, 4) || !aligned(a.pt_raw, 4) || !aligned(a.pt_cmp, 4) || !aligned(a.k_cmp_scale, 4) ||
       !aligned(a.v_cmp_scale, 4))
     return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
   const int32_t splits = resolve_splits(a.n_queries, a.num_heads, requested_splits);
   if (static_cast<int64_t>(a.n_queries) * splits > 0x7fffffffLL)
     return fail(SPA_ERR_UNSUPPORTED, "n_queries * num_splits exceeds the grid");
+  return ok();
+}
+
+// The forward entry points: shared checks, outputs, workspace, launch.
+int attn_run(spa::AttnArgs a, int32_t requested_splits, size_t workspace_bytes, cudaStream_t stream) {
+  const int st = attn_check(a, requested_splits);
+  if (st != SPA_OK || a.n_queries == 0) return st;
+  if (a.out == nullptr || a.lse == nullptr) return fail(SPA_ERR_INVALID_ARG, "q, out and lse must be non-NULL");
+  if (!aligned(a.out, 16)) return fail(SPA_ERR_ALIGNMENT, "out must be 16-byte aligned");
+  if (!aligned(a.lse, 4)) return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
+  const int32_t splits = resolve_splits(a.n_queries, a.num_heads, requested_splits);
   const size_t need = spa::attn_workspace_bytes(a.n_queries, a.num_heads, a.head_dim, splits);
   if (need > 0) {
     if (a.workspace == nullptr || workspace_bytes < need)
@@ -378,6 +387,51 @@ int spa_sparse_sink_attn_fwd_fp8(const uint16_t* q, int64_t q_stride_tok, int64_
   a.v_cmp_scale = v_cmp_scale;
   a.fp8_fnuz = fp8_format == 1;
   return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spa_sparse_sink_attn_bwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+                             int32_t num_heads, int32_t head_dim, const uint16_t* k_raw, const uint16_t* v_raw,
+                             int64_t raw_num_pages, int32_t raw_page_size, const int32_t* pt_raw,
+                             int32_t pt_raw_cols, const uint16_t* k_cmp, const uint16_t* v_cmp,
+                             int64_t cmp_num_pages, int32_t cmp_page_size, const int32_t* pt_cmp,
+                             int32_t pt_cmp_cols, const int32_t* req, int32_t n_requests,
+                             const int32_t* indptr, const int32_t* indices, const float* sink, float scale,
+                             const uint16_t* out, const float* lse, const uint16_t* dout, float* dq,
+                             float* dk_raw, float* dv_raw, float* dk_cmp, float* dv_cmp, float* dsink,
+                             int32_t num_splits, uint32_t* dev_status, spa_stream_t stream) {
+  if (pt_cmp != nullptr && n_queries > 0 && (k_cmp == nullptr || v_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
+  spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
+                              raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
+                              pt_cmp_cols, req, n_requests, indptr, indices, sink, scale, nullptr, nullptr, nullptr,
+                              dev_status);
+  a.k_cmp = k_cmp;
+  a.v_cmp = v_cmp;
+  const int st = attn_check(a, num_splits);
+  if (st != SPA_OK || n_queries == 0) return st;
+  if (out == nullptr || lse == nullptr || dout == nullptr)
+    return fail(SPA_ERR_INVALID_ARG, "out, lse and dout must be non-NULL");
+  if (dq == nullptr || dk_raw == nullptr || dv_raw == nullptr)
+    return fail(SPA_ERR_INVALID_ARG, "dq, dk_raw and dv_raw must be non-NULL");
+  if (pt_cmp != nullptr && (dk_cmp == nullptr || dv_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "dk_cmp/dv_cmp NULL with pt_cmp set");
+  if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dq, 16))
+    return fail(SPA_ERR_ALIGNMENT, "out, dout and dq must be 16-byte aligned");
+  if (!aligned(lse, 4) || !aligned(dk_raw, 4) || !aligned(dv_raw, 4) || !aligned(dk_cmp, 4) ||
+      !aligned(dv_cmp, 4) || !aligned(dsink, 4))
+    return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
+  a.num_splits = resolve_splits(n_queries, num_heads, num_splits);
+  a.o_saved = out;
+  a.lse_saved = lse;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk_raw = dk_raw;
+  a.dv_raw = dv_raw;
+  a.dk_cmp = dk_cmp;
+  a.dv_cmp = dv_cmp;
+  a.dsink = sink != nullptr ? dsink : nullptr;
+  return cuda_status(spa::launch_sparse_sink_attn_bwd(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "sparse_sink_attn_bwd launch");
 }
 
 }  // extern "C"

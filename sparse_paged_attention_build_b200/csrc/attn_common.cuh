@@ -1,0 +1,202 @@
+// Pieces shared by the attention kernels (forward and backward): the chunk
+// descriptors the resolver hands to the other warp roles, the resolver
+// itself (keys -> physical pool rows through the page tables), and the
+// host-side tensor-map encoders.
+#pragma once
+
+#include <algorithm>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "spa_device.cuh"
+#include "spa_internal.h"
+
+namespace spa {
+namespace attn {
+
+constexpr int kT = kAttnKeysPerTile;             // keys per tile
+constexpr int kChunkKeys = 768;                  // keys resolved per chunk (12 tiles)
+constexpr uint32_t kRawBit = 0x80000000u;        // row of the raw (window) pool
+constexpr uint32_t kInvalidRow = 0xFFFFFFFFu;    // padding or faulty key: zero row, no update
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+constexpr int kFlagFirst = 1;   // first chunk of its unit
+constexpr int kFlagLast = 2;    // last chunk of its unit
+constexpr int kFlagFinal = 4;   // last chunk of this CTA
+constexpr int kFlagSetStart = 8;   // the chunk starts at the first key of its query's set
+
+struct ChunkDesc {
+  int32_t i;          // query token
+  int32_t split;      // slice of the token's key set
+  int32_t key_base;   // CSR position of the chunk's first key
+  int32_t nkeys;      // keys in the chunk (tiles = ceil(nkeys / 64))
+  int32_t flags;
+  int32_t pad[3];
+};
+
+__device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) / kT; }
+
+// Keys -> physical rows for one chunk. Each lane handles keys lane, lane+32,
+// ...; the loads of each phase are issued together so the chunk costs two
+// round trips, not two per key. Prm holds the page tables and pool sizes.
+template <class Prm>
+__device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t nkeys, uint32_t* tab,
+                              int lane) {
+  constexpr int kPer = kChunkKeys / 32;
+  int32_t key[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int k = lane + 32 * e;
+    key[e] = k < nkeys ? __ldg(P.indices + key_base + k) : -2;
+  }
+  int32_t page[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    page[e] = -1;
+    const int32_t kk = key[e];
+    if (kk == -2) continue;
+    if (kk < 0) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
+    const bool raw = (kk & SPA_WINDOW_TAG) != 0;
+    const int32_t t = kk & (SPA_WINDOW_TAG - 1);
+    const int32_t* pt = raw ? P.pt_raw : P.pt_cmp;
+    const int32_t cols = raw ? P.pt_raw_cols : P.pt_cmp_cols;
+    const int32_t lp = t >> (raw ? P.raw_ps_log2 : P.cmp_ps_log2);
+    if (pt == nullptr || lp >= cols) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
+    page[e] = __ldg(pt + static_cast<int64_t>(b) * cols + lp);
+  }
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int k = lane + 32 * e;
+    const int32_t kk = key[e];
+    uint32_t row = kInvalidRow;
+    if (kk >= 0) {
+      const bool raw = (kk & SPA_WINDOW_TAG) != 0;
+      const int32_t t = kk & (SPA_WINDOW_TAG - 1);
+      const int32_t ps_log2 = raw ? P.raw_ps_log2 : P.cmp_ps_log2;
+      const int64_t pages = raw ? P.raw_pages : P.cmp_pages;
+      const int64_t pg = page[e];
+      if (pg < 0 || pg >= pages) {
+        report(P.dev_status, SPA_DEV_BAD_PAGE);
+      } else {
+        row = static_cast<uint32_t>((pg << ps_log2) + (t & ((1 << ps_log2) - 1))) | (raw ? kRawBit : 0u);
+      }
+    }
+    if (k < nkeys) tab[k] = row;
+  }
+}
+
+// The resolver warp: walks this CTA's units (query i, slice) in a fixed
+// stride, splits each slice's keys into chunks of up to kChunkKeys, resolves
+// them into the double-buffered table and publishes a descriptor per chunk.
+// An empty slice still gets one (empty) chunk so that every role sees every
+// unit. S = slices per query.
+template <class Prm>
+__device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* desc, uint64_t* tab_full,
+                              uint64_t* tab_empty, volatile int* abort_flag, int lane) {
+  int c = 0;
+  const int64_t n_units = static_cast<int64_t>(P.n_queries) * S;
+  for (int64_t u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
+    const int i = static_cast<int>(u / S);
+    const int split = static_cast<int>(u - static_cast<int64_t>(i) * S);
+    const int32_t set_begin = __ldg(P.indptr + i);
+    int32_t set_len = __ldg(P.indptr + i + 1) - set_begin;
+    const int32_t b = __ldg(P.req + i);
+    if (set_len < 0 || b < 0 || b >= P.n_requests) {
+      if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
+      set_len = 0;
+    }
+    const int tiles_total = ceil_tiles(set_len);
+    const int tile_lo = static_cast<int>((static_cast<int64_t>(tiles_total) * split) / S);
+    const int tile_hi = static_cast<int>((static_cast<int64_t>(tiles_total) * (split + 1)) / S);
+    const int32_t key_lo = tile_lo * kT;
+    const int32_t key_hi = min(tile_hi * kT, set_len);
+    const bool final_unit = u + gridDim.x >= n_units;
+    int32_t k0 = key_lo;
+    do {
+      const int slot = c & 1;
+      if (!mbar_wait(tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status)) return;
+      const int32_t n = max(0, min(kChunkKeys, key_hi - k0));   // 0: an empty slice
+      resolve_chunk(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane);
+      if (lane == 0) {
+        ChunkDesc& d = desc[slot];
+        d.i = i;
+        d.split = split;
+        d.key_base = set_begin + k0;
+        d.nkeys = n;
+        const bool last = k0 + n >= key_hi;
+        d.flags = (k0 == key_lo ? kFlagFirst : 0) | (last ? kFlagLast : 0) | (last && final_unit ? kFlagFinal : 0) |
+                  (k0 == 0 && n > 0 ? kFlagSetStart : 0);
+      }
+      __syncwarp();
+      mbar_arrive(tab_full + slot);
+      ++c;
+      k0 += n;
+    } while (k0 < key_hi);
+  }
+}
+
+// ------------------------------------------------------------------ host
+inline int sm_count_cached() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+    else
+      n = 148;
+  }
+  return n;
+}
+
+inline int log2_exact(int32_t v) {
+  int k = 0;
+  while ((1 << k) < v) ++k;
+  return k;
+}
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// A paged pool [rows, d] BF16 as a 2D tensor with a one-row, 64-column box,
+// 128-byte swizzle: the form tile::gather4 takes.
+inline bool encode_pool(CUtensorMap* m, const void* base, int64_t rows, int d) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(std::max<int64_t>(rows, 1))};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t elem[2] = {1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                              box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [N, H, d] BF16 with element strides (tok, head) as a 3D tensor {d, H, N},
+// box {64, box_rows, 1}: one token's head rows, 64 columns at a time.
+inline bool encode_q(CUtensorMap* m, const void* base, int32_t n, int32_t h, int d, int64_t stride_tok,
+                     int64_t stride_head, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(h),
+                              static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride_head) * 2, static_cast<cuuint64_t>(stride_tok) * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                              box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace attn
+}  // namespace spa

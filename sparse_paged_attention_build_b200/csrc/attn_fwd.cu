@@ -51,16 +51,13 @@
 #include <cmath>
 #include <cstring>
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "spa_device.cuh"
-#include "spa_internal.h"
+#include "attn_common.cuh"
 
 namespace spa {
 namespace {
 
-constexpr int kT = kAttnKeysPerTile;   // keys per tile
+using namespace attn;
+
 constexpr int kStagesK = 2;
 constexpr int kStagesV = 2;
 constexpr int kSoftThreads = 128;
@@ -70,11 +67,6 @@ constexpr int kKWarp0 = 6;                       // K (and Q) producer
 constexpr int kVWarp0 = 7;                       // V producer
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
-constexpr int kChunkKeys = 768;                  // keys resolved per chunk (12 tiles)
-constexpr uint32_t kRawBit = 0x80000000u;
-constexpr uint32_t kInvalidRow = 0xFFFFFFFFu;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 // A tile whose row sum of P, taken with the running max as it stands,
 // exceeds 2^16 (or is not a number) is recomputed with its exact max. P
 // therefore stays below 2^16: harmless in BF16 and in the FP32 sums, whose
@@ -82,19 +74,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kSpecBound = 65536.0f;
 // consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
 constexpr uint32_t kTabConsumers = 32 + 32 + 1 + kSoftThreads;
-
-constexpr int kFlagFirst = 1;   // first chunk of its unit
-constexpr int kFlagLast = 2;    // last chunk of its unit
-constexpr int kFlagFinal = 4;   // last chunk of this CTA
-
-struct ChunkDesc {
-  int32_t i;          // query token
-  int32_t split;      // slice of the token's key set
-  int32_t key_base;   // CSR position of the chunk's first key
-  int32_t nkeys;      // keys in the chunk (tiles = ceil(nkeys / 64))
-  int32_t flags;
-  int32_t pad[3];
-};
 
 struct Params {
   // TMA descriptors (passed as a __grid_constant__ parameter)
@@ -186,57 +165,6 @@ struct Bars {
   uint64_t* soft_sync;
 };
 
-__device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) / kT; }
-
-// ------------------------------------------------------------------ resolver
-// Keys -> physical rows for one chunk. Each lane handles keys lane, lane+32,
-// ...; the loads of each phase are issued together so the chunk costs two
-// round trips, not two per key.
-__device__ void resolve_chunk(const Params& P, int32_t b, int32_t key_base, int32_t nkeys,
-                              uint32_t* tab, int lane) {
-  constexpr int kPer = kChunkKeys / 32;
-  int32_t key[kPer];
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    const int k = lane + 32 * e;
-    key[e] = k < nkeys ? __ldg(P.indices + key_base + k) : -2;
-  }
-  int32_t page[kPer];
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    page[e] = -1;
-    const int32_t kk = key[e];
-    if (kk == -2) continue;
-    if (kk < 0) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
-    const bool raw = (kk & SPA_WINDOW_TAG) != 0;
-    const int32_t t = kk & (SPA_WINDOW_TAG - 1);
-    const int32_t* pt = raw ? P.pt_raw : P.pt_cmp;
-    const int32_t cols = raw ? P.pt_raw_cols : P.pt_cmp_cols;
-    const int32_t lp = t >> (raw ? P.raw_ps_log2 : P.cmp_ps_log2);
-    if (pt == nullptr || lp >= cols) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
-    page[e] = __ldg(pt + static_cast<int64_t>(b) * cols + lp);
-  }
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    const int k = lane + 32 * e;
-    const int32_t kk = key[e];
-    uint32_t row = kInvalidRow;
-    if (kk >= 0) {
-      const bool raw = (kk & SPA_WINDOW_TAG) != 0;
-      const int32_t t = kk & (SPA_WINDOW_TAG - 1);
-      const int32_t ps_log2 = raw ? P.raw_ps_log2 : P.cmp_ps_log2;
-      const int64_t pages = raw ? P.raw_pages : P.cmp_pages;
-      const int64_t pg = page[e];
-      if (pg < 0 || pg >= pages) {
-        report(P.dev_status, SPA_DEV_BAD_PAGE);
-      } else {
-        row = static_cast<uint32_t>((pg << ps_log2) + (t & ((1 << ps_log2) - 1))) | (raw ? kRawBit : 0u);
-      }
-    }
-    if (k < nkeys) tab[k] = row;
-  }
-}
-
 template <int D, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __grid_constant__ Params P) {
   using L = Layout<D>;
@@ -309,46 +237,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
 
   if (warp == kResolverWarp) {
     // ================================================= resolver
-    int c = 0;
-    const int64_t n_units = static_cast<int64_t>(P.n_queries) * S;
-    for (int64_t u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
-      const int i = static_cast<int>(u / S);
-      const int split = static_cast<int>(u - static_cast<int64_t>(i) * S);
-      const int32_t set_begin = __ldg(P.indptr + i);
-      int32_t set_len = __ldg(P.indptr + i + 1) - set_begin;
-      const int32_t b = __ldg(P.req + i);
-      if (set_len < 0 || b < 0 || b >= P.n_requests) {
-        if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
-        set_len = 0;
-      }
-      const int tiles_total = ceil_tiles(set_len);
-      const int tile_lo = static_cast<int>((static_cast<int64_t>(tiles_total) * split) / S);
-      const int tile_hi = static_cast<int>((static_cast<int64_t>(tiles_total) * (split + 1)) / S);
-      const int32_t key_lo = tile_lo * kT;
-      const int32_t key_hi = min(tile_hi * kT, set_len);
-      const bool final_unit = u + gridDim.x >= n_units;
-      int32_t k0 = key_lo;
-      do {
-        const int slot = c & 1;
-        if (!mbar_wait(B.tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status)) break;
-        const int32_t n = max(0, min(kChunkKeys, key_hi - k0));   // 0: an empty slice
-        resolve_chunk(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane);
-        if (lane == 0) {
-          ChunkDesc& d = desc[slot];
-          d.i = i;
-          d.split = split;
-          d.key_base = set_begin + k0;
-          d.nkeys = n;
-          const bool last = k0 + n >= key_hi;
-          d.flags = (k0 == key_lo ? kFlagFirst : 0) | (last ? kFlagLast : 0) |
-                    (last && final_unit ? kFlagFinal : 0);
-        }
-        __syncwarp();
-        mbar_arrive(B.tab_full + slot);
-        ++c;
-        k0 += n;
-      } while (k0 < key_hi);
-    }
+    resolver_loop(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane);
   } else if (warp == kKWarp0 || warp == kVWarp0) {
     // ================================================= K / V gather (TMA)
     // A tile is 16 four-row groups x D/64 column halves = "jobs"; lane j
@@ -1019,19 +908,6 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-int sm_count_cached() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      n = v;
-    else
-      n = 148;
-  }
-  return n;
-}
-
 template <int D, bool kFp8>
 cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
   using L = Layout<D>;
@@ -1065,51 +941,6 @@ cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
   sparse_sink_attn_kernel<D, kFp8><<<grid, kThreads, L::kBytes, stream>>>(P);
   return cudaGetLastError();
-}
-
-int log2_exact(int32_t v) {
-  int k = 0;
-  while ((1 << k) < v) ++k;
-  return k;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// A paged pool [rows, d] BF16 as a 2D tensor with a one-row, 64-column box,
-// 128-byte swizzle: the form tile::gather4 takes.
-bool encode_pool(CUtensorMap* m, const void* base, int64_t rows, int d) {
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(std::max<int64_t>(rows, 1))};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[2] = {64, 1};
-  const cuuint32_t elem[2] = {1, 1};
-  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                              box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// q [N, H, d] with element strides (tok, head) as a 3D tensor {d, H, N}.
-bool encode_q(CUtensorMap* m, const void* base, int32_t n, int32_t h, int d, int64_t stride_tok,
-              int64_t stride_head, int box_rows) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(h),
-                              static_cast<cuuint64_t>(n)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride_head) * 2, static_cast<cuuint64_t>(stride_tok) * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  const cuuint32_t elem[3] = {1, 1, 1};
-  return tensor_map_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                              box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace

@@ -253,6 +253,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same with either operand's major-ness chosen: a_mn_major = 1 reads A
+// as M-major (its M index contiguous), b_mn_major = 1 reads B as N-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, int a_mn_major, int b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | (static_cast<uint32_t>(a_mn_major) << 15);
+}
+
 // Shared-memory matrix descriptor for the 128-byte swizzle: start address,
 // leading and stride byte offsets (16-byte units), version 1, swizzle mode 2.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,

@@ -64,6 +64,14 @@ struct AttnArgs {
   int32_t num_splits;  // >= 1, resolved
   void* workspace;
   uint32_t* dev_status;
+  // backward only: the forward's saved O [N, H, d] BF16 and LSE [N, H], the
+  // output gradient dO [N, H, d] BF16, and the FP32 gradients it adds into
+  // (dq [N, H, d]; dk/dv shaped like their pools; dsink [H], may be NULL)
+  const uint16_t* o_saved = nullptr;
+  const float* lse_saved = nullptr;
+  const uint16_t* dout = nullptr;
+  float *dq = nullptr, *dk_raw = nullptr, *dv_raw = nullptr, *dk_cmp = nullptr, *dv_cmp = nullptr;
+  float* dsink = nullptr;
 };
 
 constexpr int kAttnKeysPerTile = 64;
@@ -74,5 +82,6 @@ constexpr int kAttnMaxClusterSplits = 8;
 size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                             int32_t num_splits);
 cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse_sink_attn_bwd(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace spa

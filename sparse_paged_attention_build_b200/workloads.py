@@ -244,3 +244,9 @@ def make(name: str, shrink: int = 1, seed_offset: int = 0, fp8_format: int = 0) 
         L = max(1024, 32768 // shrink)
         return _decode(name, seed, B, np.full(B, L), 128, 128, 128, 4, 512, 128, fp8=True, fmt=fp8_format)
     raise KeyError(name)
+
+
+def make_dout(w: Workload, seed: int = 0) -> np.ndarray:
+    """A seeded output gradient dO for a workload: BF16 bits [N, H, d], N(0,1)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([BASE_SEED, 77, seed])))
+    return _normal_bf16(rng, (w.N, w.H, w.d))

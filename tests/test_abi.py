@@ -143,7 +143,8 @@ def attn_call(L, **kw):
     (dict(scale=float("inf")), 1, "scale must be finite"),
     (dict(splits=17), 1, "num_splits must be"),
     (dict(sq=-8), 1, "negative q stride"),
-    (dict(q=None), 1, "q, out and lse"),
+    (dict(q=None), 1, "q must be non-NULL"),
+    (dict(out=None), 1, "q, out and lse"),
     (dict(vr=None), 1, "k_raw, v_raw and pt_raw"),
     (dict(idx=None), 1, "req, indptr and indices"),
     (dict(sh=129), 5, "q base and strides"),
@@ -220,3 +221,42 @@ def test_guard_matrix_kv_write(L, kw, status, clause):
 
 def test_kv_write_zero_tokens_is_a_no_op(L):
     assert kvw_call(L, n=0, kn=None, vn=None) == 0
+
+
+def bwd_call(L, **kw):
+    a = dict(q=FAKE, sq=16384, sh=128, n=4, H=128, d=128, kr=FAKE, vr=FAKE, rp=10, rps=64, ptr=FAKE,
+             ptrc=4, kc=FAKE, vc=FAKE, cp=10, cps=64, ptc=FAKE, ptcc=4, req=FAKE, B=1, ip=FAKE,
+             idx=FAKE, sink=FAKE, scale=0.088, out=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dkr=FAKE,
+             dvr=FAKE, dkc=FAKE, dvc=FAKE, dsink=FAKE, splits=1)
+    a.update(kw)
+    return L.spa_sparse_sink_attn_bwd(
+        a["q"], a["sq"], a["sh"], a["n"], a["H"], a["d"], a["kr"], a["vr"], a["rp"], a["rps"], a["ptr"],
+        a["ptrc"], a["kc"], a["vc"], a["cp"], a["cps"], a["ptc"], a["ptcc"], a["req"], a["B"], a["ip"],
+        a["idx"], a["sink"], a["scale"], a["out"], a["lse"], a["dout"], a["dq"], a["dkr"], a["dvr"],
+        a["dkc"], a["dvc"], a["dsink"], a["splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(n=-1), 1, "n_queries < 0"),
+    (dict(d=96), 2, "head_dim must be 64 or 128"),
+    (dict(rps=48), 2, "raw_page_size must be a power of two"),
+    (dict(kc=None), 1, "k_cmp/v_cmp NULL"),
+    (dict(splits=17), 1, "num_splits must be"),
+    (dict(q=None), 1, "q must be non-NULL"),
+    (dict(dout=None), 1, "out, lse and dout"),
+    (dict(lse=None), 1, "out, lse and dout"),
+    (dict(dq=None), 1, "dq, dk_raw and dv_raw"),
+    (dict(dvr=None), 1, "dq, dk_raw and dv_raw"),
+    (dict(dkc=None), 1, "dk_cmp/dv_cmp NULL"),
+    (dict(dq=FAKE + 4), 5, "out, dout and dq"),
+    (dict(dout=FAKE + 2), 5, "out, dout and dq"),
+    (dict(dkr=FAKE + 2), 5, "32-bit arrays"),
+    (dict(dsink=FAKE + 1), 5, "32-bit arrays"),
+])
+def test_guard_matrix_attention_bwd(L, kw, status, clause):
+    assert bwd_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def test_attention_bwd_zero_queries_is_a_no_op(L):
+    assert bwd_call(L, n=0, q=None, out=None, lse=None, dout=None, dq=None, dkr=None, dvr=None) == 0

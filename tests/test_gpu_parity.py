@@ -475,3 +475,191 @@ def test_graph_capture_and_two_streams(spa):
     torch.cuda.synchronize()
     assert torch.equal(b.out, ref_out) and torch.equal(b2.out, ref_out)
     assert torch.equal(b2.lse, ref_lse)
+
+
+# ---------------------------------------------------------------- backward
+# The backward reads the forward's saved O (BF16) and LSE (FP32). Parity
+# feeds both sides the same saved values (the oracle's forward, O rounded to
+# BF16 and LSE to FP32), so what is compared is the backward alone. Bar,
+# from its arithmetic: P and dS enter the tensor-core products rounded to
+# BF16 (relative 2^-9 per term) and every sum is FP32, so an element may be
+# off by a small multiple of 2^-9 of its row's magnitude:
+#   |g - ref| <= 2e-2 * rms(row of ref) + 1e-2 * |ref| + 1e-3 * rms(ref)
+# (a row: the d entries of one dq (query, head), of one dk/dv pool row, or
+# the H entries of dsink; the last term covers rows whose exact value
+# cancels to zero while their FP32 terms are of the tensor's typical size). The chain check (the CUDA forward's own O and LSE
+# into the backward) adds the forward's error to D; it is held to a
+# relative Frobenius error of 2e-2 per gradient.
+G_ROW = 2e-2
+G_REL = 1e-2
+G_FLOOR = 1e-3
+G_CHAIN = 2e-2
+
+
+def check_grad(g, ref, what):
+    g = g.detach().double().cpu().numpy() if torch.is_tensor(g) else np.asarray(g, dtype=np.float64)
+    g = g.reshape(ref.shape)
+    r2 = ref.reshape(-1, ref.shape[-1]) if ref.ndim > 1 else ref.reshape(1, -1)
+    g2 = g.reshape(r2.shape)
+    rms_row = np.sqrt(np.mean(r2 * r2, axis=1, keepdims=True))
+    rms_all = float(np.sqrt(np.mean(r2 * r2))) if r2.size else 0.0
+    err = np.abs(g2 - r2)
+    bad = err > G_ROW * rms_row + G_REL * np.abs(r2) + G_FLOOR * rms_all
+    worst = float((err / np.maximum(rms_row, 1e-2 * rms_all + 1e-30)).max()) if r2.size else 0.0
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {r2.size} out of tolerance, "
+                           f"max err {err.max():.3g}, worst err / rms(row) {worst:.3g}")
+    return worst
+
+
+@functools.lru_cache(maxsize=None)
+def dout_bits(name, shrink=1):
+    from sparse_paged_attention_build_b200 import workloads
+    return workloads.make_dout(workload(name, shrink))
+
+
+def saved_from_oracle(O, L):
+    """The oracle's forward as a forward would store it: O rounded to BF16
+    (bits), LSE rounded to FP32; and the same values in FP64 for the oracle."""
+    o_bf = torch.from_numpy(O).to(torch.float32).to(torch.bfloat16)
+    l_f32 = torch.from_numpy(L).to(torch.float32)
+    return o_bf, l_f32, o_bf.to(torch.float64).numpy(), l_f32.to(torch.float64).numpy()
+
+
+def gpu_bwd(spa, b, name, shrink, out, lse, num_splits=0, indptr=None, indices=None, sink="w"):
+    w = workload(name, shrink)
+    dO = torch.from_numpy(dout_bits(name, shrink).view(np.int16)).cuda().view(torch.bfloat16)
+    st = spa.new_status()
+    ip = b.indptr if indptr is None else indptr
+    ix = b.indices if indices is None else indices
+    s = b.sink if isinstance(sink, str) else sink
+    g = spa.sparse_sink_attn_bwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, ip, ix, s, w.scale,
+                                 out.cuda().contiguous(), lse.cuda().contiguous(), dO,
+                                 k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp, num_splits=num_splits,
+                                 dev_status=st)
+    torch.cuda.synchronize()
+    assert spa.read_status(st) == 0
+    return g
+
+
+def oracle_bwd(name, shrink, rows=None, indptr=None, indices=None, sink="w", o_saved=None, lse_saved=None):
+    import oracle
+    w = workload(name, shrink)
+    ip, idx = oracle_sets(name, shrink) if indptr is None else (indptr, indices)
+    k_cmp, v_cmp = oracle_cmp_pools(name, shrink)
+    return oracle.sparse_sink_attn_bwd(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx,
+                                       w.sink if isinstance(sink, str) else sink, w.scale, dout_bits(name, shrink),
+                                       k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp,
+                                       rows=None if rows is None else np.asarray(rows, dtype=np.int32),
+                                       o_saved=o_saved, lse_saved=lse_saved)
+
+
+def oracle_fwd_sets(name, shrink, ip, idx, sink):
+    import oracle
+    w = workload(name, shrink)
+    k_cmp, v_cmp = oracle_cmp_pools(name, shrink)
+    return oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, sink, w.scale,
+                                   k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp)
+
+
+GRAD_NAMES = ("dq", "dk_raw", "dv_raw", "dk_cmp", "dv_cmp", "dsink")
+
+
+def check_all_grads(g, r, what):
+    worst = {}
+    for n, a, ref in zip(GRAD_NAMES, g, r):
+        if ref is None:
+            assert a is None or float(a.abs().max()) == 0.0, n
+            continue
+        worst[n] = check_grad(a, ref, f"{what} {n}")
+    return worst
+
+
+def saved_case(spa, name, shrink, num_splits=0, ip=None, idx=None, sink="w"):
+    """GPU backward and oracle backward on the same saved O/LSE."""
+    w = workload(name, shrink)
+    if ip is None:
+        ip, idx = oracle_sets(name, shrink)
+    s = w.sink if isinstance(sink, str) else np.full(w.H, -np.inf, dtype=np.float32)
+    O, L = oracle_fwd_sets(name, shrink, ip, idx, s)
+    o_bf, l_f32, o64, l64 = saved_from_oracle(O, L)
+    b = batch(spa, name, shrink)
+    g = gpu_bwd(spa, b, name, shrink, o_bf, l_f32, num_splits=num_splits,
+                indptr=torch.from_numpy(ip).cuda(), indices=torch.from_numpy(idx).cuda(), sink=sink)
+    r = oracle_bwd(name, shrink, indptr=ip, indices=idx, sink=s, o_saved=o64, lse_saved=l64)
+    if sink is None:
+        r = r[:5] + (None,)
+    return g, r
+
+
+@pytest.mark.parametrize("name,shrink", [("c1", 1), ("c2", 8), ("c3", 16), ("c4", 16)])
+def test_bwd_every_element_small(spa, name, shrink):
+    g, r = saved_case(spa, name, shrink)
+    worst = check_all_grads(g, r, f"{name}/{shrink}")
+    print(name, shrink, {k: f"{v:.2e}" for k, v in worst.items()})
+
+
+@pytest.mark.parametrize("splits", [1, 3, 16])
+def test_bwd_split_counts(spa, splits):
+    g, r = saved_case(spa, "c4", 8, num_splits=splits)
+    check_all_grads(g, r, f"splits={splits}")
+
+
+def test_bwd_no_sink_and_empty_sets(spa):
+    w = workload("c1")
+    ip, idx = oracle_sets("c1")
+    keep = np.ones(w.N, dtype=bool)
+    keep[::3] = False
+    sizes = np.diff(ip) * keep
+    ip2 = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    idx2 = np.concatenate([idx[ip[i]:ip[i + 1]] for i in range(w.N) if keep[i]]).astype(np.int32)
+    for sink in ("w", None):
+        g, r = saved_case(spa, "c1", 1, ip=ip2, idx=idx2, sink=sink)
+        check_all_grads(g, r, f"empty sets, sink={sink}")
+        assert float(g[0][torch.from_numpy(~keep).cuda()].abs().max()) == 0.0
+
+
+def test_bwd_chain_from_the_cuda_forward(spa):
+    """The CUDA forward's O and LSE into the CUDA backward, against the
+    exact gradients: relative Frobenius error per gradient."""
+    name, shrink = "c3", 16
+    w = workload(name, shrink)
+    b = batch(spa, name, shrink)
+    b.step()
+    torch.cuda.synchronize()
+    g = gpu_bwd(spa, b, name, shrink, b.out, b.lse)
+    r = oracle_bwd(name, shrink)
+    for n, a, ref in zip(GRAD_NAMES, g, r):
+        if ref is None:
+            continue
+        a = a.double().cpu().numpy().reshape(ref.shape)
+        rel = np.linalg.norm(a - ref) / np.linalg.norm(ref)
+        assert rel <= G_CHAIN, f"{n}: relative error {rel:.3g}"
+
+
+def test_bwd_full_size_sampled_dq(spa):
+    """c3 at full size in the benchmark's launch configuration (the CUDA
+    forward's O/LSE for every token, the oracle's saved O/LSE for the
+    sampled tokens): dq of the sampled tokens against the oracle (a token's
+    dq depends only on its own saved O/LSE)."""
+    import oracle
+    name = "c3"
+    w = workload(name)
+    b = batch(spa, name)
+    b.step()
+    torch.cuda.synchronize()
+    rows = sample_rows(w, n_random=24)
+    O, L = oracle_attn(name, 1, rows)
+    o_bf, l_f32, o64, l64 = saved_from_oracle(O, L)
+    out, lse = b.out.clone(), b.lse.clone()
+    ridx = torch.from_numpy(rows).long().cuda()
+    out[ridx] = o_bf.cuda()
+    lse[ridx] = l_f32.cuda()
+    g = gpu_bwd(spa, b, name, 1, out, lse)
+    o_full = np.zeros((w.N, w.H, w.d))
+    l_full = np.zeros((w.N, w.H))
+    o_full[rows] = o64
+    l_full[rows] = l64
+    r = oracle_bwd(name, 1, rows=rows, o_saved=o_full, lse_saved=l_full)
+    check_grad(g[0][ridx], r[0], "c3 dq sampled")
+    for t in g[1:5]:
+        assert torch.isfinite(t).all()

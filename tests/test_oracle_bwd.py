@@ -274,8 +274,8 @@ def test_saved_o_enters_only_through_d(oracle):
     np.testing.assert_allclose(moved[0] - base[0], -pr.scale * dD[:, :, None] * PK, rtol=1e-9, atol=1e-13)
     p_sink = np.exp(pr.sink.astype(np.float64)[None, :] - L)
     np.testing.assert_allclose(moved[5] - base[5], -(p_sink * dD).sum(axis=0), rtol=1e-9, atol=1e-13)
-    np.testing.assert_allclose(moved[2], base[2], rtol=0, atol=0)
-    np.testing.assert_allclose(moved[4], base[4], rtol=0, atol=0)
+    np.testing.assert_allclose(moved[2], base[2], rtol=1e-13, atol=1e-14)   # summation order varies by thread
+    np.testing.assert_allclose(moved[4], base[4], rtol=1e-13, atol=1e-14)
 
 
 def test_saved_lse_scales_every_gradient(oracle):
