@@ -311,9 +311,9 @@ int spa_sparse_sink_attn_fwd_fp8(
  *            contiguous, 16-B aligned) and LSE (FP32 [n_queries, num_heads])
  * dout       dO, BF16 [n_queries, num_heads, head_dim], contiguous, 16-B aligned
  * dq         FP32 [n_queries, num_heads, head_dim], 16-B aligned
- * dk_raw, dv_raw  FP32 [raw_num_pages * raw_page_size, head_dim]: the raw
- *            pools' gradient rows; dk_cmp, dv_cmp likewise for the
- *            compressed pool (required when pt_cmp is set)
+ * dk_raw, dv_raw  FP32 [raw_num_pages * raw_page_size, head_dim], 16-B
+ *            aligned: the raw pools' gradient rows; dk_cmp, dv_cmp likewise
+ *            for the compressed pool (required when pt_cmp is set)
  * dsink      FP32 [num_heads] or NULL (ignored when sink is NULL)
  * Every gradient is ADDED into its array (zero them for a fresh gradient);
  * the additions are FP32 atomics, so their order, and the last bits of a

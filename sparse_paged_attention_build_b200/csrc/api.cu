@@ -415,10 +415,10 @@ int spa_sparse_sink_attn_bwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
     return fail(SPA_ERR_INVALID_ARG, "dq, dk_raw and dv_raw must be non-NULL");
   if (pt_cmp != nullptr && (dk_cmp == nullptr || dv_cmp == nullptr))
     return fail(SPA_ERR_INVALID_ARG, "dk_cmp/dv_cmp NULL with pt_cmp set");
-  if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dq, 16))
-    return fail(SPA_ERR_ALIGNMENT, "out, dout and dq must be 16-byte aligned");
-  if (!aligned(lse, 4) || !aligned(dk_raw, 4) || !aligned(dv_raw, 4) || !aligned(dk_cmp, 4) ||
-      !aligned(dv_cmp, 4) || !aligned(dsink, 4))
+  if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk_raw, 16) ||
+      !aligned(dv_raw, 16) || !aligned(dk_cmp, 16) || !aligned(dv_cmp, 16))
+    return fail(SPA_ERR_ALIGNMENT, "out, dout, dq, dk and dv must be 16-byte aligned");
+  if (!aligned(lse, 4) || !aligned(dsink, 4))
     return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
   a.num_splits = resolve_splits(n_queries, num_heads, num_splits);
   a.o_saved = out;

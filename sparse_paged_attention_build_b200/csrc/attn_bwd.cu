@@ -113,7 +113,10 @@ struct Layout {
   // p_ready, pd_free[2], g_full[2], g_free[2], dq_full, dq_free, mma_done
   static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 2 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kUsed = kMiscOff + 16;
+  // a 2 KB staging area per reducer warp: gradient rows leave through it as
+  // coalesced 16-byte reductions
+  static constexpr int kStageOff = (kMiscOff + 16 + 127) / 128 * 128;
+  static constexpr int kUsed = kStageOff + 4 * 2048;
   static constexpr int kBytes = kUsed + 1024;                   // + alignment slack
   static constexpr uint32_t kSCol = 0;
   static constexpr uint32_t kDPCol = kT;
@@ -122,6 +125,7 @@ struct Layout {
   static_assert(kDQCol + 128 <= kTmemCols, "TMEM budget");
   static_assert(kBytes <= 227 * 1024, "shared memory");
   static_assert(kPOff % 1024 == 0 && kKOff % 1024 == 0 && kVOff % 1024 == 0, "swizzle atoms");
+  static_assert(kStageOff % 16 == 0, "16-byte staging accesses");
 };
 
 struct Bars {
@@ -240,7 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
 
   if (warp == kResolverWarp) {
     // ================================================= resolver
-    resolver_loop(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane);
+    // contiguous ranges of units: concurrent CTAs then add into distant
+    // gradient rows (consecutive queries share most of their window keys)
+    resolver_loop(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane, true);
   } else if (warp == kKWarp || warp == kVWarp) {
     // ================================================= K / V gather (TMA)
     // As in the forward: lane j issues one tile::gather4 (four rows, 64
@@ -524,8 +530,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
     if (row_ok && P.dsink != nullptr && dsink_acc != 0.f) atomicAdd(P.dsink + h, dsink_acc);
   } else if (warp >= kRedWarp0) {
     // ================================================= gradient reductions
-    const int r = tid - kRedWarp0 * 32;   // TMEM lane: d index of dV^T/dK^T, head row of dQ
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    // Thread r holds TMEM lane r: the d index r of dV^T/dK^T (keys along
+    // the columns), the head row r of dQ. Rows leave through the warp's
+    // staging area so that every reduction is a 16-byte vector covering a
+    // contiguous piece of one gradient row.
+    const int wq = warp - kRedWarp0;                   // this warp's 32 d / head rows
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    float* stg = reinterpret_cast<float*>(smem + L::kStageOff + wq * 2048);
+    const bool d_ok = wq * 32 < D;                     // warp-uniform (d = 64: two warps idle)
     int c = 0, g = 0, ud = 0;
     bool ok = true, final_seen = false;
     while (ok && !final_seen) {
@@ -554,28 +566,45 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
             tc_fence_before_sync();
             mbar_arrive(B.g_free + (g & 1));
           }
-          if (r < D) {
+          if (!d_ok) continue;
 #pragma unroll
-            for (int cc = 0; cc < 32; ++cc) {
-              const int j = 32 * hk + cc;
-              const uint32_t e = j < nv ? t_rows[t * kT + j] : kInvalidRow;
-              if (e == kInvalidRow) continue;
-              const int64_t off = static_cast<int64_t>(e & ~kRawBit) * D + r;
-              const bool raw = (e & kRawBit) != 0;
-              atomicAdd((raw ? P.dv_raw : P.dv_cmp) + off, __uint_as_float(dv[cc]));
-              atomicAdd((raw ? P.dk_raw : P.dk_cmp) + off, __uint_as_float(dk[cc]));
+          for (int which = 0; which < 2; ++which) {
+            const uint32_t* vals = which == 0 ? dv : dk;
+            float* pool_raw = which == 0 ? P.dv_raw : P.dk_raw;
+            float* pool_cmp = which == 0 ? P.dv_cmp : P.dk_cmp;
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+              // 16 keys x this warp's 32 d: key-major rows of 128 bytes
+#pragma unroll
+              for (int kl = 0; kl < 16; ++kl) stg[kl * 32 + lane] = __uint_as_float(vals[16 * pass + kl]);
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int item = lane + 32 * k, kl = item >> 3, c4 = item & 7;
+                const float4 v = reinterpret_cast<const float4*>(stg)[kl * 8 + c4];
+                const int j = 32 * hk + 16 * pass + kl;
+                const uint32_t e = j < nv ? t_rows[t * kT + j] : kInvalidRow;
+                if (e == kInvalidRow) continue;
+                float* dst = ((e & kRawBit) ? pool_raw : pool_cmp) + static_cast<int64_t>(e & ~kRawBit) * D +
+                             wq * 32 + 4 * c4;
+                red_add_v4_f32(dst, v);
+              }
+              __syncwarp();   // the stage is rewritten next
             }
           }
         }
         if ((d.flags & kFlagLast) && t == ntiles - 1) {
-          // dQ of the unit: head row r, FP32, added into dq
+          // dQ of the unit (head row r), added into dq: 16 columns of the
+          // warp's 32 rows per pass through the stage, then 8 rows x 64
+          // contiguous bytes per vector reduction
           if (!__all_sync(0xffffffffu, mbar_wait(B.dq_full, ud & 1, abort_flag, P.dev_status))) {
             ok = false;
             break;
           }
           ++ud;
           tc_fence_after_sync();
-          float* dq_row = P.dq + (static_cast<int64_t>(d.i) * P.num_heads + head0 + r) * D;
+          float* dq_base = P.dq + (static_cast<int64_t>(d.i) * P.num_heads + head0 + wq * 32) * D;
+          const int swz = (lane >> 1) & 3;
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t v[32];
@@ -585,12 +614,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
               tc_fence_before_sync();
               mbar_arrive(B.dq_free);
             }
-            if (r < heads_here) {
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                atomicAdd(reinterpret_cast<float4*>(dq_row + c0 + 4 * q),
-                          make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                      __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+            for (int hf = 0; hf < 2; ++hf) {
+              float4* row = reinterpret_cast<float4*>(stg + lane * 16);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                row[q ^ swz] = make_float4(__uint_as_float(v[16 * hf + 4 * q]), __uint_as_float(v[16 * hf + 4 * q + 1]),
+                                           __uint_as_float(v[16 * hf + 4 * q + 2]), __uint_as_float(v[16 * hf + 4 * q + 3]));
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int rr = 8 * k + (lane >> 2), piece = lane & 3;
+                const float4 x = reinterpret_cast<const float4*>(stg + rr * 16)[piece ^ ((rr >> 1) & 3)];
+                if (wq * 32 + rr < heads_here)
+                  red_add_v4_f32(dq_base + static_cast<int64_t>(rr) * D + c0 + 16 * hf + 4 * piece, x);
+              }
+              __syncwarp();
             }
           }
         }

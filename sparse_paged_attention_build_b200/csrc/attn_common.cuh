@@ -88,17 +88,23 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
   }
 }
 
-// The resolver warp: walks this CTA's units (query i, slice) in a fixed
-// stride, splits each slice's keys into chunks of up to kChunkKeys, resolves
-// them into the double-buffered table and publishes a descriptor per chunk.
-// An empty slice still gets one (empty) chunk so that every role sees every
-// unit. S = slices per query.
+// The resolver warp: walks this CTA's units (query i, slice), splits each
+// slice's keys into chunks of up to kChunkKeys, resolves them into the
+// double-buffered table and publishes a descriptor per chunk. An empty slice
+// still gets one (empty) chunk so that every role sees every unit. S =
+// slices per query. The CTA's units are every gridDim.x-th one (strided) or
+// one contiguous range of about n_units / gridDim.x (contiguous: at any
+// moment the CTAs then work on queries far apart, whose windows do not
+// overlap).
 template <class Prm>
 __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* desc, uint64_t* tab_full,
-                              uint64_t* tab_empty, volatile int* abort_flag, int lane) {
+                              uint64_t* tab_empty, volatile int* abort_flag, int lane, bool contiguous = false) {
   int c = 0;
   const int64_t n_units = static_cast<int64_t>(P.n_queries) * S;
-  for (int64_t u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x) {
+  const int64_t u0 = contiguous ? (static_cast<int64_t>(blockIdx.x) * n_units) / gridDim.x : blockIdx.x;
+  const int64_t u_end = contiguous ? (static_cast<int64_t>(blockIdx.x + 1) * n_units) / gridDim.x : n_units;
+  const int64_t step = contiguous ? 1 : gridDim.x;
+  for (int64_t u = u0; u < u_end && !*abort_flag; u += step) {
     const int i = static_cast<int>(u / S);
     const int split = static_cast<int>(u - static_cast<int64_t>(i) * S);
     const int32_t set_begin = __ldg(P.indptr + i);
@@ -113,7 +119,7 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
     const int tile_hi = static_cast<int>((static_cast<int64_t>(tiles_total) * (split + 1)) / S);
     const int32_t key_lo = tile_lo * kT;
     const int32_t key_hi = min(tile_hi * kT, set_len);
-    const bool final_unit = u + gridDim.x >= n_units;
+    const bool final_unit = u + step >= u_end;
     int32_t k0 = key_lo;
     do {
       const int slot = c & 1;

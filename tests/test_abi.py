@@ -248,9 +248,10 @@ def bwd_call(L, **kw):
     (dict(dq=None), 1, "dq, dk_raw and dv_raw"),
     (dict(dvr=None), 1, "dq, dk_raw and dv_raw"),
     (dict(dkc=None), 1, "dk_cmp/dv_cmp NULL"),
-    (dict(dq=FAKE + 4), 5, "out, dout and dq"),
-    (dict(dout=FAKE + 2), 5, "out, dout and dq"),
-    (dict(dkr=FAKE + 2), 5, "32-bit arrays"),
+    (dict(dq=FAKE + 4), 5, "out, dout, dq, dk and dv"),
+    (dict(dout=FAKE + 2), 5, "out, dout, dq, dk and dv"),
+    (dict(dkr=FAKE + 4), 5, "out, dout, dq, dk and dv"),
+    (dict(lse=FAKE + 2), 5, "32-bit arrays"),
     (dict(dsink=FAKE + 1), 5, "32-bit arrays"),
 ])
 def test_guard_matrix_attention_bwd(L, kw, status, clause):
