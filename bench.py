@@ -142,7 +142,7 @@ def measured_traffic(w, args):
         return None
     rec = json.load(open(path))
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "spa_device.cuh"):
+    for f in ("attn_fwd.cu", "attn_common.cuh", "spa_device.cuh"):
         h.update(open(os.path.join(ROOT, "sparse_paged_attention_build_b200", "csrc", f), "rb").read())
     fused = w.k_cmp_fp8 is not None and args.fp8_path == "fused"
     entry = rec.get(w.name + (":fused" if fused else ""))

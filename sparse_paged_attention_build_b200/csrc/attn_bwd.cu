@@ -36,10 +36,12 @@
 //   warps 8-11  thread t owns TMEM lane t: reads dV^T/dK^T rows (d index t)
 //               and adds them into the gradient pools, and at the end of a
 //               unit reads dQ (head row t) and adds it into dq
-// TMEM columns: S [0,64), dP [64,128), two dV^T|dK^T buffers [128,256) and
+// TMEM columns: two S|dP buffers [0,128) and [128,256), dV^T|dK^T
 // [256,384), dQ [384,512). Per tile the UMMA thread issues S/dP of tile g
-// before the dQ/dV/dK products of tile g-1, so the softmax of tile g runs
-// while the tensor core does the rest of tile g-1.
+// (into buffer g&1, without waiting for the softmax of tile g-1) and then
+// the dQ/dV/dK products of tile g-1 once its P and dS are written, so the
+// softmax of consecutive tiles runs back to back while the tensor core does
+// the rest.
 #include <cmath>
 #include <cstring>
 
@@ -109,19 +111,19 @@ struct Layout {
   static constexpr int kTabOff = kPOff + 4 * kPBytes;           // [2][kChunkKeys] u32
   static constexpr int kDescOff = kTabOff + 2 * kChunkKeys * 4;
   static constexpr int kBarOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
-  // tab_full[2], tab_empty[2], qd_full, qd_empty, K ring, V ring, s_full,
-  // p_ready, pd_free[2], g_full[2], g_free[2], dq_full, dq_free, mma_done
-  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 2 + 3;
+  // tab_full[2], tab_empty[2], qd_full, qd_empty, K ring, V ring, s_full[2],
+  // p_ready, pd_free[2], g_full, g_free, dq_full, dq_free, mma_done
+  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 1 + 2 + 1 + 1 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // a 2 KB staging area per reducer warp: gradient rows leave through it as
   // coalesced 16-byte reductions
   static constexpr int kStageOff = (kMiscOff + 16 + 127) / 128 * 128;
   static constexpr int kUsed = kStageOff + 4 * 2048;
   static constexpr int kBytes = kUsed + 1024;                   // + alignment slack
-  static constexpr uint32_t kSCol = 0;
+  static constexpr uint32_t kSCol = 0;                          // buffer b: S at 128 b, dP at 128 b + 64
   static constexpr uint32_t kDPCol = kT;
-  static constexpr uint32_t kGCol = 2 * kT;                     // buffer b at kGCol + 128 b
-  static constexpr uint32_t kDQCol = kGCol + 256;
+  static constexpr uint32_t kGCol = 4 * kT;                     // dV^T, then dK^T
+  static constexpr uint32_t kDQCol = kGCol + 2 * kT;
   static_assert(kDQCol + 128 <= kTmemCols, "TMEM budget");
   static_assert(kBytes <= 227 * 1024, "shared memory");
   static_assert(kPOff % 1024 == 0 && kKOff % 1024 == 0 && kVOff % 1024 == 0, "swizzle atoms");
@@ -137,11 +139,11 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;     // [kStagesV]
   uint64_t* v_empty;
-  uint64_t* s_full;     // S and dP of the current tile in TMEM
+  uint64_t* s_full;     // [2] S and dP of buffer b in TMEM
   uint64_t* p_ready;    // P and dS of the current tile in shared memory (S/dP read)
   uint64_t* pd_free;    // [2] the products reading P/dS buffer b have completed
-  uint64_t* g_full;     // [2] dV^T/dK^T of buffer b complete
-  uint64_t* g_free;     // [2] ... and read out
+  uint64_t* g_full;     // dV^T/dK^T of the tile complete
+  uint64_t* g_free;     // ... and read out
   uint64_t* dq_full;    // dQ of the unit complete
   uint64_t* dq_free;    // ... and read out
   uint64_t* mma_done;
@@ -180,11 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
   B.v_full = B.k_empty + kStagesK;
   B.v_empty = B.v_full + kStagesV;
   B.s_full = B.v_empty + kStagesV;
-  B.p_ready = B.s_full + 1;
+  B.p_ready = B.s_full + 2;
   B.pd_free = B.p_ready + 1;
   B.g_full = B.pd_free + 2;
-  B.g_free = B.g_full + 2;
-  B.dq_full = B.g_free + 2;
+  B.g_free = B.g_full + 1;
+  B.dq_full = B.g_free + 1;
   B.dq_free = B.dq_full + 1;
   B.mma_done = B.dq_free + 1;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
@@ -212,8 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       mbar_init(B.tab_full + s, 32);
       mbar_init(B.tab_empty + s, kTabConsumers);
       mbar_init(B.pd_free + s, 1);
-      mbar_init(B.g_full + s, 1);
-      mbar_init(B.g_free + s, 128);
+      mbar_init(B.s_full + s, 1);
     }
     mbar_init(B.qd_full, 1);
     mbar_init(B.qd_empty, 1);
@@ -225,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       mbar_init(B.v_full + s, 1);
       mbar_init(B.v_empty + s, 1);
     }
-    mbar_init(B.s_full, 1);
+    mbar_init(B.g_full, 1);
+    mbar_init(B.g_free, 128);
     mbar_init(B.p_ready, kSoftThreads);
     mbar_init(B.dq_full, 1);
     mbar_init(B.dq_free, 128);
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       int pg = 0;
       // dQ, dV^T and dK^T of tile gg (its P and dS are in shared memory)
       auto issue_d = [&](int gg, bool first, bool last) -> bool {
-        if (!mbar_wait(B.g_free + (gg & 1), ((gg >> 1) & 1) ^ 1, abort_flag, P.dev_status)) return false;
+        if (!mbar_wait(B.g_free, (gg & 1) ^ 1, abort_flag, P.dev_status)) return false;
         if (first) {
           if (!mbar_wait(B.dq_free, (ud & 1) ^ 1, abort_flag, P.dev_status)) return false;
           ++ud;
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
         const uint32_t k_addr = sbase + L::kKOff + (gg % kStagesK) * L::kTileBytes;
         const uint32_t p_addr = sbase + L::kPOff + (gg & 1) * 2 * L::kPBytes;
         const uint32_t ds_addr = p_addr + L::kPBytes;
-        const uint32_t gcol = L::kGCol + (gg & 1) * 128;
+        const uint32_t gcol = L::kGCol;
 #pragma unroll
         for (int k = 0; k < kT / 16; ++k) {   // K-dim: 16 keys per step
           const uint64_t a = smem_desc_sw128(ds_addr + k * 32, 16, 1024);
@@ -365,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
         }
         tc_commit(B.k_empty + gg % kStagesK);
         tc_commit(B.pd_free + (gg & 1));
-        tc_commit(B.g_full + (gg & 1));
+        tc_commit(B.g_full);
         if (last) {
           tc_commit(B.dq_full);
           tc_commit(B.qd_empty);
@@ -392,28 +394,35 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
             ok = false;
             break;
           }
-          // S/dP are single-buffered: the softmax has read those of tile pg
-          if (pending && !mbar_wait(B.p_ready, pg & 1, abort_flag, P.dev_status)) { ok = false; break; }
+          // S/dP buffer g&1 was last read by the softmax of tile g-2, whose
+          // P/dS the dQ/dV/dK products of that tile (issued before this)
+          // waited for
           tc_fence_after_sync();
+          const uint32_t sb = (g & 1) * 128;
           const uint32_t k_addr = sbase + L::kKOff + (g % kStagesK) * L::kTileBytes;
           const uint32_t v_addr = sbase + L::kVOff + (g & 1) * L::kTileBytes;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {   // K-dim: 16 columns of d per step
             const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
             const uint32_t toff = (k >> 2) * (kT * 128) + (k & 3) * 32;
-            umma_ss(tmem + L::kSCol, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + toff, 16, 1024),
+            umma_ss(tmem + L::kSCol + sb, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + toff, 16, 1024),
                     id_s, k > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
             const uint32_t toff = (k >> 2) * (kT * 128) + (k & 3) * 32;
-            umma_ss(tmem + L::kDPCol, smem_desc_sw128(do_addr + off, 16, 1024),
+            umma_ss(tmem + L::kDPCol + sb, smem_desc_sw128(do_addr + off, 16, 1024),
                     smem_desc_sw128(v_addr + toff, 16, 1024), id_s, k > 0 ? 1u : 0u);
           }
           tc_commit(B.v_empty + (g & 1));
-          tc_commit(B.s_full);
-          if (pending && !issue_d(pg, p_first, p_last)) { ok = false; break; }
+          tc_commit(B.s_full + (g & 1));
+          // then the rest of the previous tile, once its P and dS are in
+          // shared memory: the softmax of this tile overlaps those products
+          if (pending && (!mbar_wait(B.p_ready, pg & 1, abort_flag, P.dev_status) || !issue_d(pg, p_first, p_last))) {
+            ok = false;
+            break;
+          }
           pending = true;
           pg = g;
           p_first = first;
@@ -482,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
             if ((d.flags & kFlagSetStart) && sink2 > -INFINITY) dsink_acc -= exp2_approx(sink2 - lse2) * Dh;
           }
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full, g & 1, abort_flag, P.dev_status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full + (g & 1), (g >> 1) & 1, abort_flag, P.dev_status))) {
           ok = false;
           break;
         }
@@ -498,8 +507,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t s[32], dp[32];
-          tmem_ld32(lane_addr + L::kSCol + 32 * hf, s);
-          tmem_ld32(lane_addr + L::kDPCol + 32 * hf, dp);
+          tmem_ld32(lane_addr + L::kSCol + (g & 1) * 128 + 32 * hf, s);
+          tmem_ld32(lane_addr + L::kDPCol + (g & 1) * 128 + 32 * hf, dp);
           tmem_ld_wait(s);
           tmem_ld_wait(dp);
           uint32_t pk[16], dk[16];
@@ -548,13 +557,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       const uint32_t* t_rows = tab + slot * kChunkKeys;
       const int ntiles = ceil_tiles(d.nkeys);
       for (int t = 0; t < ntiles; ++t, ++g) {
-        if (!__all_sync(0xffffffffu, mbar_wait(B.g_full + (g & 1), (g >> 1) & 1, abort_flag, P.dev_status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.g_full, g & 1, abort_flag, P.dev_status))) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
         const int nv = min(kT, d.nkeys - t * kT);
-        const uint32_t gcol = L::kGCol + (g & 1) * 128;
+        const uint32_t gcol = L::kGCol;
 #pragma unroll 1
         for (int hk = 0; hk < 2; ++hk) {
           uint32_t dv[32], dk[32];
@@ -564,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
           tmem_ld_wait(dk);
           if (hk == 1) {   // both halves are in registers: the buffer is free
             tc_fence_before_sync();
-            mbar_arrive(B.g_free + (g & 1));
+            mbar_arrive(B.g_free);
           }
           if (!d_ok) continue;
 #pragma unroll
@@ -578,16 +587,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
 #pragma unroll
               for (int kl = 0; kl < 16; ++kl) stg[kl * 32 + lane] = __uint_as_float(vals[16 * pass + kl]);
               __syncwarp();
+              // every read first, then the four reductions (their source
+              // registers stay untouched until the reductions have issued)
+              float4 v[4];
+              uint32_t e[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const int item = lane + 32 * k, kl = item >> 3, c4 = item & 7;
-                const float4 v = reinterpret_cast<const float4*>(stg)[kl * 8 + c4];
+                v[k] = reinterpret_cast<const float4*>(stg)[kl * 8 + c4];
                 const int j = 32 * hk + 16 * pass + kl;
-                const uint32_t e = j < nv ? t_rows[t * kT + j] : kInvalidRow;
-                if (e == kInvalidRow) continue;
-                float* dst = ((e & kRawBit) ? pool_raw : pool_cmp) + static_cast<int64_t>(e & ~kRawBit) * D +
+                e[k] = j < nv ? t_rows[t * kT + j] : kInvalidRow;
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (e[k] == kInvalidRow) continue;
+                const int c4 = (lane + 32 * k) & 7;
+                float* dst = ((e[k] & kRawBit) ? pool_raw : pool_cmp) + static_cast<int64_t>(e[k] & ~kRawBit) * D +
                              wq * 32 + 4 * c4;
-                red_add_v4_f32(dst, v);
+                red_add_v4_f32(dst, v[k]);
               }
               __syncwarp();   // the stage is rewritten next
             }
@@ -622,12 +639,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
                 row[q ^ swz] = make_float4(__uint_as_float(v[16 * hf + 4 * q]), __uint_as_float(v[16 * hf + 4 * q + 1]),
                                            __uint_as_float(v[16 * hf + 4 * q + 2]), __uint_as_float(v[16 * hf + 4 * q + 3]));
               __syncwarp();
+              float4 x[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const int rr = 8 * k + (lane >> 2), piece = lane & 3;
-                const float4 x = reinterpret_cast<const float4*>(stg + rr * 16)[piece ^ ((rr >> 1) & 3)];
+                x[k] = reinterpret_cast<const float4*>(stg + rr * 16)[piece ^ ((rr >> 1) & 3)];
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int rr = 8 * k + (lane >> 2), piece = lane & 3;
                 if (wq * 32 + rr < heads_here)
-                  red_add_v4_f32(dq_base + static_cast<int64_t>(rr) * D + c0 + 16 * hf + 4 * piece, x);
+                  red_add_v4_f32(dq_base + static_cast<int64_t>(rr) * D + c0 + 16 * hf + 4 * piece, x[k]);
               }
               __syncwarp();
             }
