@@ -17,6 +17,9 @@ What each function follows (page title, then section):
 * :func:`sparse_sink_attn` -- "Roadmap item 24", "Reuse and arithmetic"
   (one denominator for compressed KV, window and sink; the sink has no V;
   natural-log LSE) and "MI300X validation" (an FP64 O/LSE oracle).
+* :func:`unpack_d512_pages` -- "Roadmap item 24", review notes on the packed
+  joint KV gather (584 bytes per token for a 512-wide head, 576 of them
+  data): 448 E4M3 codes with UE8M0 scales per 64, 64 BF16 values.
 * :func:`sparse_sink_attn_bwd` -- "Roadmap item 24", the backward named as
   its follow-on item (dQ, dK/dV, d_sink): the chain rule through the forward
   above, with the sink's logit carrying no V.
@@ -86,6 +89,10 @@ def lib() -> ctypes.CDLL:
             L.oracle_dequant_fp8_pages_fmt.restype = ctypes.c_int
             L.oracle_e4m3fnuz_to_double.argtypes = [ctypes.c_uint8]
             L.oracle_e4m3fnuz_to_double.restype = dbl
+            L.oracle_ue8m0_to_double.argtypes = [ctypes.c_uint8]
+            L.oracle_ue8m0_to_double.restype = dbl
+            L.oracle_unpack_d512_pages.argtypes = [P, i64, i32, P, i32, P]
+            L.oracle_unpack_d512_pages.restype = ctypes.c_int
             L.oracle_paged_kv_write.argtypes = [P, P, i32, i32, P, P, P, i32, i32, i32, i64, P, P]
             L.oracle_paged_kv_write.restype = ctypes.c_int
             L.oracle_sparse_sink_attn.argtypes = [
@@ -284,6 +291,25 @@ def lse_merge(lse_parts, o_parts):
     lse = np.zeros(1, dtype=np.float64)
     lib().oracle_lse_merge(S, _ptr(lse_parts), _ptr(o_parts), d, _ptr(o), _ptr(lse))
     return o, float(lse[0])
+
+
+def ue8m0_to_double(code: int) -> float:
+    return lib().oracle_ue8m0_to_double(int(code))
+
+
+def unpack_d512_pages(src, page_ids, dst=None):
+    """BF16 bits [pages, page_size, 512] of the listed pages of a packed
+    cache (uint8 [pages, page_size, 584]: 448 E4M3 codes, 64 BF16, 7 UE8M0
+    scale bytes, 1 unused byte per token)."""
+    src = _c(src, np.uint8)
+    P, ps, w = src.shape
+    assert w == 584
+    page_ids = _c(page_ids, np.int32)
+    if dst is None:
+        dst = np.zeros((P, ps, 512), dtype=np.uint16)
+    assert dst.dtype == np.uint16 and dst.flags.c_contiguous and dst.shape == (P, ps, 512)
+    _check(lib().oracle_unpack_d512_pages(_ptr(src), P, ps, _ptr(page_ids), page_ids.shape[0], _ptr(dst)))
+    return dst
 
 
 def paged_kv_write(k_new, v_new, req, pos, pt, k_pool, v_pool):

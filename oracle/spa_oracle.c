@@ -235,6 +235,49 @@ int oracle_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t nu
 }
 
 /* ------------------------------------------------------------------------ */
+/* Packed D512 rows (584 bytes per token).                                   */
+/* ------------------------------------------------------------------------ */
+
+/* UE8M0 scale byte: 2^(byte - 127); 0xFF is NaN. */
+double oracle_ue8m0_to_double(uint8_t b)
+{
+    if (b == 0xFF) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
+/* The packed row of a 512-wide head, 584 bytes per token ("Roadmap item 24"
+ * review: 584 bytes per token for head width 512, 576 of them data): 448
+ * E4M3 codes (the first 448 elements), 64 BF16 values (the last 64
+ * elements, 128 bytes), then 7 UE8M0 scale bytes (one per 64 codes) and one
+ * unused byte. Element e < 448 decodes to bf16_rne(float(e4m3(code_e)) *
+ * float(2^(scale_{e/64} - 127))), one binary32 multiply; e >= 448 is copied.
+ * src: [num_pages, page_size, 584] bytes; dst: [num_pages, page_size, 512]
+ * BF16 bits; only the listed pages are written. */
+int oracle_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size,
+                             const int32_t* page_ids, int32_t n, uint16_t* dst)
+{
+    if (page_size < 1 || n < 0) return ORACLE_BAD_ARG;
+    for (int32_t k = 0; k < n; ++k) {
+        int64_t pg = page_ids[k];
+        if (pg < 0 || pg >= num_pages) return ORACLE_BAD_PAGE;
+        for (int64_t t = 0; t < page_size; ++t) {
+            int64_t row = pg * page_size + t;
+            const uint8_t* in = src + row * 584;
+            uint16_t* out = dst + row * 512;
+            for (int32_t e = 0; e < 448; ++e) {
+                float value = (float)oracle_e4m3_to_double(in[e]);
+                float scale = (float)oracle_ue8m0_to_double(in[576 + e / 64]);
+                float product = value * scale; /* one binary32 multiply */
+                out[e] = oracle_float_to_bf16_rne(product);
+            }
+            for (int32_t e = 0; e < 64; ++e)
+                out[448 + e] = (uint16_t)(in[448 + 2 * e] | (in[448 + 2 * e + 1] << 8));
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Paged KV write.                                                           */
 /* ------------------------------------------------------------------------ */
 

@@ -250,3 +250,25 @@ def make_dout(w: Workload, seed: int = 0) -> np.ndarray:
     """A seeded output gradient dO for a workload: BF16 bits [N, H, d], N(0,1)."""
     rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([BASE_SEED, 77, seed])))
     return _normal_bf16(rng, (w.N, w.H, w.d))
+
+
+PACKED_D512_BYTES = 584
+
+
+def make_packed_d512(num_pages: int, page_size: int, seed: int = 0) -> np.ndarray:
+    """A seeded packed cache of 512-wide rows, uint8 [num_pages, page_size,
+    584]: per token 448 E4M3 codes (N(0,1) values divided by a power-of-two
+    scale per 64, the smallest that keeps them within 448, encoded by
+    PyTorch's float8_e4m3fn cast), 64 BF16 N(0,1) values, 7 UE8M0 scale
+    bytes (127 + log2 of the scale) and one zero byte."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([BASE_SEED, 584, seed])))
+    x = rng.standard_normal((num_pages, page_size, 7, 64)).astype(np.float32)
+    amax = np.maximum(np.abs(x).max(axis=3), 1e-30)
+    e = np.ceil(np.log2(amax / 448.0)).astype(np.int32)                   # 2^e >= amax / 448
+    codes = torch.from_numpy(x / np.ldexp(1.0, e)[..., None].astype(np.float32)).to(torch.float8_e4m3fn)
+    out = np.zeros((num_pages, page_size, PACKED_D512_BYTES), dtype=np.uint8)
+    out[..., :448] = codes.view(torch.uint8).numpy().reshape(num_pages, page_size, 448)
+    rope = _normal_bf16(rng, (num_pages, page_size, 64))
+    out[..., 448:576] = rope.view(np.uint8).reshape(num_pages, page_size, 128)
+    out[..., 576:583] = (127 + e).astype(np.uint8)
+    return out
