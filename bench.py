@@ -235,7 +235,7 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
                     help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
-    ap.add_argument("--op", default="path", choices=["path", "kv_write", "bwd"],
+    ap.add_argument("--op", default="path", choices=["path", "kv_write", "bwd", "unpack_d512"],
                     help="path: the attention hot path (the bench line); kv_write: the paged KV write alone; "
                          "bwd: the backward of the attention alone")
     ap.add_argument("--no-e2e", action="store_true")
@@ -253,6 +253,8 @@ def main():
         return run_kv_write(args, rank, local_rank, world)
     if args.op == "bwd":
         return run_bwd(args, rank, local_rank, world)
+    if args.op == "unpack_d512":
+        return run_unpack_d512(args, rank, local_rank, world)
 
     import torch
     import torch.distributed as dist
@@ -533,6 +535,65 @@ def run_bwd(args, rank, local_rank, world):
                          "frac": tflops / pk["bf16_tflops"], "peak_source": f"{pk_kind} BF16 burst",
                          "kernel": "sparse_sink_attn_bwd_kernel", "algorithmic_flops": flops},
             "gpu_launches": args.steps, "finite_and_status_ok": bool(ok)}))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_unpack_d512(args, rank, local_rank, world):
+    """The packed 512-wide row decode alone: a seeded packed cache of
+    8192 pages x 64 tokens (584 bytes per token; a 128-request, 4096-token
+    context in 64-token pages), every page decoded to BF16; HBM GB/s
+    against the copy peak. Algorithmic bytes per token: 584 read + 1024
+    written."""
+    import torch
+    import torch.distributed as dist
+    from sparse_paged_attention_build_b200 import workloads
+    import sparse_paged_attention_build_b200 as spa
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    pages, ps = 8192 // max(1, args.shrink), 64
+    src = torch.from_numpy(workloads.make_packed_d512(pages, ps, seed=rank)).cuda()
+    ids = torch.arange(pages, dtype=torch.int32, device="cuda")
+    dst = torch.empty((pages, ps, 512), dtype=torch.bfloat16, device="cuda")
+    st = spa.new_status()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            spa.unpack_d512_pages(src, ids, dst, dev_status=st)
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(args.warmup):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record()
+        g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in evs]))
+    tokens = pages * ps
+    bytes_step = tokens * (584 + 1024) + pages * 4
+    total_bytes, ms = job_totals(bytes_step, ms, world, "cuda")
+    pk, pk_kind = peaks()
+    gbs = total_bytes / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "packed D512 row decode HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 -> bf16", "data": "synthetic",
+            "config": {"workload": f"packed 512-wide rows: {pages} pages x {ps} tokens x 584 bytes",
+                       "l2": "256 MB buffer written between timed steps (L2 flush)"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "peak_source": f"{pk_kind} HBM copy",
+                         "kernel": "unpack_d512_kernel", "algorithmic_bytes": int(bytes_step)},
+            "gpu_launches": args.steps, "status_ok": spa.read_status(st) == 0}))
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -296,6 +296,27 @@ int spa_sparse_sink_attn_fwd_fp8(
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * 6. spa_unpack_d512_pages -- packed 512-wide rows (584 bytes per token)
+ * to BF16.
+ *
+ * "Roadmap item 24 - joint compressed/window attention with sink", review
+ * notes on the packed joint KV gather: 584 bytes per token for a 512-wide
+ * head, 576 of them data. Read as: bytes 0..447 OCP E4M3 codes (elements
+ * 0..447), bytes 448..575 BF16 (elements 448..511), bytes 576..582 UE8M0
+ * scales (2^(byte-127), one per 64 codes; 0xFF is NaN), byte 583 unused.
+ * Element e < 448 -> bf16_rne(float(e4m3) * 2^(s-127)); the rest copied.
+ *
+ * src        uint8 [num_pages, page_size, 584], 8-B aligned
+ * page_ids   int32 [n_page_ids]: the pages to decode; an id outside
+ *            [0, num_pages) sets SPA_DEV_BAD_PAGE and that page is skipped
+ * dst        BF16 [num_pages, page_size, 512], 16-B aligned; pages not
+ *            listed are left untouched
+ * page_size  1 .. 4096
+ * ---------------------------------------------------------------------- */
+int spa_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size, const int32_t* page_ids,
+                          int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * 5. spa_sparse_sink_attn_bwd -- gradients of the attention with sink.
  *
  * The follow-on item of "Roadmap item 24 - joint compressed/window attention

@@ -73,6 +73,8 @@ def _load():
     L.spa_sparse_sink_attn_fwd_fp8.restype = ctypes.c_int
     L.spa_paged_kv_write.argtypes = [P, P, i32, i32, P, P, P, i32, i32, i32, i64, P, P, P, P]
     L.spa_paged_kv_write.restype = ctypes.c_int
+    L.spa_unpack_d512_pages.argtypes = [P, i64, i32, P, i32, P, P, P]
+    L.spa_unpack_d512_pages.restype = ctypes.c_int
     L.spa_sparse_sink_attn_bwd.argtypes = [
         P, i64, i64, i32, i32, i32,
         P, P, i64, i32, P, i32,
@@ -332,6 +334,24 @@ def sparse_sink_attn_bwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
         _p(dout), _p(dq), _p(dk_raw), _p(dv_raw), _p(dk_cmp), _p(dv_cmp), _p(dsink), num_splits,
         _p(dev_status), _stream(stream)))
     return dq, dk_raw, dv_raw, dk_cmp, dv_cmp, dsink
+
+
+def unpack_d512_pages(src, page_ids, dst=None, dev_status=None, stream=None):
+    """BF16 [pages, page_size, 512] of the listed pages of a packed cache
+    (uint8 [pages, page_size, 584]: 448 E4M3 codes, 64 BF16 values, 7 UE8M0
+    scale bytes, 1 unused byte per token)."""
+    _need(src, "src", torch.uint8)
+    _need(page_ids, "page_ids", torch.int32)
+    assert src.is_contiguous() and src.dim() == 3 and src.shape[2] == 584
+    P, ps, _ = src.shape
+    if dst is None:
+        dst = torch.zeros((P, ps, 512), dtype=torch.bfloat16, device=src.device)
+    _need(dst, "dst", torch.bfloat16)
+    assert dst.is_contiguous() and tuple(dst.shape) == (P, ps, 512)
+    page_ids = page_ids.contiguous()
+    _check("spa_unpack_d512_pages", lib.spa_unpack_d512_pages(
+        _p(src), P, ps, _p(page_ids), page_ids.numel(), _p(dst), _p(dev_status), _stream(stream)))
+    return dst
 
 
 def paged_kv_write(k_new, v_new, req, pos, pt, k_pool, v_pool, dev_status=None, stream=None):

@@ -173,6 +173,22 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
 }
 
 // ---------------------------------------------------------------- attention
+int spa_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size, const int32_t* page_ids,
+                          int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status, spa_stream_t stream) {
+  if (num_pages < 0) return fail(SPA_ERR_INVALID_ARG, "num_pages < 0");
+  if (page_size < 1) return fail(SPA_ERR_INVALID_ARG, "page_size < 1");
+  if (n_page_ids < 0) return fail(SPA_ERR_INVALID_ARG, "n_page_ids < 0");
+  if (page_size > 4096) return fail(SPA_ERR_UNSUPPORTED, "page_size above 4096");
+  if (n_page_ids > 0 && (src == nullptr || page_ids == nullptr || dst == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "src, page_ids and dst must be non-NULL");
+  if (!aligned(src, 8)) return fail(SPA_ERR_ALIGNMENT, "src must be 8-byte aligned");
+  if (!aligned(dst, 16)) return fail(SPA_ERR_ALIGNMENT, "dst must be 16-byte aligned");
+  if (!aligned(page_ids, 4)) return fail(SPA_ERR_ALIGNMENT, "page_ids misaligned");
+  return cuda_status(spa::launch_unpack_d512_pages(src, num_pages, page_size, page_ids, n_page_ids, dst, dev_status,
+                                                   reinterpret_cast<cudaStream_t>(stream)),
+                     "unpack_d512_pages launch");
+}
+
 int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int32_t max_set_size) {
   if (n_queries <= 0 || num_heads <= 0) return 1;
   const int64_t head_tiles = (num_heads + 127) / 128;

@@ -29,6 +29,9 @@ cudaError_t launch_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, 
                                   int32_t head_dim, const int32_t* req, const int32_t* pos, const int32_t* pt,
                                   int32_t pt_cols, int32_t n_requests, int32_t page_size, int64_t num_pages,
                                   uint16_t* k_pool, uint16_t* v_pool, uint32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size,
+                                     const int32_t* page_ids, int32_t n_page_ids, uint16_t* dst,
+                                     uint32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_pages,
                                      int32_t page_size, int32_t head_dim, const int32_t* page_ids,
                                      int32_t n_page_ids, bool fnuz, uint16_t* dst, uint32_t* dev_status,

@@ -261,3 +261,29 @@ def test_guard_matrix_attention_bwd(L, kw, status, clause):
 
 def test_attention_bwd_zero_queries_is_a_no_op(L):
     assert bwd_call(L, n=0, q=None, out=None, lse=None, dout=None, dq=None, dkr=None, dvr=None) == 0
+
+
+def unpack_call(L, **kw):
+    a = dict(src=FAKE, P=10, ps=64, ids=FAKE, n=4, dst=FAKE)
+    a.update(kw)
+    return L.spa_unpack_d512_pages(a["src"], a["P"], a["ps"], a["ids"], a["n"], a["dst"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(P=-1), 1, "num_pages < 0"),
+    (dict(ps=0), 1, "page_size < 1"),
+    (dict(n=-1), 1, "n_page_ids < 0"),
+    (dict(ps=8192), 2, "page_size above 4096"),
+    (dict(src=None), 1, "src, page_ids and dst must be non-NULL"),
+    (dict(ids=None), 1, "src, page_ids and dst must be non-NULL"),
+    (dict(src=FAKE + 4), 5, "src must be 8-byte aligned"),
+    (dict(dst=FAKE + 8), 5, "dst must be 16-byte aligned"),
+    (dict(ids=FAKE + 2), 5, "page_ids misaligned"),
+])
+def test_guard_matrix_unpack_d512(L, kw, status, clause):
+    assert unpack_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
+def test_unpack_d512_zero_pages_is_a_no_op(L):
+    assert unpack_call(L, n=0, src=None, ids=None, dst=None) == 0

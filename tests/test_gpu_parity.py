@@ -663,3 +663,47 @@ def test_bwd_full_size_sampled_dq(spa):
     check_grad(g[0][ridx], r[0], "c3 dq sampled")
     for t in g[1:5]:
         assert torch.isfinite(t).all()
+
+
+# ---------------------------------------------------------------- packed D512 rows
+@pytest.mark.parametrize("pages,ps", [(64, 64), (5, 1), (3, 128)])
+def test_unpack_d512_bit_exact(spa, pages, ps):
+    import oracle
+    from sparse_paged_attention_build_b200 import workloads
+    src = workloads.make_packed_d512(pages, ps, seed=pages + ps)
+    ids = np.random.default_rng(ps).permutation(pages)[: max(1, pages - 2)].astype(np.int32)
+    ref = oracle.unpack_d512_pages(src, ids)
+    st = spa.new_status()
+    dst = spa.unpack_d512_pages(torch.from_numpy(src).cuda(), torch.from_numpy(ids).cuda(), dev_status=st)
+    torch.cuda.synchronize()
+    assert spa.read_status(st) == 0
+    got = dst.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_unpack_d512_every_code_scale_and_bad_page(spa):
+    """Every code under scale bytes 0 (a subnormal scale), 1, 120, 127, 140
+    and 254, NaN codes and the NaN scale compared by position; a bad page id
+    is reported and skipped."""
+    import oracle
+    src = np.zeros((2, 8, 584), dtype=np.uint8)
+    codes = np.arange(256, dtype=np.uint8)
+    src[:, :, :448] = np.concatenate([codes, codes[:192]])
+    for r, sb in enumerate((0, 1, 120, 127, 140, 254, 255, 127)):
+        src[:, r, 576:583] = sb
+    src[:, :, 448:576] = np.arange(128, dtype=np.uint8)
+    ids = np.array([0, 1], dtype=np.int32)
+    ref = oracle.unpack_d512_pages(src, ids)
+    st = spa.new_status()
+    dst = spa.unpack_d512_pages(torch.from_numpy(src).cuda(), torch.from_numpy(ids).cuda(), dev_status=st)
+    torch.cuda.synchronize()
+    got = dst.view(torch.int16).cpu().numpy().view(np.uint16)
+    nan_ref = (ref & 0x7F80 == 0x7F80) & (ref & 0x7F != 0)
+    nan_got = (got & 0x7F80 == 0x7F80) & (got & 0x7F != 0)
+    assert np.array_equal(nan_ref, nan_got)
+    assert np.array_equal(got[~nan_ref], ref[~nan_ref])
+    bad = torch.tensor([0, 7], dtype=torch.int32, device="cuda")
+    st2 = spa.new_status()
+    spa.unpack_d512_pages(torch.from_numpy(src).cuda(), bad, dev_status=st2)
+    torch.cuda.synchronize()
+    assert spa.read_status(st2) & 1   # SPA_DEV_BAD_PAGE
