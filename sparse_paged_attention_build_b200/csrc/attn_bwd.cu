@@ -107,13 +107,14 @@ struct Layout {
   static constexpr int kDOOff = 2 * kHalfBytes;                 // dO [2 halves]
   static constexpr int kKOff = 4 * kHalfBytes;
   static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
-  static constexpr int kPOff = kVOff + kStagesV * kTileBytes;   // [2] x (P, dS)
-  static constexpr int kTabOff = kPOff + 4 * kPBytes;           // [2][kChunkKeys] u32
+  static constexpr int kPOff = kVOff + kStagesV * kTileBytes;   // P, then dS
+  static constexpr int kBulkOff = kPOff + 2 * kPBytes;          // [64 keys][D] FP32: a dV or dK tile
+  static constexpr int kTabOff = kBulkOff + kT * D * 4;         // [2][kChunkKeys] u32
   static constexpr int kDescOff = kTabOff + 2 * kChunkKeys * 4;
   static constexpr int kBarOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
   // tab_full[2], tab_empty[2], qd_full, qd_empty, K ring, V ring, s_full[2],
-  // p_ready, pd_free[2], g_full, g_free, dq_full, dq_free, mma_done
-  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 1 + 2 + 1 + 1 + 3;
+  // p_ready, pd_free, g_full, g_free, dq_full, dq_free, mma_done, red_sync[2]
+  static constexpr int kNumBars = 2 + 2 + 2 + 2 * kStagesK + 2 * kStagesV + 2 + 1 + 1 + 1 + 1 + 3 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // a 2 KB staging area per reducer warp: gradient rows leave through it as
   // coalesced 16-byte reductions
@@ -141,12 +142,14 @@ struct Bars {
   uint64_t* v_empty;
   uint64_t* s_full;     // [2] S and dP of buffer b in TMEM
   uint64_t* p_ready;    // P and dS of the current tile in shared memory (S/dP read)
-  uint64_t* pd_free;    // [2] the products reading P/dS buffer b have completed
+  uint64_t* pd_free;    // the products reading P/dS have completed
   uint64_t* g_full;     // dV^T/dK^T of the tile complete
   uint64_t* g_free;     // ... and read out
   uint64_t* dq_full;    // dQ of the unit complete
   uint64_t* dq_free;    // ... and read out
   uint64_t* mma_done;
+  // [2]: barrier of the reducer threads, the two used in turn (bounded)
+  uint64_t* red_sync;
 };
 
 // 8 BF16 in a 16-byte word, times 8 BF16 in another, summed in FP32.
@@ -184,11 +187,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
   B.s_full = B.v_empty + kStagesV;
   B.p_ready = B.s_full + 2;
   B.pd_free = B.p_ready + 1;
-  B.g_full = B.pd_free + 2;
+  B.g_full = B.pd_free + 1;
   B.g_free = B.g_full + 1;
   B.dq_full = B.g_free + 1;
   B.dq_free = B.dq_full + 1;
   B.mma_done = B.dq_free + 1;
+  B.red_sync = B.mma_done + 1;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + L::kDescOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
@@ -213,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
     for (int s = 0; s < 2; ++s) {
       mbar_init(B.tab_full + s, 32);
       mbar_init(B.tab_empty + s, kTabConsumers);
-      mbar_init(B.pd_free + s, 1);
       mbar_init(B.s_full + s, 1);
+      mbar_init(B.red_sync + s, 128);
     }
     mbar_init(B.qd_full, 1);
     mbar_init(B.qd_empty, 1);
@@ -226,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       mbar_init(B.v_full + s, 1);
       mbar_init(B.v_empty + s, 1);
     }
+    mbar_init(B.pd_free, 1);
     mbar_init(B.g_full, 1);
     mbar_init(B.g_free, 128);
     mbar_init(B.p_ready, kSoftThreads);
@@ -344,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
         }
         tc_fence_after_sync();
         const uint32_t k_addr = sbase + L::kKOff + (gg % kStagesK) * L::kTileBytes;
-        const uint32_t p_addr = sbase + L::kPOff + (gg & 1) * 2 * L::kPBytes;
+        const uint32_t p_addr = sbase + L::kPOff;
         const uint32_t ds_addr = p_addr + L::kPBytes;
         const uint32_t gcol = L::kGCol;
 #pragma unroll
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
           umma_ss(tmem + gcol + kT, a, b, id_g, k > 0 ? 1u : 0u);
         }
         tc_commit(B.k_empty + gg % kStagesK);
-        tc_commit(B.pd_free + (gg & 1));
+        tc_commit(B.pd_free);
         tc_commit(B.g_full);
         if (last) {
           tc_commit(B.dq_full);
@@ -497,13 +502,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
         }
         tc_fence_after_sync();
         const int nv = min(kT, d.nkeys - t * kT);
-        // P/dS buffer g&1 is free once the products of tile g-2 completed
-        if (!__all_sync(0xffffffffu, mbar_wait(B.pd_free + (g & 1), ((g >> 1) & 1) ^ 1, abort_flag, P.dev_status))) {
-          ok = false;
-          break;
-        }
-        uint8_t* pbuf = smem + L::kPOff + (g & 1) * 2 * L::kPBytes + row * 128;
+        uint8_t* pbuf = smem + L::kPOff + row * 128;
         uint8_t* dsbuf = pbuf + L::kPBytes;
+        bool stores_ok = true;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t s[32], dp[32];
@@ -523,6 +524,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
             pk[cc] = pack_bf16x2(p0, p1);
             dk[cc] = pack_bf16x2(d0, d1);
           }
+          // P/dS are free once the products of tile g-1 have completed:
+          // the first half's exponentials do not wait for that
+          if (hf == 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(B.pd_free, (g & 1) ^ 1, abort_flag, P.dev_status))) {
+            stores_ok = false;
+            break;
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int chunk = 4 * hf + q;
@@ -530,6 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
             *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             *reinterpret_cast<uint4*>(dsbuf + off) = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
           }
+        }
+        if (!stores_ok) {
+          ok = false;
+          break;
         }
         fence_proxy_async_smem();   // generic-proxy writes -> the UMMA's reads
         tc_fence_before_sync();
@@ -540,13 +552,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
   } else if (warp >= kRedWarp0) {
     // ================================================= gradient reductions
     // Thread r holds TMEM lane r: the d index r of dV^T/dK^T (keys along
-    // the columns), the head row r of dQ. Rows leave through the warp's
-    // staging area so that every reduction is a 16-byte vector covering a
-    // contiguous piece of one gradient row.
+    // the columns), the head row r of dQ. A dV or dK tile is written into
+    // the staging tile as 64 key rows of d FP32 values; then each of the
+    // first nv threads hands its key's row to the TMA unit as one bulk
+    // reduction into the gradient pool. dQ leaves through the warp's 2 KB
+    // stage as 16-byte vector reductions.
+    const int r = tid - kRedWarp0 * 32;
     const int wq = warp - kRedWarp0;                   // this warp's 32 d / head rows
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     float* stg = reinterpret_cast<float*>(smem + L::kStageOff + wq * 2048);
-    const bool d_ok = wq * 32 < D;                     // warp-uniform (d = 64: two warps idle)
+    float* bulk = reinterpret_cast<float*>(smem + L::kBulkOff);
+    const uint32_t bulk_addr = sbase + L::kBulkOff;
+    uint32_t nsync = 0;
+    // barrier of the 128 reducer threads (bounded: false once a wait gave up)
+    auto rsync = [&]() -> bool {
+      uint64_t* bar = B.red_sync + (nsync & 1);
+      const uint32_t parity = (nsync >> 1) & 1;
+      ++nsync;
+      mbar_arrive(bar);
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, P.dev_status));
+    };
     int c = 0, g = 0, ud = 0;
     bool ok = true, final_seen = false;
     while (ok && !final_seen) {
@@ -556,60 +581,50 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       final_seen = (d.flags & kFlagFinal) != 0;
       const uint32_t* t_rows = tab + slot * kChunkKeys;
       const int ntiles = ceil_tiles(d.nkeys);
-      for (int t = 0; t < ntiles; ++t, ++g) {
+      for (int t = 0; ok && t < ntiles; ++t, ++g) {
         if (!__all_sync(0xffffffffu, mbar_wait(B.g_full, g & 1, abort_flag, P.dev_status))) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
         const int nv = min(kT, d.nkeys - t * kT);
-        const uint32_t gcol = L::kGCol;
+        // this thread's key row (threads r < nv hand one row each to the TMA)
+        const uint32_t e = r < nv ? t_rows[t * kT + r] : kInvalidRow;
 #pragma unroll 1
-        for (int hk = 0; hk < 2; ++hk) {
-          uint32_t dv[32], dk[32];
-          tmem_ld32(lane_addr + gcol + 32 * hk, dv);
-          tmem_ld32(lane_addr + gcol + kT + 32 * hk, dk);
-          tmem_ld_wait(dv);
-          tmem_ld_wait(dk);
-          if (hk == 1) {   // both halves are in registers: the buffer is free
+        for (int which = 0; which < 2; ++which) {   // dV, then dK
+          // the staging tile is free once every reduction issued from it
+          // has read it
+          bulk_wait_read_all();
+          if (!rsync()) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int hk = 0; hk < 2; ++hk) {
+            uint32_t v[32];
+            tmem_ld32(lane_addr + L::kGCol + which * kT + 32 * hk, v);
+            tmem_ld_wait(v);
+            if (r < D) {
+#pragma unroll
+              for (int kk = 0; kk < 32; ++kk) bulk[(32 * hk + kk) * D + r] = __uint_as_float(v[kk]);
+            }
+          }
+          if (which == 1) {   // dV^T and dK^T have left TMEM
             tc_fence_before_sync();
             mbar_arrive(B.g_free);
           }
-          if (!d_ok) continue;
-#pragma unroll
-          for (int which = 0; which < 2; ++which) {
-            const uint32_t* vals = which == 0 ? dv : dk;
-            float* pool_raw = which == 0 ? P.dv_raw : P.dk_raw;
-            float* pool_cmp = which == 0 ? P.dv_cmp : P.dk_cmp;
-#pragma unroll
-            for (int pass = 0; pass < 2; ++pass) {
-              // 16 keys x this warp's 32 d: key-major rows of 128 bytes
-#pragma unroll
-              for (int kl = 0; kl < 16; ++kl) stg[kl * 32 + lane] = __uint_as_float(vals[16 * pass + kl]);
-              __syncwarp();
-              // every read first, then the four reductions (their source
-              // registers stay untouched until the reductions have issued)
-              float4 v[4];
-              uint32_t e[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int item = lane + 32 * k, kl = item >> 3, c4 = item & 7;
-                v[k] = reinterpret_cast<const float4*>(stg)[kl * 8 + c4];
-                const int j = 32 * hk + 16 * pass + kl;
-                e[k] = j < nv ? t_rows[t * kT + j] : kInvalidRow;
-              }
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                if (e[k] == kInvalidRow) continue;
-                const int c4 = (lane + 32 * k) & 7;
-                float* dst = ((e[k] & kRawBit) ? pool_raw : pool_cmp) + static_cast<int64_t>(e[k] & ~kRawBit) * D +
-                             wq * 32 + 4 * c4;
-                red_add_v4_f32(dst, v[k]);
-              }
-              __syncwarp();   // the stage is rewritten next
-            }
+          fence_proxy_async_smem();   // generic-proxy writes -> the TMA's reads
+          if (!rsync()) {
+            ok = false;
+            break;
           }
+          if (e != kInvalidRow) {
+            float* pool = which == 0 ? ((e & kRawBit) ? P.dv_raw : P.dv_cmp) : ((e & kRawBit) ? P.dk_raw : P.dk_cmp);
+            bulk_reduce_add_f32(pool + static_cast<int64_t>(e & ~kRawBit) * D, bulk_addr + r * D * 4, D * 4);
+          }
+          bulk_commit_group();
         }
+        if (!ok) break;
         if ((d.flags & kFlagLast) && t == ntiles - 1) {
           // dQ of the unit (head row r), added into dq: 16 columns of the
           // warp's 32 rows per pass through the stage, then 8 rows x 64
@@ -659,6 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_bwd_kernel(const
       mbar_arrive(B.tab_empty + slot);
       ++c;
     }
+    bulk_wait_all();   // every bulk reduction has completed
   }
 
   // ---- teardown: every TMEM access above has completed

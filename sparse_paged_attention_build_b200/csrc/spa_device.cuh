@@ -332,6 +332,20 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, float4 v) {
                : "memory");
 }
 
+// Bulk asynchronous reduction: `bytes` (a multiple of 16) of FP32 values
+// at shared-memory address `src` are added into global memory at `dst`
+// (16-byte aligned) by the TMA unit; tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst), "r"(src),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Every bulk operation this thread committed has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float exp2_approx(float x) {
   float y;
