@@ -1,6 +1,9 @@
 /*
- * spa.h -- C ABI of libspa.so: the forward of sparse paged attention with an
- * attention sink, for NVIDIA B200 (sm_100a).
+ * spa.h -- C ABI of libspa.so: sparse paged attention with an attention
+ * sink, for NVIDIA B200 (sm_100a). The path: the per-token key sets (1), the
+ * FP8 page decode (2), the attention forward (3, 3b with the FP8 decode in
+ * its gather); around it: the backward (3c), the paged write of new window
+ * tokens (4) and the decode of packed 512-wide rows (5).
  *
  * The method (page "Roadmap item 24 - joint compressed/window attention with
  * sink", RL-Kernel PR #628, section "Reuse and arithmetic"): for each query
@@ -238,32 +241,6 @@ int spa_sparse_sink_attn_fwd(
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * 4. spa_paged_kv_write -- new raw tokens into the paged window cache.
- *
- * Defined by "test: add block-level DeepSeek-V4 attention test", decode
- * kernel timeline and notes (the paged KV write, "swa_write" / "kvw_paged",
- * runs ahead of the sparse attention core); without the qk-norm and RoPE
- * the model fuses into it. Token j, of request b = req[j] at position
- * t = pos[j], is copied to row pt[b][t / page_size] * page_size +
- * t % page_size of k_pool and of v_pool.
- *
- * k_new, v_new  BF16 [n_tokens, head_dim] contiguous, 16-B aligned
- * head_dim      a multiple of 8
- * req, pos      int32 [n_tokens]; a request outside [0, n_requests) or a
- *               position outside the table sets SPA_DEV_BAD_INDEX, a page id
- *               outside [0, num_pages) SPA_DEV_BAD_PAGE; the token is skipped
- * pt            int32 [n_requests, pt_cols] (the raw page table)
- * page_size     power of two, 1 .. 1024
- * k_pool, v_pool BF16 [num_pages, page_size, head_dim], 16-B aligned
- * Rows not named by a token are left as they are; two tokens naming the
- * same row leave one of them there (which one is unspecified).
- * ---------------------------------------------------------------------- */
-int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_tokens, int32_t head_dim,
-                       const int32_t* req, const int32_t* pos, const int32_t* pt, int32_t pt_cols,
-                       int32_t n_requests, int32_t page_size, int64_t num_pages, uint16_t* k_pool,
-                       uint16_t* v_pool, uint32_t* dev_status, spa_stream_t stream);
-
-/* ------------------------------------------------------------------------
  * 3b. spa_sparse_sink_attn_fwd_fp8 -- the same attention over a mixed
  * cache whose compressed pool is stored in FP8, decoded inside the gather.
  *
@@ -296,28 +273,7 @@ int spa_sparse_sink_attn_fwd_fp8(
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * 6. spa_unpack_d512_pages -- packed 512-wide rows (584 bytes per token)
- * to BF16.
- *
- * "Roadmap item 24 - joint compressed/window attention with sink", review
- * notes on the packed joint KV gather: 584 bytes per token for a 512-wide
- * head, 576 of them data. Read as: bytes 0..447 OCP E4M3 codes (elements
- * 0..447), bytes 448..575 BF16 (elements 448..511), bytes 576..582 UE8M0
- * scales (2^(byte-127), one per 64 codes; 0xFF is NaN), byte 583 unused.
- * Element e < 448 -> bf16_rne(float(e4m3) * 2^(s-127)); the rest copied.
- *
- * src        uint8 [num_pages, page_size, 584], 8-B aligned
- * page_ids   int32 [n_page_ids]: the pages to decode; an id outside
- *            [0, num_pages) sets SPA_DEV_BAD_PAGE and that page is skipped
- * dst        BF16 [num_pages, page_size, 512], 16-B aligned; pages not
- *            listed are left untouched
- * page_size  1 .. 4096
- * ---------------------------------------------------------------------- */
-int spa_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size, const int32_t* page_ids,
-                          int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status, spa_stream_t stream);
-
-/* ------------------------------------------------------------------------
- * 5. spa_sparse_sink_attn_bwd -- gradients of the attention with sink.
+ * 3c. spa_sparse_sink_attn_bwd -- gradients of the attention with sink.
  *
  * The follow-on item of "Roadmap item 24 - joint compressed/window attention
  * with sink": dQ, dK/dV scattered to the pages, and d_sink, from the saved O
@@ -353,6 +309,53 @@ int spa_sparse_sink_attn_bwd(
     const float* sink, float scale, const uint16_t* out, const float* lse, const uint16_t* dout,
     float* dq, float* dk_raw, float* dv_raw, float* dk_cmp, float* dv_cmp, float* dsink,
     int32_t num_splits, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * 4. spa_paged_kv_write -- new raw tokens into the paged window cache.
+ *
+ * Defined by "test: add block-level DeepSeek-V4 attention test", decode
+ * kernel timeline and notes (the paged KV write, "swa_write" / "kvw_paged",
+ * runs ahead of the sparse attention core); without the qk-norm and RoPE
+ * the model fuses into it. Token j, of request b = req[j] at position
+ * t = pos[j], is copied to row pt[b][t / page_size] * page_size +
+ * t % page_size of k_pool and of v_pool.
+ *
+ * k_new, v_new  BF16 [n_tokens, head_dim] contiguous, 16-B aligned
+ * head_dim      a multiple of 8
+ * req, pos      int32 [n_tokens]; a request outside [0, n_requests) or a
+ *               position outside the table sets SPA_DEV_BAD_INDEX, a page id
+ *               outside [0, num_pages) SPA_DEV_BAD_PAGE; the token is skipped
+ * pt            int32 [n_requests, pt_cols] (the raw page table)
+ * page_size     power of two, 1 .. 1024
+ * k_pool, v_pool BF16 [num_pages, page_size, head_dim], 16-B aligned
+ * Rows not named by a token are left as they are; two tokens naming the
+ * same row leave one of them there (which one is unspecified).
+ * ---------------------------------------------------------------------- */
+int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_tokens, int32_t head_dim,
+                       const int32_t* req, const int32_t* pos, const int32_t* pt, int32_t pt_cols,
+                       int32_t n_requests, int32_t page_size, int64_t num_pages, uint16_t* k_pool,
+                       uint16_t* v_pool, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * 5. spa_unpack_d512_pages -- packed 512-wide rows (584 bytes per token)
+ * to BF16.
+ *
+ * "Roadmap item 24 - joint compressed/window attention with sink", review
+ * notes on the packed joint KV gather: 584 bytes per token for a 512-wide
+ * head, 576 of them data. Read as: bytes 0..447 OCP E4M3 codes (elements
+ * 0..447), bytes 448..575 BF16 (elements 448..511), bytes 576..582 UE8M0
+ * scales (2^(byte-127), one per 64 codes; 0xFF is NaN), byte 583 unused.
+ * Element e < 448 -> bf16_rne(float(e4m3) * 2^(s-127)); the rest copied.
+ *
+ * src        uint8 [num_pages, page_size, 584], 8-B aligned
+ * page_ids   int32 [n_page_ids]: the pages to decode; an id outside
+ *            [0, num_pages) sets SPA_DEV_BAD_PAGE and that page is skipped
+ * dst        BF16 [num_pages, page_size, 512], 16-B aligned; pages not
+ *            listed are left untouched
+ * page_size  1 .. 4096
+ * ---------------------------------------------------------------------- */
+int spa_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size, const int32_t* page_ids,
+                          int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status, spa_stream_t stream);
 
 #ifdef __cplusplus
 }
