@@ -33,9 +33,10 @@
 //   warp  6     K gather (TMA tile::gather4, 3-stage ring) and each unit's
 //               Q and dO (TMA boxes)
 //   warp  7     V gather (2-stage ring)
-//   warps 8-11  thread t owns TMEM lane t: reads dV^T/dK^T rows (d index t)
-//               and adds them into the gradient pools, and at the end of a
-//               unit reads dQ (head row t) and adds it into dq
+//   warps 8-11  thread t owns TMEM lane t: writes dV^T, then dK^T (d index
+//               t) into a [key][d] FP32 staging tile whose rows the TMA adds
+//               into the gradient pools (one bulk reduction per key), and at
+//               the end of a unit reads dQ (head row t) and adds it into dq
 // TMEM columns: two S|dP buffers [0,128) and [128,256), dV^T|dK^T
 // [256,384), dQ [384,512). Per tile the UMMA thread issues S/dP of tile g
 // (into buffer g&1, without waiting for the softmax of tile g-1) and then
