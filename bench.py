@@ -200,8 +200,9 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(times)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w, world, None),
+        "data": "synthetic", "config": config_of(w, world, int(ip[-1]), args.fp8_path),
         "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": threads,
+                         "cpu_model": cpu_model(),
                          "sample": f"{rows_per_step} random query tokens per step (of {w.N}), all heads, "
                                    f"FP64 C oracle with {threads} threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -241,6 +242,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=0)
+    ap.add_argument("--no-decode", dest="decode_too", action="store_false",
+                    help="prefill workloads: skip the ratio-128 decode measurement that rides along")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide requests/tokens (profiling cases only; not a bench line)")
     args = ap.parse_args()
@@ -271,8 +274,65 @@ def main():
             dist.barrier()
 
     w = workloads.make(args.workload, shrink=args.shrink, seed_offset=rank)
+    res = measure_path(w, args, args.steps, args.warmup, args.splits, local_rank, world, barrier, dist)
+
+    # The ratio-128 decode rides along in the default run, so that every
+    # bench line carries both targets of the path: the prefill's tensor
+    # roofline and the decode's HBM roofline. Same protocol (graph replay,
+    # L2 flushed between steps, CUDA events on the launching stream).
+    dec = None
+    if args.decode_too and w.kind == "prefill" and args.shrink == 1:
+        wd = workloads.make("c4", seed_offset=rank)
+        dres = measure_path(wd, args, max(args.steps, 50), args.warmup, 0, local_rank, world, barrier, dist,
+                            want_e2e=not args.no_e2e)
+        dec = {"workload": f"{wd.name}: {workloads.DESCRIPTIONS[wd.name]}",
+               "tok_per_s": dres["total_queries"] / (dres["elapsed_ms"] / 1e3),
+               "ms_per_step": dres["elapsed_ms"] / dres["steps"],
+               "attn_ms_per_launch": dres["attn_ms"], "hbm_gbs": dres["roofline"]["hbm_gbs"],
+               "pairs_per_s": dres["value"], "roofline": dres["roofline"], "clocks": dres["clocks"],
+               "num_splits": dres["num_splits"], "gpu_launches": dres["gpu_launches"],
+               "device_status": dres["status"], "config": config_of(wd, world, dres["nnz"], args.fp8_path),
+               "e2e": dres["e2e"]}
+        if dres["e2e"] is not None:
+            dec["e2e"]["tok_per_s"] = dres["total_queries"] * dres["e2e"]["value"] / max(dres["value"], 1e-30)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["elapsed_ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, world, res["nnz"], args.fp8_path),
+            "tflops": res["tflops"],
+            "roofline": res["roofline"],
+            "clocks": res["clocks"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
+            "device_status": res["status"],
+        }
+        if w.kind == "decode":
+            line["tok_per_s"] = res["total_queries"] / (res["elapsed_ms"] / 1e3)
+        if dec is not None:
+            line["decode"] = dec
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dist, want_e2e=None):
+    """Time the hot path (sets, FP8 decode, attention) on one workload:
+    graph replays, CUDA events on the launching stream, whole-job totals
+    over the ranks; the roofline of the attention launch; clocks sampled
+    during the timed region; the end-to-end figure through the public API."""
+    import torch
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+
     decode = w.kind == "decode"
-    b0 = DeviceBatch(w, num_splits=args.splits, fp8_path=args.fp8_path)
+    b0 = DeviceBatch(w, num_splits=splits, fp8_path=args.fp8_path)
     stream = torch.cuda.current_stream()
     b0.step()
     torch.cuda.synchronize()
@@ -299,7 +359,7 @@ def main():
     stream.wait_stream(cap)
     torch.cuda.synchronize()
 
-    for s in range(args.warmup):
+    for s in range(warmup):
         if flush is not None:
             flush.zero_()
         g_front.replay()
@@ -309,13 +369,13 @@ def main():
     sampler = ClockSampler(physical_gpu(local_rank))
     sampler.start()
     time.sleep(0.3)
-    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record(stream)
-    for s in range(args.steps):
+    for s in range(steps):
         if flush is not None:
             flush.zero_()
         ev[s][0].record(stream)
@@ -337,7 +397,8 @@ def main():
     else:
         elapsed_ms = start.elapsed_time(stop)
     attn_ms = float(np.mean([e1.elapsed_time(e2) for _, e1, e2 in ev]))
-    total_triples, elapsed_ms = job_totals(triples * args.steps, elapsed_ms, world, "cuda")
+    total_triples, elapsed_ms = job_totals(triples * steps, elapsed_ms, world, "cuda")
+    total_queries, _ = job_totals(w.N * steps, 0.0, world, "cuda")
     total_flops = total_triples * 4.0 * w.d
     status = b0.status_word()
 
@@ -369,30 +430,14 @@ def main():
     # end to end through the public API: pinned host inputs -> device ->
     # the three calls -> O and LSE back to the host, every step
     e2e = None
-    if not args.no_e2e:
+    if want_e2e if want_e2e is not None else not args.no_e2e:
         e2e = measure_e2e(w, b0, args, stream, world, barrier, dist)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w)
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_of(w, world, nnz, args.fp8_path),
-            "tflops": total_flops / (elapsed_ms / 1e3) / 1e12,
-            "roofline": roofline,
-            "clocks": clocks, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
-            "device_status": status,
-        }
-        if cpu is not None:
-            line["cpu_baseline"] = cpu
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
-    return 0
+    splits_used = b0.splits_used()
+    del g_front, g_attn
+    return {"value": value, "elapsed_ms": elapsed_ms, "attn_ms": attn_ms, "nnz": nnz,
+            "tflops": total_flops / (elapsed_ms / 1e3) / 1e12, "roofline": roofline, "clocks": clocks,
+            "e2e": e2e, "gpu_launches": kernels_per_step * steps, "status": status, "steps": steps,
+            "total_queries": total_queries, "num_splits": splits_used}
 
 
 def run_kv_write(args, rank, local_rank, world):
@@ -623,10 +668,8 @@ def measure_e2e(w, b0, args, stream, world, barrier, dist):
         if w.k_cmp is not None:
             host["k_cmp"] = pinned(w.k_cmp.view(np.int16), bf)
             host["v_cmp"] = pinned(w.v_cmp.view(np.int16), bf)
-    if w.k_cmp_fp8 is not None:
-        names = ("k_cmp_fp8", "v_cmp_fp8", "k_cmp_scale", "v_cmp_scale")
-        for k in names + (() if b0.fused else ("cmp_page_ids",)):
-            host[k] = pinned(getattr(w, k))
+    if w.k_cmp_fp8 is not None and not b0.fused:
+        host["cmp_page_ids"] = pinned(w.cmp_page_ids)
     dev = {k: getattr(b0, k) for k in host}
     h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
     out_h = torch.empty(b0.out.shape, dtype=bf).pin_memory()
@@ -654,13 +697,29 @@ def measure_e2e(w, b0, args, stream, world, barrier, dist):
     e.synchronize()
     ms = s.elapsed_time(e)
     total, ms = job_totals(b0.nnz() * w.H * steps, ms, world, "cuda")
+    copies = ("per-step inputs host->device (q, positions, requests, top-k, page tables, sink"
+              + (", the step's raw and compressed K/V" if w.kind == "prefill" else "")
+              + "), O and LSE device->host"
+              + ("; the paged KV caches stay resident on the device (decode)" if w.kind == "decode" else ""))
     return {"value": total / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": ms / steps, "steps": steps}
+            "ms_per_step": ms / steps, "steps": steps, "copies": copies}
 
 
-def cpu_baseline(w, budget_s=15.0):
-    """The FP64 oracle on a bounded sample of the same workload."""
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(w, budget_s=15.0, budget_1t_s=5.0):
+    """The FP64 oracle on a bounded sample of the same workload: once with
+    every host thread, once single-threaded."""
     import oracle
     threads = os.cpu_count() or 1
     ip, idx = oracle.build_kv_sets(w.pos, w.W, w.ratio, w.topk)
@@ -670,19 +729,23 @@ def cpu_baseline(w, budget_s=15.0):
         v_cmp = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids)
     rng = np.random.default_rng(1)
 
-    def run(n):
+    def run(n, nthreads):
         rows = np.sort(rng.choice(w.N, size=min(n, w.N), replace=False)).astype(np.int32)
         t0 = time.perf_counter()
         oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, w.sink, w.scale,
-                                k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp, rows=rows, threads=threads)
+                                k_cmp=k_cmp, v_cmp=v_cmp, pt_cmp=w.pt_cmp, rows=rows, threads=nthreads)
         return time.perf_counter() - t0, int((ip[rows + 1] - ip[rows]).sum()) * w.H, rows.size
 
-    dt, _, n = run(threads)
+    dt, _, n = run(threads, threads)
     n2 = int(max(threads, min(w.N, n * budget_s / max(dt, 1e-3))))
-    dt, tri, n2 = run(n2)
+    dt, tri, n2 = run(n2, threads)
+    dt1, _, m = run(1, 1)
+    m2 = int(max(1, min(w.N, m * budget_1t_s / max(dt1, 1e-3))))
+    dt1, tri1, m2 = run(m2, 1)
     return {"kind": "oracle", "value": tri / dt, "unit": UNIT, "cores": threads,
+            "cpu_model": cpu_model(), "value_1_thread": tri1 / dt1,
             "sample": f"{n2} random query tokens of {w.N} (all {w.H} heads), FP64 C oracle, "
-                      f"{threads} threads, {dt:.1f} s"}
+                      f"{threads} threads, {dt:.1f} s; single-threaded: {m2} query tokens, {dt1:.1f} s"}
 
 
 if __name__ == "__main__":

@@ -64,6 +64,10 @@ typedef enum {
 #define SPA_DEV_BAD_INDEX 2u   /* key/position/request outside its table              */
 #define SPA_DEV_CAPACITY  4u   /* the key sets overflowed `capacity`                  */
 #define SPA_DEV_TIMEOUT   8u   /* a bounded wait inside a kernel ran out              */
+#define SPA_DEV_SCRATCH_RACE 16u /* two set builds that may run at the same time used
+                                  the same scan scratch (one workspace for both, or
+                                  overlapping spa_build_kv_sets_noalloc calls); the
+                                  sets of that call are wrong                          */
 
 /* A key is a compressed-group index g (0 <= g < 2^30) or
  * SPA_WINDOW_TAG | t for raw token t (0 <= t < 2^30). Ascending key order is
@@ -139,9 +143,13 @@ int spa_build_kv_sets(const int32_t* pos, int32_t n_queries, int32_t window, int
  *
  * The first call on each device looks up the scratch array's device address
  * (with that device current) and caches it; make that first call before any
- * stream capture on the device. All calls share the one array: calls that
- * may overlap on the GPU (different streams, or graph replays running
- * concurrently) race on it and must be serialised by the caller.
+ * stream capture on the device. A device reset (cudaDeviceReset) creates a
+ * new context: the next call looks the address up again, and it too must
+ * come before any capture. All calls share the one array: calls that may
+ * overlap on the GPU (different streams, or graph replays running
+ * concurrently) race on it and must be serialised by the caller. Such a
+ * race gives wrong sets, never an access outside the array: a CTA whose
+ * ticket lies past its own grid sets SPA_DEV_SCRATCH_RACE and stops.
  * ---------------------------------------------------------------------- */
 int spa_build_kv_sets_noalloc(const int32_t* pos, int32_t n_queries, int32_t window, int32_t ratio,
                               const int32_t* topk, int32_t topk_width, int32_t* indptr,

@@ -22,7 +22,7 @@ import os
 import torch
 
 WINDOW_TAG = 1 << 30
-DEV_BAD_PAGE, DEV_BAD_INDEX, DEV_CAPACITY, DEV_TIMEOUT = 1, 2, 4, 8
+DEV_BAD_PAGE, DEV_BAD_INDEX, DEV_CAPACITY, DEV_TIMEOUT, DEV_SCRATCH_RACE = 1, 2, 4, 8, 16
 STATUS = {0: "SPA_OK", 1: "SPA_ERR_INVALID_ARG", 2: "SPA_ERR_UNSUPPORTED", 3: "SPA_ERR_CAPACITY",
           4: "SPA_ERR_WORKSPACE", 5: "SPA_ERR_ALIGNMENT", 6: "SPA_ERR_CUDA"}
 

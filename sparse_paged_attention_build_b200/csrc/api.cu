@@ -3,6 +3,7 @@
 // before anything is enqueued and leaves a message for
 // spa_last_error_detail(). No call allocates, frees or synchronises.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -36,25 +37,34 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool pow2_in(int32_t v, int32_t lo, int32_t hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
 
-int sm_count() {
-  static int cached = 0;
-  if (cached == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-      cached = n;
-    else
-      cached = 148;
-  }
-  return cached;
-}
-
 int32_t resolve_splits(int32_t n_queries, int32_t num_heads, int32_t requested) {
   if (requested > 0) return requested;
   return spa_sparse_sink_attn_choose_splits(n_queries, num_heads, 0);
 }
 
 }  // namespace
+
+namespace spa {
+
+// SM count of the current device, looked up once per device (148 if the
+// query fails). Each device has its own slot, written at most once with
+// the same value, so concurrent callers on different threads agree.
+int device_sm_count() {
+  constexpr int kSlots = 64;
+  static std::atomic<int> cache[kSlots];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kSlots) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < kSlots) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+}  // namespace spa
 
 extern "C" {
 
@@ -193,7 +203,7 @@ int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int
   if (n_queries <= 0 || num_heads <= 0) return 1;
   const int64_t head_tiles = (num_heads + 127) / 128;
   const int64_t units = static_cast<int64_t>(n_queries) * head_tiles;
-  const int64_t slots = 2 * static_cast<int64_t>(sm_count());   // persistent CTAs, two per SM
+  const int64_t slots = 2 * static_cast<int64_t>(spa::device_sm_count());   // persistent CTAs, two per SM
   int64_t s = 1;
   if (units <= slots / 2) {
     // A small batch (decode) leaves CTAs idle: cut each set into slices

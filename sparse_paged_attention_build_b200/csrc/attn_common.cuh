@@ -145,19 +145,6 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
 }
 
 // ------------------------------------------------------------------ host
-inline int sm_count_cached() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      n = v;
-    else
-      n = 148;
-  }
-  return n;
-}
-
 inline int log2_exact(int32_t v) {
   int k = 0;
   while ((1 << k) < v) ++k;

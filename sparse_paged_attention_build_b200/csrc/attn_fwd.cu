@@ -937,7 +937,7 @@ cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }
-  const int64_t slots = std::max<int64_t>(1, (2 * static_cast<int64_t>(sm_count_cached())) / head_tiles);
+  const int64_t slots = std::max<int64_t>(1, (2 * static_cast<int64_t>(device_sm_count())) / head_tiles);
   dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
   sparse_sink_attn_kernel<D, kFp8><<<grid, kThreads, L::kBytes, stream>>>(P);
   return cudaGetLastError();

@@ -22,6 +22,8 @@
 #include <climits>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "spa_device.cuh"
 #include "spa_internal.h"
 
@@ -194,6 +196,14 @@ __global__ void __launch_bounds__(kSetsWarps * 32) build_kv_sets_kernel(const Se
   if (threadIdx.x == 0) s_tile = atomicAdd(P.tile_ticket, 1u);
   __syncthreads();
   const uint32_t tile = s_tile;
+  // A ticket past this launch's grid only comes from another launch using
+  // the same scratch at the same time (a shared workspace, or overlapping
+  // calls of the no-allocation entry point). The status words of such a
+  // tile lie outside what this launch cleared: touch none of them.
+  if (tile >= gridDim.x) {
+    if (threadIdx.x == 0) report(P.dev_status, SPA_DEV_SCRATCH_RACE);
+    return;
+  }
   const int64_t q0 = static_cast<int64_t>(tile) * P.per_cta;
   const int nq = static_cast<int>(min(static_cast<int64_t>(P.per_cta), static_cast<int64_t>(P.n) - q0));
 
@@ -276,19 +286,6 @@ int sort_width_for(int32_t topk_width) {
   return w;
 }
 
-int sm_count_for_sets() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      n = v;
-    else
-      n = 148;
-  }
-  return n;
-}
-
 }  // namespace
 
 // An upper bound of the scratch the launcher uses (it uses fewer status
@@ -298,18 +295,28 @@ size_t build_kv_sets_workspace_bytes(int32_t n_queries) {
   return static_cast<size_t>(tiles) * sizeof(uint64_t) + 16;
 }
 
-cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
-                                 const int32_t* topk, int32_t topk_width, int32_t* indptr,
-                                 int32_t* indices, int64_t capacity, void* ws,
-                                 uint32_t* dev_status, cudaStream_t stream) {
+namespace {
+
+// Enqueue the set builder with its look-back status words at `tile_status`
+// (one per CTA) and its CTA ticket at `ticket`; both are cleared first.
+cudaError_t launch_sets(const int32_t* pos, int32_t n, int32_t window, int32_t ratio, const int32_t* topk,
+                        int32_t topk_width, int32_t* indptr, int32_t* indices, int64_t capacity,
+                        uint64_t* tile_status, uint32_t* ticket, bool ticket_follows_status,
+                        uint32_t* dev_status, cudaStream_t stream) {
   if (n == 0) return cudaMemsetAsync(indptr, 0, sizeof(int32_t), stream);
   // about two CTAs per SM, each with a contiguous block of queries
-  const int64_t slots = 2 * static_cast<int64_t>(sm_count_for_sets());
+  const int64_t slots = 2 * static_cast<int64_t>(device_sm_count());
   int64_t per_cta = (static_cast<int64_t>(n) + slots - 1) / slots;
   per_cta = per_cta < kSetsQueriesPerCta ? kSetsQueriesPerCta : (per_cta > kMaxPerCta ? kMaxPerCta : per_cta);
   const int64_t tiles = (static_cast<int64_t>(n) + per_cta - 1) / per_cta;
-  const size_t ws_used = static_cast<size_t>(tiles) * sizeof(uint64_t) + 16;
-  cudaError_t err = cudaMemsetAsync(ws, 0, ws_used, stream);
+  const size_t status_bytes = static_cast<size_t>(tiles) * sizeof(uint64_t);
+  cudaError_t err;
+  if (ticket_follows_status) {   // one clear covers both
+    err = cudaMemsetAsync(tile_status, 0, status_bytes + 16, stream);
+  } else {
+    err = cudaMemsetAsync(tile_status, 0, status_bytes, stream);
+    if (err == cudaSuccess) err = cudaMemsetAsync(ticket, 0, 16, stream);
+  }
   if (err != cudaSuccess) return err;
   SetsParams P;
   P.pos = pos;
@@ -326,8 +333,8 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
   P.indptr = indptr;
   P.indices = indices;
   P.capacity = capacity;
-  P.tile_status = static_cast<uint64_t*>(ws);
-  P.tile_ticket = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + tiles * sizeof(uint64_t));
+  P.tile_status = tile_status;
+  P.tile_ticket = ticket;
   P.dev_status = dev_status;
   const size_t smem = static_cast<size_t>(kSetsWarps) * P.buf_words * sizeof(int32_t) +
                       static_cast<size_t>(per_cta) * sizeof(int64_t);
@@ -338,6 +345,25 @@ cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, 
   }
   build_kv_sets_kernel<<<static_cast<unsigned>(tiles), kSetsWarps * 32, smem, stream>>>(P);
   return cudaGetLastError();
+}
+
+size_t sets_tiles(int32_t n) {
+  const int64_t slots = 2 * static_cast<int64_t>(device_sm_count());
+  int64_t per_cta = (static_cast<int64_t>(n) + slots - 1) / slots;
+  per_cta = per_cta < kSetsQueriesPerCta ? kSetsQueriesPerCta : (per_cta > kMaxPerCta ? kMaxPerCta : per_cta);
+  return static_cast<size_t>((static_cast<int64_t>(n) + per_cta - 1) / per_cta);
+}
+
+}  // namespace
+
+cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
+                                 const int32_t* topk, int32_t topk_width, int32_t* indptr,
+                                 int32_t* indices, int64_t capacity, void* ws,
+                                 uint32_t* dev_status, cudaStream_t stream) {
+  uint64_t* status = static_cast<uint64_t*>(ws);
+  uint32_t* ticket = reinterpret_cast<uint32_t*>(status + (n > 0 ? sets_tiles(n) : 0));
+  return launch_sets(pos, n, window, ratio, topk, topk_width, indptr, indices, capacity, status, ticket, true,
+                     dev_status, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -355,23 +381,53 @@ static_assert(kNoAllocScratchBytes == 1048576 + 16, "the documented limit");
 static __device__ __align__(256) uint64_t g_sets_scratch[kNoAllocScratchBytes / sizeof(uint64_t)];
 
 // Host code cannot pass &g_sets_scratch to a kernel: on the host that name
-// is only a stand-in. Its device address is looked up once per device, with
-// that device current, and cached.
+// is only a stand-in. Its device address is looked up once per device (and
+// context: a device reset makes a new context and a new address), with that
+// device current, and cached.
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
+
+// Unique id of the current context (0 if the driver cannot say).
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 cudaError_t scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_sets_scratch);
     if (err != cudaSuccess) return err;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -388,10 +444,15 @@ cudaError_t launch_build_kv_sets_no_alloc(const int32_t* pos, int32_t n, int32_t
   void* scratch = nullptr;
   cudaError_t err = scratch_for_current_device(&scratch);
   if (err != cudaSuccess) return err;
-  // the same kernel as the workspace entry point; the launcher clears the
-  // part of the scratch this call uses before the kernel runs
-  return launch_build_kv_sets(pos, n, window, ratio, topk, topk_width, indptr, indices, capacity,
-                              scratch, dev_status, stream);
+  // The same kernel as the workspace entry point. The status words start
+  // at the array's base; the CTA ticket sits in the array's last 16 bytes,
+  // past the status words of the largest call, so that no call's ticket
+  // ever lands on another call's status words. The launcher clears both
+  // before the kernel runs.
+  uint64_t* status = static_cast<uint64_t*>(scratch);
+  uint32_t* ticket = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + kNoAllocScratchBytes - 16);
+  return launch_sets(pos, n, window, ratio, topk, topk_width, indptr, indices, capacity, status, ticket, false,
+                     dev_status, stream);
 }
 
 }  // namespace spa

@@ -8,6 +8,9 @@
 
 namespace spa {
 
+// SM count of the current device (cached per device).
+int device_sm_count();
+
 constexpr int kSetsQueriesPerCta = 8;      // one warp per query
 constexpr int kMaxTopkWidth = 2048;
 

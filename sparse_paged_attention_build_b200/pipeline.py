@@ -107,6 +107,13 @@ class DeviceBatch:
         self.dequant(stream)
         self.attend(stream)
 
+    def splits_used(self) -> int:
+        """Slices per query the attention runs with (0 resolves to the
+        library's automatic choice)."""
+        if self.num_splits > 0:
+            return self.num_splits
+        return int(lib.spa_sparse_sink_attn_choose_splits(self.w.N, self.w.H, 0))
+
     def kernels_per_step(self) -> int:
         return 1 + (2 if self.fp8 and not self.fused else 0) + 1
 

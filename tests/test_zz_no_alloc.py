@@ -76,3 +76,54 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
             assert int(status.item()) == 0, (w.name, call)
             assert np.array_equal(indptr.cpu().numpy(), ref_ip), (w.name, call)
             assert np.array_equal(indices[: ref_ip[-1]].cpu().numpy(), ref_idx), (w.name, call)
+
+
+@pytest.mark.gpu
+def test_noalloc_replayed_from_a_cuda_graph():
+    """One warm-up call (it looks up the scratch address), then the call
+    captured on a side stream and replayed twice with new positions in the
+    same input buffer: each replay gives the workspace entry point's sets."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_paged_attention_build_b200 as spa
+    from sparse_paged_attention_build_b200 import workloads
+
+    so = _abi()
+    w = workloads.make("c1")
+    rng = np.random.default_rng(7)
+    pos_sets = [w.pos, rng.permutation(w.pos).astype(np.int32)]
+    max_pos = int(w.pos.max())
+    cap = spa.kv_sets_capacity(w.N, w.W, w.ratio, w.K, True, max_pos)
+    pos = torch.from_numpy(w.pos).cuda()
+    topk = torch.from_numpy(w.topk).cuda()
+    indptr = torch.empty(w.N + 1, dtype=torch.int32, device="cuda")
+    indices = torch.empty(cap, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def call(stream):
+        return so.spa_build_kv_sets_noalloc(_ptr(pos), w.N, w.W, w.ratio, _ptr(topk), w.K, _ptr(indptr),
+                                            _ptr(indices), cap, _ptr(status), ctypes.c_void_p(stream.cuda_stream))
+
+    assert call(torch.cuda.current_stream()) == 0, so.spa_last_error_detail()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            assert call(side) == 0, so.spa_last_error_detail()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for p in pos_sets:
+        pos.copy_(torch.from_numpy(p))
+        indptr.fill_(-1)
+        indices.fill_(-1)
+        g.replay()
+        torch.cuda.synchronize()
+        ref_ip, ref_idx = spa.build_kv_sets(pos, w.W, w.ratio, topk, capacity=cap)
+        torch.cuda.synchronize()
+        ref_ip = ref_ip.cpu().numpy()
+        assert int(status.item()) == 0
+        assert np.array_equal(indptr.cpu().numpy(), ref_ip)
+        assert np.array_equal(indices[: ref_ip[-1]].cpu().numpy(), ref_idx[: ref_ip[-1]].cpu().numpy())
+    del g
