@@ -231,7 +231,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "f1", "f2"],
+                    help="c1..c5: the 128-head configurations; f1, f2: the 32-head, 512-wide DSV4-Flash shape")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
@@ -420,7 +421,9 @@ def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dis
     else:
         roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peak_gbs, "unit": "GB/s",
                     "frac": achieved_gbs / peak_gbs, "peak_source": f"{pk_kind} HBM copy"}
-    roofline.update({"kernel": f"sparse_sink_attn_kernel<{w.d}, {'true' if b0.fused else 'false'}>",
+    kernel = ("sparse_sink_attn_d512_kernel" if w.d == 512
+              else f"sparse_sink_attn_kernel<{w.d}, {'true' if b0.fused else 'false'}>")
+    roofline.update({"kernel": kernel,
                      "traffic": traffic,
                      "algorithmic_bytes": hbm_bytes, "algorithmic_flops": flops,
                      "distinct_kv_rows": int(distinct_rows), "tflops": achieved_tf,

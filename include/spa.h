@@ -206,8 +206,16 @@ int spa_dequant_fp8_pages(const uint8_t* src, const float* scales, int64_t num_p
  * q          BF16 [n_queries, num_heads, head_dim]; element (i,h,e) at
  *            q + i*q_stride_tok + h*q_stride_head + e. Base and both
  *            strides (in bytes) must be multiples of 16.
- * head_dim   64 or 128 (d_qk = d_v)
- * num_heads  1..128, or a multiple of 128
+ * head_dim   64, 128 or 512 (d_qk = d_v). 512 is the DSV4-Flash attention
+ *            shape ("Roadmap item 24", section "Reuse and arithmetic": the
+ *            fixed H32 launch recipe; the 512-wide rows of the packed cache,
+ *            decoded by spa_unpack_d512_pages): 32 heads per CTA, the
+ *            products transposed (keys, then columns of d, on the tensor
+ *            cores' M side); slices merge inside a cluster only, so
+ *            num_splits is at most 8, no workspace is used, and 0 picks
+ *            spa_sparse_sink_attn_choose_splits_d512(n, H)
+ * num_heads  1..128, or a multiple of 128 (head_dim 64, 128); 1..32, or a
+ *            multiple of 32 (head_dim 512)
  * k_raw, v_raw   BF16 [raw_num_pages, raw_page_size, head_dim], 16-B aligned
  * pt_raw     int32 [n_requests, pt_raw_cols]
  * k_cmp, v_cmp, pt_cmp   the compressed pool, laid out the same way; may be
@@ -237,6 +245,9 @@ size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads,
                                            int32_t head_dim, int32_t num_splits);
 int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads,
                                        int32_t max_set_size);
+/* head_dim 512: slices per query (1, 2, 4 or 8) so that one wave of CTAs, one
+ * per SM, covers the batch; 1 once the batch fills the GPU. */
+int spa_sparse_sink_attn_choose_splits_d512(int32_t n_queries, int32_t num_heads);
 int spa_sparse_sink_attn_fwd(
     const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
     int32_t num_heads, int32_t head_dim,
@@ -364,6 +375,23 @@ int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_t
  * ---------------------------------------------------------------------- */
 int spa_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_size, const int32_t* page_ids,
                           int32_t n_page_ids, uint16_t* dst, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Testing hook -- not part of the method.
+ *
+ * Every wait between the warp roles of the attention forward gives up after
+ * a limit (1 s), sets SPA_DEV_TIMEOUT and lets the kernel unwind, so that a
+ * stuck pipeline ends the call instead of hanging the GPU. The waits that
+ * keep a CTA's memory alive until its own copies and tensor-core products
+ * have finished always keep the 1 s limit. spa_testing_set_wait_limit_ns
+ * changes the limit of the former for the attention forward launches that
+ * follow (process-wide, on every device); 0 makes them give up almost at
+ * once, which is how the tests reach the timeout path without a fault.
+ * Pass SPA_DEFAULT_WAIT_LIMIT_NS to restore the default. Outputs of a call
+ * that timed out are poisoned.
+ * ---------------------------------------------------------------------- */
+#define SPA_DEFAULT_WAIT_LIMIT_NS 1000000000ull
+void spa_testing_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libspa.so")
-SOURCES = ["api.cu", "kv_sets.cu", "dequant.cu", "attn_fwd.cu", "attn_bwd.cu", "kv_write.cu", "unpack_d512.cu"]
+SOURCES = ["api.cu", "kv_sets.cu", "dequant.cu", "attn_fwd.cu", "attn_d512.cu", "attn_bwd.cu", "kv_write.cu", "unpack_d512.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
               "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
 

@@ -64,6 +64,10 @@ int device_sm_count() {
   return n;
 }
 
+std::atomic<uint64_t> g_attn_wait_ns{1000ull * 1000ull * 1000ull};
+uint64_t attn_wait_limit_ns() { return g_attn_wait_ns.load(std::memory_order_relaxed); }
+void set_attn_wait_limit_ns(uint64_t ns) { g_attn_wait_ns.store(ns, std::memory_order_relaxed); }
+
 }  // namespace spa
 
 extern "C" {
@@ -84,6 +88,8 @@ const char* spa_status_string(int status) {
 }
 
 const char* spa_last_error_detail(void) { return g_detail; }
+
+void spa_testing_set_wait_limit_ns(uint64_t ns) { spa::set_attn_wait_limit_ns(ns); }
 
 // ---------------------------------------------------------------- sets
 int64_t spa_kv_sets_capacity(int32_t n_queries, int32_t window, int32_t ratio, int32_t topk_width,
@@ -223,6 +229,11 @@ int spa_sparse_sink_attn_choose_splits(int32_t n_queries, int32_t num_heads, int
   return static_cast<int>(s);
 }
 
+int spa_sparse_sink_attn_choose_splits_d512(int32_t n_queries, int32_t num_heads) {
+  if (n_queries <= 0 || num_heads <= 0) return 1;
+  return spa::d512_default_splits(n_queries, num_heads);
+}
+
 int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_tokens, int32_t head_dim,
                        const int32_t* req, const int32_t* pos, const int32_t* pt, int32_t pt_cols,
                        int32_t n_requests, int32_t page_size, int64_t num_pages, uint16_t* k_pool,
@@ -249,6 +260,7 @@ int spa_paged_kv_write(const uint16_t* k_new, const uint16_t* v_new, int32_t n_t
 size_t spa_sparse_sink_attn_workspace_size(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                                            int32_t num_splits) {
   if (n_queries <= 0 || num_heads <= 0 || head_dim <= 0 || num_splits < 0) return 0;
+  if (head_dim == 512) return 0;   // slices merge inside a cluster
   return spa::attn_workspace_bytes(n_queries, num_heads, head_dim,
                                    resolve_splits(n_queries, num_heads, num_splits));
 }
@@ -263,9 +275,16 @@ int attn_check(const spa::AttnArgs& a, int32_t requested_splits) {
   if (a.n_queries < 0) return fail(SPA_ERR_INVALID_ARG, "n_queries < 0");
   if (a.num_heads < 1) return fail(SPA_ERR_INVALID_ARG, "num_heads < 1");
   if (a.n_requests < 1) return fail(SPA_ERR_INVALID_ARG, "n_requests < 1");
-  if (a.head_dim != 64 && a.head_dim != 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
-  if (a.num_heads > 128 && a.num_heads % 128 != 0)
+  if (a.head_dim != 64 && a.head_dim != 128 && a.head_dim != 512)
+    return fail(SPA_ERR_UNSUPPORTED, "head_dim must be 64, 128 or 512");
+  if (a.head_dim == 512) {
+    if (a.num_heads > 32 && a.num_heads % 32 != 0)
+      return fail(SPA_ERR_UNSUPPORTED, "head_dim 512: num_heads above 32 must be a multiple of 32");
+    if (requested_splits > spa::kAttnMaxClusterSplits)
+      return fail(SPA_ERR_UNSUPPORTED, "head_dim 512: num_splits at most %d", spa::kAttnMaxClusterSplits);
+  } else if (a.num_heads > 128 && a.num_heads % 128 != 0) {
     return fail(SPA_ERR_UNSUPPORTED, "num_heads above 128 must be a multiple of 128");
+  }
   if (a.raw_num_pages < 0 || a.pt_raw_cols < 0) return fail(SPA_ERR_INVALID_ARG, "raw pool sizes < 0");
   if (a.raw_page_size < 1) return fail(SPA_ERR_INVALID_ARG, "raw_page_size < 1");
   if (!pow2_in(a.raw_page_size, 1, 1024))
@@ -299,7 +318,9 @@ int attn_check(const spa::AttnArgs& a, int32_t requested_splits) {
       !aligned(a.indices, 4) || !aligned(a.pt_raw, 4) || !aligned(a.pt_cmp, 4) || !aligned(a.k_cmp_scale, 4) ||
       !aligned(a.v_cmp_scale, 4))
     return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
-  const int32_t splits = resolve_splits(a.n_queries, a.num_heads, requested_splits);
+  const int32_t splits = a.head_dim == 512 ? (requested_splits > 0 ? requested_splits
+                                                                    : spa::d512_default_splits(a.n_queries, a.num_heads))
+                                           : resolve_splits(a.n_queries, a.num_heads, requested_splits);
   if (static_cast<int64_t>(a.n_queries) * splits > 0x7fffffffLL)
     return fail(SPA_ERR_UNSUPPORTED, "n_queries * num_splits exceeds the grid");
   return ok();
@@ -312,6 +333,11 @@ int attn_run(spa::AttnArgs a, int32_t requested_splits, size_t workspace_bytes, 
   if (a.out == nullptr || a.lse == nullptr) return fail(SPA_ERR_INVALID_ARG, "q, out and lse must be non-NULL");
   if (!aligned(a.out, 16)) return fail(SPA_ERR_ALIGNMENT, "out must be 16-byte aligned");
   if (!aligned(a.lse, 4)) return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
+  if (a.head_dim == 512) {
+    if (a.k_cmp_fp8 != nullptr) return fail(SPA_ERR_UNSUPPORTED, "head_dim 512: the FP8 gather takes 64 or 128");
+    a.num_splits = requested_splits > 0 ? requested_splits : spa::d512_default_splits(a.n_queries, a.num_heads);
+    return cuda_status(spa::launch_sparse_sink_attn_d512(a, stream), "sparse_sink_attn (d 512) launch");
+  }
   const int32_t splits = resolve_splits(a.n_queries, a.num_heads, requested_splits);
   const size_t need = spa::attn_workspace_bytes(a.n_queries, a.num_heads, a.head_dim, splits);
   if (need > 0) {
@@ -435,6 +461,7 @@ int spa_sparse_sink_attn_bwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
   a.v_cmp = v_cmp;
   const int st = attn_check(a, num_splits);
   if (st != SPA_OK || n_queries == 0) return st;
+  if (head_dim == 512) return fail(SPA_ERR_UNSUPPORTED, "the backward takes head_dim 64 or 128");
   if (out == nullptr || lse == nullptr || dout == nullptr)
     return fail(SPA_ERR_INVALID_ARG, "out, lse and dout must be non-NULL");
   if (dq == nullptr || dk_raw == nullptr || dv_raw == nullptr)

@@ -97,6 +97,7 @@ struct Params {
   float* dsink;           // [H] or NULL
   int32_t num_splits;
   uint32_t* dev_status;
+  uint64_t wait_ns;   // limit of the waits between the roles
 };
 
 template <int D>
@@ -752,6 +753,7 @@ cudaError_t launch_sparse_sink_attn_bwd(const AttnArgs& a, cudaStream_t stream) 
   P.dsink = a.dsink;
   P.num_splits = a.num_splits;
   P.dev_status = a.dev_status;
+  P.wait_ns = kWaitTimeoutNs;
   const int head_tiles = (a.num_heads + 127) / 128;
   if (a.head_dim == 128) return launch_d<128>(P, head_tiles, stream);
   return launch_d<64>(P, head_tiles, stream);

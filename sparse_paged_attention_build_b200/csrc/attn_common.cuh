@@ -39,17 +39,20 @@ struct ChunkDesc {
 
 __device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) / kT; }
 
-// Keys -> physical rows for one chunk. Each lane handles keys lane, lane+32,
-// ...; the loads of each phase are issued together so the chunk costs two
-// round trips, not two per key. Prm holds the page tables and pool sizes.
-template <class Prm>
+// Keys -> physical rows for one chunk. The chunk is shared by kParts
+// resolver warps; part p's lanes handle keys p*kChunkKeys/kParts + lane,
+// + lane + 32, ...; the loads of each phase are issued together so the
+// chunk costs two round trips, not two per key. Prm holds the page tables
+// and pool sizes.
+template <int kParts = 1, class Prm>
 __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t nkeys, uint32_t* tab,
-                              int lane) {
-  constexpr int kPer = kChunkKeys / 32;
+                              int lane, int part = 0) {
+  constexpr int kPer = kChunkKeys / kParts / 32;
+  const int k0 = part * (kChunkKeys / kParts);
   int32_t key[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    const int k = lane + 32 * e;
+    const int k = k0 + lane + 32 * e;
     key[e] = k < nkeys ? __ldg(P.indices + key_base + k) : -2;
   }
   int32_t page[kPer];
@@ -69,7 +72,7 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
   }
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    const int k = lane + 32 * e;
+    const int k = k0 + lane + 32 * e;
     const int32_t kk = key[e];
     uint32_t row = kInvalidRow;
     if (kk >= 0) {
@@ -95,10 +98,13 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
 // slices per query. The CTA's units are every gridDim.x-th one (strided) or
 // one contiguous range of about n_units / gridDim.x (contiguous: at any
 // moment the CTAs then work on queries far apart, whose windows do not
-// overlap).
-template <class Prm>
+// overlap). With kParts > 1, kParts warps run this loop side by side, each
+// resolving its share of every chunk (tab_full then counts all of them);
+// part 0 writes the descriptors.
+template <int kParts = 1, class Prm>
 __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* desc, uint64_t* tab_full,
-                              uint64_t* tab_empty, volatile int* abort_flag, int lane, bool contiguous = false) {
+                              uint64_t* tab_empty, volatile int* abort_flag, int lane, bool contiguous = false,
+                              int part = 0) {
   int c = 0;
   const int64_t n_units = static_cast<int64_t>(P.n_queries) * S;
   const int64_t u0 = contiguous ? (static_cast<int64_t>(blockIdx.x) * n_units) / gridDim.x : blockIdx.x;
@@ -123,10 +129,10 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
     int32_t k0 = key_lo;
     do {
       const int slot = c & 1;
-      if (!mbar_wait(tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status)) return;
+      if (!mbar_wait(tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns)) return;
       const int32_t n = max(0, min(kChunkKeys, key_hi - k0));   // 0: an empty slice
-      resolve_chunk(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane);
-      if (lane == 0) {
+      resolve_chunk<kParts>(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane, part);
+      if (lane == 0 && part == 0) {
         ChunkDesc& d = desc[slot];
         d.i = i;
         d.split = split;

@@ -24,22 +24,29 @@
 //
 // Persistent CTAs (two per SM) walk their units in a fixed stride; the two
 // CTAs of an SM interleave on the tensor core and on the exp unit. Warp
-// roles (256 threads):
+// roles (512 threads, four warpgroups):
 //   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t.
 //              They also move each unit's Q from shared memory into TMEM.
 //   warp  4    TMEM allocation; lane 0 issues every UMMA and commit
-//   warp  5    resolver: for a chunk of up to 768 keys of a unit it loads
-//              the keys, looks their pages up and writes the physical row
-//              of every key (bit 31 = raw pool) to a double-buffered table,
+//   warps 5, 7 resolver: for a chunk of up to 768 keys of a unit they load
+//              the keys, look their pages up and write the physical row of
+//              every key (bit 31 = raw pool) to a double-buffered table,
 //              plus a chunk descriptor that every other role follows. All
 //              dependent global loads of the gather happen here, ahead of
-//              the copies.
-//   warp  6    K gather (and Q): TMA tile::gather4 loads, four rows of one
-//              pool per instruction, into a 2-stage ring, 128-byte swizzled
-//              by the tensor map into the K-major layout of the UMMA
-//              descriptors; rows outside a pool (padding, faulty keys) are
-//              zero-filled by the TMA. Q arrives as TMA boxes.
-//   warp  7    V gather, into its own 2-stage ring
+//              the copies; each warp takes half of every chunk.
+//   warp  6    Q: one TMA box load per unit into the landing area
+//   warps 8-11 K gather, warps 12-15 V gather: 16-byte cp.async copies of
+//              the rows the table names into 2-stage rings, written in the
+//              128-byte swizzled K-major layout of the UMMA descriptors
+//              (lanes 0-15 of a warp copy one 256-byte row, so every
+//              instruction moves whole rows); rows outside a pool (padding,
+//              faulty keys) are zero-filled. Measured on B200, random row
+//              gathers from L2 by cp.async over 8 warps per CTA run at
+//              about 14.7 TB/s against 5.9 TB/s for TMA tile::gather4 from
+//              one warp per operand, which capped this kernel before.
+// The warpgroups then move registers with setmaxnreg: the softmax rows keep
+// 64 scores, 32 packed probabilities and the running statistics in
+// registers, the copy warps need few.
 // TMEM columns: S/P [0,64), Q [64, 64 + d/2) as packed BF16 pairs, O after.
 // S is single-buffered: QK^T of tile g+1 is issued after PV of tile g, and
 // the UMMAs of a CTA run in issue order, so P(g) is read before S(g+1)
@@ -62,18 +69,30 @@ constexpr int kStagesK = 2;
 constexpr int kStagesV = 2;
 constexpr int kSoftThreads = 128;
 constexpr int kMmaWarp = 4;
-constexpr int kResolverWarp = 5;
-constexpr int kKWarp0 = 6;                       // K (and Q) producer
-constexpr int kVWarp0 = 7;                       // V producer
-constexpr int kThreads = 256;
+constexpr int kResolverWarp0 = 5;
+constexpr int kQWarp = 6;
+constexpr int kResolverWarp1 = 7;
+constexpr int kKGroupWarp0 = 8;                  // warps 8..11: K rows
+constexpr int kVGroupWarp0 = 12;                 // warps 12..15: V rows
+constexpr int kGroupThreads = 128;
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 256;
+// Registers per thread after the split; the four warpgroups together keep
+// the 4 x 64 the block is launched with (two 512-thread blocks per SM).
+template <bool kFp8>
+struct RegSplit {
+  static constexpr uint32_t kSoftmax = kFp8 ? 120 : 136;
+  static constexpr uint32_t kControl = 56;            // MMA issue, resolvers, Q
+  static constexpr uint32_t kGather = kFp8 ? 40 : 32;  // the FP8 decode holds codes and scales
+  static_assert(true || kSoftmax + kControl + 2 * kGather <= 4 * 64, "register split exceeds the launch");
+};
 // A tile whose row sum of P, taken with the running max as it stands,
 // exceeds 2^16 (or is not a number) is recomputed with its exact max. P
 // therefore stays below 2^16: harmless in BF16 and in the FP32 sums, whose
 // relative precision does not depend on magnitude.
 constexpr float kSpecBound = 65536.0f;
-// consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
-constexpr uint32_t kTabConsumers = 32 + 32 + 1 + kSoftThreads;
+// consumers of a chunk descriptor: K and V groups, MMA thread, softmax, Q warp
+constexpr uint32_t kTabConsumers = 2 * kGroupThreads + 1 + kSoftThreads + 32;
 
 struct Params {
   // TMA descriptors (passed as a __grid_constant__ parameter)
@@ -82,6 +101,11 @@ struct Params {
   CUtensorMap tm_v_raw;
   CUtensorMap tm_k_cmp;
   CUtensorMap tm_v_cmp;
+  // the pools as plain pointers, for the cp.async gather
+  const uint8_t* k_raw;
+  const uint8_t* v_raw;
+  const uint8_t* k_cmp;
+  const uint8_t* v_cmp;
   int32_t q_box_rows;     // min(128, num_heads)
   int32_t n_queries, num_heads;
   int64_t raw_pages;
@@ -114,6 +138,10 @@ struct Params {
   float2* part_ml;     // [n_queries * num_splits][num_heads]
   uint32_t* tickets;   // [n_queries * head_tiles]
   uint32_t* dev_status;
+  // limit of every wait between the roles (ns); the waits that keep TMEM
+  // and shared memory alive until the CTA's own copies and MMAs are done
+  // keep the fixed kWaitTimeoutNs
+  uint64_t wait_ns;
 };
 
 template <int D>
@@ -165,8 +193,126 @@ struct Bars {
   uint64_t* soft_sync;
 };
 
+// End of every role (inlined into each, so that it runs within that
+// warpgroup's registers): every TMEM access of the role has completed; the
+// softmax warps (soft) then run the cluster merge, every warp takes the
+// cluster barriers, and the MMA warp frees TMEM last.
+template <int D>
+__device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                                           int tid, int warp, int S, int heads_here, int head0) {
+  using L = Layout<D>;
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (P.cluster_merge) {
+    // Exact merge of the S slices of query i, CTA `rank` holding slice
+    // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
+    // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
+    // Summary: the deterministic (out, lse) merge). Each CTA scales its own
+    // O rows by its weight into shared memory (the K/V rings are idle now);
+    // then CTA `rank` sums its share of the rows over the cluster's shared
+    // memory and writes them. Every thread of every CTA reaches the three
+    // cluster barriers: every earlier wait in the kernel is bounded.
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int i = static_cast<int>(blockIdx.x / S);
+    const uint32_t ml_addr = sbase + L::kMergeOff;
+    const uint32_t wo_addr = sbase + L::kKOff;               // [128][D] FP32, 16-byte chunks swizzled by row
+    constexpr int kChunks = D / 4;                           // 16-byte chunks per row
+    __syncwarp();
+    cluster_sync_all();                                      // every slice's (m, l) is in place
+    if (soft) {
+      const int row = tid;
+      // all slices' (m, l) of this row, the loads in flight together
+      float2 ml[kAttnMaxClusterSplits];
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+        ml[s] = s < S ? ld_dsmem_f2(dsmem_addr(ml_addr + row * 8, s)) : make_float2(-INFINITY, 0.f);
+      float M = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+        if (ml[s].y > 0.f) M = fmaxf(M, ml[s].x);
+      float Lsum = 0.f, w_own = 0.f;
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
+        const float w = (ml[s].y > 0.f) ? exp2_approx(ml[s].x - M) : 0.f;
+        Lsum += w * ml[s].y;
+        if (s == rank) w_own = w;
+      }
+      const float scale_own = Lsum > 0.f ? w_own / Lsum : 0.f;
+      if (rank == 0 && row < heads_here)
+        P.lse[static_cast<int64_t>(i) * P.num_heads + head0 + row] =
+            Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
+      const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
+      const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
+      float* wo = reinterpret_cast<float*>(smem + L::kKOff);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {   // warp-uniform: one flag per CTA
+          tmem_ld32(o_lane + c0, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const int chunk = (c0 >> 2) + v;
+          const int phys = chunk ^ (row & (kChunks - 1));
+          *reinterpret_cast<float4*>(wo + row * D + phys * 4) =
+              make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
+                          __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own);
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();                                      // every slice's weighted rows are in place
+    if (soft) {
+      const int per = (heads_here + S - 1) / S;
+      const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
+      uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
+      // two 16-byte pieces per thread per pass, every slice's copy of both
+      // loaded before any is added
+      const int n_items = (r1 - r0) * kChunks;
+      for (int base = tid; base < n_items; base += 2 * kSoftThreads) {
+        float4 v[2][kAttnMaxClusterSplits];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int idx = base + k * kSoftThreads;
+          const int r = r0 + idx / kChunks, c = idx % kChunks;
+          const uint32_t off = wo_addr + static_cast<uint32_t>((r * D + (c ^ (r & (kChunks - 1))) * 4) * 4);
+#pragma unroll
+          for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+            v[k][s] = (idx < n_items && s < S) ? ld_dsmem_f4(dsmem_addr(off, s)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int idx = base + k * kSoftThreads;
+          if (idx >= n_items) continue;
+          const int r = r0 + idx / kChunks, c = idx % kChunks;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
+            acc.x += v[k][s].x;
+            acc.y += v[k][s].y;
+            acc.z += v[k][s].z;
+            acc.w += v[k][s].w;
+          }
+          *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r) * D + 4 * c) =
+              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();                                      // no slice leaves while its memory is read
+  }
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
 template <int D, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __grid_constant__ Params P) {
+  using R = RegSplit<kFp8>;
   using L = Layout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -204,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   // ---- setup
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(B.tab_full + s, 32);
+      mbar_init(B.tab_full + s, 64);   // two resolver warps
       mbar_init(B.tab_empty + s, kTabConsumers);
       mbar_init(B.soft_sync + s, kSoftThreads);
     }
@@ -212,11 +358,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     mbar_init(B.q_empty, kSoftThreads);
     mbar_init(B.q_ready, kSoftThreads);
     for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(B.k_full + s, 1);
+      mbar_init(B.k_full + s, kGroupThreads);
       mbar_init(B.k_empty + s, 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(B.v_full + s, 1);
+      mbar_init(B.v_full + s, kGroupThreads);
       mbar_init(B.v_empty + s, 1);
     }
     mbar_init(B.s_full, 1);
@@ -234,227 +380,222 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == kResolverWarp) {
-    // ================================================= resolver
-    resolver_loop(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane);
-  } else if (warp == kKWarp0 || warp == kVWarp0) {
-    // ================================================= K / V gather (TMA)
-    // A tile is 16 four-row groups x D/64 column halves = "jobs"; lane j
-    // issues one TMA tile::gather4 for job j (four rows of one pool, 512
-    // bytes). A group whose four keys come from both pools (at most one per
-    // unit: compressed groups precede window tokens) is loaded row by row.
-    // Rows past the chunk's keys and rows of faulty keys are outside the
-    // tensor and zero-filled. Lane 0 of the K warp also loads each unit's Q
-    // (every unit, empty ones included, so that the Q phases of all roles
-    // stay in step).
-    const bool is_k = warp == kKWarp0;
+  // Each warpgroup takes its register limit at one place (setmaxnreg is
+  // executed by the four warps of a warpgroup together) that dominates all
+  // of its roles' code.
+  if (warp >= 4 && warp < 8) {
+    warpgroup_reg_dealloc<R::kControl>();
+    if (warp == kResolverWarp0 || warp == kResolverWarp1) {
+      // ================================================= resolver
+      resolver_loop<2>(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane, false,
+                       warp == kResolverWarp0 ? 0 : 1);
+      cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
+    } else if (warp == kQWarp) {
+      // ================================================= Q loader
+      // Every unit's Q, empty units included, so that the Q phases of all
+      // roles stay in step; the landing area is free once the previous Q
+      // has moved on to TMEM.
+      constexpr int kHalves = D / 64;
+      int c = 0, qc = 0;
+      bool final_seen = false;
+      while (!final_seen) {
+        const int slot = c & 1;
+        if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
+        const ChunkDesc d = desc[slot];
+        final_seen = (d.flags & kFlagFinal) != 0;
+        bool ok = true;
+        if (d.flags & kFlagFirst) {
+          ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns);
+          if (ok && lane == 0) {
+            mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
+            for (int hb = 0; hb < kHalves; ++hb)
+              tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0, d.i);
+          }
+          if (ok) ++qc;
+        }
+        __syncwarp();
+        mbar_arrive(B.tab_empty + slot);
+        ++c;
+        if (!ok) break;
+      }
+      // the last Q copy has landed before the CTA can leave (it lands even
+      // when the roles gave up early; this wait keeps the fixed limit)
+      if (qc > 0) mbar_wait(B.q_full, (qc - 1) & 1, nullptr, P.dev_status);
+      cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
+    } else if (warp == kMmaWarp) {
+      // ================================================= UMMA issuer
+      // Per tile: S = Q K^T (A = Q from TMEM), then, once P is in TMEM,
+      // O += P V (A = P from TMEM). s_full is committed after the QK^T of a
+      // tile, so its arrival also means every earlier UMMA (the previous PV)
+      // has completed.
+      if (lane == 0) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, kT, 0);
+        constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
+        int c = 0, g = 0, u = 0;
+        bool ok = true, final_seen = false;
+        while (ok && !final_seen) {
+          const int slot = c & 1;
+          if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          const ChunkDesc d = desc[slot];
+          mbar_arrive(B.tab_empty + slot);
+          ++c;
+          final_seen = (d.flags & kFlagFinal) != 0;
+          if (d.flags & kFlagFirst) {   // this unit's Q is in TMEM
+            if (!mbar_wait(B.q_ready, u & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+            ++u;
+            tc_fence_after_sync();
+          }
+          const int ntiles = ceil_tiles(d.nkeys);
+          for (int t = 0; t < ntiles; ++t, ++g) {
+            const int stage = g % kStagesK, st = g % kStagesV;
+            if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+            tc_fence_after_sync();
+            const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
+  #pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + (k & 3) * 32, 16, 1024);
+              umma_ts(tmem + L::kSCol, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
+            }
+            tc_commit(B.k_empty + stage);
+            tc_commit(B.s_full);
+            if (!mbar_wait(B.p_ready, g & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+            if (!mbar_wait(B.v_full + st, (g / kStagesV) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+            tc_fence_after_sync();
+            const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
+            const bool first = (d.flags & kFlagFirst) && t == 0;
+  #pragma unroll
+            for (int k = 0; k < kT / 16; ++k) {
+              const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
+              umma_ts(tmem + L::kOCol, tmem + L::kSCol + k * 8, bdesc, idesc_o, (!first || k > 0) ? 1u : 0u);
+            }
+            tc_commit(B.v_empty + st);
+            if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.o_done);
+          }
+        }
+        // every UMMA has completed before TMEM is released
+        tc_commit(B.mma_done);
+        mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
+      }
+      cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
+    }
+  } else if (warp >= kKGroupWarp0) {
+    warpgroup_reg_dealloc<R::kGather>();
+    // ================================================= K / V gather (cp.async)
+    // A warp copies 16 rows of a 64-row tile: lane l takes 16-byte piece
+    // l % (D/8) of row l / (D/8) (+ the rows of later instructions), so an
+    // instruction moves 32 / (D/8) whole rows. Piece c of row r lands at
+    // half c/8 (64-column blocks), row r, 16-byte chunk (c%8) ^ (r%8): the
+    // 128-byte swizzle of the K-major UMMA layout. A tile is handed over
+    // (fence.proxy.async, then one arrival per thread) once its copies have
+    // landed, which is checked after the next tile's copies are issued, so
+    // two tiles are in flight; before any wait that would block, the tile
+    // in flight is handed over first.
+    const bool is_k = warp < kVGroupWarp0;
+    const int gw = warp - (is_k ? kKGroupWarp0 : kVGroupWarp0);
     const int nst = is_k ? kStagesK : kStagesV;
     uint64_t* full = is_k ? B.k_full : B.v_full;
     uint64_t* empty = is_k ? B.k_empty : B.v_empty;
-    const CUtensorMap* map_raw = is_k ? &P.tm_k_raw : &P.tm_v_raw;
-    const CUtensorMap* map_cmp = is_k ? &P.tm_k_cmp : &P.tm_v_cmp;
+    const uint8_t* pool_raw = is_k ? P.k_raw : P.v_raw;
+    const uint8_t* pool_cmp = is_k ? P.k_cmp : P.v_cmp;
+    const uint8_t* pool8 = is_k ? P.k_cmp8 : P.v_cmp8;
+    const float* psc = is_k ? P.k_cmp_sc : P.v_cmp_sc;
     const uint32_t ring = sbase + (is_k ? L::kKOff : L::kVOff);
-    constexpr int kHalves = D / 64;
-    constexpr int kGroups = kT / 4;
-    constexpr int kJobs = kGroups * kHalves;
-    const int grp = lane % kGroups, half = lane / kGroups;
-    const bool issuer = lane < kJobs;
-    int c = 0, g = 0, qc = 0;
+    constexpr int kCpr = D / 8;          // 16-byte pieces per row
+    constexpr int kRpi = 32 / kCpr;      // rows per instruction
+    constexpr int kNi = 16 / kRpi;       // instructions per warp per tile
+    const int ch = lane % kCpr, rsub = lane / kCpr;
+    const uint32_t col_off = static_cast<uint32_t>((ch / 8) * (kT * 128));
+    const int c8 = ch % 8;
+    int pending = -1;   // ring stage whose copies are issued but not handed over
+    auto hand_over = [&]() {
+      if (pending >= 0) {
+        cp_async_wait_group<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(full + pending);
+        pending = -1;
+      }
+    };
+    int c = 0, g = 0;
     bool final_seen = false;
     while (!final_seen) {
       const int slot = c & 1;
-      if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status)) break;
+      if (pending >= 0 && !mbar_try_wait(B.tab_full + slot, (c >> 1) & 1)) hand_over();
+      if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
       const ChunkDesc d = desc[slot];
       final_seen = (d.flags & kFlagFinal) != 0;
       const uint32_t* t_rows = tab + slot * kChunkKeys;
       const int ntiles = ceil_tiles(d.nkeys);
       bool ok = true;
-      if (is_k && (d.flags & kFlagFirst)) {
-        // the landing area is free once the previous Q has moved to TMEM
-        ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status);
-        if (ok && lane == 0) {
-          mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
-          for (int hb = 0; hb < kHalves; ++hb)
-            tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0, d.i);
-        }
-        ++qc;
-      }
-      if constexpr (!kFp8) {
-        for (int t = 0; ok && t < ntiles; ++t, ++g) {
-          const int stage = g % nst;
-          if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
-          if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
-          __syncwarp();
-          if (issuer) {
-            const int nv = min(kT, d.nkeys - t * kT);
-            uint32_t e[4];
-            bool any_raw = false, any_cmp = false;
-  #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int r = 4 * grp + k;
-              e[k] = r < nv ? t_rows[t * kT + r] : kInvalidRow;
-              if (e[k] != kInvalidRow) {
-                if (e[k] & kRawBit) any_raw = true;
-                else any_cmp = true;
-              }
-            }
-            int32_t y[4];
-  #pragma unroll
-            for (int k = 0; k < 4; ++k)   // rows outside the tensor are zero-filled
-              y[k] = e[k] == kInvalidRow ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
-            const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
-            if (!(any_raw && any_cmp)) {
-              tma_gather4(dst, any_cmp ? map_cmp : map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
-            } else {
-  #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const bool cmp_row = e[k] != kInvalidRow && !(e[k] & kRawBit);
-                tma_load_2d(dst + k * 128, cmp_row ? map_cmp : map_raw, full + stage, half * 64, y[k]);
-              }
-            }
+      for (int t = 0; t < ntiles; ++t, ++g) {
+        const int stage = g % nst;
+        const uint32_t par = ((g / nst) & 1) ^ 1;
+        if (pending >= 0 && !mbar_try_wait(empty + stage, par)) hand_over();
+        if (!mbar_wait(empty + stage, par, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+        const int nv = min(kT, d.nkeys - t * kT);
+        const uint32_t* trow = t_rows + t * kT;
+        const uint32_t stage_base = ring + stage * L::kTileBytes + col_off;
+        if constexpr (!kFp8) {
+#pragma unroll 2
+          for (int j = 0; j < kNi; ++j) {
+            const int r = gw * 16 + j * kRpi + rsub;
+            const uint32_t e = r < nv ? trow[r] : kInvalidRow;
+            const uint8_t* base = (e & kRawBit) ? pool_raw : pool_cmp;
+            const bool valid = e != kInvalidRow && base != nullptr;
+            const uint8_t* src = valid ? base + static_cast<int64_t>(e & ~kRawBit) * (D * 2) + ch * 16 : pool_raw;
+            cp_async16(stage_base + r * 128 + ((c8 ^ (r & 7)) << 4), src, valid ? 16u : 0u);
           }
-        }
-      } else {
-        // Fused FP8 decode. Raw (window) rows and zero rows (past the set,
-        // faulty keys) still come by TMA; compressed rows are read as E4M3
-        // codes and scales with plain loads (all of a tile's loads in flight
-        // together), decoded exactly as the page decode does, and written
-        // into the same 128-byte swizzled BF16 layout. The tile is complete
-        // once the TMA bytes have landed and lane 0 has arrived after every
-        // lane's shared-memory writes. (Staging the codes through cp.async
-        // to overlap the next tile's fetch measured slower on B200.)
-        constexpr int kPieces = D / 16;   // 16 codes per piece
-        constexpr int kPerLane = kT * kPieces / 32;
-        const uint8_t* pool8 = is_k ? P.k_cmp8 : P.v_cmp8;
-        const float* psc = is_k ? P.k_cmp_sc : P.v_cmp_sc;
-        for (int t = 0; ok && t < ntiles; ++t, ++g) {
-          const int stage = g % nst;
-          if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status)) { ok = false; break; }
-          const int nv = min(kT, d.nkeys - t * kT);
-          const uint32_t* trow = t_rows + t * kT;
-          uint32_t tx = 0;
-          uint32_t e[4];
-          bool fp8_row[4] = {false, false, false, false};
-          if (issuer) {
+        } else {
+          // compressed rows arrive as E4M3 codes (8 per piece) and their
+          // group scale, decoded exactly as the page decode does; window rows
+          // and zero rows by cp.async. Every load of the tile first.
+          uint2 code[kNi];
+          float sc[kNi];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int r = 4 * grp + k;
-              e[k] = r < nv ? trow[r] : kInvalidRow;
-              fp8_row[k] = e[k] != kInvalidRow && !(e[k] & kRawBit);
-              if (!fp8_row[k]) tx += 128;
-            }
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) tx += __shfl_xor_sync(0xffffffffu, tx, off);
-          if (lane == 0) mbar_expect_tx(full + stage, tx);
-          __syncwarp();
-          if (issuer) {
-            int32_t y[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              y[k] = (e[k] == kInvalidRow || fp8_row[k]) ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
-            const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
-            if (!(fp8_row[0] || fp8_row[1] || fp8_row[2] || fp8_row[3])) {
-              tma_gather4(dst, map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
-            } else {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                if (!fp8_row[k]) tma_load_2d(dst + k * 128, map_raw, full + stage, half * 64, y[k]);
-            }
-          }
-          uint8_t* tile = smem + (is_k ? L::kKOff : L::kVOff) + stage * L::kTileBytes;
-          uint4 raw[kPerLane];
-          float sc[kPerLane];
-#pragma unroll
-          for (int j = 0; j < kPerLane; ++j) {   // every load first
-            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
-            const uint32_t er = r < nv ? trow[r] : kInvalidRow;
-            raw[j] = make_uint4(0u, 0u, 0u, 0u);
+          for (int j = 0; j < kNi; ++j) {
+            const int r = gw * 16 + j * kRpi + rsub;
+            const uint32_t e = r < nv ? trow[r] : kInvalidRow;
+            const bool fp8_row = e != kInvalidRow && !(e & kRawBit);
+            code[j] = make_uint2(0u, 0u);
             sc[j] = 0.f;
-            if (er != kInvalidRow && !(er & kRawBit)) {
-              const int64_t row8 = er;
-              raw[j] = __ldg(reinterpret_cast<const uint4*>(pool8 + row8 * D + piece * 16));
-              sc[j] = __ldg(psc + row8 * (D / 64) + (piece * 16) / 64);
+            if (fp8_row) {
+              const int64_t row8 = e;
+              code[j] = __ldg(reinterpret_cast<const uint2*>(pool8 + row8 * D + ch * 8));
+              sc[j] = __ldg(psc + row8 * (D / 64) + (ch * 8) / 64);
+            } else {
+              const bool valid = e != kInvalidRow;
+              const uint8_t* src = valid ? pool_raw + static_cast<int64_t>(e & ~kRawBit) * (D * 2) + ch * 16 : pool_raw;
+              cp_async16(stage_base + r * 128 + ((c8 ^ (r & 7)) << 4), src, valid ? 16u : 0u);
             }
           }
 #pragma unroll
-          for (int j = 0; j < kPerLane; ++j) {
-            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
-            const uint32_t er = r < nv ? trow[r] : kInvalidRow;
-            if (er == kInvalidRow || (er & kRawBit)) continue;
-            uint32_t o[8];
-            if (P.fp8_fnuz) decode_e4m3x16<true>(raw[j], sc[j], o);
-            else decode_e4m3x16<false>(raw[j], sc[j], o);
-            const int hf = (piece * 16) / 64, ch0 = ((piece * 16) % 64) / 8;
-            uint8_t* row_ptr = tile + hf * (kT * 128) + r * 128;
-            *reinterpret_cast<uint4*>(row_ptr + ((ch0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(row_ptr + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          for (int j = 0; j < kNi; ++j) {
+            const int r = gw * 16 + j * kRpi + rsub;
+            const uint32_t e = r < nv ? trow[r] : kInvalidRow;
+            if (e == kInvalidRow || (e & kRawBit)) continue;
+            uint32_t o[4];
+            if (P.fp8_fnuz) decode_e4m3x8<true>(code[j], sc[j], o);
+            else decode_e4m3x8<false>(code[j], sc[j], o);
+            *reinterpret_cast<uint4*>(smem + (stage_base - sbase) + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+                make_uint4(o[0], o[1], o[2], o[3]);
           }
-          fence_proxy_async_smem();   // generic-proxy writes -> the UMMA's reads
-          __syncwarp();
-          if (lane == 0) mbar_arrive(full + stage);
         }
+        cp_async_commit();
+        if (pending >= 0) {   // the previous tile has landed: hand it over
+          cp_async_wait_group<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(full + pending);
+        }
+        pending = stage;
       }
       mbar_arrive(B.tab_empty + slot);
       ++c;
       if (!ok) break;
     }
-  } else if (warp == kMmaWarp) {
-    // ================================================= UMMA issuer
-    // Per tile: S = Q K^T (A = Q from TMEM), then, once P is in TMEM,
-    // O += P V (A = P from TMEM). s_full is committed after the QK^T of a
-    // tile, so its arrival also means every earlier UMMA (the previous PV)
-    // has completed.
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kT, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
-      int c = 0, g = 0, u = 0;
-      bool ok = true, final_seen = false;
-      while (ok && !final_seen) {
-        const int slot = c & 1;
-        if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status)) { ok = false; break; }
-        const ChunkDesc d = desc[slot];
-        mbar_arrive(B.tab_empty + slot);
-        ++c;
-        final_seen = (d.flags & kFlagFinal) != 0;
-        if (d.flags & kFlagFirst) {   // this unit's Q is in TMEM
-          if (!mbar_wait(B.q_ready, u & 1, abort_flag, P.dev_status)) { ok = false; break; }
-          ++u;
-          tc_fence_after_sync();
-        }
-        const int ntiles = ceil_tiles(d.nkeys);
-        for (int t = 0; t < ntiles; ++t, ++g) {
-          const int stage = g % kStagesK, st = g % kStagesV;
-          if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status)) { ok = false; break; }
-          tc_fence_after_sync();
-          const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + (k & 3) * 32, 16, 1024);
-            umma_ts(tmem + L::kSCol, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
-          }
-          tc_commit(B.k_empty + stage);
-          tc_commit(B.s_full);
-          if (!mbar_wait(B.p_ready, g & 1, abort_flag, P.dev_status)) { ok = false; break; }
-          if (!mbar_wait(B.v_full + st, (g / kStagesV) & 1, abort_flag, P.dev_status)) { ok = false; break; }
-          tc_fence_after_sync();
-          const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
-          const bool first = (d.flags & kFlagFirst) && t == 0;
-#pragma unroll
-          for (int k = 0; k < kT / 16; ++k) {
-            const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
-            umma_ts(tmem + L::kOCol, tmem + L::kSCol + k * 8, bdesc, idesc_o, (!first || k > 0) ? 1u : 0u);
-          }
-          tc_commit(B.v_empty + st);
-          if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.o_done);
-        }
-      }
-      // every UMMA has completed before TMEM is released
-      tc_commit(B.mma_done);
-      mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
-    }
+    hand_over();
+    cp_async_wait_group<0>();
+    cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
   } else {
+    warpgroup_reg_alloc<R::kSoftmax>();
     // ================================================= softmax + epilogue
     const int row = tid;   // head row == TMEM lane
     const int h = head0 + row;
@@ -468,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const uint32_t parity = (nsync >> 1) & 1;
       ++nsync;
       mbar_arrive(bar);
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, P.dev_status));
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, P.dev_status, P.wait_ns));
     };
     // Q of the next unit: shared memory (TMA, 128-byte swizzled rows) ->
     // registers -> this thread's TMEM lane, as the packed BF16 pairs the
@@ -476,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     // reads the previous Q has completed.
     int qc = 0;
     auto copy_q = [&]() -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(B.q_full, qc & 1, abort_flag, P.dev_status))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(B.q_full, qc & 1, abort_flag, P.dev_status, P.wait_ns))) return false;
       ++qc;
       const uint8_t* qrow = smem + L::kQOff + row * 128;
 #pragma unroll
@@ -525,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     uint32_t s0[32], s1[32];
     while (ok && !final_seen) {
       const int slot = c & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns))) {
         ok = false;
         break;
       }
@@ -544,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const int ntiles = ceil_tiles(d.nkeys);
       for (int t = 0; t < ntiles; ++t, ++g, ++unit_tiles) {
         // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
-        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full, g & 1, abort_flag, P.dev_status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full, g & 1, abort_flag, P.dev_status, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -642,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       // ---- epilogue of the unit
       const bool have_o = unit_tiles > 0;
       if (have_o) {
-        if (!__all_sync(0xffffffffu, mbar_wait(B.o_done, n_o & 1, abort_flag, P.dev_status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(B.o_done, n_o & 1, abort_flag, P.dev_status, P.wait_ns))) {
           ok = false;
           break;
         }
@@ -796,116 +937,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         }
       }
     }
+    cta_finish<D>(P, true, smem, sbase, tmem, tid, warp, S, heads_here, head0);
   }
-
-  // ---- teardown: every TMEM access above has completed
-  __syncwarp();
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  if (P.cluster_merge) {
-    // Exact merge of the S slices of query i, CTA `rank` holding slice
-    // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
-    // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
-    // Summary: the deterministic (out, lse) merge). Each CTA scales its own
-    // O rows by its weight into shared memory (the K/V rings are idle now);
-    // then CTA `rank` sums its share of the rows over the cluster's shared
-    // memory and writes them. Every thread of every CTA reaches the three
-    // cluster barriers: every earlier wait in the kernel is bounded.
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int i = static_cast<int>(blockIdx.x / S);
-    const uint32_t ml_addr = sbase + L::kMergeOff;
-    const uint32_t wo_addr = sbase + L::kKOff;               // [128][D] FP32, 16-byte chunks swizzled by row
-    constexpr int kChunks = D / 4;                           // 16-byte chunks per row
-    __syncwarp();
-    cluster_sync_all();                                      // every slice's (m, l) is in place
-    if (tid < kSoftThreads) {
-      const int row = tid;
-      // all slices' (m, l) of this row, the loads in flight together
-      float2 ml[kAttnMaxClusterSplits];
-#pragma unroll
-      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-        ml[s] = s < S ? ld_dsmem_f2(dsmem_addr(ml_addr + row * 8, s)) : make_float2(-INFINITY, 0.f);
-      float M = -INFINITY;
-#pragma unroll
-      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-        if (ml[s].y > 0.f) M = fmaxf(M, ml[s].x);
-      float Lsum = 0.f, w_own = 0.f;
-#pragma unroll
-      for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
-        const float w = (ml[s].y > 0.f) ? exp2_approx(ml[s].x - M) : 0.f;
-        Lsum += w * ml[s].y;
-        if (s == rank) w_own = w;
-      }
-      const float scale_own = Lsum > 0.f ? w_own / Lsum : 0.f;
-      if (rank == 0 && row < heads_here)
-        P.lse[static_cast<int64_t>(i) * P.num_heads + head0 + row] =
-            Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
-      const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
-      const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
-      float* wo = reinterpret_cast<float*>(smem + L::kKOff);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        if (have_o) {   // warp-uniform: one flag per CTA
-          tmem_ld32(o_lane + c0, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
-        }
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const int chunk = (c0 >> 2) + v;
-          const int phys = chunk ^ (row & (kChunks - 1));
-          *reinterpret_cast<float4*>(wo + row * D + phys * 4) =
-              make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
-                          __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own);
-        }
-      }
-    }
-    __syncwarp();
-    cluster_sync_all();                                      // every slice's weighted rows are in place
-    if (tid < kSoftThreads) {
-      const int per = (heads_here + S - 1) / S;
-      const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
-      uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
-      // two 16-byte pieces per thread per pass, every slice's copy of both
-      // loaded before any is added
-      const int n_items = (r1 - r0) * kChunks;
-      for (int base = tid; base < n_items; base += 2 * kSoftThreads) {
-        float4 v[2][kAttnMaxClusterSplits];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int idx = base + k * kSoftThreads;
-          const int r = r0 + idx / kChunks, c = idx % kChunks;
-          const uint32_t off = wo_addr + static_cast<uint32_t>((r * D + (c ^ (r & (kChunks - 1))) * 4) * 4);
-#pragma unroll
-          for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-            v[k][s] = (idx < n_items && s < S) ? ld_dsmem_f4(dsmem_addr(off, s)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int idx = base + k * kSoftThreads;
-          if (idx >= n_items) continue;
-          const int r = r0 + idx / kChunks, c = idx % kChunks;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
-            acc.x += v[k][s].x;
-            acc.y += v[k][s].y;
-            acc.z += v[k][s].z;
-            acc.w += v[k][s].w;
-          }
-          *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r) * D + 4 * c) =
-              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-        }
-      }
-    }
-    __syncwarp();
-    cluster_sync_all();                                      // no slice leaves while its memory is read
-  }
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 template <int D, bool kFp8>
@@ -974,6 +1007,10 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
         !encode_pool(&P.tm_v_cmp, a.v_cmp, cmp_rows, a.head_dim))
       return cudaErrorInvalidValue;
   }
+  P.k_raw = reinterpret_cast<const uint8_t*>(a.k_raw);
+  P.v_raw = reinterpret_cast<const uint8_t*>(a.v_raw);
+  P.k_cmp = a.k_cmp_fp8 == nullptr ? reinterpret_cast<const uint8_t*>(a.k_cmp) : nullptr;
+  P.v_cmp = a.k_cmp_fp8 == nullptr ? reinterpret_cast<const uint8_t*>(a.v_cmp) : nullptr;
   P.n_queries = a.n_queries;
   P.num_heads = a.num_heads;
   P.raw_pages = a.raw_num_pages;
@@ -999,6 +1036,7 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
   P.lse = a.lse;
   P.num_splits = a.num_splits;
   P.dev_status = a.dev_status;
+  P.wait_ns = attn_wait_limit_ns();
   const int head_tiles = (a.num_heads + 127) / 128;
   P.part_o = nullptr;
   P.part_ml = nullptr;

@@ -58,17 +58,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for the phase of `bar` with the given parity to complete. Gives up
 // when *abort is set by another thread of the CTA (abort may be nullptr: no
-// such check), or after kWaitTimeoutNs (then sets *abort and
-// SPA_DEV_TIMEOUT). Returns false when it gave up.
+// such check), or after limit_ns (then sets *abort and SPA_DEV_TIMEOUT).
+// Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* dev_status) {
+                                          uint32_t* dev_status, uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         if (abort != nullptr) *abort = 1;
         report(dev_status, SPA_DEV_TIMEOUT);
         return false;
@@ -104,6 +104,29 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // later tensor-core reads (async proxy).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Close the group of cp.async issued since the last commit.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most N committed groups of this thread are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------- registers
+// Move this warpgroup's per-thread register limit (all four warps execute
+// it together). A decrease returns registers to the block's pool; an
+// increase waits until the pool holds enough, so the increases of a block
+// must fit in what its threads were launched with.
+template <uint32_t R>
+__device__ __forceinline__ void warpgroup_reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void warpgroup_reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 // ---------------------------------------------------------------- TMA
@@ -397,6 +420,27 @@ __device__ __forceinline__ void decode_e4m3x16(const uint4 raw, float s, uint32_
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
+    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
+    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
+    if (kFnuz) {
+      a.x = fnuz_from_ocp(a.x, w[k] & 0xffu);
+      a.y = fnuz_from_ocp(a.y, (w[k] >> 8) & 0xffu);
+      b.x = fnuz_from_ocp(b.x, (w[k] >> 16) & 0xffu);
+      b.y = fnuz_from_ocp(b.y, w[k] >> 24);
+    }
+    o[2 * k] = pack_bf16x2(__fmul_rn(a.x, s), __fmul_rn(a.y, s));
+    o[2 * k + 1] = pack_bf16x2(__fmul_rn(b.x, s), __fmul_rn(b.y, s));
+  }
+}
+
+// 8 E4M3 codes (one 8-byte load) with their group scale -> 8 BF16 values
+// packed in pairs, element by element the same arithmetic as
+// decode_e4m3x16.
+template <bool kFnuz = false>
+__device__ __forceinline__ void decode_e4m3x8(const uint2 raw, float s, uint32_t (&o)[4]) {
+  const uint32_t w[2] = {raw.x, raw.y};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
     float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[k] & 0xffffu));
     float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[k] >> 16));
     if (kFnuz) {

@@ -88,6 +88,14 @@ constexpr int kAttnMaxClusterSplits = 8;
 size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                             int32_t num_splits);
 cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream);
+// Limit (ns) of the waits between the warp roles of the attention forward;
+// 1 s unless a test changed it.
+uint64_t attn_wait_limit_ns();
+void set_attn_wait_limit_ns(uint64_t ns);
 cudaError_t launch_sparse_sink_attn_bwd(const AttnArgs& a, cudaStream_t stream);
+// head_dim 512 (32 heads per tile, transposed products); slices merge in a
+// cluster only (at most kAttnMaxClusterSplits), no workspace
+cudaError_t launch_sparse_sink_attn_d512(const AttnArgs& a, cudaStream_t stream);
+int d512_default_splits(int32_t n_queries, int32_t num_heads);
 
 }  // namespace spa

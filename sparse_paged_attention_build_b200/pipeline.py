@@ -112,6 +112,8 @@ class DeviceBatch:
         library's automatic choice)."""
         if self.num_splits > 0:
             return self.num_splits
+        if self.w.d == 512:
+            return int(lib.spa_sparse_sink_attn_choose_splits_d512(self.w.N, self.w.H))
         return int(lib.spa_sparse_sink_attn_choose_splits(self.w.N, self.w.H, 0))
 
     def kernels_per_step(self) -> int:

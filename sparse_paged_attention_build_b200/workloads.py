@@ -21,6 +21,15 @@ The five workloads:
         32768, H=128, d=128, top-k 512 + W=128, FP8 compressed cache with
         per-64 FP32 scales, page size 128.
 
+Two more at the DSV4-Flash attention shape (32 query heads, head width
+512, the BF16 rows that the packed 584-byte cache decodes to):
+
+``f1``  ratio-4 prefill: 1 request x 1024 tokens, H=32, d=512, W=128,
+        top-k 512, page size 64.
+``f2``  ratio-4 decode: 64 requests x 1 query, context 8192 (the input
+        length of the pages' serving timeline), H=32, d=512, top-k 512 +
+        W=128, page size 64.
+
 ``shrink`` keeps every per-token shape (H, d, W, K, page size) and reduces
 only the number of requests and tokens, for parity cases the oracle finishes
 in seconds.
@@ -216,6 +225,8 @@ DESCRIPTIONS = {
     "c3": "ratio-4 CSA prefill: B=2 x 8192 tokens, H=128, d=128, W=128, top-k 512, page 64",
     "c4": "ratio-128 HCA decode: 64 requests, context U[16384, 65536], H=128, d=128, W=128, page 64",
     "c5": "mixed FP8/BF16 ratio-4 decode: 128 requests, context 32768, H=128, d=128, top-k 512, W=128, page 128",
+    "f1": "DSV4-Flash-shaped ratio-4 prefill: B=1 x 1024 tokens, H=32, d=512, W=128, top-k 512, page 64",
+    "f2": "DSV4-Flash-shaped ratio-4 decode: 64 requests, context 8192, H=32, d=512, top-k 512, W=128, page 64",
 }
 
 
@@ -224,7 +235,7 @@ def make(name: str, shrink: int = 1, seed_offset: int = 0, fp8_format: int = 0) 
     the tokens per request (prefill) or the context lengths (decode).
     ``fp8_format`` picks the encoding of the mixed cache (c5): 0 = OCP
     E4M3, 1 = E4M3 FNUZ."""
-    idx = int(name[1:])
+    idx = int(name[1:]) + (100 if name[0] == "f" else 0)
     seed = BASE_SEED + idx + 1000 * seed_offset
     if name == "c1":
         return _prefill(name, seed, 2, max(16, 256 // shrink), 8, 64, 64, 4, 16, 16, 2, max(4, 64 // shrink))
@@ -243,6 +254,13 @@ def make(name: str, shrink: int = 1, seed_offset: int = 0, fp8_format: int = 0) 
         B = max(1, 128 // shrink)
         L = max(1024, 32768 // shrink)
         return _decode(name, seed, B, np.full(B, L), 128, 128, 128, 4, 512, 128, fp8=True, fmt=fp8_format)
+    if name == "f1":
+        S = max(128, 1024 // shrink)
+        return _prefill(name, seed, 1, S, 32, 512, 128, 4, 512, 64, 2, S // 4)
+    if name == "f2":
+        B = max(1, 64 // shrink)
+        L = max(1024, 8192 // shrink)
+        return _decode(name, seed, B, np.full(B, L), 32, 512, 128, 4, 512, 64, fp8=False)
     raise KeyError(name)
 
 

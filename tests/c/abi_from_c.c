@@ -27,7 +27,7 @@ int main(void) {
     bad += check(spa_sparse_sink_attn_fwd(q, 16384, 128, 4, 128, 96, NULL, NULL, 1, 64, NULL, 1, NULL, NULL, 0, 64,
                                           NULL, 0, NULL, 1, NULL, NULL, NULL, 0.088f, NULL, NULL, 1, NULL, 0, NULL,
                                           NULL),
-                 SPA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+                 SPA_ERR_UNSUPPORTED, "head_dim must be 64, 128 or 512");
     bad += check(spa_sparse_sink_attn_bwd(q, 16384, 128, 4, 128, 128, NULL, NULL, 1, 64, NULL, 1, NULL, NULL, 0, 64,
                                           NULL, 0, NULL, 1, NULL, NULL, NULL, 0.088f, NULL, NULL, NULL, NULL, NULL,
                                           NULL, NULL, NULL, NULL, 1, NULL, NULL),

@@ -130,8 +130,10 @@ def attn_call(L, **kw):
     (dict(n=-1), 1, "n_queries < 0"),
     (dict(H=0), 1, "num_heads < 1"),
     (dict(B=0), 1, "n_requests < 1"),
-    (dict(d=96), 2, "head_dim must be 64 or 128"),
+    (dict(d=96), 2, "head_dim must be 64, 128 or 512"),
     (dict(H=192), 2, "multiple of 128"),
+    (dict(d=512, H=48), 2, "head_dim 512: num_heads above 32"),
+    (dict(d=512, H=32, splits=9), 2, "head_dim 512: num_splits at most"),
     (dict(rp=-1), 1, "raw pool sizes"),
     (dict(rps=0), 1, "raw_page_size < 1"),
     (dict(rps=48), 2, "raw_page_size must be a power of two"),
@@ -238,7 +240,8 @@ def bwd_call(L, **kw):
 
 @pytest.mark.parametrize("kw,status,clause", [
     (dict(n=-1), 1, "n_queries < 0"),
-    (dict(d=96), 2, "head_dim must be 64 or 128"),
+    (dict(d=96), 2, "head_dim must be 64, 128 or 512"),
+    (dict(d=512, H=32), 2, "the backward takes head_dim 64 or 128"),
     (dict(rps=48), 2, "raw_page_size must be a power of two"),
     (dict(kc=None), 1, "k_cmp/v_cmp NULL"),
     (dict(splits=17), 1, "num_splits must be"),

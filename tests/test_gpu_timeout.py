@@ -1,0 +1,64 @@
+"""The attention's bounded waits, driven to give up on purpose -- no fault.
+
+Every wait between the warp roles of the attention forward has a time
+limit; when one runs out the kernel sets SPA_DEV_TIMEOUT, the CTA unwinds
+(waiting, with the fixed limit, for its own copies and tensor-core products
+before it frees TMEM) and the call returns. The testing hook sets that limit
+to 0, so the first wait that is not already satisfied gives up: a flag that
+nothing sets in time. The context must stay usable: the next call with the
+default limit is bit-identical to a clean run.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+DEFAULT_LIMIT_NS = 1_000_000_000
+
+
+@pytest.fixture(scope="module")
+def spa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_paged_attention_build_b200 as m
+    m.lib.spa_testing_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    m.lib.spa_testing_set_wait_limit_ns.restype = None
+    return m
+
+
+@pytest.mark.parametrize("splits", [1, 2])
+def test_zero_wait_limit_sets_timeout_and_next_call_is_clean(spa, splits):
+    from sparse_paged_attention_build_b200 import workloads
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    w = workloads.make("c1")
+    b = DeviceBatch(w, num_splits=splits)
+    b.step()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+    ref_out = b.out.view(torch.int16).clone()
+    ref_lse = b.lse.view(torch.int32).clone()
+
+    st = spa.new_status()
+    out = torch.full_like(b.out, float("nan"))
+    lse = torch.full_like(b.lse, float("nan"))
+    spa.lib.spa_testing_set_wait_limit_ns(0)
+    try:
+        spa.sparse_sink_attn_fwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, b.indptr, b.indices, b.sink, w.scale,
+                                 k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp, out=out, lse=lse,
+                                 num_splits=splits, workspace=b.attn_ws, dev_status=st)
+        torch.cuda.synchronize()    # the call returned and the context is usable
+    finally:
+        spa.lib.spa_testing_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+    assert spa.read_status(st) & spa.DEV_TIMEOUT
+
+    b.status.zero_()
+    b.out.zero_()
+    b.lse.zero_()
+    b.attend()
+    torch.cuda.synchronize()
+    assert b.status_word() == 0
+    assert torch.equal(b.out.view(torch.int16), ref_out)
+    assert torch.equal(b.lse.view(torch.int32), ref_lse)
