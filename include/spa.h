@@ -383,15 +383,17 @@ int spa_unpack_d512_pages(const uint8_t* src, int64_t num_pages, int32_t page_si
  * a limit (1 s), sets SPA_DEV_TIMEOUT and lets the kernel unwind, so that a
  * stuck pipeline ends the call instead of hanging the GPU. The waits that
  * keep a CTA's memory alive until its own copies and tensor-core products
- * have finished always keep the 1 s limit. spa_testing_set_wait_limit_ns
- * changes the limit of the former for the attention forward launches that
- * follow (process-wide, on every device); 0 makes them give up almost at
- * once, which is how the tests reach the timeout path without a fault.
- * Pass SPA_DEFAULT_WAIT_LIMIT_NS to restore the default. Outputs of a call
- * that timed out are poisoned.
+ * have finished always keep the 1 s limit.
+ *
+ * spa_testing_stall_attention(limit_ns) with limit_ns > 0 makes the forward
+ * launches that follow (both head-width kernels; process-wide, every
+ * device) wait, in every CTA, on a barrier that nothing ever arrives at,
+ * with limit_ns as the limit of every wait between the roles: each CTA
+ * times out there and unwinds, and the call returns with SPA_DEV_TIMEOUT
+ * set and poisoned outputs. That is how the tests reach the timeout path
+ * without a fault. limit_ns = 0 restores normal launches.
  * ---------------------------------------------------------------------- */
-#define SPA_DEFAULT_WAIT_LIMIT_NS 1000000000ull
-void spa_testing_set_wait_limit_ns(uint64_t ns);
+void spa_testing_stall_attention(uint64_t limit_ns);
 
 #ifdef __cplusplus
 }

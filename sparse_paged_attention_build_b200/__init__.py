@@ -61,8 +61,8 @@ def _load():
     L.spa_sparse_sink_attn_choose_splits.restype = ctypes.c_int
     L.spa_sparse_sink_attn_choose_splits_d512.argtypes = [i32, i32]
     L.spa_sparse_sink_attn_choose_splits_d512.restype = ctypes.c_int
-    L.spa_testing_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
-    L.spa_testing_set_wait_limit_ns.restype = None
+    L.spa_testing_stall_attention.argtypes = [ctypes.c_uint64]
+    L.spa_testing_stall_attention.restype = None
     L.spa_sparse_sink_attn_fwd.argtypes = [
         P, i64, i64, i32, i32, i32,
         P, P, i64, i32, P, i32,

@@ -64,9 +64,15 @@ int device_sm_count() {
   return n;
 }
 
-std::atomic<uint64_t> g_attn_wait_ns{1000ull * 1000ull * 1000ull};
-uint64_t attn_wait_limit_ns() { return g_attn_wait_ns.load(std::memory_order_relaxed); }
-void set_attn_wait_limit_ns(uint64_t ns) { g_attn_wait_ns.store(ns, std::memory_order_relaxed); }
+// 0: normal launches; otherwise every CTA stalls on a barrier nothing
+// arrives at, and every wait between the roles uses this limit (ns)
+std::atomic<uint64_t> g_attn_stall_ns{0};
+uint64_t attn_wait_limit_ns() {
+  const uint64_t v = g_attn_stall_ns.load(std::memory_order_relaxed);
+  return v != 0 ? v : kWaitTimeoutNsHost;
+}
+bool attn_stall() { return g_attn_stall_ns.load(std::memory_order_relaxed) != 0; }
+void set_attn_stall_ns(uint64_t ns) { g_attn_stall_ns.store(ns, std::memory_order_relaxed); }
 
 }  // namespace spa
 
@@ -89,7 +95,7 @@ const char* spa_status_string(int status) {
 
 const char* spa_last_error_detail(void) { return g_detail; }
 
-void spa_testing_set_wait_limit_ns(uint64_t ns) { spa::set_attn_wait_limit_ns(ns); }
+void spa_testing_stall_attention(uint64_t limit_ns) { spa::set_attn_stall_ns(limit_ns); }
 
 // ---------------------------------------------------------------- sets
 int64_t spa_kv_sets_capacity(int32_t n_queries, int32_t window, int32_t ratio, int32_t topk_width,

@@ -119,6 +119,18 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
     if (set_len < 0 || b < 0 || b >= P.n_requests) {
       if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
       set_len = 0;
+    } else {
+      // The page-table rows of this request into L2 while the keys load,
+      // so that the lookup after them (the third dependent load of the
+      // chunk) hits L2: up to 64 lines (8 KB) of each table per lane group.
+      const int32_t* rows[2] = {P.pt_raw + static_cast<int64_t>(b) * P.pt_raw_cols,
+                                P.pt_cmp ? P.pt_cmp + static_cast<int64_t>(b) * P.pt_cmp_cols : nullptr};
+      const int32_t cols[2] = {P.pt_raw_cols, P.pt_cmp ? P.pt_cmp_cols : 0};
+#pragma unroll
+      for (int tb = 0; tb < 2; ++tb) {
+        const int lines = min(64, (cols[tb] + 31) / 32);
+        for (int ln = lane; ln < lines; ln += 32) prefetch_l2(rows[tb] + 32 * ln);
+      }
     }
     const int tiles_total = ceil_tiles(set_len);
     const int tile_lo = static_cast<int>((static_cast<int64_t>(tiles_total) * split) / S);

@@ -101,6 +101,7 @@ struct Params {
   int32_t num_splits;   // slices per query; > 1: one cluster of that many CTAs per query
   uint32_t* dev_status;
   uint64_t wait_ns;
+  int32_t stall;        // testing: every CTA waits on a barrier nothing arrives at
 };
 
 struct Layout {
@@ -119,7 +120,7 @@ struct Layout {
   static constexpr int kBarOff = kMaxOff + 4 * kHT * 4;
   static constexpr int kNumBars = 2 + 2 + 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1 + 1 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 32 + 1024;
+  static constexpr int kBytes = kMiscOff + 48 + 1024;   // misc: TMEM slot, abort, have_o, votes, stall barrier at +32
   static_assert(kBytes <= 227 * 1024, "shared memory");
   static_assert(kKStages * kChunkBytes == kHT * kD * 4, "the merge reuses the K ring for [32][512] FP32");
 };
@@ -151,6 +152,18 @@ struct SoftSync {
   }
 };
 
+// Bytes of the merge's receive slots [S][32 heads][widest column range]
+// FP32, the largest over 2..8 slices.
+constexpr int merge_rx_bytes_max() {
+  int m = 0;
+  for (int S = 2; S <= kAttnMaxClusterSplits; ++S) {
+    const int per = (kD / S) & ~3;
+    const int b = S * kHT * (kD - (S - 1) * per) * 4;
+    m = b > m ? b : m;
+  }
+  return m;
+}
+
 // End of every role (inlined into each): the cluster merge of the slices
 // by the softmax threads, the cluster barriers for every warp, TMEM freed
 // by the MMA warp last.
@@ -165,13 +178,23 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
   if (S > 1) {
     // Exact merge of the S slices of query i (page "[WS2] Add CP-aware
     // Attention contract and dispatch metadata", Summary: the deterministic
-    // (out, lse) merge): w_s = 2^(m_s - M) / L per head; each CTA scales its
-    // own O^T by its weight into shared memory as [head][d] FP32, then CTA
-    // `rank` sums its share of d over the cluster and writes BF16 O.
+    // (out, lse) merge): w_s = 2^(m_s - M) / L per head. CTA r owns columns
+    // [r*per, ...) of d. Each CTA scales its O^T by its weights into its own
+    // shared memory as [head][d] FP32, then stores every 16-byte piece
+    // straight into its owner's receive slots (posted stores, slot = the
+    // sender's rank); after the second cluster barrier each owner sums its
+    // slots locally and writes BF16 O. Nothing is read or written remotely
+    // after that barrier, so no third one is needed.
     const int rank = static_cast<int>(cluster_ctarank());
     const int i = static_cast<int>(blockIdx.x / S);
+    const int per = (kD / S) & ~3;   // 16-byte pieces; the last rank takes the rest
+    const int own_e0 = rank * per, own_e1 = rank == S - 1 ? kD : own_e0 + per;
+    const int span = kD - (S - 1) * per;   // the widest range (the last rank's)
     float* head_w = reinterpret_cast<float*>(smem + L::kHeadOff + 2 * kHT * 4);
     const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 8) != 0;
+    // receive slots [S][32 heads][span] FP32 after the K ring (idle by now)
+    static_assert(L::kPOff + 2 * L::kPBytes - L::kVOff >= merge_rx_bytes_max(), "receive slots fit the idle V ring and P");
+    const uint32_t rx_addr = sbase + L::kVOff;
     __syncwarp();
     cluster_sync_all();   // every slice's (m, l) is in place
     if (soft) {
@@ -216,31 +239,35 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
 #pragma unroll
         for (int h = 0; h < kHT; ++h) wo[h * kD + 128 * b + tid] = __uint_as_float(o[h]) * w[h];
       }
+      (*ss)();   // this CTA's scaled rows are in place
+      for (int item = tid; item < kHT * (kD / 4); item += kSoftThreads) {
+        const int h = item / (kD / 4), e = 4 * (item % (kD / 4));
+        const int owner = min(e / per, S - 1);
+        const int e_rel = e - owner * per;
+        const float4 v = *reinterpret_cast<const float4*>(wo + h * kD + e);
+        st_dsmem_f4(dsmem_addr(rx_addr + static_cast<uint32_t>(((rank * kHT + h) * span + e_rel) * 4), owner), v);
+      }
     }
     __syncwarp();
-    cluster_sync_all();   // every slice's weighted O is in place
+    cluster_sync_all();   // every slice's pieces have arrived
     if (soft) {
-      const int per = (kD / S) & ~3;   // 16-byte pieces; the last rank takes the rest
-      const int e0 = rank * per, e1 = rank == S - 1 ? kD : e0 + per;
-      const int n4 = (e1 - e0) / 4;
-      const uint32_t wo_addr = sbase + L::kKOff;
+      const int n4 = (own_e1 - own_e0) / 4;
+      const float* rx = reinterpret_cast<const float*>(smem + L::kVOff);
       for (int item = tid; item < kHT * n4; item += kSoftThreads) {
-        const int h = item / n4, e = e0 + 4 * (item % n4);
+        const int h = item / n4, e_rel = 4 * (item % n4);
         if (h >= heads_here) continue;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < S; ++s) {
-          const float4 v = ld_dsmem_f4(dsmem_addr(wo_addr + static_cast<uint32_t>((h * kD + e) * 4), s));
+          const float4 v = *reinterpret_cast<const float4*>(rx + (s * kHT + h) * span + e_rel);
           acc.x += v.x;
           acc.y += v.y;
           acc.z += v.z;
           acc.w += v.w;
         }
-        *reinterpret_cast<uint2*>(P.out + (static_cast<int64_t>(i) * P.num_heads + head0 + h) * kD + e) =
+        *reinterpret_cast<uint2*>(P.out + (static_cast<int64_t>(i) * P.num_heads + head0 + h) * kD + own_e0 + e_rel) =
             make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
       }
     }
-    __syncwarp();
-    cluster_sync_all();   // no slice leaves while its memory is read
   }
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
@@ -311,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
     *abort_flag = 0;
     *reinterpret_cast<int*>(smem + L::kMiscOff + 8) = 0;
     for (int k = 0; k < 3; ++k) reinterpret_cast<uint32_t*>(smem + L::kMiscOff + 16)[k] = 0u;
+    mbar_init(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 32), 1);   // never arrived at
     mbar_init_fence();
   }
   if (tid < kHT) {
@@ -343,19 +371,31 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
     warpgroup_reg_dealloc<kRegControl>();
     if (warp == kResolverWarp) {
       // ================================================= resolver
+      // testing stall: a wait that only its limit ends, then the CTA unwinds
+      if (P.stall) mbar_wait(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 32), 0, abort_flag, P.dev_status, P.wait_ns);
       resolver_loop(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane);
       cta_finish(P, false, smem, sbase, tmem, tid, warp, head0, heads_here, &ss);
     } else if (warp == kQWarp) {
       // ================================================= Q loader
-      int c = 0, qc = 0;
-      bool final_seen = false;
+      // The CTA's first unit is unit blockIdx.x (units are strided over the
+      // CTAs): its Q is loaded at once, while the resolver fetches its keys.
+      int c = 0, qc = 1;
+      bool final_seen = false, first_issued = true;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kNChunks);
+        for (int cb = 0; cb < kNChunks; ++cb)
+          tma_load_3d(sbase + L::kQOff + cb * (kHT * 128), &P.tm_q, B.q_full, cb * 64, head0,
+                      static_cast<int32_t>(blockIdx.x / S));
+      }
       while (!final_seen) {
         const int slot = c & 1;
         if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
         const ChunkDesc d = desc[slot];
         final_seen = (d.flags & kFlagFinal) != 0;
         bool ok = true;
-        if (d.flags & kFlagFirst) {
+        if ((d.flags & kFlagFirst) && first_issued) {
+          first_issued = false;   // the first unit's Q is on its way
+        } else if (d.flags & kFlagFirst) {
           // the previous unit's last S^T product has read Q
           ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns);
           if (ok && lane == 0) {
@@ -815,6 +855,7 @@ cudaError_t launch_sparse_sink_attn_d512(const AttnArgs& a, cudaStream_t stream)
   P.num_splits = a.num_splits;
   P.dev_status = a.dev_status;
   P.wait_ns = attn_wait_limit_ns();
+  P.stall = attn_stall() ? 1 : 0;
   static bool configured = false;
   if (!configured) {
     cudaError_t err = cudaFuncSetAttribute(sparse_sink_attn_d512_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

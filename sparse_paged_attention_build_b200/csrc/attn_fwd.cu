@@ -12,9 +12,11 @@
 // Work unit = (query token i, slice s of its key set, 128-head tile). All
 // heads of the unit share every K/V row, so the unit is a dense MQA problem
 // with M = 128 heads:
-//   S  = Q[128 x d] . K_tile[64 x d]^T      tcgen05.mma, Q in TMEM, K in SMEM
+//   S  = Q[128 x d] . K_half[32 x d]^T      tcgen05.mma, Q in TMEM, K in SMEM
 //   P  = exp2(S*scale*log2e - m)  (BF16)    softmax warps, TMEM -> regs -> TMEM
-//   O += P[128 x 64] . V_tile[64 x d]        tcgen05.mma, P in TMEM, V in SMEM
+//   O += P[128 x 32] . V_half[32 x d]        tcgen05.mma, P in TMEM, V in SMEM
+// K and V arrive in tiles of 64 rows; the products and the softmax take each
+// tile in two halves of 32 keys.
 // Both products take their A operand from TMEM: measured on B200, an
 // M = 128, N = 64 product with both operands in shared memory is bound by
 // shared-memory bandwidth at two thirds of the tensor rate, while with A in
@@ -47,10 +49,13 @@
 // The warpgroups then move registers with setmaxnreg: the softmax rows keep
 // 64 scores, 32 packed probabilities and the running statistics in
 // registers, the copy warps need few.
-// TMEM columns: S/P [0,64), Q [64, 64 + d/2) as packed BF16 pairs, O after.
-// S is single-buffered: QK^T of tile g+1 is issued after PV of tile g, and
-// the UMMAs of a CTA run in issue order, so P(g) is read before S(g+1)
-// overwrites it; the other CTA on the SM fills the tensor core meanwhile.
+// TMEM columns: two S/P buffers [0,64) of 32 columns each, Q [64, 64 + d/2)
+// as packed BF16 pairs, O after. S of half tile j+1 is computed while the
+// softmax of half j runs (issue order QK(j+1), then PV(j)); P(j) overwrites
+// the first 16 columns of its buffer and is read by PV(j) before QK(j+2)
+// reuses that buffer, since the UMMAs of a CTA run in issue order. (With one
+// 64-column S buffer the softmax and the product round trip ran in series,
+// about 950 + 1400 cycles per 64 keys for a CTA on B200.)
 // The softmax first takes P with the running max as it stands and only
 // recomputes a tile whose row sum leaves a fixed bound (see kSpecBound);
 // O/l and LSE use the same max, so the result is exact in exact arithmetic.
@@ -81,9 +86,9 @@ constexpr uint32_t kTmemCols = 256;
 // the 4 x 64 the block is launched with (two 512-thread blocks per SM).
 template <bool kFp8>
 struct RegSplit {
-  static constexpr uint32_t kSoftmax = kFp8 ? 120 : 136;
-  static constexpr uint32_t kControl = 56;            // MMA issue, resolvers, Q
-  static constexpr uint32_t kGather = kFp8 ? 40 : 32;  // the FP8 decode holds codes and scales
+  static constexpr uint32_t kSoftmax = kFp8 ? 96 : 112;
+  static constexpr uint32_t kControl = 64;            // MMA issue, resolvers, Q
+  static constexpr uint32_t kGather = kFp8 ? 48 : 40;  // the FP8 decode holds codes and scales
   static_assert(true || kSoftmax + kControl + 2 * kGather <= 4 * 64, "register split exceeds the launch");
 };
 // A tile whose row sum of P, taken with the running max as it stands,
@@ -91,6 +96,12 @@ struct RegSplit {
 // therefore stays below 2^16: harmless in BF16 and in the FP32 sums, whose
 // relative precision does not depend on magnitude.
 constexpr float kSpecBound = 65536.0f;
+// The tensor cores and the softmax work on half tiles of 32 keys with two S
+// buffers in TMEM: S of half j+1 is computed while the softmax of half j
+// runs, and P of half j (BF16, over the first kSub/2 columns of its S
+// buffer) is read by the PV product before S of half j+2 overwrites it (the
+// products of a CTA run in issue order).
+constexpr int kSub = 32;
 // consumers of a chunk descriptor: K and V groups, MMA thread, softmax, Q warp
 constexpr uint32_t kTabConsumers = 2 * kGroupThreads + 1 + kSoftThreads + 32;
 
@@ -142,6 +153,7 @@ struct Params {
   // and shared memory alive until the CTA's own copies and MMAs are done
   // keep the fixed kWaitTimeoutNs
   uint64_t wait_ns;
+  int32_t stall;       // testing: every CTA waits on a barrier nothing arrives at
 };
 
 template <int D>
@@ -158,16 +170,16 @@ struct Layout {
   static constexpr int kMergeOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
   static constexpr int kBarOff = kMergeOff + kAttnMaxSplits * 128 * 4;
   // tab_full[2], tab_empty[2], q_full, q_empty, q_ready, K ring, V ring,
-  // s_full, p_ready, o_done, mma_done, soft_sync[2]
-  static constexpr int kNumBars = 2 + 2 + 3 + 2 * kStagesK + 2 * kStagesV + 1 + 1 + 1 + 1 + 2;
+  // s_full[2], p_ready[2], o_ready, o_done, mma_done, soft_sync[2]
+  static constexpr int kNumBars = 2 + 2 + 3 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 1 + 1 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kUsed = kMiscOff + 16;
+  static constexpr int kUsed = kMiscOff + 32;   // + the testing stall barrier at kMiscOff + 16
   // + alignment slack; at least 80 KB so that no more than two CTAs share an
   // SM (TMEM holds two 256-column allocations)
   static constexpr int kBytes = (kUsed + 1024) < 80 * 1024 ? 80 * 1024 : (kUsed + 1024);
-  static constexpr uint32_t kSCol = 0;
-  static constexpr uint32_t kQCol = kT;
-  static constexpr uint32_t kOCol = kT + D / 2;
+  static constexpr uint32_t kSCol = 0;                      // S buffers [2][kSub]
+  static constexpr uint32_t kQCol = 2 * kSub;
+  static constexpr uint32_t kOCol = 2 * kSub + D / 2;
   static_assert(kOCol + D <= kTmemCols, "TMEM budget");
   static_assert((kBytes + 1024) * 2 <= 228 * 1024, "two CTAs per SM");
   static_assert(kMergeOff % 16 == 0, "staging alignment");
@@ -183,8 +195,10 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;     // [kStagesV]
   uint64_t* v_empty;
-  uint64_t* s_full;     // S of the current tile (also: every earlier UMMA done)
-  uint64_t* p_ready;    // P of the current tile in TMEM
+  uint64_t* s_full;     // [2]: S of a half tile in its buffer
+  uint64_t* p_ready;    // [2]: P of a half tile in its S buffer (one barrier per buffer: the
+                        // softmax may finish two half tiles before the UMMA issuer waits)
+  uint64_t* o_ready;    // one phase per half tile: its PV product has completed
   uint64_t* o_done;     // last PV of a unit complete
   uint64_t* mma_done;
   // [2]: barrier of the softmax threads, the two used in turn. An mbarrier
@@ -209,21 +223,32 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
     // Exact merge of the S slices of query i, CTA `rank` holding slice
     // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
     // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
-    // Summary: the deterministic (out, lse) merge). Each CTA scales its own
-    // O rows by its weight into shared memory (the K/V rings are idle now);
-    // then CTA `rank` sums its share of the rows over the cluster's shared
-    // memory and writes them. Every thread of every CTA reaches the three
-    // cluster barriers: every earlier wait in the kernel is bounded.
+    // Summary: the deterministic (out, lse) merge). CTA r owns rows
+    // [r*per, (r+1)*per) of the output. After the first cluster barrier
+    // every CTA reads all slices' (m, l) of its rows (one round trip of
+    // distributed shared memory), scales its O rows by its weight and
+    // stores each row straight into its owner's idle K/V ring (posted
+    // stores, slot = the sender's rank); after the second barrier each owner
+    // sums its slots locally and writes BF16 O. No shared memory is read or
+    // written remotely after the second barrier, so no third one is needed.
+    // Every thread of every CTA reaches both barriers: every earlier wait in
+    // the kernel is bounded.
     const int rank = static_cast<int>(cluster_ctarank());
     const int i = static_cast<int>(blockIdx.x / S);
     const uint32_t ml_addr = sbase + L::kMergeOff;
-    const uint32_t wo_addr = sbase + L::kKOff;               // [128][D] FP32, 16-byte chunks swizzled by row
+    const uint32_t rx_addr = sbase + L::kKOff;               // [S][per][D] FP32, 16-byte chunks swizzled by row
     constexpr int kChunks = D / 4;                           // 16-byte chunks per row
+    const int per = (128 + S - 1) / S;
+    // the slots (S * per <= 128 + S - 1 rows of D FP32) fill the K/V rings
+    // and may run on into the chunk tables, all idle by now
+    static_assert(L::kTabOff - L::kKOff + 2 * kChunkKeys * 4 >= (128 + kAttnMaxClusterSplits - 1) * D * 4,
+                  "receive slots fit the idle rings and tables");
+    static_assert(L::kTabOff == L::kVOff + kStagesV * L::kTileBytes && L::kVOff == L::kKOff + kStagesK * L::kTileBytes,
+                  "rings and tables are contiguous");
     __syncwarp();
-    cluster_sync_all();                                      // every slice's (m, l) is in place
+    cluster_sync_all();                                      // every slice's (m, l) is in place; rings idle
     if (soft) {
       const int row = tid;
-      // all slices' (m, l) of this row, the loads in flight together
       float2 ml[kAttnMaxClusterSplits];
 #pragma unroll
       for (int s = 0; s < kAttnMaxClusterSplits; ++s)
@@ -245,7 +270,8 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
             Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
       const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
       const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
-      float* wo = reinterpret_cast<float*>(smem + L::kKOff);
+      const int owner = row / per, rr = row - owner * per;
+      const uint32_t dst = dsmem_addr(rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 4), owner);
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -259,53 +285,35 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const int chunk = (c0 >> 2) + v;
-          const int phys = chunk ^ (row & (kChunks - 1));
-          *reinterpret_cast<float4*>(wo + row * D + phys * 4) =
-              make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
-                          __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own);
+          const int phys = chunk ^ (rr & (kChunks - 1));
+          st_dsmem_f4(dst + phys * 16,
+                      make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
+                                  __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own));
         }
       }
     }
     __syncwarp();
-    cluster_sync_all();                                      // every slice's weighted rows are in place
+    cluster_sync_all();                                      // every slice's weighted rows have arrived
     if (soft) {
-      const int per = (heads_here + S - 1) / S;
       const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
+      const float* rx = reinterpret_cast<const float*>(smem + L::kKOff);
       uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
-      // two 16-byte pieces per thread per pass, every slice's copy of both
-      // loaded before any is added
       const int n_items = (r1 - r0) * kChunks;
-      for (int base = tid; base < n_items; base += 2 * kSoftThreads) {
-        float4 v[2][kAttnMaxClusterSplits];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int idx = base + k * kSoftThreads;
-          const int r = r0 + idx / kChunks, c = idx % kChunks;
-          const uint32_t off = wo_addr + static_cast<uint32_t>((r * D + (c ^ (r & (kChunks - 1))) * 4) * 4);
-#pragma unroll
-          for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-            v[k][s] = (idx < n_items && s < S) ? ld_dsmem_f4(dsmem_addr(off, s)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int idx = tid; idx < n_items; idx += kSoftThreads) {
+        const int rr = idx / kChunks, c = idx % kChunks;
+        const int phys = c ^ (rr & (kChunks - 1));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+          const float4 v = *reinterpret_cast<const float4*>(rx + ((s * per + rr) * D) + phys * 4);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
         }
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int idx = base + k * kSoftThreads;
-          if (idx >= n_items) continue;
-          const int r = r0 + idx / kChunks, c = idx % kChunks;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
-            acc.x += v[k][s].x;
-            acc.y += v[k][s].y;
-            acc.z += v[k][s].z;
-            acc.w += v[k][s].w;
-          }
-          *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r) * D + 4 * c) =
-              make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-        }
+        *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r0 + rr) * D + 4 * c) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
       }
     }
-    __syncwarp();
-    cluster_sync_all();                                      // no slice leaves while its memory is read
   }
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
@@ -330,8 +338,9 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   B.v_full = B.k_empty + kStagesK;
   B.v_empty = B.v_full + kStagesV;
   B.s_full = B.v_empty + kStagesV;
-  B.p_ready = B.s_full + 1;
-  B.o_done = B.p_ready + 1;
+  B.p_ready = B.s_full + 2;
+  B.o_ready = B.p_ready + 2;
+  B.o_done = B.o_ready + 1;
   B.mma_done = B.o_done + 1;
   B.soft_sync = B.mma_done + 1;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
@@ -366,10 +375,14 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       mbar_init(B.v_empty + s, 1);
     }
     mbar_init(B.s_full, 1);
+    mbar_init(B.s_full + 1, 1);
     mbar_init(B.p_ready, kSoftThreads);
+    mbar_init(B.p_ready + 1, kSoftThreads);
+    mbar_init(B.o_ready, 1);
     mbar_init(B.o_done, 1);
     mbar_init(B.mma_done, 1);
     *abort_flag = 0;
+    mbar_init(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 16), 1);   // never arrived at
     mbar_init_fence();
   }
   if (warp == kMmaWarp) {
@@ -387,6 +400,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     warpgroup_reg_dealloc<R::kControl>();
     if (warp == kResolverWarp0 || warp == kResolverWarp1) {
       // ================================================= resolver
+      // testing stall: a wait that only its limit ends, then the CTA unwinds
+      if (P.stall) mbar_wait(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 16), 0, abort_flag, P.dev_status, P.wait_ns);
       resolver_loop<2>(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane, false,
                        warp == kResolverWarp0 ? 0 : 1);
       cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
@@ -394,17 +409,29 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       // ================================================= Q loader
       // Every unit's Q, empty units included, so that the Q phases of all
       // roles stay in step; the landing area is free once the previous Q
-      // has moved on to TMEM.
+      // has moved on to TMEM. The CTA's first unit is unit blockIdx.x (units
+      // are strided over the CTAs), so its Q is loaded at once, while the
+      // resolver is still fetching its keys.
       constexpr int kHalves = D / 64;
       int c = 0, qc = 0;
-      bool final_seen = false;
+      bool final_seen = false, first_issued = false;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
+        for (int hb = 0; hb < kHalves; ++hb)
+          tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0,
+                      static_cast<int32_t>(blockIdx.x / S));
+      }
+      first_issued = true;
+      qc = 1;
       while (!final_seen) {
         const int slot = c & 1;
         if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
         const ChunkDesc d = desc[slot];
         final_seen = (d.flags & kFlagFinal) != 0;
         bool ok = true;
-        if (d.flags & kFlagFirst) {
+        if ((d.flags & kFlagFirst) && first_issued) {
+          first_issued = false;   // the first unit's Q is on its way
+        } else if (d.flags & kFlagFirst) {
           ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns);
           if (ok && lane == 0) {
             mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
@@ -424,15 +451,39 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
     } else if (warp == kMmaWarp) {
       // ================================================= UMMA issuer
-      // Per tile: S = Q K^T (A = Q from TMEM), then, once P is in TMEM,
-      // O += P V (A = P from TMEM). s_full is committed after the QK^T of a
-      // tile, so its arrival also means every earlier UMMA (the previous PV)
-      // has completed.
+      // Half tile x: S[x%2] = Q K_x^T (A = Q from TMEM); once its P is in
+      // TMEM, O += P_x V_x (A = P from TMEM). The issue order is QK(x+1)
+      // before PV(x), so the softmax of half x overlaps the product of the
+      // next S; QK(x+2) comes after PV(x), which read P(x) from the same
+      // buffer.
       if (lane == 0) {
-        constexpr uint32_t idesc_s = idesc_bf16_f32(128, kT, 0);
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, kSub, 0);
         constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
-        int c = 0, g = 0, u = 0;
+        int c = 0, g = 0, u = 0, x = 0;
         bool ok = true, final_seen = false;
+        // the half tile whose PV is still to be issued
+        int pend = -1, pend_v = 0, pend_hf = 0;
+        bool pend_first = false, pend_last_of_tile = false, pend_last_of_unit = false;
+        auto issue_pv = [&]() -> bool {
+          if (!mbar_wait(B.p_ready + (pend & 1), (pend >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) return false;
+          const int st = pend_v % kStagesV;
+          if (pend_hf == 0 &&
+              !mbar_wait(B.v_full + st, (pend_v / kStagesV) & 1, abort_flag, P.dev_status, P.wait_ns))
+            return false;
+          tc_fence_after_sync();
+          const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes + pend_hf * (kSub * 128);
+          const uint32_t p_col = tmem + L::kSCol + (pend & 1) * kSub;
+#pragma unroll
+          for (int k = 0; k < kSub / 16; ++k) {
+            const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
+            umma_ts(tmem + L::kOCol, p_col + k * 8, bdesc, idesc_o, (!pend_first || k > 0) ? 1u : 0u);
+          }
+          tc_commit(B.o_ready);
+          if (pend_last_of_tile) tc_commit(B.v_empty + st);
+          if (pend_last_of_unit) tc_commit(B.o_done);
+          pend = -1;
+          return true;
+        };
         while (ok && !final_seen) {
           const int slot = c & 1;
           if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
@@ -446,32 +497,33 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
             tc_fence_after_sync();
           }
           const int ntiles = ceil_tiles(d.nkeys);
-          for (int t = 0; t < ntiles; ++t, ++g) {
-            const int stage = g % kStagesK, st = g % kStagesV;
+          for (int t = 0; ok && t < ntiles; ++t, ++g) {
+            const int stage = g % kStagesK;
             if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
             tc_fence_after_sync();
             const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
-  #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + (k & 3) * 32, 16, 1024);
-              umma_ts(tmem + L::kSCol, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
+            const int nv = min(kT, d.nkeys - t * kT);
+            const int nsub = (nv + kSub - 1) / kSub;
+            for (int hf = 0; hf < nsub; ++hf, ++x) {
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k) {
+                const uint64_t bdesc =
+                    smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + hf * (kSub * 128) + (k & 3) * 32, 16, 1024);
+                umma_ts(tmem + L::kSCol + (x & 1) * kSub, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
+              }
+              if (hf == nsub - 1) tc_commit(B.k_empty + stage);
+              tc_commit(B.s_full + (x & 1));
+              if (pend >= 0 && !issue_pv()) { ok = false; break; }
+              pend = x;
+              pend_v = g;
+              pend_hf = hf;
+              pend_first = (d.flags & kFlagFirst) && t == 0 && hf == 0;
+              pend_last_of_tile = hf == nsub - 1;
+              pend_last_of_unit = (d.flags & kFlagLast) && t == ntiles - 1 && hf == nsub - 1;
             }
-            tc_commit(B.k_empty + stage);
-            tc_commit(B.s_full);
-            if (!mbar_wait(B.p_ready, g & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
-            if (!mbar_wait(B.v_full + st, (g / kStagesV) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
-            tc_fence_after_sync();
-            const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
-            const bool first = (d.flags & kFlagFirst) && t == 0;
-  #pragma unroll
-            for (int k = 0; k < kT / 16; ++k) {
-              const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
-              umma_ts(tmem + L::kOCol, tmem + L::kSCol + k * 8, bdesc, idesc_o, (!first || k > 0) ? 1u : 0u);
-            }
-            tc_commit(B.v_empty + st);
-            if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.o_done);
           }
         }
+        if (ok && pend >= 0) issue_pv();
         // every UMMA has completed before TMEM is released
         tc_commit(B.mma_done);
         mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
@@ -659,11 +711,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       piece = lane & 3;
       return reinterpret_cast<const uint4*>(stage + r * 64)[piece ^ ((r >> 1) & 3)];
     };
-    int c = 0, g = 0, n_o = 0;
+    int c = 0, x = 0, n_o = 0;
     bool ok = copy_q(), final_seen = false;
     float m = -INFINITY, l = 0.f;
-    int unit_tiles = 0;
-    uint32_t s0[32], s1[32];
+    int unit_subs = 0;
+    uint32_t s0[32];
     while (ok && !final_seen) {
       const int slot = c & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns))) {
@@ -675,103 +727,106 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       ++c;
       final_seen = (d.flags & kFlagFinal) != 0;
       if (d.flags & kFlagFirst) {
-        unit_tiles = 0;
+        unit_subs = 0;
         // the sink logit seeds the max of every slice (any reference point
         // is exact; this one is usually within the bound of the scores) but
         // joins the denominator only once, in slice 0
         m = sink2;
         l = (d.split == 0 && sink2 > -INFINITY) ? 1.f : 0.f;
       }
+      // the chunk's keys in half tiles of kSub, as the UMMA issuer cuts them
       const int ntiles = ceil_tiles(d.nkeys);
-      for (int t = 0; t < ntiles; ++t, ++g, ++unit_tiles) {
-        // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
-        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full, g & 1, abort_flag, P.dev_status, P.wait_ns))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const int nv = min(kT, d.nkeys - t * kT);
-        // Speculative pass: P with the running max as it stands. Only when
-        // some row's tile sum leaves the bound (NaN and +inf, from a max
-        // still at -inf, included) is the exact tile max taken and P
-        // recomputed, so the max reduction stays off the common path. S is
-        // still intact in TMEM for that second pass.
-        auto load_s = [&]() {
-          tmem_ld32(lane_addr + L::kSCol, s0);
-          tmem_ld32(lane_addr + L::kSCol + 32, s1);
-          tmem_ld_wait(s0);
-          tmem_ld_wait(s1);
-          if (nv < kT) {   // columns past the set: -inf, so they add nothing
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int nv_tile = min(kT, d.nkeys - t * kT);
+        const int nsub = (nv_tile + kSub - 1) / kSub;
+        for (int hf = 0; hf < nsub; ++hf, ++x, ++unit_subs) {
+          // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(B.s_full + (x & 1), (x >> 1) & 1, abort_flag, P.dev_status, P.wait_ns))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const int nv = min(kSub, nv_tile - hf * kSub);
+          const uint32_t s_col = lane_addr + L::kSCol + (x & 1) * kSub;
+          // Speculative pass: P with the running max as it stands. Only when
+          // some row's sum leaves the bound (NaN and +inf, from a max still
+          // at -inf, included) is the exact max taken and P recomputed, so
+          // the max reduction stays off the common path. S is still intact
+          // in TMEM for that second pass.
+          auto load_s = [&]() {
+            tmem_ld32(s_col, s0);
+            tmem_ld_wait(s0);
+            if (nv < kSub) {   // columns past the set: -inf, so they add nothing
 #pragma unroll
-            for (int cc = 0; cc < 32; ++cc) {
-              if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
-              if (cc + 32 >= nv) s1[cc] = __float_as_uint(-INFINITY);
+              for (int cc = 0; cc < 32; ++cc)
+                if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
             }
-          }
-        };
-        uint32_t pk[32];
-        auto exp_pass = [&]() -> float {
-          const float neg_m = -m;
-          float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+          };
+          uint32_t pk[16];
+          auto exp_pass = [&]() -> float {
+            const float neg_m = -m;
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
-            const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
-            const float p2 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc]), P.scale_log2, neg_m));
-            const float p3 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc + 1]), P.scale_log2, neg_m));
-            sum4[cc & 3] += (p0 + p1) + (p2 + p3);
-            pk[cc] = pack_bf16x2(p0, p1);
-            pk[cc + 16] = pack_bf16x2(p2, p3);
-          }
-          return (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-        };
-        load_s();
-        float lsum = exp_pass();
-        const bool flag = row_ok && !(lsum <= kSpecBound);
-        if (__any_sync(0xffffffffu, flag)) {
+            for (int cc = 0; cc < 16; ++cc) {
+              const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
+              const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
+              sum4[cc & 3] += p0 + p1;
+              pk[cc] = pack_bf16x2(p0, p1);
+            }
+            return (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+          };
           load_s();
-          // row max: eight independent chains of 3-input max and a tree
-          float mx8[8];
+          float lsum = exp_pass();
+          const bool flag = row_ok && !(lsum <= kSpecBound);
+          if (__any_sync(0xffffffffu, flag)) {
+            load_s();
+            // row max: eight independent chains of 3-input max and a tree
+            float mx8[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mx8[k] = fmax3(__uint_as_float(s0[k]), __uint_as_float(s1[k]), __uint_as_float(s0[k + 8]));
+            for (int k = 0; k < 8; ++k)
+              mx8[k] = fmax3(__uint_as_float(s0[k]), __uint_as_float(s0[k + 8]), __uint_as_float(s0[k + 16]));
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mx8[k] = fmax3(mx8[k], __uint_as_float(s1[k + 8]), __uint_as_float(s0[k + 16]));
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mx8[k] = fmax3(mx8[k], __uint_as_float(s1[k + 16]), __uint_as_float(s0[k + 24]));
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s1[k + 24]));
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          const float tmax = mx * P.scale_log2;
-          // a flagged row's tile max lies above its running max
-          const bool move = flag && (tmax > m || m == -INFINITY);
-          const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
-          l *= alpha;
-          if (move) m = tmax;
-          if (unit_tiles > 0 && __any_sync(0xffffffffu, move)) {
-            // rows whose max moved rescale their O row (alpha = 1
-            // elsewhere); the previous PV has completed (s_full)
+            for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s0[k + 24]));
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float tmax = mx * P.scale_log2;
+            // a flagged row's max lies above its running max
+            const bool move = flag && (tmax > m || m == -INFINITY);
+            const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
+            l *= alpha;
+            if (move) m = tmax;
+            if (unit_subs > 0 && __any_sync(0xffffffffu, move)) {
+              // rows whose max moved rescale their O row (alpha = 1
+              // elsewhere), once the PV of the previous half tile has
+              // completed: phases before it have, the next one cannot have
+              // (it needs this half's P), so the parity names it
+              if (!__all_sync(0xffffffffu, mbar_wait(B.o_ready, (x - 1) & 1, abort_flag, P.dev_status,
+                                                     P.wait_ns))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after_sync();
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(lane_addr + L::kOCol + c0, o);
-              tmem_ld_wait(o);
+              for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(lane_addr + L::kOCol + c0, o);
+                tmem_ld_wait(o);
 #pragma unroll
-              for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
-              tmem_st32(lane_addr + L::kOCol + c0, o);
+                for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
+                tmem_st32(lane_addr + L::kOCol + c0, o);
+              }
             }
+            lsum = exp_pass();
           }
-          lsum = exp_pass();
+          l += lsum;
+          tmem_st16(s_col, pk);   // P over the first kSub/2 columns of this S buffer
+          tmem_st_wait();
+          tc_fence_before_sync();
+          mbar_arrive(B.p_ready + (x & 1));
         }
-        l += lsum;
-        tmem_st32(lane_addr + L::kSCol, pk);   // P overwrites the first 32 columns of S
-        tmem_st_wait();
-        tc_fence_before_sync();
-        mbar_arrive(B.p_ready);
       }
+      const bool have_o = unit_subs > 0;
       if (!ok || !(d.flags & kFlagLast)) continue;
       // The next unit's Q goes to TMEM first (every QK^T of this unit has
       // completed: its S was seen), so its first QK^T overlaps this epilogue.
@@ -781,7 +836,6 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       }
 
       // ---- epilogue of the unit
-      const bool have_o = unit_tiles > 0;
       if (have_o) {
         if (!__all_sync(0xffffffffu, mbar_wait(B.o_done, n_o & 1, abort_flag, P.dev_status, P.wait_ns))) {
           ok = false;
@@ -1037,6 +1091,7 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
   P.num_splits = a.num_splits;
   P.dev_status = a.dev_status;
   P.wait_ns = attn_wait_limit_ns();
+  P.stall = attn_stall() ? 1 : 0;
   const int head_tiles = (a.num_heads + 127) / 128;
   P.part_o = nullptr;
   P.part_ml = nullptr;

@@ -80,7 +80,7 @@ struct SetsParams {
   uint32_t* dev_status;
 };
 
-constexpr int kSetsWarps = kSetsQueriesPerCta;   // warps per CTA
+constexpr int kSetsWarps = 16;   // warps per CTA, one query each at a time
 constexpr int kMaxPerCta = 2048;
 
 __device__ __forceinline__ int64_t warp_sum64(int64_t v) {

@@ -167,6 +167,13 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
+// Posted store of 16 bytes into the shared memory of a CTA of the cluster
+// (address from dsmem_addr); visible to it after the next cluster barrier.
+__device__ __forceinline__ void st_dsmem_f4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 // Every thread of every CTA of the cluster, convergently: shared-memory
 // writes before it are visible to the whole cluster after it.
 __device__ __forceinline__ void cluster_sync_all() {
@@ -368,6 +375,11 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // ... and has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Bring the 128-byte line holding p into L2 (no value, no fault reported).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float exp2_approx(float x) {

@@ -11,7 +11,7 @@ namespace spa {
 // SM count of the current device (cached per device).
 int device_sm_count();
 
-constexpr int kSetsQueriesPerCta = 8;      // one warp per query
+constexpr int kSetsQueriesPerCta = 8;      // fewest queries a set-builder CTA owns
 constexpr int kMaxTopkWidth = 2048;
 
 size_t build_kv_sets_workspace_bytes(int32_t n_queries);
@@ -88,10 +88,13 @@ constexpr int kAttnMaxClusterSplits = 8;
 size_t attn_workspace_bytes(int32_t n_queries, int32_t num_heads, int32_t head_dim,
                             int32_t num_splits);
 cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream);
-// Limit (ns) of the waits between the warp roles of the attention forward;
-// 1 s unless a test changed it.
+// Limit (ns) of the waits between the warp roles of the attention forward
+// (1 s), and the testing stall: when set, every CTA of the next forward
+// launches waits on a barrier nothing arrives at, with the stall's limit.
+constexpr uint64_t kWaitTimeoutNsHost = 1000ull * 1000ull * 1000ull;
 uint64_t attn_wait_limit_ns();
-void set_attn_wait_limit_ns(uint64_t ns);
+bool attn_stall();
+void set_attn_stall_ns(uint64_t ns);
 cudaError_t launch_sparse_sink_attn_bwd(const AttnArgs& a, cudaStream_t stream);
 // head_dim 512 (32 heads per tile, transposed products); slices merge in a
 // cluster only (at most kAttnMaxClusterSplits), no workspace

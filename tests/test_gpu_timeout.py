@@ -3,10 +3,11 @@
 Every wait between the warp roles of the attention forward has a time
 limit; when one runs out the kernel sets SPA_DEV_TIMEOUT, the CTA unwinds
 (waiting, with the fixed limit, for its own copies and tensor-core products
-before it frees TMEM) and the call returns. The testing hook sets that limit
-to 0, so the first wait that is not already satisfied gives up: a flag that
-nothing sets in time. The context must stay usable: the next call with the
-default limit is bit-identical to a clean run.
+before it frees TMEM) and the call returns. The testing hook makes every
+CTA wait on a barrier that nothing arrives at (a flag that nothing sets),
+with a 2 ms limit: that wait always runs out, the others then give up on
+the CTA's abort flag. The context must stay usable: the next normal call is
+bit-identical to a clean run.
 """
 import ctypes
 
@@ -16,7 +17,7 @@ import torch
 
 pytestmark = pytest.mark.gpu
 
-DEFAULT_LIMIT_NS = 1_000_000_000
+STALL_LIMIT_NS = 2_000_000
 
 
 @pytest.fixture(scope="module")
@@ -24,16 +25,16 @@ def spa():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     import sparse_paged_attention_build_b200 as m
-    m.lib.spa_testing_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
-    m.lib.spa_testing_set_wait_limit_ns.restype = None
+    m.lib.spa_testing_stall_attention.argtypes = [ctypes.c_uint64]
+    m.lib.spa_testing_stall_attention.restype = None
     return m
 
 
-@pytest.mark.parametrize("splits", [1, 2])
-def test_zero_wait_limit_sets_timeout_and_next_call_is_clean(spa, splits):
+@pytest.mark.parametrize("name,shrink,splits", [("c1", 1, 1), ("c1", 1, 2), ("c4", 16, 12), ("f2", 8, 2)])
+def test_stalled_wait_sets_timeout_and_next_call_is_clean(spa, name, shrink, splits):
     from sparse_paged_attention_build_b200 import workloads
     from sparse_paged_attention_build_b200.pipeline import DeviceBatch
-    w = workloads.make("c1")
+    w = workloads.make(name, shrink=shrink)
     b = DeviceBatch(w, num_splits=splits)
     b.step()
     torch.cuda.synchronize()
@@ -44,14 +45,14 @@ def test_zero_wait_limit_sets_timeout_and_next_call_is_clean(spa, splits):
     st = spa.new_status()
     out = torch.full_like(b.out, float("nan"))
     lse = torch.full_like(b.lse, float("nan"))
-    spa.lib.spa_testing_set_wait_limit_ns(0)
+    spa.lib.spa_testing_stall_attention(STALL_LIMIT_NS)
     try:
         spa.sparse_sink_attn_fwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, b.indptr, b.indices, b.sink, w.scale,
                                  k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp, out=out, lse=lse,
                                  num_splits=splits, workspace=b.attn_ws, dev_status=st)
         torch.cuda.synchronize()    # the call returned and the context is usable
     finally:
-        spa.lib.spa_testing_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+        spa.lib.spa_testing_stall_attention(0)
     assert spa.read_status(st) & spa.DEV_TIMEOUT
 
     b.status.zero_()
