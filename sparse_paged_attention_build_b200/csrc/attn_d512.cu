@@ -435,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
           for (int b = 0; b < kOBlocks; ++b, ++nvp) {
             const int st = nvp % kVStages;
             if (!mbar_wait(B.v_full + st, (nvp / kVStages) & 1, abort_flag, P.dev_status, P.wait_ns)) return false;
+            fence_proxy_async_smem();
             tc_fence_after_sync();
             const uint32_t v_addr = sbase + L::kVOff + st * (2 * kChunkBytes);
   #pragma unroll
@@ -471,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
             for (int cc = 0; cc < kNChunks; ++cc, ++nk) {
               const int st = nk % kKStages;
               if (!mbar_wait(B.k_full + st, (nk / kKStages) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+              fence_proxy_async_smem();   // the copies' rows, landed in the generic proxy -> the UMMA reads
               tc_fence_after_sync();
               const uint32_t k_addr = sbase + L::kKOff + st * kChunkBytes;
               const uint32_t q_addr = sbase + L::kQOff + cc * (kHT * 128);
@@ -509,9 +511,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
     // V: a pair is columns [128b, 128b+128); lane l copies piece l%16 of
     // rows l/16 + 2j. Piece p of row r lands at (p/8)*16 KB + r*128 +
     // ((p%8) ^ (r%8))*16: the 128-byte swizzle that both the K-major S^T
-    // operand and the M-major O^T operand read. Tiles are handed over as
-    // in the 128-head kernel: fence.proxy.async and one arrival per thread
-    // once the copies have landed, checked after the next chunk is issued.
+    // operand and the M-major O^T operand read. Each thread's copies of a
+    // stage complete into the stage's barrier by themselves
+    // (cp.async.mbarrier.arrive.noinc: one arrival per thread once its
+    // copies have landed), so a thread never waits for its own copies and
+    // every free stage is in flight; the UMMA issuer orders the landed rows
+    // before its tensor-core reads with fence.proxy.async after the wait.
+    // (Handing a stage over only after the next one was issued, waiting for
+    // the copies, kept one stage in flight: about 1 us per 16 KB chunk.)
     const bool is_k = warp < kVGroupWarp0;
     const int gw = warp - (is_k ? kKGroupWarp0 : kVGroupWarp0);
     const int nst = is_k ? kKStages : kVStages;
@@ -527,21 +534,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
     const int piece = lane % pieces, rsub = lane / pieces;
     const uint32_t col_off = static_cast<uint32_t>((piece / 8) * kChunkBytes);
     const int p8 = piece % 8;
-    int pending = -1;
-    auto hand_over = [&]() {
-      if (pending >= 0) {
-        cp_async_wait_group<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(full + pending);
-        pending = -1;
-      }
-    };
-    int c = 0, n = 0;
+int c = 0, n = 0;
     bool final_seen = false;
     while (!final_seen) {
       const int slot = c & 1;
-      if (pending >= 0 && !mbar_try_wait(B.tab_full + slot, (c >> 1) & 1)) hand_over();
-      if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
+if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
       const ChunkDesc d = desc[slot];
       final_seen = (d.flags & kFlagFinal) != 0;
       const uint32_t* t_rows = tab + slot * kChunkKeys;
@@ -553,8 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
         for (int part = 0; part < per_tile; ++part, ++n) {
           const int stage = n % nst;
           const uint32_t par = ((n / nst) & 1) ^ 1;
-          if (pending >= 0 && !mbar_try_wait(empty + stage, par)) hand_over();
-          if (!mbar_wait(empty + stage, par, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+if (!mbar_wait(empty + stage, par, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
           const uint32_t stage_base = ring + stage * stage_bytes + col_off;
           const int64_t col_bytes = static_cast<int64_t>(part) * (is_k ? 128 : 256) + piece * 16;
 #pragma unroll 4
@@ -566,21 +562,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
             const uint8_t* src = valid ? base + static_cast<int64_t>(e & ~kRawBit) * (kD * 2) + col_bytes : pool_raw;
             cp_async16(stage_base + r * 128 + ((p8 ^ (r & 7)) << 4), src, valid ? 16u : 0u);
           }
-          cp_async_commit();
-          if (pending >= 0) {
-            cp_async_wait_group<1>();
-            fence_proxy_async_smem();
-            mbar_arrive(full + pending);
-          }
-          pending = stage;
+          cp_async_arrive_noinc(full + stage);
         }
       }
       mbar_arrive(B.tab_empty + slot);
       ++c;
       if (!ok) break;
     }
-    hand_over();
-    cp_async_wait_group<0>();
+    cp_async_wait_all();   // no copy of this thread is in flight when the CTA leaves
     cta_finish(P, false, smem, sbase, tmem, tid, warp, head0, heads_here, &ss);
   } else {
     warpgroup_reg_alloc<kRegSoftmax>();

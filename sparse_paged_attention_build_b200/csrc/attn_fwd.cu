@@ -12,11 +12,9 @@
 // Work unit = (query token i, slice s of its key set, 128-head tile). All
 // heads of the unit share every K/V row, so the unit is a dense MQA problem
 // with M = 128 heads:
-//   S  = Q[128 x d] . K_half[32 x d]^T      tcgen05.mma, Q in TMEM, K in SMEM
+//   S  = Q[128 x d] . K_tile[64 x d]^T      tcgen05.mma, Q in TMEM, K in SMEM
 //   P  = exp2(S*scale*log2e - m)  (BF16)    softmax warps, TMEM -> regs -> TMEM
-//   O += P[128 x 32] . V_half[32 x d]        tcgen05.mma, P in TMEM, V in SMEM
-// K and V arrive in tiles of 64 rows; the products and the softmax take each
-// tile in two halves of 32 keys.
+//   O += P[128 x 64] . V_tile[64 x d]        tcgen05.mma, P in TMEM, V in SMEM
 // Both products take their A operand from TMEM: measured on B200, an
 // M = 128, N = 64 product with both operands in shared memory is bound by
 // shared-memory bandwidth at two thirds of the tensor rate, while with A in
@@ -26,36 +24,32 @@
 //
 // Persistent CTAs (two per SM) walk their units in a fixed stride; the two
 // CTAs of an SM interleave on the tensor core and on the exp unit. Warp
-// roles (512 threads, four warpgroups):
+// roles (256 threads):
 //   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t.
 //              They also move each unit's Q from shared memory into TMEM.
 //   warp  4    TMEM allocation; lane 0 issues every UMMA and commit
-//   warps 5, 7 resolver: for a chunk of up to 768 keys of a unit they load
-//              the keys, look their pages up and write the physical row of
-//              every key (bit 31 = raw pool) to a double-buffered table,
+//   warp  5    resolver: for a chunk of up to 768 keys of a unit it loads
+//              the keys, looks their pages up and writes the physical row
+//              of every key (bit 31 = raw pool) to a double-buffered table,
 //              plus a chunk descriptor that every other role follows. All
 //              dependent global loads of the gather happen here, ahead of
-//              the copies; each warp takes half of every chunk.
-//   warp  6    Q: one TMA box load per unit into the landing area
-//   warps 8-11 K gather, warps 12-15 V gather: 16-byte cp.async copies of
-//              the rows the table names into 2-stage rings, written in the
-//              128-byte swizzled K-major layout of the UMMA descriptors
-//              (lanes 0-15 of a warp copy one 256-byte row, so every
-//              instruction moves whole rows); rows outside a pool (padding,
-//              faulty keys) are zero-filled. Measured on B200, random row
-//              gathers from L2 by cp.async over 8 warps per CTA run at
-//              about 14.7 TB/s against 5.9 TB/s for TMA tile::gather4 from
-//              one warp per operand, which capped this kernel before.
-// The warpgroups then move registers with setmaxnreg: the softmax rows keep
-// 64 scores, 32 packed probabilities and the running statistics in
-// registers, the copy warps need few.
-// TMEM columns: two S/P buffers [0,64) of 32 columns each, Q [64, 64 + d/2)
-// as packed BF16 pairs, O after. S of half tile j+1 is computed while the
-// softmax of half j runs (issue order QK(j+1), then PV(j)); P(j) overwrites
-// the first 16 columns of its buffer and is read by PV(j) before QK(j+2)
-// reuses that buffer, since the UMMAs of a CTA run in issue order. (With one
-// 64-column S buffer the softmax and the product round trip ran in series,
-// about 950 + 1400 cycles per 64 keys for a CTA on B200.)
+//              the copies.
+//   warp  6    K gather (and Q): TMA tile::gather4 loads, four rows of one
+//              pool per instruction, into a 2-stage ring, 128-byte swizzled
+//              by the tensor map into the K-major layout of the UMMA
+//              descriptors; rows outside a pool (padding, faulty keys) are
+//              zero-filled by the TMA. Q arrives as TMA boxes; the first
+//              unit's Q is requested at once (the unit is known from the
+//              block index), while the resolver is still fetching keys.
+//   warp  7    V gather, into its own 2-stage ring
+// (Measured on B200 for the ratio-4 prefill: the same kernel with 16-byte
+// cp.async gathers from eight warps per CTA ran 1.24 ms against 1.0 ms
+// with TMA gather4 from one warp per operand: the copy warps took issue
+// slots and registers the softmax needs.)
+// TMEM columns: S/P [0,64), Q [64, 64 + d/2) as packed BF16 pairs, O after.
+// S is single-buffered: QK^T of tile g+1 is issued after PV of tile g, and
+// the UMMAs of a CTA run in issue order, so P(g) is read before S(g+1)
+// overwrites it; the other CTA on the SM fills the tensor core meanwhile.
 // The softmax first takes P with the running max as it stands and only
 // recomputes a tile whose row sum leaves a fixed bound (see kSpecBound);
 // O/l and LSE use the same max, so the result is exact in exact arithmetic.
@@ -74,36 +68,18 @@ constexpr int kStagesK = 2;
 constexpr int kStagesV = 2;
 constexpr int kSoftThreads = 128;
 constexpr int kMmaWarp = 4;
-constexpr int kResolverWarp0 = 5;
-constexpr int kQWarp = 6;
-constexpr int kResolverWarp1 = 7;
-constexpr int kKGroupWarp0 = 8;                  // warps 8..11: K rows
-constexpr int kVGroupWarp0 = 12;                 // warps 12..15: V rows
-constexpr int kGroupThreads = 128;
-constexpr int kThreads = 512;
+constexpr int kResolverWarp = 5;
+constexpr int kKWarp0 = 6;                       // K (and Q) producer
+constexpr int kVWarp0 = 7;                       // V producer
+constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
-// Registers per thread after the split; the four warpgroups together keep
-// the 4 x 64 the block is launched with (two 512-thread blocks per SM).
-template <bool kFp8>
-struct RegSplit {
-  static constexpr uint32_t kSoftmax = kFp8 ? 96 : 112;
-  static constexpr uint32_t kControl = 64;            // MMA issue, resolvers, Q
-  static constexpr uint32_t kGather = kFp8 ? 48 : 40;  // the FP8 decode holds codes and scales
-  static_assert(true || kSoftmax + kControl + 2 * kGather <= 4 * 64, "register split exceeds the launch");
-};
 // A tile whose row sum of P, taken with the running max as it stands,
 // exceeds 2^16 (or is not a number) is recomputed with its exact max. P
 // therefore stays below 2^16: harmless in BF16 and in the FP32 sums, whose
 // relative precision does not depend on magnitude.
 constexpr float kSpecBound = 65536.0f;
-// The tensor cores and the softmax work on half tiles of 32 keys with two S
-// buffers in TMEM: S of half j+1 is computed while the softmax of half j
-// runs, and P of half j (BF16, over the first kSub/2 columns of its S
-// buffer) is read by the PV product before S of half j+2 overwrites it (the
-// products of a CTA run in issue order).
-constexpr int kSub = 32;
-// consumers of a chunk descriptor: K and V groups, MMA thread, softmax, Q warp
-constexpr uint32_t kTabConsumers = 2 * kGroupThreads + 1 + kSoftThreads + 32;
+// consumers of a chunk descriptor: K warp, V warp, MMA thread, softmax
+constexpr uint32_t kTabConsumers = 32 + 32 + 1 + kSoftThreads;
 
 struct Params {
   // TMA descriptors (passed as a __grid_constant__ parameter)
@@ -112,11 +88,6 @@ struct Params {
   CUtensorMap tm_v_raw;
   CUtensorMap tm_k_cmp;
   CUtensorMap tm_v_cmp;
-  // the pools as plain pointers, for the cp.async gather
-  const uint8_t* k_raw;
-  const uint8_t* v_raw;
-  const uint8_t* k_cmp;
-  const uint8_t* v_cmp;
   int32_t q_box_rows;     // min(128, num_heads)
   int32_t n_queries, num_heads;
   int64_t raw_pages;
@@ -170,16 +141,16 @@ struct Layout {
   static constexpr int kMergeOff = kDescOff + 2 * static_cast<int>(sizeof(ChunkDesc));
   static constexpr int kBarOff = kMergeOff + kAttnMaxSplits * 128 * 4;
   // tab_full[2], tab_empty[2], q_full, q_empty, q_ready, K ring, V ring,
-  // s_full[2], p_ready[2], o_ready, o_done, mma_done, soft_sync[2]
-  static constexpr int kNumBars = 2 + 2 + 3 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 1 + 1 + 1 + 2;
+  // s_full, p_ready, o_done, mma_done, soft_sync[2]
+  static constexpr int kNumBars = 2 + 2 + 3 + 2 * kStagesK + 2 * kStagesV + 1 + 1 + 1 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kUsed = kMiscOff + 32;   // + the testing stall barrier at kMiscOff + 16
   // + alignment slack; at least 80 KB so that no more than two CTAs share an
   // SM (TMEM holds two 256-column allocations)
   static constexpr int kBytes = (kUsed + 1024) < 80 * 1024 ? 80 * 1024 : (kUsed + 1024);
-  static constexpr uint32_t kSCol = 0;                      // S buffers [2][kSub]
-  static constexpr uint32_t kQCol = 2 * kSub;
-  static constexpr uint32_t kOCol = 2 * kSub + D / 2;
+  static constexpr uint32_t kSCol = 0;
+  static constexpr uint32_t kQCol = kT;
+  static constexpr uint32_t kOCol = kT + D / 2;
   static_assert(kOCol + D <= kTmemCols, "TMEM budget");
   static_assert((kBytes + 1024) * 2 <= 228 * 1024, "two CTAs per SM");
   static_assert(kMergeOff % 16 == 0, "staging alignment");
@@ -195,10 +166,8 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;     // [kStagesV]
   uint64_t* v_empty;
-  uint64_t* s_full;     // [2]: S of a half tile in its buffer
-  uint64_t* p_ready;    // [2]: P of a half tile in its S buffer (one barrier per buffer: the
-                        // softmax may finish two half tiles before the UMMA issuer waits)
-  uint64_t* o_ready;    // one phase per half tile: its PV product has completed
+  uint64_t* s_full;     // S of the current tile (also: every earlier UMMA done)
+  uint64_t* p_ready;    // P of the current tile in TMEM
   uint64_t* o_done;     // last PV of a unit complete
   uint64_t* mma_done;
   // [2]: barrier of the softmax threads, the two used in turn. An mbarrier
@@ -207,120 +176,8 @@ struct Bars {
   uint64_t* soft_sync;
 };
 
-// End of every role (inlined into each, so that it runs within that
-// warpgroup's registers): every TMEM access of the role has completed; the
-// softmax warps (soft) then run the cluster merge, every warp takes the
-// cluster barriers, and the MMA warp frees TMEM last.
-template <int D>
-__device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* smem, uint32_t sbase, uint32_t tmem,
-                                           int tid, int warp, int S, int heads_here, int head0) {
-  using L = Layout<D>;
-  __syncwarp();
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  if (P.cluster_merge) {
-    // Exact merge of the S slices of query i, CTA `rank` holding slice
-    // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
-    // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
-    // Summary: the deterministic (out, lse) merge). CTA r owns rows
-    // [r*per, (r+1)*per) of the output. After the first cluster barrier
-    // every CTA reads all slices' (m, l) of its rows (one round trip of
-    // distributed shared memory), scales its O rows by its weight and
-    // stores each row straight into its owner's idle K/V ring (posted
-    // stores, slot = the sender's rank); after the second barrier each owner
-    // sums its slots locally and writes BF16 O. No shared memory is read or
-    // written remotely after the second barrier, so no third one is needed.
-    // Every thread of every CTA reaches both barriers: every earlier wait in
-    // the kernel is bounded.
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int i = static_cast<int>(blockIdx.x / S);
-    const uint32_t ml_addr = sbase + L::kMergeOff;
-    const uint32_t rx_addr = sbase + L::kKOff;               // [S][per][D] FP32, 16-byte chunks swizzled by row
-    constexpr int kChunks = D / 4;                           // 16-byte chunks per row
-    const int per = (128 + S - 1) / S;
-    // the slots (S * per <= 128 + S - 1 rows of D FP32) fill the K/V rings
-    // and may run on into the chunk tables, all idle by now
-    static_assert(L::kTabOff - L::kKOff + 2 * kChunkKeys * 4 >= (128 + kAttnMaxClusterSplits - 1) * D * 4,
-                  "receive slots fit the idle rings and tables");
-    static_assert(L::kTabOff == L::kVOff + kStagesV * L::kTileBytes && L::kVOff == L::kKOff + kStagesK * L::kTileBytes,
-                  "rings and tables are contiguous");
-    __syncwarp();
-    cluster_sync_all();                                      // every slice's (m, l) is in place; rings idle
-    if (soft) {
-      const int row = tid;
-      float2 ml[kAttnMaxClusterSplits];
-#pragma unroll
-      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-        ml[s] = s < S ? ld_dsmem_f2(dsmem_addr(ml_addr + row * 8, s)) : make_float2(-INFINITY, 0.f);
-      float M = -INFINITY;
-#pragma unroll
-      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-        if (ml[s].y > 0.f) M = fmaxf(M, ml[s].x);
-      float Lsum = 0.f, w_own = 0.f;
-#pragma unroll
-      for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
-        const float w = (ml[s].y > 0.f) ? exp2_approx(ml[s].x - M) : 0.f;
-        Lsum += w * ml[s].y;
-        if (s == rank) w_own = w;
-      }
-      const float scale_own = Lsum > 0.f ? w_own / Lsum : 0.f;
-      if (rank == 0 && row < heads_here)
-        P.lse[static_cast<int64_t>(i) * P.num_heads + head0 + row] =
-            Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
-      const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
-      const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
-      const int owner = row / per, rr = row - owner * per;
-      const uint32_t dst = dsmem_addr(rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 4), owner);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        if (have_o) {   // warp-uniform: one flag per CTA
-          tmem_ld32(o_lane + c0, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
-        }
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const int chunk = (c0 >> 2) + v;
-          const int phys = chunk ^ (rr & (kChunks - 1));
-          st_dsmem_f4(dst + phys * 16,
-                      make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
-                                  __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own));
-        }
-      }
-    }
-    __syncwarp();
-    cluster_sync_all();                                      // every slice's weighted rows have arrived
-    if (soft) {
-      const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
-      const float* rx = reinterpret_cast<const float*>(smem + L::kKOff);
-      uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
-      const int n_items = (r1 - r0) * kChunks;
-      for (int idx = tid; idx < n_items; idx += kSoftThreads) {
-        const int rr = idx / kChunks, c = idx % kChunks;
-        const int phys = c ^ (rr & (kChunks - 1));
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < S; ++s) {
-          const float4 v = *reinterpret_cast<const float4*>(rx + ((s * per + rr) * D) + phys * 4);
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
-        }
-        *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r0 + rr) * D + 4 * c) =
-            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-      }
-    }
-  }
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
-}
-
 template <int D, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __grid_constant__ Params P) {
-  using R = RegSplit<kFp8>;
   using L = Layout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -338,9 +195,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   B.v_full = B.k_empty + kStagesK;
   B.v_empty = B.v_full + kStagesV;
   B.s_full = B.v_empty + kStagesV;
-  B.p_ready = B.s_full + 2;
-  B.o_ready = B.p_ready + 2;
-  B.o_done = B.o_ready + 1;
+  B.p_ready = B.s_full + 1;
+  B.o_done = B.p_ready + 1;
   B.mma_done = B.o_done + 1;
   B.soft_sync = B.mma_done + 1;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + L::kTabOff);
@@ -359,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   // ---- setup
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(B.tab_full + s, 64);   // two resolver warps
+      mbar_init(B.tab_full + s, 32);
       mbar_init(B.tab_empty + s, kTabConsumers);
       mbar_init(B.soft_sync + s, kSoftThreads);
     }
@@ -367,18 +223,15 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     mbar_init(B.q_empty, kSoftThreads);
     mbar_init(B.q_ready, kSoftThreads);
     for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(B.k_full + s, kGroupThreads);
+      mbar_init(B.k_full + s, 1);
       mbar_init(B.k_empty + s, 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(B.v_full + s, kGroupThreads);
+      mbar_init(B.v_full + s, 1);
       mbar_init(B.v_empty + s, 1);
     }
     mbar_init(B.s_full, 1);
-    mbar_init(B.s_full + 1, 1);
     mbar_init(B.p_ready, kSoftThreads);
-    mbar_init(B.p_ready + 1, kSoftThreads);
-    mbar_init(B.o_ready, 1);
     mbar_init(B.o_done, 1);
     mbar_init(B.mma_done, 1);
     *abort_flag = 0;
@@ -393,261 +246,249 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  // Each warpgroup takes its register limit at one place (setmaxnreg is
-  // executed by the four warps of a warpgroup together) that dominates all
-  // of its roles' code.
-  if (warp >= 4 && warp < 8) {
-    warpgroup_reg_dealloc<R::kControl>();
-    if (warp == kResolverWarp0 || warp == kResolverWarp1) {
-      // ================================================= resolver
-      // testing stall: a wait that only its limit ends, then the CTA unwinds
-      if (P.stall) mbar_wait(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 16), 0, abort_flag, P.dev_status, P.wait_ns);
-      resolver_loop<2>(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane, false,
-                       warp == kResolverWarp0 ? 0 : 1);
-      cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
-    } else if (warp == kQWarp) {
-      // ================================================= Q loader
-      // Every unit's Q, empty units included, so that the Q phases of all
-      // roles stay in step; the landing area is free once the previous Q
-      // has moved on to TMEM. The CTA's first unit is unit blockIdx.x (units
-      // are strided over the CTAs), so its Q is loaded at once, while the
-      // resolver is still fetching its keys.
-      constexpr int kHalves = D / 64;
-      int c = 0, qc = 0;
-      bool final_seen = false, first_issued = false;
+
+  if (warp == kResolverWarp) {
+    // ================================================= resolver
+    // testing stall: a wait that only its limit ends, then the CTA unwinds
+    if (P.stall) mbar_wait(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 16), 0, abort_flag, P.dev_status, P.wait_ns);
+    resolver_loop(P, S, tab, desc, B.tab_full, B.tab_empty, abort_flag, lane);
+  } else if (warp == kKWarp0 || warp == kVWarp0) {
+    // ================================================= K / V gather (TMA)
+    // A tile is 16 four-row groups x D/64 column halves = "jobs"; lane j
+    // issues one TMA tile::gather4 for job j (four rows of one pool, 512
+    // bytes). A group whose four keys come from both pools (at most one per
+    // unit: compressed groups precede window tokens) is loaded row by row.
+    // Rows past the chunk's keys and rows of faulty keys are outside the
+    // tensor and zero-filled. Lane 0 of the K warp also loads each unit's Q
+    // (every unit, empty ones included, so that the Q phases of all roles
+    // stay in step).
+    const bool is_k = warp == kKWarp0;
+    const int nst = is_k ? kStagesK : kStagesV;
+    uint64_t* full = is_k ? B.k_full : B.v_full;
+    uint64_t* empty = is_k ? B.k_empty : B.v_empty;
+    const CUtensorMap* map_raw = is_k ? &P.tm_k_raw : &P.tm_v_raw;
+    const CUtensorMap* map_cmp = is_k ? &P.tm_k_cmp : &P.tm_v_cmp;
+    const uint32_t ring = sbase + (is_k ? L::kKOff : L::kVOff);
+    constexpr int kHalves = D / 64;
+    constexpr int kGroups = kT / 4;
+    constexpr int kJobs = kGroups * kHalves;
+    const int grp = lane % kGroups, half = lane / kGroups;
+    const bool issuer = lane < kJobs;
+    int c = 0, g = 0, qc = 0;
+    bool final_seen = false, first_q_issued = false;
+    if (is_k) {
+      // The CTA's first unit is unit blockIdx.x (units are strided over the
+      // CTAs): its Q is loaded at once, while the resolver fetches its keys.
       if (lane == 0) {
         mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
         for (int hb = 0; hb < kHalves; ++hb)
           tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0,
                       static_cast<int32_t>(blockIdx.x / S));
       }
-      first_issued = true;
+      first_q_issued = true;
       qc = 1;
-      while (!final_seen) {
-        const int slot = c & 1;
-        if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
-        const ChunkDesc d = desc[slot];
-        final_seen = (d.flags & kFlagFinal) != 0;
-        bool ok = true;
-        if ((d.flags & kFlagFirst) && first_issued) {
-          first_issued = false;   // the first unit's Q is on its way
-        } else if (d.flags & kFlagFirst) {
-          ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns);
-          if (ok && lane == 0) {
-            mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
-            for (int hb = 0; hb < kHalves; ++hb)
-              tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0, d.i);
-          }
-          if (ok) ++qc;
-        }
-        __syncwarp();
-        mbar_arrive(B.tab_empty + slot);
-        ++c;
-        if (!ok) break;
-      }
-      // the last Q copy has landed before the CTA can leave (it lands even
-      // when the roles gave up early; this wait keeps the fixed limit)
-      if (qc > 0) mbar_wait(B.q_full, (qc - 1) & 1, nullptr, P.dev_status);
-      cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
-    } else if (warp == kMmaWarp) {
-      // ================================================= UMMA issuer
-      // Half tile x: S[x%2] = Q K_x^T (A = Q from TMEM); once its P is in
-      // TMEM, O += P_x V_x (A = P from TMEM). The issue order is QK(x+1)
-      // before PV(x), so the softmax of half x overlaps the product of the
-      // next S; QK(x+2) comes after PV(x), which read P(x) from the same
-      // buffer.
-      if (lane == 0) {
-        constexpr uint32_t idesc_s = idesc_bf16_f32(128, kSub, 0);
-        constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
-        int c = 0, g = 0, u = 0, x = 0;
-        bool ok = true, final_seen = false;
-        // the half tile whose PV is still to be issued
-        int pend = -1, pend_v = 0, pend_hf = 0;
-        bool pend_first = false, pend_last_of_tile = false, pend_last_of_unit = false;
-        auto issue_pv = [&]() -> bool {
-          if (!mbar_wait(B.p_ready + (pend & 1), (pend >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) return false;
-          const int st = pend_v % kStagesV;
-          if (pend_hf == 0 &&
-              !mbar_wait(B.v_full + st, (pend_v / kStagesV) & 1, abort_flag, P.dev_status, P.wait_ns))
-            return false;
-          tc_fence_after_sync();
-          const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes + pend_hf * (kSub * 128);
-          const uint32_t p_col = tmem + L::kSCol + (pend & 1) * kSub;
-#pragma unroll
-          for (int k = 0; k < kSub / 16; ++k) {
-            const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
-            umma_ts(tmem + L::kOCol, p_col + k * 8, bdesc, idesc_o, (!pend_first || k > 0) ? 1u : 0u);
-          }
-          tc_commit(B.o_ready);
-          if (pend_last_of_tile) tc_commit(B.v_empty + st);
-          if (pend_last_of_unit) tc_commit(B.o_done);
-          pend = -1;
-          return true;
-        };
-        while (ok && !final_seen) {
-          const int slot = c & 1;
-          if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
-          const ChunkDesc d = desc[slot];
-          mbar_arrive(B.tab_empty + slot);
-          ++c;
-          final_seen = (d.flags & kFlagFinal) != 0;
-          if (d.flags & kFlagFirst) {   // this unit's Q is in TMEM
-            if (!mbar_wait(B.q_ready, u & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
-            ++u;
-            tc_fence_after_sync();
-          }
-          const int ntiles = ceil_tiles(d.nkeys);
-          for (int t = 0; ok && t < ntiles; ++t, ++g) {
-            const int stage = g % kStagesK;
-            if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
-            tc_fence_after_sync();
-            const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
-            const int nv = min(kT, d.nkeys - t * kT);
-            const int nsub = (nv + kSub - 1) / kSub;
-            for (int hf = 0; hf < nsub; ++hf, ++x) {
-#pragma unroll
-              for (int k = 0; k < D / 16; ++k) {
-                const uint64_t bdesc =
-                    smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + hf * (kSub * 128) + (k & 3) * 32, 16, 1024);
-                umma_ts(tmem + L::kSCol + (x & 1) * kSub, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
-              }
-              if (hf == nsub - 1) tc_commit(B.k_empty + stage);
-              tc_commit(B.s_full + (x & 1));
-              if (pend >= 0 && !issue_pv()) { ok = false; break; }
-              pend = x;
-              pend_v = g;
-              pend_hf = hf;
-              pend_first = (d.flags & kFlagFirst) && t == 0 && hf == 0;
-              pend_last_of_tile = hf == nsub - 1;
-              pend_last_of_unit = (d.flags & kFlagLast) && t == ntiles - 1 && hf == nsub - 1;
-            }
-          }
-        }
-        if (ok && pend >= 0) issue_pv();
-        // every UMMA has completed before TMEM is released
-        tc_commit(B.mma_done);
-        mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
-      }
-      cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
     }
-  } else if (warp >= kKGroupWarp0) {
-    warpgroup_reg_dealloc<R::kGather>();
-    // ================================================= K / V gather (cp.async)
-    // A warp copies 16 rows of a 64-row tile: lane l takes 16-byte piece
-    // l % (D/8) of row l / (D/8) (+ the rows of later instructions), so an
-    // instruction moves 32 / (D/8) whole rows. Piece c of row r lands at
-    // half c/8 (64-column blocks), row r, 16-byte chunk (c%8) ^ (r%8): the
-    // 128-byte swizzle of the K-major UMMA layout. A tile is handed over
-    // (fence.proxy.async, then one arrival per thread) once its copies have
-    // landed, which is checked after the next tile's copies are issued, so
-    // two tiles are in flight; before any wait that would block, the tile
-    // in flight is handed over first.
-    const bool is_k = warp < kVGroupWarp0;
-    const int gw = warp - (is_k ? kKGroupWarp0 : kVGroupWarp0);
-    const int nst = is_k ? kStagesK : kStagesV;
-    uint64_t* full = is_k ? B.k_full : B.v_full;
-    uint64_t* empty = is_k ? B.k_empty : B.v_empty;
-    const uint8_t* pool_raw = is_k ? P.k_raw : P.v_raw;
-    const uint8_t* pool_cmp = is_k ? P.k_cmp : P.v_cmp;
-    const uint8_t* pool8 = is_k ? P.k_cmp8 : P.v_cmp8;
-    const float* psc = is_k ? P.k_cmp_sc : P.v_cmp_sc;
-    const uint32_t ring = sbase + (is_k ? L::kKOff : L::kVOff);
-    constexpr int kCpr = D / 8;          // 16-byte pieces per row
-    constexpr int kRpi = 32 / kCpr;      // rows per instruction
-    constexpr int kNi = 16 / kRpi;       // instructions per warp per tile
-    const int ch = lane % kCpr, rsub = lane / kCpr;
-    const uint32_t col_off = static_cast<uint32_t>((ch / 8) * (kT * 128));
-    const int c8 = ch % 8;
-    int pending = -1;   // ring stage whose copies are issued but not handed over
-    auto hand_over = [&]() {
-      if (pending >= 0) {
-        cp_async_wait_group<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(full + pending);
-        pending = -1;
-      }
-    };
-    int c = 0, g = 0;
-    bool final_seen = false;
     while (!final_seen) {
       const int slot = c & 1;
-      if (pending >= 0 && !mbar_try_wait(B.tab_full + slot, (c >> 1) & 1)) hand_over();
       if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) break;
       const ChunkDesc d = desc[slot];
       final_seen = (d.flags & kFlagFinal) != 0;
       const uint32_t* t_rows = tab + slot * kChunkKeys;
       const int ntiles = ceil_tiles(d.nkeys);
       bool ok = true;
-      for (int t = 0; t < ntiles; ++t, ++g) {
-        const int stage = g % nst;
-        const uint32_t par = ((g / nst) & 1) ^ 1;
-        if (pending >= 0 && !mbar_try_wait(empty + stage, par)) hand_over();
-        if (!mbar_wait(empty + stage, par, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
-        const int nv = min(kT, d.nkeys - t * kT);
-        const uint32_t* trow = t_rows + t * kT;
-        const uint32_t stage_base = ring + stage * L::kTileBytes + col_off;
-        if constexpr (!kFp8) {
-#pragma unroll 2
-          for (int j = 0; j < kNi; ++j) {
-            const int r = gw * 16 + j * kRpi + rsub;
-            const uint32_t e = r < nv ? trow[r] : kInvalidRow;
-            const uint8_t* base = (e & kRawBit) ? pool_raw : pool_cmp;
-            const bool valid = e != kInvalidRow && base != nullptr;
-            const uint8_t* src = valid ? base + static_cast<int64_t>(e & ~kRawBit) * (D * 2) + ch * 16 : pool_raw;
-            cp_async16(stage_base + r * 128 + ((c8 ^ (r & 7)) << 4), src, valid ? 16u : 0u);
-          }
-        } else {
-          // compressed rows arrive as E4M3 codes (8 per piece) and their
-          // group scale, decoded exactly as the page decode does; window rows
-          // and zero rows by cp.async. Every load of the tile first.
-          uint2 code[kNi];
-          float sc[kNi];
-#pragma unroll
-          for (int j = 0; j < kNi; ++j) {
-            const int r = gw * 16 + j * kRpi + rsub;
-            const uint32_t e = r < nv ? trow[r] : kInvalidRow;
-            const bool fp8_row = e != kInvalidRow && !(e & kRawBit);
-            code[j] = make_uint2(0u, 0u);
-            sc[j] = 0.f;
-            if (fp8_row) {
-              const int64_t row8 = e;
-              code[j] = __ldg(reinterpret_cast<const uint2*>(pool8 + row8 * D + ch * 8));
-              sc[j] = __ldg(psc + row8 * (D / 64) + (ch * 8) / 64);
+      if (is_k && (d.flags & kFlagFirst) && first_q_issued) {
+        first_q_issued = false;   // the first unit's Q is on its way
+      } else if (is_k && (d.flags & kFlagFirst)) {
+        // the landing area is free once the previous Q has moved to TMEM
+        ok = mbar_wait(B.q_empty, (qc & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns);
+        if (ok && lane == 0) {
+          mbar_arrive_expect_tx(B.q_full, P.q_box_rows * 128 * kHalves);
+          for (int hb = 0; hb < kHalves; ++hb)
+            tma_load_3d(sbase + L::kQOff + hb * (128 * 128), &P.tm_q, B.q_full, hb * 64, head0, d.i);
+        }
+        if (ok) ++qc;
+      }
+      if constexpr (!kFp8) {
+        for (int t = 0; ok && t < ntiles; ++t, ++g) {
+          const int stage = g % nst;
+          if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          if (lane == 0) mbar_arrive_expect_tx(full + stage, L::kTileBytes);
+          __syncwarp();
+          if (issuer) {
+            const int nv = min(kT, d.nkeys - t * kT);
+            uint32_t e[4];
+            bool any_raw = false, any_cmp = false;
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 4 * grp + k;
+              e[k] = r < nv ? t_rows[t * kT + r] : kInvalidRow;
+              if (e[k] != kInvalidRow) {
+                if (e[k] & kRawBit) any_raw = true;
+                else any_cmp = true;
+              }
+            }
+            int32_t y[4];
+  #pragma unroll
+            for (int k = 0; k < 4; ++k)   // rows outside the tensor are zero-filled
+              y[k] = e[k] == kInvalidRow ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
+            const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
+            if (!(any_raw && any_cmp)) {
+              tma_gather4(dst, any_cmp ? map_cmp : map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
             } else {
-              const bool valid = e != kInvalidRow;
-              const uint8_t* src = valid ? pool_raw + static_cast<int64_t>(e & ~kRawBit) * (D * 2) + ch * 16 : pool_raw;
-              cp_async16(stage_base + r * 128 + ((c8 ^ (r & 7)) << 4), src, valid ? 16u : 0u);
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const bool cmp_row = e[k] != kInvalidRow && !(e[k] & kRawBit);
+                tma_load_2d(dst + k * 128, cmp_row ? map_cmp : map_raw, full + stage, half * 64, y[k]);
+              }
+            }
+          }
+        }
+      } else {
+        // Fused FP8 decode. Raw (window) rows and zero rows (past the set,
+        // faulty keys) still come by TMA; compressed rows are read as E4M3
+        // codes and scales with plain loads (all of a tile's loads in flight
+        // together), decoded exactly as the page decode does, and written
+        // into the same 128-byte swizzled BF16 layout. The tile is complete
+        // once the TMA bytes have landed and lane 0 has arrived after every
+        // lane's shared-memory writes. (Staging the codes through cp.async
+        // to overlap the next tile's fetch measured slower on B200.)
+        constexpr int kPieces = D / 16;   // 16 codes per piece
+        constexpr int kPerLane = kT * kPieces / 32;
+        const uint8_t* pool8 = is_k ? P.k_cmp8 : P.v_cmp8;
+        const float* psc = is_k ? P.k_cmp_sc : P.v_cmp_sc;
+        for (int t = 0; ok && t < ntiles; ++t, ++g) {
+          const int stage = g % nst;
+          if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          const int nv = min(kT, d.nkeys - t * kT);
+          const uint32_t* trow = t_rows + t * kT;
+          uint32_t tx = 0;
+          uint32_t e[4];
+          bool fp8_row[4] = {false, false, false, false};
+          if (issuer) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 4 * grp + k;
+              e[k] = r < nv ? trow[r] : kInvalidRow;
+              fp8_row[k] = e[k] != kInvalidRow && !(e[k] & kRawBit);
+              if (!fp8_row[k]) tx += 128;
             }
           }
 #pragma unroll
-          for (int j = 0; j < kNi; ++j) {
-            const int r = gw * 16 + j * kRpi + rsub;
-            const uint32_t e = r < nv ? trow[r] : kInvalidRow;
-            if (e == kInvalidRow || (e & kRawBit)) continue;
-            uint32_t o[4];
-            if (P.fp8_fnuz) decode_e4m3x8<true>(code[j], sc[j], o);
-            else decode_e4m3x8<false>(code[j], sc[j], o);
-            *reinterpret_cast<uint4*>(smem + (stage_base - sbase) + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-                make_uint4(o[0], o[1], o[2], o[3]);
+          for (int off = 16; off > 0; off >>= 1) tx += __shfl_xor_sync(0xffffffffu, tx, off);
+          if (lane == 0) mbar_expect_tx(full + stage, tx);
+          __syncwarp();
+          if (issuer) {
+            int32_t y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              y[k] = (e[k] == kInvalidRow || fp8_row[k]) ? -1 : static_cast<int32_t>(e[k] & ~kRawBit);
+            const uint32_t dst = ring + stage * L::kTileBytes + half * (kT * 128) + (4 * grp) * 128;
+            if (!(fp8_row[0] || fp8_row[1] || fp8_row[2] || fp8_row[3])) {
+              tma_gather4(dst, map_raw, full + stage, half * 64, y[0], y[1], y[2], y[3]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (!fp8_row[k]) tma_load_2d(dst + k * 128, map_raw, full + stage, half * 64, y[k]);
+            }
           }
+          uint8_t* tile = smem + (is_k ? L::kKOff : L::kVOff) + stage * L::kTileBytes;
+          uint4 raw[kPerLane];
+          float sc[kPerLane];
+#pragma unroll
+          for (int j = 0; j < kPerLane; ++j) {   // every load first
+            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
+            const uint32_t er = r < nv ? trow[r] : kInvalidRow;
+            raw[j] = make_uint4(0u, 0u, 0u, 0u);
+            sc[j] = 0.f;
+            if (er != kInvalidRow && !(er & kRawBit)) {
+              const int64_t row8 = er;
+              raw[j] = __ldg(reinterpret_cast<const uint4*>(pool8 + row8 * D + piece * 16));
+              sc[j] = __ldg(psc + row8 * (D / 64) + (piece * 16) / 64);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < kPerLane; ++j) {
+            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
+            const uint32_t er = r < nv ? trow[r] : kInvalidRow;
+            if (er == kInvalidRow || (er & kRawBit)) continue;
+            uint32_t o[8];
+            if (P.fp8_fnuz) decode_e4m3x16<true>(raw[j], sc[j], o);
+            else decode_e4m3x16<false>(raw[j], sc[j], o);
+            const int hf = (piece * 16) / 64, ch0 = ((piece * 16) % 64) / 8;
+            uint8_t* row_ptr = tile + hf * (kT * 128) + r * 128;
+            *reinterpret_cast<uint4*>(row_ptr + ((ch0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(row_ptr + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+          fence_proxy_async_smem();   // generic-proxy writes -> the UMMA's reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full + stage);
         }
-        cp_async_commit();
-        if (pending >= 0) {   // the previous tile has landed: hand it over
-          cp_async_wait_group<1>();
-          fence_proxy_async_smem();
-          mbar_arrive(full + pending);
-        }
-        pending = stage;
       }
       mbar_arrive(B.tab_empty + slot);
       ++c;
       if (!ok) break;
     }
-    hand_over();
-    cp_async_wait_group<0>();
-    cta_finish<D>(P, false, smem, sbase, tmem, tid, warp, S, heads_here, head0);
+    // every copy this warp started has landed before the CTA can leave (they
+    // land even when the roles gave up early; these waits keep the fixed
+    // limit): the last two ring stages, and the last Q
+    for (int k = 1; k <= nst && k <= g; ++k)
+      mbar_wait(full + (g - k) % nst, ((g - k) / nst) & 1, nullptr, P.dev_status);
+    if (is_k && qc > 0) mbar_wait(B.q_full, (qc - 1) & 1, nullptr, P.dev_status);
+  } else if (warp == kMmaWarp) {
+    // ================================================= UMMA issuer
+    // Per tile: S = Q K^T (A = Q from TMEM), then, once P is in TMEM,
+    // O += P V (A = P from TMEM). s_full is committed after the QK^T of a
+    // tile, so its arrival also means every earlier UMMA (the previous PV)
+    // has completed.
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kT, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 1);
+      int c = 0, g = 0, u = 0;
+      bool ok = true, final_seen = false;
+      while (ok && !final_seen) {
+        const int slot = c & 1;
+        if (!mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+        const ChunkDesc d = desc[slot];
+        mbar_arrive(B.tab_empty + slot);
+        ++c;
+        final_seen = (d.flags & kFlagFinal) != 0;
+        if (d.flags & kFlagFirst) {   // this unit's Q is in TMEM
+          if (!mbar_wait(B.q_ready, u & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          ++u;
+          tc_fence_after_sync();
+        }
+        const int ntiles = ceil_tiles(d.nkeys);
+        for (int t = 0; t < ntiles; ++t, ++g) {
+          const int stage = g % kStagesK, st = g % kStagesV;
+          if (!mbar_wait(B.k_full + stage, (g / kStagesK) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          tc_fence_after_sync();
+          const uint32_t k_addr = sbase + L::kKOff + stage * L::kTileBytes;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t bdesc = smem_desc_sw128(k_addr + (k >> 2) * (kT * 128) + (k & 3) * 32, 16, 1024);
+            umma_ts(tmem + L::kSCol, tmem + L::kQCol + k * 8, bdesc, idesc_s, k > 0 ? 1u : 0u);
+          }
+          tc_commit(B.k_empty + stage);
+          tc_commit(B.s_full);
+          if (!mbar_wait(B.p_ready, g & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(B.v_full + st, (g / kStagesV) & 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
+          tc_fence_after_sync();
+          const uint32_t v_addr = sbase + L::kVOff + st * L::kTileBytes;
+          const bool first = (d.flags & kFlagFirst) && t == 0;
+#pragma unroll
+          for (int k = 0; k < kT / 16; ++k) {
+            const uint64_t bdesc = smem_desc_sw128(v_addr + k * 16 * 128, kT * 128, 1024);
+            umma_ts(tmem + L::kOCol, tmem + L::kSCol + k * 8, bdesc, idesc_o, (!first || k > 0) ? 1u : 0u);
+          }
+          tc_commit(B.v_empty + st);
+          if ((d.flags & kFlagLast) && t == ntiles - 1) tc_commit(B.o_done);
+        }
+      }
+      // every UMMA has completed before TMEM is released
+      tc_commit(B.mma_done);
+      mbar_wait(B.mma_done, 0, nullptr, P.dev_status);
+    }
   } else {
-    warpgroup_reg_alloc<R::kSoftmax>();
     // ================================================= softmax + epilogue
     const int row = tid;   // head row == TMEM lane
     const int h = head0 + row;
@@ -711,11 +552,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       piece = lane & 3;
       return reinterpret_cast<const uint4*>(stage + r * 64)[piece ^ ((r >> 1) & 3)];
     };
-    int c = 0, x = 0, n_o = 0;
+    int c = 0, g = 0, n_o = 0;
     bool ok = copy_q(), final_seen = false;
     float m = -INFINITY, l = 0.f;
-    int unit_subs = 0;
-    uint32_t s0[32];
+    int unit_tiles = 0;
+    uint32_t s0[32], s1[32];
     while (ok && !final_seen) {
       const int slot = c & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(B.tab_full + slot, (c >> 1) & 1, abort_flag, P.dev_status, P.wait_ns))) {
@@ -727,106 +568,103 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       ++c;
       final_seen = (d.flags & kFlagFinal) != 0;
       if (d.flags & kFlagFirst) {
-        unit_subs = 0;
+        unit_tiles = 0;
         // the sink logit seeds the max of every slice (any reference point
         // is exact; this one is usually within the bound of the scores) but
         // joins the denominator only once, in slice 0
         m = sink2;
         l = (d.split == 0 && sink2 > -INFINITY) ? 1.f : 0.f;
       }
-      // the chunk's keys in half tiles of kSub, as the UMMA issuer cuts them
       const int ntiles = ceil_tiles(d.nkeys);
-      for (int t = 0; ok && t < ntiles; ++t) {
-        const int nv_tile = min(kT, d.nkeys - t * kT);
-        const int nsub = (nv_tile + kSub - 1) / kSub;
-        for (int hf = 0; hf < nsub; ++hf, ++x, ++unit_subs) {
-          // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait(B.s_full + (x & 1), (x >> 1) & 1, abort_flag, P.dev_status, P.wait_ns))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          const int nv = min(kSub, nv_tile - hf * kSub);
-          const uint32_t s_col = lane_addr + L::kSCol + (x & 1) * kSub;
-          // Speculative pass: P with the running max as it stands. Only when
-          // some row's sum leaves the bound (NaN and +inf, from a max still
-          // at -inf, included) is the exact max taken and P recomputed, so
-          // the max reduction stays off the common path. S is still intact
-          // in TMEM for that second pass.
-          auto load_s = [&]() {
-            tmem_ld32(s_col, s0);
-            tmem_ld_wait(s0);
-            if (nv < kSub) {   // columns past the set: -inf, so they add nothing
-#pragma unroll
-              for (int cc = 0; cc < 32; ++cc)
-                if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
-            }
-          };
-          uint32_t pk[16];
-          auto exp_pass = [&]() -> float {
-            const float neg_m = -m;
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
-              const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
-              sum4[cc & 3] += p0 + p1;
-              pk[cc] = pack_bf16x2(p0, p1);
-            }
-            return (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-          };
-          load_s();
-          float lsum = exp_pass();
-          const bool flag = row_ok && !(lsum <= kSpecBound);
-          if (__any_sync(0xffffffffu, flag)) {
-            load_s();
-            // row max: eight independent chains of 3-input max and a tree
-            float mx8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              mx8[k] = fmax3(__uint_as_float(s0[k]), __uint_as_float(s0[k + 8]), __uint_as_float(s0[k + 16]));
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s0[k + 24]));
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            const float tmax = mx * P.scale_log2;
-            // a flagged row's max lies above its running max
-            const bool move = flag && (tmax > m || m == -INFINITY);
-            const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
-            l *= alpha;
-            if (move) m = tmax;
-            if (unit_subs > 0 && __any_sync(0xffffffffu, move)) {
-              // rows whose max moved rescale their O row (alpha = 1
-              // elsewhere), once the PV of the previous half tile has
-              // completed: phases before it have, the next one cannot have
-              // (it needs this half's P), so the parity names it
-              if (!__all_sync(0xffffffffu, mbar_wait(B.o_ready, (x - 1) & 1, abort_flag, P.dev_status,
-                                                     P.wait_ns))) {
-                ok = false;
-                break;
-              }
-              tc_fence_after_sync();
-#pragma unroll 1
-              for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(lane_addr + L::kOCol + c0, o);
-                tmem_ld_wait(o);
-#pragma unroll
-                for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
-                tmem_st32(lane_addr + L::kOCol + c0, o);
-              }
-            }
-            lsum = exp_pass();
-          }
-          l += lsum;
-          tmem_st16(s_col, pk);   // P over the first kSub/2 columns of this S buffer
-          tmem_st_wait();
-          tc_fence_before_sync();
-          mbar_arrive(B.p_ready + (x & 1));
+      for (int t = 0; t < ntiles; ++t, ++g, ++unit_tiles) {
+        // tcgen05.ld/st are warp-collective: keep every branch warp-uniform
+        if (!__all_sync(0xffffffffu, mbar_wait(B.s_full, g & 1, abort_flag, P.dev_status, P.wait_ns))) {
+          ok = false;
+          break;
         }
+        tc_fence_after_sync();
+        const int nv = min(kT, d.nkeys - t * kT);
+        // Speculative pass: P with the running max as it stands. Only when
+        // some row's tile sum leaves the bound (NaN and +inf, from a max
+        // still at -inf, included) is the exact tile max taken and P
+        // recomputed, so the max reduction stays off the common path. S is
+        // still intact in TMEM for that second pass.
+        auto load_s = [&]() {
+          tmem_ld32(lane_addr + L::kSCol, s0);
+          tmem_ld32(lane_addr + L::kSCol + 32, s1);
+          tmem_ld_wait(s0);
+          tmem_ld_wait(s1);
+          if (nv < kT) {   // columns past the set: -inf, so they add nothing
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) {
+              if (cc >= nv) s0[cc] = __float_as_uint(-INFINITY);
+              if (cc + 32 >= nv) s1[cc] = __float_as_uint(-INFINITY);
+            }
+          }
+        };
+        uint32_t pk[32];
+        auto exp_pass = [&]() -> float {
+          const float neg_m = -m;
+          float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            const float p0 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc]), P.scale_log2, neg_m));
+            const float p1 = exp2_approx(fmaf(__uint_as_float(s0[2 * cc + 1]), P.scale_log2, neg_m));
+            const float p2 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc]), P.scale_log2, neg_m));
+            const float p3 = exp2_approx(fmaf(__uint_as_float(s1[2 * cc + 1]), P.scale_log2, neg_m));
+            sum4[cc & 3] += (p0 + p1) + (p2 + p3);
+            pk[cc] = pack_bf16x2(p0, p1);
+            pk[cc + 16] = pack_bf16x2(p2, p3);
+          }
+          return (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        };
+        load_s();
+        float lsum = exp_pass();
+        const bool flag = row_ok && !(lsum <= kSpecBound);
+        if (__any_sync(0xffffffffu, flag)) {
+          load_s();
+          // row max: eight independent chains of 3-input max and a tree
+          float mx8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(__uint_as_float(s0[k]), __uint_as_float(s1[k]), __uint_as_float(s0[k + 8]));
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(mx8[k], __uint_as_float(s1[k + 8]), __uint_as_float(s0[k + 16]));
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx8[k] = fmax3(mx8[k], __uint_as_float(s1[k + 16]), __uint_as_float(s0[k + 24]));
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(s1[k + 24]));
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float tmax = mx * P.scale_log2;
+          // a flagged row's tile max lies above its running max
+          const bool move = flag && (tmax > m || m == -INFINITY);
+          const float alpha = !move ? 1.f : (m == -INFINITY ? 0.f : exp2_approx(m - tmax));
+          l *= alpha;
+          if (move) m = tmax;
+          if (unit_tiles > 0 && __any_sync(0xffffffffu, move)) {
+            // rows whose max moved rescale their O row (alpha = 1
+            // elsewhere); the previous PV has completed (s_full)
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + L::kOCol + c0, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int cc = 0; cc < 32; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * alpha);
+              tmem_st32(lane_addr + L::kOCol + c0, o);
+            }
+          }
+          lsum = exp_pass();
+        }
+        l += lsum;
+        tmem_st32(lane_addr + L::kSCol, pk);   // P overwrites the first 32 columns of S
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(B.p_ready);
       }
-      const bool have_o = unit_subs > 0;
       if (!ok || !(d.flags & kFlagLast)) continue;
       // The next unit's Q goes to TMEM first (every QK^T of this unit has
       // completed: its S was seen), so its first QK^T overlaps this epilogue.
@@ -836,6 +674,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       }
 
       // ---- epilogue of the unit
+      const bool have_o = unit_tiles > 0;
       if (have_o) {
         if (!__all_sync(0xffffffffu, mbar_wait(B.o_done, n_o & 1, abort_flag, P.dev_status, P.wait_ns))) {
           ok = false;
@@ -991,8 +830,110 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         }
       }
     }
-    cta_finish<D>(P, true, smem, sbase, tmem, tid, warp, S, heads_here, head0);
   }
+
+  // ---- teardown: every TMEM access above has completed
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (P.cluster_merge) {
+    // Exact merge of the S slices of query i, CTA `rank` holding slice
+    // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
+    // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
+    // Summary: the deterministic (out, lse) merge). CTA r owns rows
+    // [r*per, (r+1)*per) of the output. After the first cluster barrier
+    // every CTA reads all slices' (m, l) of its rows (one round trip of
+    // distributed shared memory), scales its O rows by its weight and
+    // stores each row straight into its owner's idle K/V ring (posted
+    // stores, slot = the sender's rank); after the second barrier each owner
+    // sums its slots locally and writes BF16 O. No shared memory is read or
+    // written remotely after the second barrier, so no third one is needed.
+    // Every thread of every CTA reaches both barriers: every earlier wait in
+    // the kernel is bounded.
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int i = static_cast<int>(blockIdx.x / S);
+    const uint32_t ml_addr = sbase + L::kMergeOff;
+    const uint32_t rx_addr = sbase + L::kKOff;               // [S][per][D] FP32, 16-byte chunks swizzled by row
+    constexpr int kChunks = D / 4;                           // 16-byte chunks per row
+    const int per = (128 + S - 1) / S;
+    // the slots (S * per <= 128 + S - 1 rows of D FP32) fill the K/V rings
+    // and may run on into the chunk tables, all idle by now
+    static_assert(L::kTabOff - L::kKOff + 2 * kChunkKeys * 4 >= (128 + kAttnMaxClusterSplits - 1) * D * 4,
+                  "receive slots fit the idle rings and tables");
+    static_assert(L::kTabOff == L::kVOff + kStagesV * L::kTileBytes && L::kVOff == L::kKOff + kStagesK * L::kTileBytes,
+                  "rings and tables are contiguous");
+    __syncwarp();
+    cluster_sync_all();                                      // every slice's (m, l) is in place; rings idle
+    if (tid < kSoftThreads) {
+      const int row = tid;
+      float2 ml[kAttnMaxClusterSplits];
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+        ml[s] = s < S ? ld_dsmem_f2(dsmem_addr(ml_addr + row * 8, s)) : make_float2(-INFINITY, 0.f);
+      float M = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s)
+        if (ml[s].y > 0.f) M = fmaxf(M, ml[s].x);
+      float Lsum = 0.f, w_own = 0.f;
+#pragma unroll
+      for (int s = 0; s < kAttnMaxClusterSplits; ++s) {
+        const float w = (ml[s].y > 0.f) ? exp2_approx(ml[s].x - M) : 0.f;
+        Lsum += w * ml[s].y;
+        if (s == rank) w_own = w;
+      }
+      const float scale_own = Lsum > 0.f ? w_own / Lsum : 0.f;
+      if (rank == 0 && row < heads_here)
+        P.lse[static_cast<int64_t>(i) * P.num_heads + head0 + row] =
+            Lsum > 0.f ? (M + log2_approx(Lsum)) * kLn2 : -INFINITY;
+      const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
+      const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
+      const int owner = row / per, rr = row - owner * per;
+      const uint32_t dst = dsmem_addr(rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 4), owner);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {   // warp-uniform: one flag per CTA
+          tmem_ld32(o_lane + c0, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const int chunk = (c0 >> 2) + v;
+          const int phys = chunk ^ (rr & (kChunks - 1));
+          st_dsmem_f4(dst + phys * 16,
+                      make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
+                                  __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own));
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();                                      // every slice's weighted rows have arrived
+    if (tid < kSoftThreads) {
+      const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
+      const float* rx = reinterpret_cast<const float*>(smem + L::kKOff);
+      uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
+      const int n_items = (r1 - r0) * kChunks;
+      for (int idx = tid; idx < n_items; idx += kSoftThreads) {
+        const int rr = idx / kChunks, c = idx % kChunks;
+        const int phys = c ^ (rr & (kChunks - 1));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+          const float4 v = *reinterpret_cast<const float4*>(rx + ((s * per + rr) * D) + phys * 4);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r0 + rr) * D + 4 * c) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+      }
+    }
+  }
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 template <int D, bool kFp8>
@@ -1061,10 +1002,6 @@ cudaError_t launch_sparse_sink_attn(const AttnArgs& a, cudaStream_t stream) {
         !encode_pool(&P.tm_v_cmp, a.v_cmp, cmp_rows, a.head_dim))
       return cudaErrorInvalidValue;
   }
-  P.k_raw = reinterpret_cast<const uint8_t*>(a.k_raw);
-  P.v_raw = reinterpret_cast<const uint8_t*>(a.v_raw);
-  P.k_cmp = a.k_cmp_fp8 == nullptr ? reinterpret_cast<const uint8_t*>(a.k_cmp) : nullptr;
-  P.v_cmp = a.k_cmp_fp8 == nullptr ? reinterpret_cast<const uint8_t*>(a.v_cmp) : nullptr;
   P.n_queries = a.n_queries;
   P.num_heads = a.num_heads;
   P.raw_pages = a.raw_num_pages;
