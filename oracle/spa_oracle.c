@@ -508,13 +508,17 @@ void oracle_lse_merge(int32_t n_parts, const double* lse_parts, const double* o_
  *   dq = scale sum_j ds_j k_j, dk_j += scale ds_j q, dv_j += p_j dO,
  *   dsink_h += -p_c D (the sink's logit has no V, so its dp is 0).
  * dq is written ([n_rows, H, d]); dk/dv are ADDED into arrays shaped like
- * the pools ([pages * page_size, d]); dsink (may be NULL) is added into. */
+ * the pools ([pages * page_size, d]); dsink (may be NULL) is added into.
+ * The per-query contributions to dk/dv/dsink are added in query order
+ * whatever the thread count, so repeated calls give identical sums. */
 typedef struct {
     attn_job A;
     const uint16_t* dout;            /* BF16 bits [N, H, d], contiguous */
     const double* o_saved;           /* [N, H, d] or NULL */
     const double* lse_saved;         /* [N, H] or NULL */
     double *dq, *dk_raw, *dv_raw, *dk_cmp, *dv_cmp, *dsink;
+    int32_t next_commit;             /* the next row whose sums may be added */
+    pthread_cond_t turn;
 } bwd_job;
 
 static int one_query_bwd(bwd_job* G, int32_t r, double* kbuf, double* vbuf, double* s,
@@ -596,8 +600,11 @@ static void* bwd_worker(void* arg)
     int32_t cap = 0, d = J->d;
     double *kbuf = NULL, *vbuf = NULL, *s = NULL, *dkb = NULL, *dvb = NULL;
     int64_t* rowb = NULL; int* rawb = NULL;
-    double* dsink_loc = (double*)calloc((size_t)J->H, sizeof(double));
-    if (!dsink_loc) { pthread_mutex_lock(&J->lock); J->status = ORACLE_NO_MEMORY; pthread_mutex_unlock(&J->lock); return NULL; }
+    double* dsink_loc = (double*)malloc((size_t)J->H * sizeof(double));   /* this query's dsink */
+    if (!dsink_loc) {
+        pthread_mutex_lock(&J->lock); J->status = ORACLE_NO_MEMORY;
+        pthread_cond_broadcast(&G->turn); pthread_mutex_unlock(&J->lock); return NULL;
+    }
     for (;;) {
         pthread_mutex_lock(&J->lock);
         int32_t r = J->status ? J->n_rows : J->next_row++;
@@ -618,30 +625,36 @@ static void* bwd_worker(void* arg)
             rawb = (int*)malloc((size_t)cap * sizeof(int));
             if (!kbuf || !vbuf || !s || !dkb || !dvb || !rowb || !rawb) {
                 pthread_mutex_lock(&J->lock); J->status = ORACLE_NO_MEMORY;
-                pthread_mutex_unlock(&J->lock); break;
+                pthread_cond_broadcast(&G->turn); pthread_mutex_unlock(&J->lock); break;
             }
         }
+        for (int32_t h = 0; h < J->H; ++h) dsink_loc[h] = 0.0;
         int st = one_query_bwd(G, r, kbuf, vbuf, s, dkb, dvb, rowb, rawb, dsink_loc);
         pthread_mutex_lock(&J->lock);
         if (st) {
             if (!J->status) J->status = st;
+            pthread_cond_broadcast(&G->turn);
         } else {
-            /* this query's key-row gradients into the pool-shaped sums */
-            for (int32_t j = 0; j < n; ++j) {
-                double* dk = (rawb[j] ? G->dk_raw : G->dk_cmp) + rowb[j] * d;
-                double* dv = (rawb[j] ? G->dv_raw : G->dv_cmp) + rowb[j] * d;
-                for (int32_t e = 0; e < d; ++e) {
-                    dk[e] += dkb[(int64_t)j * d + e];
-                    dv[e] += dvb[(int64_t)j * d + e];
+            /* this query's key-row gradients into the pool-shaped sums, in
+             * query order: wait until every earlier row has been added */
+            while (G->next_commit != r && !J->status) pthread_cond_wait(&G->turn, &J->lock);
+            if (!J->status) {
+                for (int32_t j = 0; j < n; ++j) {
+                    double* dk = (rawb[j] ? G->dk_raw : G->dk_cmp) + rowb[j] * d;
+                    double* dv = (rawb[j] ? G->dv_raw : G->dv_cmp) + rowb[j] * d;
+                    for (int32_t e = 0; e < d; ++e) {
+                        dk[e] += dkb[(int64_t)j * d + e];
+                        dv[e] += dvb[(int64_t)j * d + e];
+                    }
                 }
+                if (G->dsink)
+                    for (int32_t h = 0; h < J->H; ++h) G->dsink[h] += dsink_loc[h];
+                ++G->next_commit;
+                pthread_cond_broadcast(&G->turn);
             }
         }
         pthread_mutex_unlock(&J->lock);
     }
-    pthread_mutex_lock(&J->lock);
-    if (G->dsink)
-        for (int32_t h = 0; h < J->H; ++h) G->dsink[h] += dsink_loc[h];
-    pthread_mutex_unlock(&J->lock);
     free(kbuf); free(vbuf); free(s); free(dkb); free(dvb); free(rowb); free(rawb); free(dsink_loc);
     return NULL;
 }
@@ -668,6 +681,8 @@ int oracle_sparse_sink_attn_bwd(
     G.A = A;
     G.dout = dout; G.o_saved = o_saved; G.lse_saved = lse_saved; G.dq = dq; G.dk_raw = dk_raw; G.dv_raw = dv_raw;
     G.dk_cmp = dk_cmp; G.dv_cmp = dv_cmp; G.dsink = dsink;
+    G.next_commit = 0;
+    pthread_cond_init(&G.turn, NULL);
     if (n_threads < 1) n_threads = 1;
     if (n_threads > 256) n_threads = 256;
     pthread_t tid[256];
@@ -676,5 +691,6 @@ int oracle_sparse_sink_attn_bwd(
         if (pthread_create(&tid[started], NULL, bwd_worker, &G) == 0) ++started;
     bwd_worker(&G);
     for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    pthread_cond_destroy(&G.turn);
     return G.A.status;
 }
