@@ -845,22 +845,24 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     // [r*per, (r+1)*per) of the output. After the first cluster barrier
     // every CTA reads all slices' (m, l) of its rows (one round trip of
     // distributed shared memory), scales its O rows by its weight and
-    // stores each row straight into its owner's idle K/V ring (posted
-    // stores, slot = the sender's rank); after the second barrier each owner
-    // sums its slots locally and writes BF16 O. No shared memory is read or
-    // written remotely after the second barrier, so no third one is needed.
-    // Every thread of every CTA reaches both barriers: every earlier wait in
-    // the kernel is bounded.
+    // stores each row as FP16 straight into its owner's idle K/V ring
+    // (posted remote stores, slot = the sender's rank; its own rows with
+    // local stores); after the second barrier each owner sums its slots in
+    // FP32 and writes BF16 O. A weighted row is at most max|v| in magnitude
+    // and FP16 keeps 11 bits, more than the BF16 output; the remote stores
+    // (about 12 bytes per clock per SM on B200) move half the bytes of FP32
+    // rows. No shared memory is read or written remotely after the second
+    // barrier, so no third one is needed. Every thread of every CTA reaches
+    // both barriers: every earlier wait in the kernel is bounded.
     const int rank = static_cast<int>(cluster_ctarank());
     const int i = static_cast<int>(blockIdx.x / S);
     const uint32_t ml_addr = sbase + L::kMergeOff;
-    const uint32_t rx_addr = sbase + L::kKOff;               // [S][per][D] FP32, 16-byte chunks swizzled by row
-    constexpr int kChunks = D / 4;                           // 16-byte chunks per row
+    const uint32_t rx_addr = sbase + L::kKOff;               // [S][per][D] FP16, 16-byte chunks swizzled by row
+    constexpr int kChunks = D / 8;                           // 16-byte chunks per row
     const int per = (128 + S - 1) / S;
-    // the slots (S * per <= 128 + S - 1 rows of D FP32) fill the K/V rings
-    // and may run on into the chunk tables, all idle by now
-    static_assert(L::kTabOff - L::kKOff + 2 * kChunkKeys * 4 >= (128 + kAttnMaxClusterSplits - 1) * D * 4,
-                  "receive slots fit the idle rings and tables");
+    // the slots (S * per <= 128 + S - 1 rows of D FP16) fit the idle K/V rings
+    static_assert(L::kTabOff - L::kKOff >= (128 + kAttnMaxClusterSplits - 1) * D * 2,
+                  "receive slots fit the idle rings");
     static_assert(L::kTabOff == L::kVOff + kStagesV * L::kTileBytes && L::kVOff == L::kKOff + kStagesK * L::kTileBytes,
                   "rings and tables are contiguous");
     __syncwarp();
@@ -889,7 +891,9 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
       const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
       const int owner = row / per, rr = row - owner * per;
-      const uint32_t dst = dsmem_addr(rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 4), owner);
+      const uint32_t slot = rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 2);
+      const uint32_t dst = dsmem_addr(slot, owner);
+      const bool local = owner == rank;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -901,12 +905,19 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           for (int cc = 0; cc < 32; ++cc) o[cc] = 0u;
         }
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const int chunk = (c0 >> 2) + v;
+        for (int v = 0; v < 4; ++v) {   // 8 columns per 16-byte chunk
+          const int chunk = (c0 >> 3) + v;
           const int phys = chunk ^ (rr & (kChunks - 1));
-          st_dsmem_f4(dst + phys * 16,
-                      make_float4(__uint_as_float(o[4 * v]) * scale_own, __uint_as_float(o[4 * v + 1]) * scale_own,
-                                  __uint_as_float(o[4 * v + 2]) * scale_own, __uint_as_float(o[4 * v + 3]) * scale_own));
+          uint32_t h[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            h[k] = pack_f16x2(__uint_as_float(o[8 * v + 2 * k]) * scale_own,
+                              __uint_as_float(o[8 * v + 2 * k + 1]) * scale_own);
+          if (local)
+            *reinterpret_cast<uint4*>(smem + (slot - sbase) + phys * 16) = make_uint4(h[0], h[1], h[2], h[3]);
+          else
+            st_dsmem_f4(dst + phys * 16, make_float4(__uint_as_float(h[0]), __uint_as_float(h[1]),
+                                                     __uint_as_float(h[2]), __uint_as_float(h[3])));
         }
       }
     }
@@ -914,22 +925,26 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     cluster_sync_all();                                      // every slice's weighted rows have arrived
     if (tid < kSoftThreads) {
       const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
-      const float* rx = reinterpret_cast<const float*>(smem + L::kKOff);
+      const uint8_t* rx = smem + L::kKOff;
       uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
       const int n_items = (r1 - r0) * kChunks;
       for (int idx = tid; idx < n_items; idx += kSoftThreads) {
         const int rr = idx / kChunks, c = idx % kChunks;
         const int phys = c ^ (rr & (kChunks - 1));
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int s = 0; s < S; ++s) {
-          const float4 v = *reinterpret_cast<const float4*>(rx + ((s * per + rr) * D) + phys * 4);
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
+          const uint4 v = *reinterpret_cast<const uint4*>(rx + ((s * per + rr) * D) * 2 + phys * 16);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_f16x2(w4[k]);
+            acc[2 * k] += f.x;
+            acc[2 * k + 1] += f.y;
+          }
         }
-        *reinterpret_cast<uint2*>(obase + static_cast<int64_t>(r0 + rr) * D + 4 * c) =
-            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        *reinterpret_cast<uint4*>(obase + static_cast<int64_t>(r0 + rr) * D + 8 * c) =
+            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                       pack_bf16x2(acc[6], acc[7]));
       }
     }
   }
