@@ -153,12 +153,12 @@ struct SoftSync {
 };
 
 // Bytes of the merge's receive slots [S][32 heads][widest column range]
-// FP32, the largest over 2..8 slices.
+// FP16, the largest over 2..8 slices.
 constexpr int merge_rx_bytes_max() {
   int m = 0;
   for (int S = 2; S <= kAttnMaxClusterSplits; ++S) {
-    const int per = (kD / S) & ~3;
-    const int b = S * kHT * (kD - (S - 1) * per) * 4;
+    const int per = (kD / S) & ~7;
+    const int b = S * kHT * (kD - (S - 1) * per) * 2;
     m = b > m ? b : m;
   }
   return m;
@@ -180,19 +180,21 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
     // Attention contract and dispatch metadata", Summary: the deterministic
     // (out, lse) merge): w_s = 2^(m_s - M) / L per head. CTA r owns columns
     // [r*per, ...) of d. Each CTA scales its O^T by its weights into its own
-    // shared memory as [head][d] FP32, then stores every 16-byte piece
-    // straight into its owner's receive slots (posted stores, slot = the
-    // sender's rank); after the second cluster barrier each owner sums its
-    // slots locally and writes BF16 O. Nothing is read or written remotely
+    // shared memory as [head][d] FP32, then stores every 8-column piece as
+    // FP16 (16 bytes) straight into its owner's receive slots (posted
+    // remote stores, slot = the sender's rank; its own columns with local
+    // stores); after the second cluster barrier each owner sums its slots
+    // in FP32 and writes BF16 O. FP16 keeps more bits than the BF16 output
+    // and halves the remote bytes. Nothing is read or written remotely
     // after that barrier, so no third one is needed.
     const int rank = static_cast<int>(cluster_ctarank());
     const int i = static_cast<int>(blockIdx.x / S);
-    const int per = (kD / S) & ~3;   // 16-byte pieces; the last rank takes the rest
+    const int per = (kD / S) & ~7;   // 8-column pieces; the last rank takes the rest
     const int own_e0 = rank * per, own_e1 = rank == S - 1 ? kD : own_e0 + per;
     const int span = kD - (S - 1) * per;   // the widest range (the last rank's)
     float* head_w = reinterpret_cast<float*>(smem + L::kHeadOff + 2 * kHT * 4);
     const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 8) != 0;
-    // receive slots [S][32 heads][span] FP32 after the K ring (idle by now)
+    // receive slots [S][32 heads][span] FP16 after the K ring (idle by now)
     static_assert(L::kPOff + 2 * L::kPBytes - L::kVOff >= merge_rx_bytes_max(), "receive slots fit the idle V ring and P");
     const uint32_t rx_addr = sbase + L::kVOff;
     __syncwarp();
@@ -240,32 +242,43 @@ __device__ __forceinline__ void cta_finish(const Params& P, bool soft, uint8_t* 
         for (int h = 0; h < kHT; ++h) wo[h * kD + 128 * b + tid] = __uint_as_float(o[h]) * w[h];
       }
       (*ss)();   // this CTA's scaled rows are in place
-      for (int item = tid; item < kHT * (kD / 4); item += kSoftThreads) {
-        const int h = item / (kD / 4), e = 4 * (item % (kD / 4));
+      for (int item = tid; item < kHT * (kD / 8); item += kSoftThreads) {
+        const int h = item / (kD / 8), e = 8 * (item % (kD / 8));
         const int owner = min(e / per, S - 1);
         const int e_rel = e - owner * per;
-        const float4 v = *reinterpret_cast<const float4*>(wo + h * kD + e);
-        st_dsmem_f4(dsmem_addr(rx_addr + static_cast<uint32_t>(((rank * kHT + h) * span + e_rel) * 4), owner), v);
+        const float4 a = *reinterpret_cast<const float4*>(wo + h * kD + e);
+        const float4 b = *reinterpret_cast<const float4*>(wo + h * kD + e + 4);
+        const uint4 v = make_uint4(pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b.x, b.y), pack_f16x2(b.z, b.w));
+        const uint32_t slot = rx_addr + static_cast<uint32_t>(((rank * kHT + h) * span + e_rel) * 2);
+        if (owner == rank)
+          *reinterpret_cast<uint4*>(smem + (slot - sbase)) = v;
+        else
+          st_dsmem_f4(dsmem_addr(slot, owner), make_float4(__uint_as_float(v.x), __uint_as_float(v.y),
+                                                           __uint_as_float(v.z), __uint_as_float(v.w)));
       }
     }
     __syncwarp();
     cluster_sync_all();   // every slice's pieces have arrived
     if (soft) {
-      const int n4 = (own_e1 - own_e0) / 4;
-      const float* rx = reinterpret_cast<const float*>(smem + L::kVOff);
-      for (int item = tid; item < kHT * n4; item += kSoftThreads) {
-        const int h = item / n4, e_rel = 4 * (item % n4);
+      const int n8 = (own_e1 - own_e0) / 8;
+      const uint8_t* rx = smem + L::kVOff;
+      for (int item = tid; item < kHT * n8; item += kSoftThreads) {
+        const int h = item / n8, e_rel = 8 * (item % n8);
         if (h >= heads_here) continue;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int s = 0; s < S; ++s) {
-          const float4 v = *reinterpret_cast<const float4*>(rx + (s * kHT + h) * span + e_rel);
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
+          const uint4 v = *reinterpret_cast<const uint4*>(rx + ((s * kHT + h) * span + e_rel) * 2);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_f16x2(w4[k]);
+            acc[2 * k] += f.x;
+            acc[2 * k + 1] += f.y;
+          }
         }
-        *reinterpret_cast<uint2*>(P.out + (static_cast<int64_t>(i) * P.num_heads + head0 + h) * kD + own_e0 + e_rel) =
-            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        *reinterpret_cast<uint4*>(P.out + (static_cast<int64_t>(i) * P.num_heads + head0 + h) * kD + own_e0 + e_rel) =
+            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                       pack_bf16x2(acc[6], acc[7]));
       }
     }
   }
