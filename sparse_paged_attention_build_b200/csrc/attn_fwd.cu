@@ -714,9 +714,12 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         if (row_ok)
           P.lse[static_cast<int64_t>(i) * P.num_heads + h] = l > 0.f ? (m + log2_approx(l)) * kLn2 : -INFINITY;
       } else if (P.cluster_merge) {
-        // this CTA's (m, l) rows for the cluster merge at the end; O stays
-        // in TMEM
-        reinterpret_cast<float2*>(smem + L::kMergeOff)[row] = make_float2(m, l);
+        // this CTA's (m, l) rows for the cluster merge at the end, into slot
+        // `split` of every CTA of the cluster (posted stores, so that after
+        // the first cluster barrier every (m, l) is local); O stays in TMEM
+        const uint32_t ml_slot = sbase + L::kMergeOff + static_cast<uint32_t>((d.split * 128 + row) * 8);
+#pragma unroll 1
+        for (int s = 0; s < S; ++s) st_dsmem_f2(dsmem_addr(ml_slot, s), make_float2(m, l));
         if (tid == 0) *reinterpret_cast<int*>(smem + L::kMiscOff + 12) = have_o ? 1 : 0;
       } else {
         // partial result of this slice (no normalisation); the last slice
@@ -843,8 +846,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
     // Summary: the deterministic (out, lse) merge). CTA r owns rows
     // [r*per, (r+1)*per) of the output. After the first cluster barrier
-    // every CTA reads all slices' (m, l) of its rows (one round trip of
-    // distributed shared memory), scales its O rows by its weight and
+    // every CTA has all slices' (m, l) of its rows (each slice stored its
+    // own into every CTA before the barrier), scales its O rows by its weight and
     // stores each row as FP16 straight into its owner's idle K/V ring
     // (posted remote stores, slot = the sender's rank; its own rows with
     // local stores); after the second barrier each owner sums its slots in
@@ -856,7 +859,8 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     // both barriers: every earlier wait in the kernel is bounded.
     const int rank = static_cast<int>(cluster_ctarank());
     const int i = static_cast<int>(blockIdx.x / S);
-    const uint32_t ml_addr = sbase + L::kMergeOff;
+    const float2* ml_all = reinterpret_cast<const float2*>(smem + L::kMergeOff);   // [S][128] (m, l)
+    static_assert(kAttnMaxClusterSplits * 128 * 8 <= kAttnMaxSplits * 128 * 4, "(m, l) slots fit the merge area");
     const uint32_t rx_addr = sbase + L::kKOff;               // [S][per][D] FP16, 16-byte chunks swizzled by row
     constexpr int kChunks = D / 8;                           // 16-byte chunks per row
     const int per = (128 + S - 1) / S;
@@ -872,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       float2 ml[kAttnMaxClusterSplits];
 #pragma unroll
       for (int s = 0; s < kAttnMaxClusterSplits; ++s)
-        ml[s] = s < S ? ld_dsmem_f2(dsmem_addr(ml_addr + row * 8, s)) : make_float2(-INFINITY, 0.f);
+        ml[s] = s < S ? ml_all[s * 128 + row] : make_float2(-INFINITY, 0.f);
       float M = -INFINITY;
 #pragma unroll
       for (int s = 0; s < kAttnMaxClusterSplits; ++s)

@@ -174,6 +174,10 @@ __device__ __forceinline__ void st_dsmem_f4(uint32_t addr, float4 v) {
                : "memory");
 }
 
+__device__ __forceinline__ void st_dsmem_f2(uint32_t addr, float2 v) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
+
 // Every thread of every CTA of the cluster, convergently: shared-memory
 // writes before it are visible to the whole cluster after it.
 __device__ __forceinline__ void cluster_sync_all() {
