@@ -377,6 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_sink_attn_d512_kernel(cons
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // everything above is private to the CTA; every global read below may
+  // depend on the previous kernel of the stream (the sets, the pools, Q)
+  grid_dep_wait();
   SoftSync ss{B.soft_sync, abort_flag, P.dev_status, P.wait_ns};
 
   // one setmaxnreg per warpgroup, dominating all of its roles
@@ -871,16 +874,19 @@ cudaError_t launch_sparse_sink_attn_d512(const AttnArgs& a, cudaStream_t stream)
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Layout::kBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start early
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (a.num_splits > 1) {
     // one unit per CTA, the slices of a query in one cluster
     cfg.gridDim = dim3(static_cast<unsigned>(units), head_tiles);
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(a.num_splits);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(a.num_splits);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   } else {
     // persistent: one CTA per SM, units strided over the CTAs
     const int64_t slots = std::max<int64_t>(1, static_cast<int64_t>(device_sm_count()) / head_tiles);

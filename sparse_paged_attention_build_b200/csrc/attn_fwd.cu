@@ -246,6 +246,9 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // everything above is private to the CTA; every global read below may
+  // depend on the previous kernel of the stream (the sets, the pools, Q)
+  grid_dep_wait();
 
   if (warp == kResolverWarp) {
     // ================================================= resolver
@@ -973,20 +976,32 @@ cudaError_t launch_d(const Params& P, int head_tiles, cudaStream_t stream) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = L::kBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(P.num_splits);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start early
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t err = cudaLaunchKernelEx(&cfg, sparse_sink_attn_kernel<D, kFp8>, P);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }
   const int64_t slots = std::max<int64_t>(1, (2 * static_cast<int64_t>(device_sm_count())) / head_tiles);
-  dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
-  sparse_sink_attn_kernel<D, kFp8><<<grid, kThreads, L::kBytes, stream>>>(P);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(units, slots)), head_tiles);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start early
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, sparse_sink_attn_kernel<D, kFp8>, P);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

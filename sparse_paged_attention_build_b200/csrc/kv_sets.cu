@@ -194,6 +194,9 @@ __global__ void __launch_bounds__(kSetsWarps * 32) build_kv_sets_kernel(const Se
   int32_t* buf = sets_smem + warp * P.buf_words;
   int64_t* prefix = reinterpret_cast<int64_t*>(sets_smem + kSetsWarps * P.buf_words);
   if (threadIdx.x == 0) s_tile = atomicAdd(P.tile_ticket, 1u);
+  // the attention launched next may start its setup now (it waits for this
+  // grid to finish before it reads the sets)
+  grid_dep_launch();
   __syncthreads();
   const uint32_t tile = s_tile;
   // A ticket past this launch's grid only comes from another launch using

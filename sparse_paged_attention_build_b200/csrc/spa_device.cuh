@@ -224,6 +224,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
+// ---------------------------------------------------------------- launch order
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start (set up shared memory, barriers, TMEM) while the
+// previous kernel of the stream still runs. grid_dep_wait() returns once
+// that kernel has completed and its writes are visible (at once if it has);
+// grid_dep_launch() lets the next such kernel start before this one ends.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 // TMEM allocation: executed by one whole warp; the TMEM address lands in
 // shared memory at `slot`.
