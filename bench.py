@@ -535,6 +535,13 @@ def run_bwd(args, rank, local_rank, world):
     dO = torch.from_numpy(workloads.make_dout(w).view(np.int16)).cuda().view(torch.bfloat16)
     torch.cuda.synchronize()
     pairs = int(b.indptr[-1].item()) * w.H
+    # FP32 reduction bytes per call: each 64-key tile of a unit adds one
+    # [64 keys x d] block into dK and one into dV (bulk reductions), and
+    # every slice of a query adds its [H x d] block into dq
+    set_sizes = np.diff(b.indptr.cpu().numpy().astype(np.int64))
+    splits_used = args.splits if args.splits > 0 else spa.choose_splits(w.N, w.H, 0)
+    red_dkdv = int(np.sum((set_sizes + 63) // 64)) * 2 * 64 * w.d * 4
+    red_dq = int(splits_used) * w.N * w.H * w.d * 4
     st = spa.new_status()
     grads = spa.sparse_sink_attn_bwd(b.q, b.k_raw, b.v_raw, b.pt_raw, b.req, b.indptr, b.indices, b.sink,
                                      w.scale, out, lse, dO, k_cmp=b.k_cmp, v_cmp=b.v_cmp, pt_cmp=b.pt_cmp,
@@ -578,7 +585,8 @@ def run_bwd(args, rank, local_rank, world):
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{w.name}: {workloads.DESCRIPTIONS[w.name]}", "pairs": int(pairs),
                        "num_splits": args.splits, "l2": "256 MB buffer written between timed steps (L2 flush)",
-                       "gradient zeroing": "not timed (the call adds into the gradients)"},
+                       "gradient zeroing": "not timed (the call adds into the gradients)",
+                       "reduction_bytes": {"dk_dv": red_dkdv, "dq": red_dq, "total": red_dkdv + red_dq}},
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": tflops / pk["bf16_tflops"], "peak_source": f"{pk_kind} BF16 burst",
                          "kernel": "sparse_sink_attn_bwd_kernel", "algorithmic_flops": flops},
