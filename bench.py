@@ -211,6 +211,19 @@ def run_reference(args, rank, world):
     return 0
 
 
+def sets_mode(w, args):
+    """Where the step builds its key sets: "inline" (inside the attention
+    kernel) for workloads without a top-k list and with a BF16 cache when
+    --sets is auto, else as asked."""
+    if args.sets != "auto":
+        return args.sets
+    return "inline" if (w.topk is None and w.k_cmp_fp8 is None) else "csr"
+
+
+SETS_TEXT = {"csr": "spa_build_kv_sets, then the attention reads the CSR sets",
+             "inline": "built inside the attention kernel (spa_sparse_sink_attn_fwd_all_groups)"}
+
+
 def config_of(w, world, nnz, fp8_path=None):
     from sparse_paged_attention_build_b200 import workloads
     c = {"workload": f"{w.name}: {workloads.DESCRIPTIONS[w.name]}", "n_queries": w.N, "heads": w.H,
@@ -235,6 +248,10 @@ def main():
                     help="c1..c5: the 128-head configurations; f1, f2: the 32-head, 512-wide DSV4-Flash shape")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--sets", default="auto", choices=["auto", "csr", "inline"],
+                    help="csr: spa_build_kv_sets, then the attention reads the CSR sets; inline: sets "
+                         "without a top-k list built inside the attention kernel; auto: inline where the "
+                         "workload has no top-k list and a BF16 cache")
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
                     help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
     ap.add_argument("--op", default="path", choices=["path", "kv_write", "bwd", "unpack_d512"],
@@ -293,7 +310,7 @@ def main():
                "pairs_per_s": dres["value"], "roofline": dres["roofline"], "clocks": dres["clocks"],
                "num_splits": dres["num_splits"], "gpu_launches": dres["gpu_launches"],
                "device_status": dres["status"], "config": config_of(wd, world, dres["nnz"], args.fp8_path),
-               "e2e": dres["e2e"]}
+               "sets": SETS_TEXT[dres["sets"]], "e2e": dres["e2e"]}
         if dres["e2e"] is not None:
             dec["e2e"]["tok_per_s"] = dres["total_queries"] * dres["e2e"]["value"] / max(dres["value"], 1e-30)
 
@@ -310,7 +327,7 @@ def main():
             "tflops": res["tflops"],
             "roofline": res["roofline"],
             "clocks": res["clocks"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
-            "device_status": res["status"],
+            "device_status": res["status"], "sets": SETS_TEXT[res["sets"]],
         }
         if w.kind == "decode":
             line["tok_per_s"] = res["total_queries"] / (res["elapsed_ms"] / 1e3)
@@ -333,8 +350,10 @@ def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dis
     from sparse_paged_attention_build_b200.pipeline import DeviceBatch
 
     decode = w.kind == "decode"
-    b0 = DeviceBatch(w, num_splits=splits, fp8_path=args.fp8_path)
+    sets = sets_mode(w, args)
+    b0 = DeviceBatch(w, num_splits=splits, fp8_path=args.fp8_path, sets=sets)
     stream = torch.cuda.current_stream()
+    b0.build_sets()   # the CSR sets, for the counts below (inside the step only on the csr path)
     b0.step()
     torch.cuda.synchronize()
     nnz = b0.nnz()
@@ -348,13 +367,18 @@ def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dis
     # The step is replayed from two CUDA graphs (set build + FP8 decode, then
     # attention) so that host-side launch cost does not enter the device
     # timings; the graphs launch exactly the library's kernels.
-    g_front, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    # (With the sets built inside the attention kernel and no FP8 decode, the
+    # first graph would be empty: the step is the attention alone.)
+    has_front = not b0.inline_sets or (b0.fp8 and not b0.fused)
+    g_front, g_attn = (torch.cuda.CUDAGraph() if has_front else None), torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
-        with torch.cuda.graph(g_front, stream=cap):
-            b0.build_sets()
-            b0.dequant()
+        if has_front:
+            with torch.cuda.graph(g_front, stream=cap):
+                if not b0.inline_sets:
+                    b0.build_sets()
+                b0.dequant()
         with torch.cuda.graph(g_attn, stream=cap):
             b0.attend()
     stream.wait_stream(cap)
@@ -363,7 +387,8 @@ def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dis
     for s in range(warmup):
         if flush is not None:
             flush.zero_()
-        g_front.replay()
+        if has_front:
+            g_front.replay()
         g_attn.replay()
     torch.cuda.synchronize()
 
@@ -380,7 +405,8 @@ def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dis
         if flush is not None:
             flush.zero_()
         ev[s][0].record(stream)
-        g_front.replay()
+        if has_front:
+            g_front.replay()
         ev[s][1].record(stream)
         g_attn.replay()
         ev[s][2].record(stream)
@@ -440,7 +466,7 @@ def measure_path(w, args, steps, warmup, splits, local_rank, world, barrier, dis
     return {"value": value, "elapsed_ms": elapsed_ms, "attn_ms": attn_ms, "nnz": nnz,
             "tflops": total_flops / (elapsed_ms / 1e3) / 1e12, "roofline": roofline, "clocks": clocks,
             "e2e": e2e, "gpu_launches": kernels_per_step * steps, "status": status, "steps": steps,
-            "total_queries": total_queries, "num_splits": splits_used}
+            "total_queries": total_queries, "num_splits": splits_used, "sets": sets}
 
 
 def run_kv_write(args, rank, local_rank, world):

@@ -260,6 +260,40 @@ int spa_sparse_sink_attn_fwd(
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * 3a. spa_sparse_sink_attn_fwd_all_groups -- spa_sparse_sink_attn_fwd over
+ * the sets spa_build_kv_sets builds without a top-k list, built inside the
+ * attention kernel from the positions instead of read from CSR arrays.
+ *
+ * Same sets ("Roadmap item 24", "Contracts and lifetime"; the block-level
+ * test's layer types: ratio 0 = the window alone, 128 = HCA, every complete
+ * group): for query i at position p = pos[i],
+ *   set_i = ascending({ g : 0 <= g < floor((p+1)/ratio) }      (ratio > 0)
+ *                     U { SPA_WINDOW_TAG | t : max(0, p-W+1) <= t <= p })
+ * The keys and their order are those of spa_build_kv_sets, so O and LSE are
+ * bit-identical to spa_build_kv_sets followed by spa_sparse_sink_attn_fwd
+ * with the same num_splits. In the decode timeline of the block-level test
+ * the set build precedes the core; here it costs no launch and no round
+ * trip through indptr/indices.
+ *
+ * Arguments as for spa_sparse_sink_attn_fwd, without indptr/indices, plus:
+ * pos      int32 [n_queries], 0 <= pos < 2^30 (else SPA_DEV_BAD_INDEX and an
+ *          empty set for that query)
+ * window   W >= 1
+ * ratio    0, 4 or 128; ratio > 0 needs the compressed pool (k_cmp, v_cmp,
+ *          pt_cmp non-NULL)
+ * ---------------------------------------------------------------------- */
+int spa_sparse_sink_attn_fwd_all_groups(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+    int32_t num_heads, int32_t head_dim,
+    const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+    const int32_t* pt_raw, int32_t pt_raw_cols,
+    const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages, int32_t cmp_page_size,
+    const int32_t* pt_cmp, int32_t pt_cmp_cols,
+    const int32_t* req, int32_t n_requests, const int32_t* pos, int32_t window, int32_t ratio,
+    const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
+    void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * 3b. spa_sparse_sink_attn_fwd_fp8 -- the same attention over a mixed
  * cache whose compressed pool is stored in FP8, decoded inside the gather.
  *

@@ -69,6 +69,12 @@ def _load():
         P, P, i64, i32, P, i32,
         P, i32, P, P, P, ctypes.c_float, P, P, i32, P, sz, P, P]
     L.spa_sparse_sink_attn_fwd.restype = ctypes.c_int
+    L.spa_sparse_sink_attn_fwd_all_groups.argtypes = [
+        P, i64, i64, i32, i32, i32,
+        P, P, i64, i32, P, i32,
+        P, P, i64, i32, P, i32,
+        P, i32, P, i32, i32, P, ctypes.c_float, P, P, i32, P, sz, P, P]
+    L.spa_sparse_sink_attn_fwd_all_groups.restype = ctypes.c_int
     L.spa_sparse_sink_attn_fwd_fp8.argtypes = [
         P, i64, i64, i32, i32, i32,
         P, P, i64, i32, P, i32,
@@ -234,6 +240,48 @@ def sparse_sink_attn_fwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
         1 if k_cmp is None else k_cmp.shape[1],
         _p(None if pt_cmp is None else pt_cmp.contiguous()), 0 if pt_cmp is None else pt_cmp.shape[1],
         _p(req.contiguous()), pt_raw.shape[0], _p(indptr.contiguous()), _p(indices.contiguous()),
+        _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
+        _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
+    return out, lse
+
+
+def sparse_sink_attn_fwd_all_groups(q, k_raw, v_raw, pt_raw, req, pos, window, ratio, sink, scale,
+                                    k_cmp=None, v_cmp=None, pt_cmp=None, out=None, lse=None, num_splits=0,
+                                    workspace=None, dev_status=None, stream=None):
+    """sparse_sink_attn_fwd over the sets spa_build_kv_sets builds without a
+    top-k list (every complete ratio-`ratio` group, then the window of
+    `window` tokens), built inside the kernel from pos (int32 [N])."""
+    _need(q, "q", torch.bfloat16)
+    for name, t in (("k_raw", k_raw), ("v_raw", v_raw)):
+        _need(t, name, torch.bfloat16)
+        assert t.is_contiguous(), name
+    for name, t in (("pt_raw", pt_raw), ("req", req), ("pos", pos)):
+        _need(t, name, torch.int32)
+    N, H, d = q.shape
+    if q.stride(2) != 1:
+        raise ValueError("q's last dimension must be contiguous")
+    if pt_cmp is not None:
+        _need(pt_cmp, "pt_cmp", torch.int32)
+        _need(k_cmp, "k_cmp", torch.bfloat16)
+        _need(v_cmp, "v_cmp", torch.bfloat16)
+        assert k_cmp.is_contiguous() and v_cmp.is_contiguous()
+    if sink is not None:
+        _need(sink, "sink", torch.float32)
+    if out is None:
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((N, H), dtype=torch.float32, device=q.device)
+    ws_bytes = attn_workspace_size(N, H, d, num_splits)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    pt_raw = pt_raw.contiguous()
+    _check("spa_sparse_sink_attn_fwd_all_groups", lib.spa_sparse_sink_attn_fwd_all_groups(
+        _p(q), q.stride(0), q.stride(1), N, H, d,
+        _p(k_raw), _p(v_raw), k_raw.shape[0], k_raw.shape[1], _p(pt_raw), pt_raw.shape[1],
+        _p(k_cmp), _p(v_cmp), 0 if k_cmp is None else k_cmp.shape[0],
+        1 if k_cmp is None else k_cmp.shape[1],
+        _p(None if pt_cmp is None else pt_cmp.contiguous()), 0 if pt_cmp is None else pt_cmp.shape[1],
+        _p(req.contiguous()), pt_raw.shape[0], _p(pos.contiguous()), int(window), int(ratio),
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
     return out, lse

@@ -313,14 +313,15 @@ int attn_check(const spa::AttnArgs& a, int32_t requested_splits) {
   if (a.q == nullptr) return fail(SPA_ERR_INVALID_ARG, "q must be non-NULL");
   if (a.k_raw == nullptr || a.v_raw == nullptr || a.pt_raw == nullptr)
     return fail(SPA_ERR_INVALID_ARG, "k_raw, v_raw and pt_raw must be non-NULL");
-  if (a.req == nullptr || a.indptr == nullptr || a.indices == nullptr)
+  if (a.req == nullptr) return fail(SPA_ERR_INVALID_ARG, "req must be non-NULL");
+  if (a.set_pos == nullptr && (a.indptr == nullptr || a.indices == nullptr))
     return fail(SPA_ERR_INVALID_ARG, "req, indptr and indices must be non-NULL");
   if (!aligned(a.q, 16) || (a.q_stride_tok * 2) % 16 != 0 || (a.q_stride_head * 2) % 16 != 0)
     return fail(SPA_ERR_ALIGNMENT, "q base and strides must be 16-byte multiples");
   if (!aligned(a.k_raw, 16) || !aligned(a.v_raw, 16) || !aligned(a.k_cmp, 16) || !aligned(a.v_cmp, 16) ||
       !aligned(a.k_cmp_fp8, 16) || !aligned(a.v_cmp_fp8, 16))
     return fail(SPA_ERR_ALIGNMENT, "K/V pools must be 16-byte aligned");
-  if (!aligned(a.sink, 4) || !aligned(a.req, 4) || !aligned(a.indptr, 4) ||
+  if (!aligned(a.sink, 4) || !aligned(a.req, 4) || !aligned(a.indptr, 4) || !aligned(a.set_pos, 4) ||
       !aligned(a.indices, 4) || !aligned(a.pt_raw, 4) || !aligned(a.pt_cmp, 4) || !aligned(a.k_cmp_scale, 4) ||
       !aligned(a.v_cmp_scale, 4))
     return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
@@ -416,6 +417,35 @@ int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
                               dev_status);
   a.k_cmp = k_cmp;
   a.v_cmp = v_cmp;
+  return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spa_sparse_sink_attn_fwd_all_groups(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head,
+                                        int32_t n_queries, int32_t num_heads, int32_t head_dim,
+                                        const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages,
+                                        int32_t raw_page_size, const int32_t* pt_raw, int32_t pt_raw_cols,
+                                        const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages,
+                                        int32_t cmp_page_size, const int32_t* pt_cmp, int32_t pt_cmp_cols,
+                                        const int32_t* req, int32_t n_requests, const int32_t* pos,
+                                        int32_t window, int32_t ratio, const float* sink, float scale,
+                                        uint16_t* out, float* lse, int32_t num_splits, void* workspace,
+                                        size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
+  if (window < 1) return fail(SPA_ERR_INVALID_ARG, "window must be >= 1");
+  if (ratio != 0 && ratio != 4 && ratio != 128) return fail(SPA_ERR_UNSUPPORTED, "ratio must be 0, 4 or 128");
+  if (ratio > 0 && n_queries > 0 && (pt_cmp == nullptr || k_cmp == nullptr || v_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "ratio > 0 needs the compressed pool (k_cmp, v_cmp, pt_cmp)");
+  if (pt_cmp != nullptr && n_queries > 0 && (k_cmp == nullptr || v_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
+  if (pos == nullptr && n_queries > 0) return fail(SPA_ERR_INVALID_ARG, "pos must be non-NULL");
+  spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
+                              raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
+                              pt_cmp_cols, req, n_requests, nullptr, nullptr, sink, scale, out, lse, workspace,
+                              dev_status);
+  a.k_cmp = k_cmp;
+  a.v_cmp = v_cmp;
+  a.set_pos = pos;
+  a.set_window = window;
+  a.set_ratio = ratio;
   return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -44,16 +44,23 @@ __device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) /
 // + lane + 32, ...; the loads of each phase are issued together so the
 // chunk costs two round trips, not two per key. Prm holds the page tables
 // and pool sizes.
+// With inl_groups >= 0 the keys are not read from `indices` but are the
+// set's closed form: position k of the set is group k below inl_groups and
+// window token inl_wstart + k - inl_groups after it (key_base is then the
+// chunk's position in the set).
 template <int kParts = 1, class Prm>
 __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t nkeys, uint32_t* tab,
-                              int lane, int part = 0) {
+                              int lane, int part = 0, int32_t inl_groups = -1, int32_t inl_wstart = 0) {
   constexpr int kPer = kChunkKeys / kParts / 32;
   const int k0 = part * (kChunkKeys / kParts);
   int32_t key[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int k = k0 + lane + 32 * e;
-    key[e] = k < nkeys ? __ldg(P.indices + key_base + k) : -2;
+    const int32_t at = key_base + k;
+    key[e] = k >= nkeys ? -2
+             : inl_groups < 0 ? __ldg(P.indices + at)
+             : at < inl_groups ? at : (SPA_WINDOW_TAG | (inl_wstart + at - inl_groups));
   }
   int32_t page[kPer];
 #pragma unroll
@@ -113,9 +120,20 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
   for (int64_t u = u0; u < u_end && !*abort_flag; u += step) {
     const int i = static_cast<int>(u / S);
     const int split = static_cast<int>(u - static_cast<int64_t>(i) * S);
-    const int32_t set_begin = __ldg(P.indptr + i);
-    int32_t set_len = __ldg(P.indptr + i + 1) - set_begin;
+    int32_t set_begin = 0, set_len, inl_groups = -1, inl_wstart = 0;
     const int32_t b = __ldg(P.req + i);
+    if (P.set_pos != nullptr) {
+      // the set built here: every complete group, then the window
+      const int32_t pos = __ldg(P.set_pos + i);
+      const bool pos_ok = pos >= 0 && pos < SPA_WINDOW_TAG;
+      const int32_t wn = pos_ok ? min(P.set_window, pos + 1) : 0;
+      inl_groups = (pos_ok && P.set_ratio > 0) ? (pos + 1) / P.set_ratio : 0;
+      inl_wstart = pos + 1 - wn;
+      set_len = pos_ok ? inl_groups + wn : -1;
+    } else {
+      set_begin = __ldg(P.indptr + i);
+      set_len = __ldg(P.indptr + i + 1) - set_begin;
+    }
     if (set_len < 0 || b < 0 || b >= P.n_requests) {
       if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
       set_len = 0;
@@ -143,7 +161,7 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
       const int slot = c & 1;
       if (!mbar_wait(tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns)) return;
       const int32_t n = max(0, min(kChunkKeys, key_hi - k0));   // 0: an empty slice
-      resolve_chunk<kParts>(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane, part);
+      resolve_chunk<kParts>(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane, part, inl_groups, inl_wstart);
       if (lane == 0 && part == 0) {
         ChunkDesc& d = desc[slot];
         d.i = i;

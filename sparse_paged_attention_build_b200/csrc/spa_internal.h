@@ -63,6 +63,10 @@ struct AttnArgs {
   int32_t n_requests;
   const int32_t* indptr;
   const int32_t* indices;
+  // sets built inside the kernel (NULL: read indptr/indices): positions,
+  // window W and ratio; the set is every complete group, then the window
+  const int32_t* set_pos = nullptr;
+  int32_t set_window = 0, set_ratio = 0;
   const float* sink;
   float scale;
   uint16_t* out;

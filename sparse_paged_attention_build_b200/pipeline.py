@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 from . import (build_kv_sets, dequant_fp8_pages, kv_sets_capacity, sparse_sink_attn_fwd, sparse_sink_attn_fwd_fp8,
-               attn_workspace_size, new_status, read_status)
+               sparse_sink_attn_fwd_all_groups, attn_workspace_size, new_status, read_status)
 from . import lib
 
 
@@ -28,8 +28,16 @@ def _dev(a, dtype=None, device="cuda"):
 class DeviceBatch:
     """A workload resident in device memory, with its outputs."""
 
-    def __init__(self, w, device="cuda", num_splits=0, fp8_path="decode"):
+    def __init__(self, w, device="cuda", num_splits=0, fp8_path="decode", sets="csr"):
         self.w = w
+        # "csr": the sets are built by spa_build_kv_sets, then read by the
+        # attention; "inline": sets without a top-k list are built inside the
+        # attention kernel (spa_sparse_sink_attn_fwd_all_groups)
+        if sets not in ("csr", "inline"):
+            raise ValueError("sets is 'csr' or 'inline'")
+        if sets == "inline" and (w.topk is not None or w.k_cmp_fp8 is not None):
+            raise ValueError("sets built inside the kernel need a workload without top-k and a BF16 cache")
+        self.inline_sets = sets == "inline"
         self.device = device
         bf16 = torch.bfloat16
         self.q = _dev(w.q.view(np.int16), bf16, device)
@@ -95,6 +103,13 @@ class DeviceBatch:
                                      lse=self.lse, num_splits=self.num_splits, workspace=self.attn_ws,
                                      dev_status=self.status, stream=stream, fp8_format=self.w.fp8_format)
             return
+        if self.inline_sets:
+            sparse_sink_attn_fwd_all_groups(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.pos, w.W,
+                                            w.ratio, self.sink, w.scale, k_cmp=self.k_cmp, v_cmp=self.v_cmp,
+                                            pt_cmp=self.pt_cmp, out=self.out, lse=self.lse,
+                                            num_splits=self.num_splits, workspace=self.attn_ws,
+                                            dev_status=self.status, stream=stream)
+            return
         sparse_sink_attn_fwd(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.indptr,
                              self.indices, self.sink, w.scale, k_cmp=self.k_cmp, v_cmp=self.v_cmp,
                              pt_cmp=self.pt_cmp, out=self.out, lse=self.lse,
@@ -102,8 +117,10 @@ class DeviceBatch:
                              dev_status=self.status, stream=stream)
 
     def step(self, stream=None):
-        """The whole hot path: sets, decode (mixed cache), attention."""
-        self.build_sets(stream)
+        """The whole hot path: sets, decode (mixed cache), attention (the
+        sets inside the attention kernel with sets="inline")."""
+        if not self.inline_sets:
+            self.build_sets(stream)
         self.dequant(stream)
         self.attend(stream)
 
@@ -117,9 +134,10 @@ class DeviceBatch:
         return int(lib.spa_sparse_sink_attn_choose_splits(self.w.N, self.w.H, 0))
 
     def kernels_per_step(self) -> int:
-        return 1 + (2 if self.fp8 and not self.fused else 0) + 1
+        return (0 if self.inline_sets else 1) + (2 if self.fp8 and not self.fused else 0) + 1
 
     def nnz(self) -> int:
+        """Keys in all sets (from the CSR arrays: run build_sets first)."""
         return int(self.indptr[-1].item())
 
     def status_word(self) -> int:
