@@ -49,7 +49,7 @@ def _no_topk(w, ratio=None):
 
 @pytest.mark.parametrize("name,shrink,splits", [
     ("c4", 1, 0), ("c4", 1, 1), ("c4", 4, 2), ("c4", 8, 3), ("c4", 16, 12),   # ratio 128 (HCA)
-    ("c2", 8, 0), ("c2", 8, 4),                                              # ratio 0 (window only)
+    ("c2", 1, 0), ("c2", 8, 4),                                              # ratio 0 (window only)
 ])
 def test_inline_sets_bit_identical_to_csr(spa, name, shrink, splits):
     from sparse_paged_attention_build_b200 import workloads
