@@ -212,16 +212,19 @@ def run_reference(args, rank, world):
 
 
 def sets_mode(w, args):
-    """Where the step builds its key sets: "inline" (inside the attention
-    kernel) for workloads without a top-k list and with a BF16 cache when
-    --sets is auto, else as asked."""
+    """Where the step builds its key sets when --sets is auto: "inline"
+    (inside the attention kernel) where that is the cheaper place (see
+    pipeline.prefer_inline_sets), else "csr"; otherwise as asked."""
+    import torch
+    from sparse_paged_attention_build_b200.pipeline import prefer_inline_sets
     if args.sets != "auto":
         return args.sets
-    return "inline" if (w.topk is None and w.k_cmp_fp8 is None) else "csr"
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return "inline" if prefer_inline_sets(w, args.fp8_path, args.splits, sms) else "csr"
 
 
 SETS_TEXT = {"csr": "spa_build_kv_sets, then the attention reads the CSR sets",
-             "inline": "built inside the attention kernel (spa_sparse_sink_attn_fwd_all_groups)"}
+             "inline": "built inside the attention kernel (spa_sparse_sink_attn_fwd_inline_sets)"}
 
 
 def config_of(w, world, nnz, fp8_path=None):
@@ -249,9 +252,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--sets", default="auto", choices=["auto", "csr", "inline"],
-                    help="csr: spa_build_kv_sets, then the attention reads the CSR sets; inline: sets "
-                         "without a top-k list built inside the attention kernel; auto: inline where the "
-                         "workload has no top-k list and a BF16 cache")
+                    help="csr: spa_build_kv_sets, then the attention reads the CSR sets; inline: the "
+                         "sets built inside the attention kernel; auto: inline without a top-k list, or "
+                         "with one for batches of at most 8 units per SM")
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
                     help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
     ap.add_argument("--op", default="path", choices=["path", "kv_write", "bwd", "unpack_d512"],

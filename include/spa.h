@@ -260,36 +260,47 @@ int spa_sparse_sink_attn_fwd(
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * 3a. spa_sparse_sink_attn_fwd_all_groups -- spa_sparse_sink_attn_fwd over
- * the sets spa_build_kv_sets builds without a top-k list, built inside the
- * attention kernel from the positions instead of read from CSR arrays.
+ * 3a. spa_sparse_sink_attn_fwd_inline_sets -- spa_sparse_sink_attn_fwd over
+ * the sets spa_build_kv_sets builds, built inside the attention kernel from
+ * the builder's own inputs (positions, top-k rows, W, ratio) instead of read
+ * from CSR arrays.
  *
- * Same sets ("Roadmap item 24", "Contracts and lifetime"; the block-level
- * test's layer types: ratio 0 = the window alone, 128 = HCA, every complete
- * group): for query i at position p = pos[i],
- *   set_i = ascending({ g : 0 <= g < floor((p+1)/ratio) }      (ratio > 0)
- *                     U { SPA_WINDOW_TAG | t : max(0, p-W+1) <= t <= p })
+ * Same sets as section 1 ("Roadmap item 24", "Contracts and lifetime"; the
+ * block-level test's layer types and its "Validation" rule on top-k): for
+ * query i at position p = pos[i] and G = floor((p+1)/ratio),
+ *   groups = none (ratio 0); { g : 0 <= g < G } (topk == NULL);
+ *            { topk[i][j] : 0 <= topk[i][j] < G }, repeats removed (else)
+ *   set_i  = ascending(groups U { SPA_WINDOW_TAG | t : max(0, p-W+1) <= t <= p })
  * The keys and their order are those of spa_build_kv_sets, so O and LSE are
  * bit-identical to spa_build_kv_sets followed by spa_sparse_sink_attn_fwd
  * with the same num_splits. In the decode timeline of the block-level test
  * the set build precedes the core; here it costs no launch and no round
- * trip through indptr/indices.
+ * trip through indptr/indices. A top-k row is reduced to its sorted groups
+ * by the kernel's resolver warp once per (query, slice) unit, which costs a
+ * CTA a few microseconds per unit: for large batches with top-k rows the
+ * separate spa_build_kv_sets is the cheaper place.
  *
  * Arguments as for spa_sparse_sink_attn_fwd, without indptr/indices, plus:
- * pos      int32 [n_queries], 0 <= pos < 2^30 (else SPA_DEV_BAD_INDEX and an
- *          empty set for that query)
- * window   W >= 1
- * ratio    0, 4 or 128; ratio > 0 needs the compressed pool (k_cmp, v_cmp,
- *          pt_cmp non-NULL)
+ * pos        int32 [n_queries], 0 <= pos < 2^30 (else SPA_DEV_BAD_INDEX and
+ *            an empty set for that query)
+ * topk       int32 [n_queries, topk_width] row-major, 4-byte aligned, or
+ *            NULL; entries < 0 (and those >= G) pick nothing. Ignored when
+ *            ratio = 0.
+ * topk_width 0 <= topk_width <= 512 (wider rows: SPA_ERR_UNSUPPORTED; build
+ *            them with spa_build_kv_sets)
+ * window     W >= 1
+ * ratio      0, 4 or 128; ratio > 0 needs the compressed pool (k_cmp, v_cmp,
+ *            pt_cmp non-NULL)
  * ---------------------------------------------------------------------- */
-int spa_sparse_sink_attn_fwd_all_groups(
+int spa_sparse_sink_attn_fwd_inline_sets(
     const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
     int32_t num_heads, int32_t head_dim,
     const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
     const int32_t* pt_raw, int32_t pt_raw_cols,
     const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages, int32_t cmp_page_size,
     const int32_t* pt_cmp, int32_t pt_cmp_cols,
-    const int32_t* req, int32_t n_requests, const int32_t* pos, int32_t window, int32_t ratio,
+    const int32_t* req, int32_t n_requests, const int32_t* pos,
+    const int32_t* topk, int32_t topk_width, int32_t window, int32_t ratio,
     const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 

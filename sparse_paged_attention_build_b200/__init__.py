@@ -69,12 +69,12 @@ def _load():
         P, P, i64, i32, P, i32,
         P, i32, P, P, P, ctypes.c_float, P, P, i32, P, sz, P, P]
     L.spa_sparse_sink_attn_fwd.restype = ctypes.c_int
-    L.spa_sparse_sink_attn_fwd_all_groups.argtypes = [
+    L.spa_sparse_sink_attn_fwd_inline_sets.argtypes = [
         P, i64, i64, i32, i32, i32,
         P, P, i64, i32, P, i32,
         P, P, i64, i32, P, i32,
-        P, i32, P, i32, i32, P, ctypes.c_float, P, P, i32, P, sz, P, P]
-    L.spa_sparse_sink_attn_fwd_all_groups.restype = ctypes.c_int
+        P, i32, P, P, i32, i32, i32, P, ctypes.c_float, P, P, i32, P, sz, P, P]
+    L.spa_sparse_sink_attn_fwd_inline_sets.restype = ctypes.c_int
     L.spa_sparse_sink_attn_fwd_fp8.argtypes = [
         P, i64, i64, i32, i32, i32,
         P, P, i64, i32, P, i32,
@@ -245,18 +245,21 @@ def sparse_sink_attn_fwd(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, sc
     return out, lse
 
 
-def sparse_sink_attn_fwd_all_groups(q, k_raw, v_raw, pt_raw, req, pos, window, ratio, sink, scale,
-                                    k_cmp=None, v_cmp=None, pt_cmp=None, out=None, lse=None, num_splits=0,
-                                    workspace=None, dev_status=None, stream=None):
-    """sparse_sink_attn_fwd over the sets spa_build_kv_sets builds without a
-    top-k list (every complete ratio-`ratio` group, then the window of
-    `window` tokens), built inside the kernel from pos (int32 [N])."""
+def sparse_sink_attn_fwd_inline_sets(q, k_raw, v_raw, pt_raw, req, pos, topk, window, ratio, sink, scale,
+                                     k_cmp=None, v_cmp=None, pt_cmp=None, out=None, lse=None, num_splits=0,
+                                     workspace=None, dev_status=None, stream=None):
+    """sparse_sink_attn_fwd over the sets spa_build_kv_sets builds from pos
+    (int32 [N]), topk (int32 [N, K] with K <= 512, or None: every complete
+    group), window and ratio, built inside the attention kernel."""
     _need(q, "q", torch.bfloat16)
     for name, t in (("k_raw", k_raw), ("v_raw", v_raw)):
         _need(t, name, torch.bfloat16)
         assert t.is_contiguous(), name
     for name, t in (("pt_raw", pt_raw), ("req", req), ("pos", pos)):
         _need(t, name, torch.int32)
+    if topk is not None:
+        _need(topk, "topk", torch.int32)
+        topk = topk.contiguous()
     N, H, d = q.shape
     if q.stride(2) != 1:
         raise ValueError("q's last dimension must be contiguous")
@@ -275,13 +278,14 @@ def sparse_sink_attn_fwd_all_groups(q, k_raw, v_raw, pt_raw, req, pos, window, r
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     pt_raw = pt_raw.contiguous()
-    _check("spa_sparse_sink_attn_fwd_all_groups", lib.spa_sparse_sink_attn_fwd_all_groups(
+    _check("spa_sparse_sink_attn_fwd_inline_sets", lib.spa_sparse_sink_attn_fwd_inline_sets(
         _p(q), q.stride(0), q.stride(1), N, H, d,
         _p(k_raw), _p(v_raw), k_raw.shape[0], k_raw.shape[1], _p(pt_raw), pt_raw.shape[1],
         _p(k_cmp), _p(v_cmp), 0 if k_cmp is None else k_cmp.shape[0],
         1 if k_cmp is None else k_cmp.shape[1],
         _p(None if pt_cmp is None else pt_cmp.contiguous()), 0 if pt_cmp is None else pt_cmp.shape[1],
-        _p(req.contiguous()), pt_raw.shape[0], _p(pos.contiguous()), int(window), int(ratio),
+        _p(req.contiguous()), pt_raw.shape[0], _p(pos.contiguous()), _p(topk),
+        0 if topk is None else topk.shape[1], int(window), int(ratio),
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
     return out, lse

@@ -420,23 +420,28 @@ int spa_sparse_sink_attn_fwd(const uint16_t* q, int64_t q_stride_tok, int64_t q_
   return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int spa_sparse_sink_attn_fwd_all_groups(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head,
-                                        int32_t n_queries, int32_t num_heads, int32_t head_dim,
-                                        const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages,
-                                        int32_t raw_page_size, const int32_t* pt_raw, int32_t pt_raw_cols,
-                                        const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages,
-                                        int32_t cmp_page_size, const int32_t* pt_cmp, int32_t pt_cmp_cols,
-                                        const int32_t* req, int32_t n_requests, const int32_t* pos,
-                                        int32_t window, int32_t ratio, const float* sink, float scale,
-                                        uint16_t* out, float* lse, int32_t num_splits, void* workspace,
-                                        size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream) {
+int spa_sparse_sink_attn_fwd_inline_sets(const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head,
+                                         int32_t n_queries, int32_t num_heads, int32_t head_dim,
+                                         const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages,
+                                         int32_t raw_page_size, const int32_t* pt_raw, int32_t pt_raw_cols,
+                                         const uint16_t* k_cmp, const uint16_t* v_cmp, int64_t cmp_num_pages,
+                                         int32_t cmp_page_size, const int32_t* pt_cmp, int32_t pt_cmp_cols,
+                                         const int32_t* req, int32_t n_requests, const int32_t* pos,
+                                         const int32_t* topk, int32_t topk_width, int32_t window, int32_t ratio,
+                                         const float* sink, float scale, uint16_t* out, float* lse,
+                                         int32_t num_splits, void* workspace, size_t workspace_bytes,
+                                         uint32_t* dev_status, spa_stream_t stream) {
   if (window < 1) return fail(SPA_ERR_INVALID_ARG, "window must be >= 1");
   if (ratio != 0 && ratio != 4 && ratio != 128) return fail(SPA_ERR_UNSUPPORTED, "ratio must be 0, 4 or 128");
+  if (topk_width < 0) return fail(SPA_ERR_INVALID_ARG, "topk_width < 0");
+  if (ratio > 0 && topk != nullptr && topk_width > spa::kInlineTopkMaxWidth)
+    return fail(SPA_ERR_UNSUPPORTED, "topk_width > %d (sets built in the kernel)", spa::kInlineTopkMaxWidth);
   if (ratio > 0 && n_queries > 0 && (pt_cmp == nullptr || k_cmp == nullptr || v_cmp == nullptr))
     return fail(SPA_ERR_INVALID_ARG, "ratio > 0 needs the compressed pool (k_cmp, v_cmp, pt_cmp)");
   if (pt_cmp != nullptr && n_queries > 0 && (k_cmp == nullptr || v_cmp == nullptr))
     return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
   if (pos == nullptr && n_queries > 0) return fail(SPA_ERR_INVALID_ARG, "pos must be non-NULL");
+  if (!aligned(topk, 4)) return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
   spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
                               raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
                               pt_cmp_cols, req, n_requests, nullptr, nullptr, sink, scale, out, lse, workspace,
@@ -446,6 +451,9 @@ int spa_sparse_sink_attn_fwd_all_groups(const uint16_t* q, int64_t q_stride_tok,
   a.set_pos = pos;
   a.set_window = window;
   a.set_ratio = ratio;
+  // with ratio 0 the row picks nothing: the set is the window alone
+  a.set_topk = ratio > 0 ? topk : nullptr;
+  a.set_topk_width = ratio > 0 && topk != nullptr ? topk_width : 0;
   return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 

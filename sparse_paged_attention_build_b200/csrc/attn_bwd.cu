@@ -85,11 +85,14 @@ struct Params {
   int32_t n_requests;
   const int32_t* indptr;
   const int32_t* indices;
-  // non-NULL: the sets are built in the resolver from the positions (every
-  // complete ratio-set_ratio group, then the window of set_window tokens)
-  // instead of read from indptr/indices
+  // non-NULL: the sets are built in the resolver from the positions (the
+  // complete ratio-set_ratio groups -- all of them, or those the set_topk
+  // row picks, sorted -- then the window of set_window tokens) instead of
+  // read from indptr/indices
   const int32_t* set_pos;
   int32_t set_window, set_ratio;
+  const int32_t* set_topk;   // [n_queries, set_topk_width] or NULL
+  int32_t set_topk_width;
   const float* sink;
   float scale, scale_log2;
   const uint16_t* o;      // saved O [N, H, d]
@@ -748,6 +751,8 @@ cudaError_t launch_sparse_sink_attn_bwd(const AttnArgs& a, cudaStream_t stream) 
   P.set_pos = a.set_pos;
   P.set_window = a.set_window;
   P.set_ratio = a.set_ratio;
+  P.set_topk = a.set_topk;
+  P.set_topk_width = a.set_topk_width;
   P.sink = a.sink;
   P.scale = a.scale;
   P.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634);

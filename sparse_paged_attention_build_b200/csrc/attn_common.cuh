@@ -5,6 +5,7 @@
 #pragma once
 
 #include <algorithm>
+#include <climits>
 #include <cstdint>
 
 #include <cuda.h>
@@ -44,13 +45,16 @@ __device__ __forceinline__ int ceil_tiles(int nkeys) { return (nkeys + kT - 1) /
 // + lane + 32, ...; the loads of each phase are issued together so the
 // chunk costs two round trips, not two per key. Prm holds the page tables
 // and pool sizes.
-// With inl_groups >= 0 the keys are not read from `indices` but are the
-// set's closed form: position k of the set is group k below inl_groups and
-// window token inl_wstart + k - inl_groups after it (key_base is then the
-// chunk's position in the set).
+// With inl_groups >= 0 the keys are not read from `indices` but built:
+// position k of the set is group k below inl_groups (or group inl_list[k],
+// a sorted list in shared memory, when inl_list is set) and window token
+// inl_wstart + k - inl_groups after it (key_base is then the chunk's
+// position in the set). inl_list may be this chunk's own table slot: every
+// lane reads its keys before any lane writes a row.
 template <int kParts = 1, class Prm>
 __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t nkeys, uint32_t* tab,
-                              int lane, int part = 0, int32_t inl_groups = -1, int32_t inl_wstart = 0) {
+                              int lane, int part = 0, int32_t inl_groups = -1, int32_t inl_wstart = 0,
+                              const int32_t* inl_list = nullptr) {
   constexpr int kPer = kChunkKeys / kParts / 32;
   const int k0 = part * (kChunkKeys / kParts);
   int32_t key[kPer];
@@ -60,8 +64,10 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
     const int32_t at = key_base + k;
     key[e] = k >= nkeys ? -2
              : inl_groups < 0 ? __ldg(P.indices + at)
-             : at < inl_groups ? at : (SPA_WINDOW_TAG | (inl_wstart + at - inl_groups));
+             : at < inl_groups ? (inl_list != nullptr ? inl_list[at] : at)
+             : (SPA_WINDOW_TAG | (inl_wstart + at - inl_groups));
   }
+  __syncwarp();
   int32_t page[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
@@ -98,6 +104,97 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
   }
 }
 
+// ---- the complete groups a query's top-k row picks (sets built here)
+// The row's entries j < width, loaded 16 per lane (entry 32 r + lane in
+// register r, -1 past the width), become the ascending list of distinct
+// groups g with 0 <= g < n_complete, written to `area` (kWords words of
+// shared memory); returns the count.
+constexpr int kInlineTopkMax = kInlineTopkMaxWidth;
+constexpr int kTopkRegs = kInlineTopkMax / 32;
+static_assert(kInlineTopkMax % 32 == 0, "whole registers per lane");
+static_assert(kInlineTopkMax <= kChunkKeys, "the list of a unit fits its first chunk's table slot");
+
+__device__ __forceinline__ void load_topk_row(const int32_t* row, int width, int lane, int32_t (&g)[kTopkRegs]) {
+#pragma unroll
+  for (int r = 0; r < kTopkRegs; ++r) g[r] = 32 * r + lane < width ? __ldg(row + 32 * r + lane) : -1;
+}
+
+// Through bitmaps rather than a sort (a sort of 512 entries costs about ten
+// times the instructions, and the resolver shares its issue slots with a
+// softmax warp): a window [w0, hi) of groups gets one bit per group in the
+// free part of `area` after the `total` groups listed so far; every entry
+// in the window sets its bit (repeats fall together); the words come back
+// into registers (word 32 r + lane in register r) and the set bits'
+// indices are appended, ascending, over the bitmap. One window covers up to
+// 32 * (kWords - total) >= 32 * (kWords - kInlineTopkMax) groups, so sets
+// with up to 32 * kWords complete groups take one pass; past that the next
+// window starts at the smallest entry not yet listed, so there are at most
+// as many passes as windows holding an entry.
+template <int kWords>
+__device__ __forceinline__ int32_t pick_groups(const int32_t (&g)[kTopkRegs], int32_t n_complete, int lane,
+                                               int32_t* area) {
+  constexpr int kR = kWords / 32;
+  static_assert(kWords % 32 == 0 && kWords > kInlineTopkMax, "room for a window after the longest list");
+  int32_t total = 0;
+  int32_t w0 = 0;
+  while (w0 < n_complete) {
+    const int64_t span_end = w0 + 32LL * (kWords - total);
+    const int32_t hi = span_end < n_complete ? static_cast<int32_t>(span_end) : n_complete;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(area + total);
+    const int words = (hi - w0 + 31) >> 5;   // <= kWords - total
+    for (int w = lane; w < words; w += 32) bits[w] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < kTopkRegs; ++r)
+      if (g[r] >= w0 && g[r] < hi) atomicOr(bits + ((g[r] - w0) >> 5), 1u << ((g[r] - w0) & 31));
+    __syncwarp();
+    uint32_t m[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) m[r] = 32 * r + lane < words ? bits[32 * r + lane] : 0u;
+    __syncwarp();   // every word is read before the list overwrites them
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      if (32 * r >= words) continue;   // uniform across the warp
+      const int32_t c = __popc(m[r]);
+      int32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int32_t at = total + incl - c;
+      const int32_t base = w0 + (32 * r + lane) * 32;
+      for (uint32_t bm = m[r]; bm != 0u; bm &= bm - 1u) area[at++] = base + (__ffs(bm) - 1);
+      total += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    if (hi >= n_complete) break;
+    int32_t nxt = INT_MAX;
+#pragma unroll
+    for (int r = 0; r < kTopkRegs; ++r)
+      if (g[r] >= hi && g[r] < n_complete) nxt = min(nxt, g[r]);
+    nxt = __reduce_min_sync(0xffffffffu, nxt);
+    if (nxt == INT_MAX) break;
+    w0 = nxt;
+  }
+  return total;
+}
+
+// A unit's picked groups, listed in the table slot `area` once the slot is
+// free (its barrier `empty` at `parity`); the row's loads are in flight
+// during the wait. Returns the count, or -1 when the wait gave up. Kept out
+// of line: inlined into the resolver loop, the code grows the kernel enough
+// to slow every launch of it, whether or not a launch takes this path.
+static __device__ __noinline__ int32_t picked_groups_in_slot(const int32_t* row, int width, int32_t n_complete, int lane,
+                                                             int32_t* area, uint64_t* empty, uint32_t parity,
+                                                             volatile int* abort_flag, uint32_t* dev_status,
+                                                             uint64_t wait_ns) {
+  int32_t g[kTopkRegs];
+  load_topk_row(row, width, lane, g);
+  if (!mbar_wait(empty, parity, abort_flag, dev_status, wait_ns)) return -1;
+  return pick_groups<kChunkKeys>(g, n_complete, lane, area);
+}
+
 // The resolver warp: walks this CTA's units (query i, slice), splits each
 // slice's keys into chunks of up to kChunkKeys, resolves them into the
 // double-buffered table and publishes a descriptor per chunk. An empty slice
@@ -108,6 +205,12 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
 // overlap). With kParts > 1, kParts warps run this loop side by side, each
 // resolving its share of every chunk (tab_full then counts all of them);
 // part 0 writes the descriptors.
+// Sets built here from top-k rows: before a unit's first chunk the resolver
+// waits for that chunk's table slot, builds the unit's sorted groups in it
+// (the set's length depends on their count), and the chunk reads its keys
+// from that list before its rows overwrite it. Every group position lies in
+// the unit's first chunk (at most kInlineTopkMax <= kChunkKeys of them, at
+// the front of the set).
 template <int kParts = 1, class Prm>
 __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* desc, uint64_t* tab_full,
                               uint64_t* tab_empty, volatile int* abort_flag, int lane, bool contiguous = false,
@@ -117,27 +220,14 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
   const int64_t u0 = contiguous ? (static_cast<int64_t>(blockIdx.x) * n_units) / gridDim.x : blockIdx.x;
   const int64_t u_end = contiguous ? (static_cast<int64_t>(blockIdx.x + 1) * n_units) / gridDim.x : n_units;
   const int64_t step = contiguous ? 1 : gridDim.x;
+  const bool picked = P.set_pos != nullptr && P.set_topk != nullptr && kParts == 1;
   for (int64_t u = u0; u < u_end && !*abort_flag; u += step) {
     const int i = static_cast<int>(u / S);
     const int split = static_cast<int>(u - static_cast<int64_t>(i) * S);
     int32_t set_begin = 0, set_len, inl_groups = -1, inl_wstart = 0;
     const int32_t b = __ldg(P.req + i);
-    if (P.set_pos != nullptr) {
-      // the set built here: every complete group, then the window
-      const int32_t pos = __ldg(P.set_pos + i);
-      const bool pos_ok = pos >= 0 && pos < SPA_WINDOW_TAG;
-      const int32_t wn = pos_ok ? min(P.set_window, pos + 1) : 0;
-      inl_groups = (pos_ok && P.set_ratio > 0) ? (pos + 1) / P.set_ratio : 0;
-      inl_wstart = pos + 1 - wn;
-      set_len = pos_ok ? inl_groups + wn : -1;
-    } else {
-      set_begin = __ldg(P.indptr + i);
-      set_len = __ldg(P.indptr + i + 1) - set_begin;
-    }
-    if (set_len < 0 || b < 0 || b >= P.n_requests) {
-      if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
-      set_len = 0;
-    } else {
+    const bool b_ok = b >= 0 && b < P.n_requests;
+    if (b_ok) {
       // The page-table rows of this request into L2 while the keys load,
       // so that the lookup after them (the third dependent load of the
       // chunk) hits L2: up to 64 lines (8 KB) of each table per lane group.
@@ -150,6 +240,33 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
         for (int ln = lane; ln < lines; ln += 32) prefetch_l2(rows[tb] + 32 * ln);
       }
     }
+    bool slot_held = false;   // the first chunk's slot is already waited for
+    if (P.set_pos != nullptr) {
+      // the set built here: the complete groups (all of them, or those the
+      // top-k row picks, sorted, repeats removed), then the window
+      const int32_t pos = __ldg(P.set_pos + i);
+      const bool pos_ok = pos >= 0 && pos < SPA_WINDOW_TAG;
+      const int32_t wn = pos_ok ? min(P.set_window, pos + 1) : 0;
+      inl_groups = (pos_ok && P.set_ratio > 0) ? (pos + 1) / P.set_ratio : 0;
+      if (picked) {
+        inl_groups = picked_groups_in_slot(P.set_topk + static_cast<int64_t>(i) * P.set_topk_width,
+                                           P.set_topk_width, inl_groups, lane,
+                                           reinterpret_cast<int32_t*>(tab + (c & 1) * kChunkKeys),
+                                           tab_empty + (c & 1), ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status,
+                                           P.wait_ns);
+        if (inl_groups < 0) return;
+        slot_held = true;
+      }
+      inl_wstart = pos + 1 - wn;
+      set_len = pos_ok ? inl_groups + wn : -1;
+    } else {
+      set_begin = __ldg(P.indptr + i);
+      set_len = __ldg(P.indptr + i + 1) - set_begin;
+    }
+    if (set_len < 0 || !b_ok) {
+      if (lane == 0) report(P.dev_status, SPA_DEV_BAD_INDEX);
+      set_len = 0;
+    }
     const int tiles_total = ceil_tiles(set_len);
     const int tile_lo = static_cast<int>((static_cast<int64_t>(tiles_total) * split) / S);
     const int tile_hi = static_cast<int>((static_cast<int64_t>(tiles_total) * (split + 1)) / S);
@@ -159,9 +276,12 @@ __device__ void resolver_loop(const Prm& P, int S, uint32_t* tab, ChunkDesc* des
     int32_t k0 = key_lo;
     do {
       const int slot = c & 1;
-      if (!mbar_wait(tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns)) return;
+      if (!slot_held && !mbar_wait(tab_empty + slot, ((c >> 1) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns))
+        return;
       const int32_t n = max(0, min(kChunkKeys, key_hi - k0));   // 0: an empty slice
-      resolve_chunk<kParts>(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane, part, inl_groups, inl_wstart);
+      resolve_chunk<kParts>(P, b, set_begin + k0, n, tab + slot * kChunkKeys, lane, part, inl_groups, inl_wstart,
+                            slot_held ? reinterpret_cast<const int32_t*>(tab + slot * kChunkKeys) : nullptr);
+      slot_held = false;
       if (lane == 0 && part == 0) {
         ChunkDesc& d = desc[slot];
         d.i = i;

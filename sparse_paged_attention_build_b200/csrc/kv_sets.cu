@@ -8,8 +8,8 @@
 // complete groups outnumber it.
 //
 // A CTA owns a block of consecutive queries, one warp per query at a time.
-// A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio))
-// into a shared-memory bitmap over the complete groups -- setting a bit drops
+// A warp filters its top-k row (keeps 0 <= g < floor((p+1)/ratio)) into a
+// shared-memory bitmap over the complete groups -- setting a bit drops
 // repeats and reading the words in order yields the ascending list -- and
 // counts the set bits; when the complete groups outnumber the bitmap it
 // sorts the row with a bitonic network instead. The window adds min(p+1, W)
@@ -17,8 +17,11 @@
 // by a decoupled look-back over the CTAs before it (CTA order taken from an
 // atomic ticket, so every predecessor is already running; one warp reads 32
 // predecessors per step), then recomputes every set and writes its indptr
-// entry and its keys: the distinct groups ascending, then the window tokens
-// ascending with the window tag. Integer only; no floating point anywhere.
+// entry and its keys: the distinct groups ascending (listed in shared
+// memory, then copied out coalesced), then the window tokens ascending with
+// the window tag. A warp writes its queries in the reverse of the counting
+// order, so the bitmap of its first one is still in place. Integer only; no
+// floating point anywhere.
 #include <climits>
 #include <mutex>
 
@@ -81,6 +84,8 @@ struct SetsParams {
 };
 
 constexpr int kSetsWarps = 16;   // warps per CTA, one query each at a time
+constexpr int kRowStep = 512;    // top-k entries a warp loads at once
+constexpr int kRegWords = 16;    // bitmap words per lane held in registers while writing a list
 constexpr int kMaxPerCta = 2048;
 
 __device__ __forceinline__ int64_t warp_sum64(int64_t v) {
@@ -92,8 +97,10 @@ __device__ __forceinline__ int64_t warp_sum64(int64_t v) {
 // The key set of query i, by one warp (all lanes call together). Returns
 // the number of keys; when `write` is set, stores them at
 // indices[start ..) ascending (entries at or past `limit` are dropped).
+// `bitmap_ready`: buf still holds this query's bitmap from the counting
+// pass (the warp's last query there is its first here).
 __device__ int64_t one_query(const SetsParams& P, int64_t i, int32_t* buf, int lane, bool write,
-                             int64_t start, int64_t limit) {
+                             int64_t start, int64_t limit, bool bitmap_ready = false) {
   const int32_t p = P.pos[i];
   if (p < 0 || p >= SPA_WINDOW_TAG) {
     if (lane == 0 && !write) report(P.dev_status, SPA_DEV_BAD_INDEX);
@@ -114,26 +121,70 @@ __device__ int64_t one_query(const SetsParams& P, int64_t i, int32_t* buf, int l
     // bitmap over the complete groups: marking a bit removes repeats,
     // reading the words in order gives the ascending list
     uint32_t* bm = reinterpret_cast<uint32_t*>(buf);
-    for (int w = lane; w < words; w += 32) bm[w] = 0u;
-    __syncwarp();
-    const int32_t* row = P.topk + i * P.topk_width;
-    for (int j = lane; j < P.topk_width; j += 32) {
-      const int32_t g = row[j];
-      if (g >= 0 && g < n_complete) atomicOr(bm + (g >> 5), 1u << (g & 31));
-    }
-    __syncwarp();
-    int64_t written = 0;
-    for (int w0 = 0; w0 < words; w0 += 32) {
-      const int w = w0 + lane;
-      uint32_t bits = w < words ? bm[w] : 0u;
-      const int cnt = __popc(bits);
-      int incl = cnt;
+    if (!bitmap_ready) {
+      for (int w = lane; w < words; w += 32) bm[w] = 0u;
+      __syncwarp();
+      const int32_t* row = P.topk + i * P.topk_width;
+      // 512 entries per step with all 16 loads of a lane in flight together
+      // (one round trip per step rather than one per entry)
+      for (int j0 = 0; j0 < P.topk_width; j0 += kRowStep) {
+        int32_t g[kRowStep / 32];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+        for (int r = 0; r < kRowStep / 32; ++r) {
+          const int j = j0 + 32 * r + lane;
+          g[r] = j < P.topk_width ? __ldg(row + j) : -1;
+        }
+#pragma unroll
+        for (int r = 0; r < kRowStep / 32; ++r)
+          if (g[r] >= 0 && g[r] < n_complete) atomicOr(bm + (g[r] >> 5), 1u << (g[r] & 31));
       }
-      if (write) {
+      __syncwarp();
+    }
+    if (!write) {
+      // counting needs only the number of set bits; the bitmap stays
+      int32_t cnt = 0;
+      for (int w = lane; w < words; w += 32) cnt += __popc(bm[w]);
+      n_groups = warp_sum64(cnt);
+    } else if (words <= 32 * kRegWords) {
+      // every word into registers (word 32 r + lane in register r), then
+      // the ascending list over the bitmap in shared memory and one
+      // coalesced copy of it
+      uint32_t m[kRegWords];
+#pragma unroll
+      for (int r = 0; r < kRegWords; ++r) m[r] = 32 * r + lane < words ? bm[32 * r + lane] : 0u;
+      __syncwarp();
+      int32_t total = 0;
+#pragma unroll
+      for (int r = 0; r < kRegWords; ++r) {
+        if (32 * r >= words) continue;   // uniform across the warp
+        const int cnt = __popc(m[r]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int32_t at = total + incl - cnt;
+        const int32_t base = (32 * r + lane) * 32;
+        for (uint32_t bits = m[r]; bits != 0u; bits &= bits - 1u) buf[at++] = base + (__ffs(bits) - 1);
+        total += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      __syncwarp();
+      for (int k = lane; k < total; k += 32)
+        if (start + k < limit) P.indices[start + k] = buf[k];
+      n_groups = total;
+    } else {
+      int64_t written = 0;
+      for (int w0 = 0; w0 < words; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t bits = w < words ? bm[w] : 0u;
+        const int cnt = __popc(bits);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
         int64_t dst = start + written + (incl - cnt);
         while (bits) {
           const int bit = __ffs(bits) - 1;
@@ -141,16 +192,25 @@ __device__ int64_t one_query(const SetsParams& P, int64_t i, int32_t* buf, int l
           ++dst;
           bits &= bits - 1u;
         }
+        written += __shfl_sync(0xffffffffu, incl, 31);
       }
-      written += __shfl_sync(0xffffffffu, incl, 31);
+      n_groups = written;
     }
-    n_groups = written;
     __syncwarp();   // the bitmap is rebuilt by the next query
   } else if (listed) {
     const int32_t* row = P.topk + i * P.topk_width;
-    for (int j = lane; j < P.sort_width; j += 32) {
-      const int32_t g = j < P.topk_width ? row[j] : -1;
-      buf[j] = (g >= 0 && g < n_complete) ? g : INT_MAX;
+    for (int j0 = 0; j0 < P.sort_width; j0 += kRowStep) {
+      int32_t g[kRowStep / 32];
+#pragma unroll
+      for (int r = 0; r < kRowStep / 32; ++r) {
+        const int j = j0 + 32 * r + lane;
+        g[r] = j < P.topk_width ? __ldg(row + j) : -1;
+      }
+#pragma unroll
+      for (int r = 0; r < kRowStep / 32; ++r) {
+        const int j = j0 + 32 * r + lane;
+        if (j < P.sort_width) buf[j] = (g[r] >= 0 && g[r] < n_complete) ? g[r] : INT_MAX;
+      }
     }
     __syncwarp();
     warp_bitonic_sort(buf, P.sort_width, lane);
@@ -210,9 +270,11 @@ __global__ void __launch_bounds__(kSetsWarps * 32) build_kv_sets_kernel(const Se
   const int64_t q0 = static_cast<int64_t>(tile) * P.per_cta;
   const int nq = static_cast<int>(min(static_cast<int64_t>(P.per_cta), static_cast<int64_t>(P.n) - q0));
 
+  int last_q = -1;
   for (int q = warp; q < nq; q += kSetsWarps) {
     const int64_t c = one_query(P, q0 + q, buf, lane, false, 0, 0);
     if (lane == 0) prefix[q] = c;
+    last_q = q;
   }
   __syncthreads();
 
@@ -270,10 +332,12 @@ __global__ void __launch_bounds__(kSetsWarps * 32) build_kv_sets_kernel(const Se
 
   const int64_t base = s_base;
   const int64_t limit = P.capacity < INT_MAX ? P.capacity : INT_MAX;
-  for (int q = warp; q < nq; q += kSetsWarps) {
+  // the warp's queries in reverse order: the first one's bitmap is still
+  // in its buffer from the counting pass
+  for (int q = last_q; q >= 0; q -= kSetsWarps) {
     const int64_t i = q0 + q;
     const int64_t start = base + prefix[q];
-    const int64_t c = one_query(P, i, buf, lane, true, start, limit);
+    const int64_t c = one_query(P, i, buf, lane, true, start, limit, q == last_q);
     if (lane == 0) {
       const int64_t end = start + c;
       if (end > P.capacity || end > INT_MAX) report(P.dev_status, SPA_DEV_CAPACITY);

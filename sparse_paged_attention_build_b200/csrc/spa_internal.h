@@ -13,6 +13,8 @@ int device_sm_count();
 
 constexpr int kSetsQueriesPerCta = 8;      // fewest queries a set-builder CTA owns
 constexpr int kMaxTopkWidth = 2048;
+// widest top-k row whose groups the attention's resolver sorts itself
+constexpr int kInlineTopkMaxWidth = 512;
 
 size_t build_kv_sets_workspace_bytes(int32_t n_queries);
 cudaError_t launch_build_kv_sets(const int32_t* pos, int32_t n, int32_t window, int32_t ratio,
@@ -64,9 +66,13 @@ struct AttnArgs {
   const int32_t* indptr;
   const int32_t* indices;
   // sets built inside the kernel (NULL: read indptr/indices): positions,
-  // window W and ratio; the set is every complete group, then the window
+  // window W and ratio, and the top-k rows [n_queries, set_topk_width]
+  // (NULL: every complete group); the set is the complete groups, sorted,
+  // then the window
   const int32_t* set_pos = nullptr;
   int32_t set_window = 0, set_ratio = 0;
+  const int32_t* set_topk = nullptr;
+  int32_t set_topk_width = 0;
   const float* sink;
   float scale;
   uint16_t* out;

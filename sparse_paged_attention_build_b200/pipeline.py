@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 from . import (build_kv_sets, dequant_fp8_pages, kv_sets_capacity, sparse_sink_attn_fwd, sparse_sink_attn_fwd_fp8,
-               sparse_sink_attn_fwd_all_groups, attn_workspace_size, new_status, read_status)
+               sparse_sink_attn_fwd_inline_sets, attn_workspace_size, new_status, read_status)
 from . import lib
 
 
@@ -25,18 +25,58 @@ def _dev(a, dtype=None, device="cuda"):
     return t.to(device)
 
 
+INLINE_TOPK_MAX = 512   # widest top-k row the attention kernel sorts itself
+
+
+def inline_sets_supported(w, fp8_path="decode") -> bool:
+    """Whether the attention kernel can build this workload's sets itself:
+    top-k rows of at most INLINE_TOPK_MAX entries (or none), and the BF16
+    attention (a mixed cache decoded to BF16 first, not inside the gather)."""
+    fused = w.k_cmp_fp8 is not None and fp8_path == "fused"
+    return not fused and (w.topk is None or w.topk.shape[1] <= INLINE_TOPK_MAX)
+
+
+def splits_for(w, num_splits=0) -> int:
+    """Slices per query the attention runs a workload with (0: the
+    library's automatic choice)."""
+    if num_splits > 0:
+        return num_splits
+    if w.d == 512:
+        return int(lib.spa_sparse_sink_attn_choose_splits_d512(w.N, w.H))
+    return int(lib.spa_sparse_sink_attn_choose_splits(w.N, w.H, 0))
+
+
+def prefer_inline_sets(w, fp8_path="decode", num_splits=0, sm_count=148) -> bool:
+    """Where the sets are cheaper to build: inside the attention kernel
+    without a top-k list (a closed form, no extra launch) or for small
+    batches with one; a separate build kernel for large batches with top-k
+    rows. Measured on B200: picking a unit's groups from its row costs the
+    CTA about 3 us of its critical path (its resolver shares issue slots
+    with a softmax warp), 16k ratio-4 prefill queries lost 0.17 ms that way
+    against a 0.02 ms build launch, while 64 to 1024 queries gained 2-6 us
+    per step."""
+    if not inline_sets_supported(w, fp8_path):
+        return False
+    if w.topk is None:
+        return True
+    return w.N * splits_for(w, num_splits) <= 8 * sm_count
+
+
 class DeviceBatch:
     """A workload resident in device memory, with its outputs."""
 
     def __init__(self, w, device="cuda", num_splits=0, fp8_path="decode", sets="csr"):
         self.w = w
         # "csr": the sets are built by spa_build_kv_sets, then read by the
-        # attention; "inline": sets without a top-k list are built inside the
-        # attention kernel (spa_sparse_sink_attn_fwd_all_groups)
+        # attention; "inline": the sets are built inside the attention kernel
+        # (spa_sparse_sink_attn_fwd_inline_sets), from the same inputs
         if sets not in ("csr", "inline"):
             raise ValueError("sets is 'csr' or 'inline'")
-        if sets == "inline" and (w.topk is not None or w.k_cmp_fp8 is not None):
-            raise ValueError("sets built inside the kernel need a workload without top-k and a BF16 cache")
+        if fp8_path not in ("fused", "decode"):
+            raise ValueError("fp8_path is 'fused' or 'decode'")
+        if sets == "inline" and not inline_sets_supported(w, fp8_path):
+            raise ValueError("sets built inside the kernel need top-k rows of at most 512 entries and no FP8 "
+                             "decode inside the gather")
         self.inline_sets = sets == "inline"
         self.device = device
         bf16 = torch.bfloat16
@@ -50,8 +90,6 @@ class DeviceBatch:
         self.pt_cmp = _dev(w.pt_cmp, None, device)
         self.sink = _dev(w.sink, None, device)
         self.fp8 = w.k_cmp_fp8 is not None
-        if fp8_path not in ("fused", "decode"):
-            raise ValueError("fp8_path is 'fused' or 'decode'")
         # mixed cache: decode inside the attention gather ("fused"), or decode
         # the pages to a BF16 pool first ("decode")
         self.fused = self.fp8 and fp8_path == "fused"
@@ -104,11 +142,11 @@ class DeviceBatch:
                                      dev_status=self.status, stream=stream, fp8_format=self.w.fp8_format)
             return
         if self.inline_sets:
-            sparse_sink_attn_fwd_all_groups(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.pos, w.W,
-                                            w.ratio, self.sink, w.scale, k_cmp=self.k_cmp, v_cmp=self.v_cmp,
-                                            pt_cmp=self.pt_cmp, out=self.out, lse=self.lse,
-                                            num_splits=self.num_splits, workspace=self.attn_ws,
-                                            dev_status=self.status, stream=stream)
+            sparse_sink_attn_fwd_inline_sets(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.pos,
+                                             self.topk, w.W, w.ratio, self.sink, w.scale, k_cmp=self.k_cmp,
+                                             v_cmp=self.v_cmp, pt_cmp=self.pt_cmp, out=self.out, lse=self.lse,
+                                             num_splits=self.num_splits, workspace=self.attn_ws,
+                                             dev_status=self.status, stream=stream)
             return
         sparse_sink_attn_fwd(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.indptr,
                              self.indices, self.sink, w.scale, k_cmp=self.k_cmp, v_cmp=self.v_cmp,
@@ -127,11 +165,7 @@ class DeviceBatch:
     def splits_used(self) -> int:
         """Slices per query the attention runs with (0 resolves to the
         library's automatic choice)."""
-        if self.num_splits > 0:
-            return self.num_splits
-        if self.w.d == 512:
-            return int(lib.spa_sparse_sink_attn_choose_splits_d512(self.w.N, self.w.H))
-        return int(lib.spa_sparse_sink_attn_choose_splits(self.w.N, self.w.H, 0))
+        return splits_for(self.w, self.num_splits)
 
     def kernels_per_step(self) -> int:
         return (0 if self.inline_sets else 1) + (2 if self.fp8 and not self.fused else 0) + 1

@@ -165,20 +165,24 @@ def test_attention_zero_queries_is_a_no_op(L):
     assert attn_call(L, n=0, q=None, out=None, lse=None) == 0
 
 
-def attn_all_groups_call(L, **kw):
+def attn_inline_call(L, **kw):
     a = dict(q=FAKE, sq=16384, sh=128, n=4, H=128, d=128, kr=FAKE, vr=FAKE, rp=10, rps=64, ptr=FAKE,
-             ptrc=4, kc=FAKE, vc=FAKE, cp=10, cps=64, ptc=FAKE, ptcc=4, req=FAKE, B=1, pos=FAKE, W=128,
-             ratio=128, sink=FAKE, scale=0.088, out=FAKE, lse=FAKE, splits=1, ws=None, wsb=0)
+             ptrc=4, kc=FAKE, vc=FAKE, cp=10, cps=64, ptc=FAKE, ptcc=4, req=FAKE, B=1, pos=FAKE, topk=None,
+             K=0, W=128, ratio=128, sink=FAKE, scale=0.088, out=FAKE, lse=FAKE, splits=1, ws=None, wsb=0)
     a.update(kw)
-    return L.spa_sparse_sink_attn_fwd_all_groups(
+    return L.spa_sparse_sink_attn_fwd_inline_sets(
         a["q"], a["sq"], a["sh"], a["n"], a["H"], a["d"], a["kr"], a["vr"], a["rp"], a["rps"], a["ptr"],
         a["ptrc"], a["kc"], a["vc"], a["cp"], a["cps"], a["ptc"], a["ptcc"], a["req"], a["B"], a["pos"],
-        a["W"], a["ratio"], a["sink"], a["scale"], a["out"], a["lse"], a["splits"], a["ws"], a["wsb"], None, None)
+        a["topk"], a["K"], a["W"], a["ratio"], a["sink"], a["scale"], a["out"], a["lse"], a["splits"], a["ws"],
+        a["wsb"], None, None)
 
 
 @pytest.mark.parametrize("kw,status,clause", [
     (dict(W=0), 1, "window must be >= 1"),
     (dict(ratio=3), 2, "ratio must be 0, 4 or 128"),
+    (dict(K=-1), 1, "topk_width < 0"),
+    (dict(ratio=4, topk=FAKE, K=513), 2, "topk_width > 512"),
+    (dict(ratio=4, topk=FAKE + 2, K=16), 5, "32-bit arrays"),
     (dict(ptc=None), 1, "ratio > 0 needs the compressed pool"),
     (dict(kc=None), 1, "ratio > 0 needs the compressed pool"),
     (dict(ratio=0, ptc=FAKE, vc=None), 1, "k_cmp/v_cmp NULL"),
@@ -189,14 +193,20 @@ def attn_all_groups_call(L, **kw):
     (dict(d=96), 2, "head_dim must be 64, 128 or 512"),
     (dict(splits=12), 4, "workspace needs"),
 ])
-def test_guard_matrix_attention_all_groups(L, kw, status, clause):
-    assert attn_all_groups_call(L, **kw) == status
+def test_guard_matrix_attention_inline_sets(L, kw, status, clause):
+    assert attn_inline_call(L, **kw) == status
     assert clause in L.spa_last_error_detail().decode()
 
 
-def test_attention_all_groups_window_only_needs_no_compressed_pool(L):
+def test_attention_inline_sets_window_only_needs_no_compressed_pool(L):
     # ratio 0: the window alone; only the zero-query call runs on the CPU
-    assert attn_all_groups_call(L, ratio=0, ptc=None, kc=None, vc=None, n=0, q=None, out=None, lse=None) == 0
+    assert attn_inline_call(L, ratio=0, ptc=None, kc=None, vc=None, n=0, q=None, out=None, lse=None) == 0
+
+
+def test_attention_inline_sets_ignores_topk_width_at_ratio_0(L):
+    # ratio 0 picks no group, so a row of any width is accepted (and unread)
+    assert attn_inline_call(L, ratio=0, topk=FAKE, K=4096, ptc=None, kc=None, vc=None, n=0, q=None, out=None,
+                            lse=None) == 0
 
 
 def attn8_call(L, **kw):

@@ -1,11 +1,12 @@
-"""GPU: attention over sets built inside the kernel (no top-k list).
+"""GPU: attention over sets built inside the kernel.
 
-spa_sparse_sink_attn_fwd_all_groups builds, per query, the set
-spa_build_kv_sets builds without a top-k list (every complete group, then
-the window) in its resolver. The keys and their order are the same, so its
-O and LSE must be bit-identical to spa_build_kv_sets followed by
+spa_sparse_sink_attn_fwd_inline_sets builds, per query, the set
+spa_build_kv_sets builds from the same inputs (the complete groups -- all of
+them, or those a top-k row picks, sorted, repeats removed -- then the
+window) in its resolver. The keys and their order are the same, so its O
+and LSE must be bit-identical to spa_build_kv_sets followed by
 spa_sparse_sink_attn_fwd at the same split count -- including the status
-word and the empty-set rows of faulty positions. One case is also checked
+word and the empty-set rows of faulty positions. Two cases are also checked
 against the FP64 oracle directly, at the method's tolerance.
 """
 import dataclasses
@@ -71,6 +72,62 @@ def test_inline_sets_every_complete_group(spa, name, shrink, splits):
     _assert_identical(csr, inl, f"{name}/{shrink} without top-k, splits={splits}")
 
 
+@pytest.mark.parametrize("name,shrink,splits", [
+    ("c1", 1, 0), ("c1", 1, 1), ("c1", 1, 3),       # top-k 16, d = 64
+    ("c3", 16, 0), ("c3", 16, 2), ("c3", 1, 0),     # top-k 512, d = 128; the full prefill the bench times
+    ("f1", 8, 0), ("f2", 8, 0), ("f2", 8, 3),       # top-k 512, d = 512
+    ("c5", 8, 0), ("c5", 8, 4),                     # top-k 512, mixed cache decoded to BF16 first
+])
+def test_inline_sets_from_topk_rows(spa, name, shrink, splits):
+    from sparse_paged_attention_build_b200 import workloads
+    w = workloads.make(name, shrink=shrink)
+    assert w.topk is not None
+    csr, inl = _both(w, splits)
+    assert csr.status_word() == 0
+    _assert_identical(csr, inl, f"{name}/{shrink} splits={splits}")
+
+
+def _planted_topk(w, width, seed):
+    """Top-k rows of `width` entries with repeats, padding (-1, -7), groups
+    that are not complete yet and values past 2^30 planted in them."""
+    rng = np.random.default_rng(seed)
+    n_groups = (w.pos.astype(np.int64) + 1) // w.ratio
+    top = rng.integers(0, np.maximum(n_groups, 1)[:, None] + 40, size=(w.N, width)).astype(np.int64)
+    kind = rng.integers(0, 10, size=top.shape)
+    top[kind == 0] = -1
+    top[kind == 1] = -7
+    top[kind == 2] = (1 << 30) + 5
+    rep = rng.integers(0, width, size=top.shape)
+    top[kind == 3] = np.take_along_axis(top, rep, axis=1)[kind == 3]
+    return np.ascontiguousarray(top.astype(np.int32))
+
+
+@pytest.mark.parametrize("width", [1, 2, 31, 33, 300, 512])
+def test_inline_sets_planted_topk_rows(spa, width):
+    """Rows of any width up to 512 (not only powers of two), with repeats,
+    padding, incomplete groups and huge values: each picks the same groups
+    on both paths."""
+    from sparse_paged_attention_build_b200 import workloads
+    w = workloads.make("c3", shrink=16)
+    w = dataclasses.replace(w, topk=_planted_topk(w, width, seed=width), K=width)
+    csr, inl = _both(w, 2)
+    assert csr.status_word() == 0
+    _assert_identical(csr, inl, f"planted rows of width {width}")
+
+
+@pytest.mark.parametrize("splits", [0, 3])
+def test_inline_sets_past_16384_groups(spa, splits):
+    """Contexts whose complete groups outnumber 16384 (the resolver's bitmap)
+    take its sorting network instead; one request stays below."""
+    from sparse_paged_attention_build_b200 import workloads
+    w = workloads._decode("long", 11, 4, np.array([70000, 65541, 100000, 16000]), 8, 64, 128, 4, 512, 64,
+                          fp8=False)
+    assert ((w.pos.astype(np.int64) + 1) // 4 > 16384).sum() == 3
+    csr, inl = _both(w, splits)
+    assert csr.status_word() == 0
+    _assert_identical(csr, inl, f"long contexts, splits={splits}")
+
+
 def test_inline_sets_faulty_positions(spa):
     """A position outside [0, 2^30) gives SPA_DEV_BAD_INDEX and an empty set
     (O = 0, LSE = the sink) on both paths."""
@@ -86,11 +143,12 @@ def test_inline_sets_faulty_positions(spa):
     np.testing.assert_allclose(inl.lse[0].cpu().numpy(), w.sink, rtol=0, atol=1e-6)
 
 
-def test_inline_sets_against_the_oracle(spa):
+@pytest.mark.parametrize("name,shrink", [("c4", 16), ("c3", 16)])
+def test_inline_sets_against_the_oracle(spa, name, shrink):
     import oracle
     from sparse_paged_attention_build_b200 import workloads
     from sparse_paged_attention_build_b200.pipeline import DeviceBatch
-    w = workloads.make("c4", shrink=16)
+    w = workloads.make(name, shrink=shrink)
     b = DeviceBatch(w, sets="inline")
     b.step()
     torch.cuda.synchronize()
