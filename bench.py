@@ -213,18 +213,17 @@ def run_reference(args, rank, world):
 
 def sets_mode(w, args):
     """Where the step builds its key sets when --sets is auto: "inline"
-    (inside the attention kernel) where that is the cheaper place (see
-    pipeline.prefer_inline_sets), else "csr"; otherwise as asked."""
-    import torch
-    from sparse_paged_attention_build_b200.pipeline import prefer_inline_sets
+    (inside the attention kernel, which measured faster than a separate
+    build on every workload) wherever the kernel can (top-k rows of at most
+    512 entries), else "csr"; otherwise as asked."""
+    from sparse_paged_attention_build_b200.pipeline import inline_sets_supported
     if args.sets != "auto":
         return args.sets
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    return "inline" if prefer_inline_sets(w, args.fp8_path, args.splits, sms) else "csr"
+    return "inline" if inline_sets_supported(w) else "csr"
 
 
 SETS_TEXT = {"csr": "spa_build_kv_sets, then the attention reads the CSR sets",
-             "inline": "built inside the attention kernel (spa_sparse_sink_attn_fwd_inline_sets)"}
+             "inline": "built inside the attention kernel (the *_inline_sets call)"}
 
 
 def config_of(w, world, nnz, fp8_path=None):
@@ -253,8 +252,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--sets", default="auto", choices=["auto", "csr", "inline"],
                     help="csr: spa_build_kv_sets, then the attention reads the CSR sets; inline: the "
-                         "sets built inside the attention kernel; auto: inline without a top-k list, or "
-                         "with one for batches of at most 8 units per SM")
+                         "sets built inside the attention kernel; auto: inline wherever the kernel can "
+                         "(top-k rows of at most 512 entries)")
     ap.add_argument("--fp8-path", default="fused", choices=["fused", "decode"],
                     help="mixed FP8 cache: decode inside the attention gather, or decode the pages first")
     ap.add_argument("--op", default="path", choices=["path", "kv_write", "bwd", "unpack_d512"],

@@ -276,9 +276,7 @@ int spa_sparse_sink_attn_fwd(
  * with the same num_splits. In the decode timeline of the block-level test
  * the set build precedes the core; here it costs no launch and no round
  * trip through indptr/indices. A top-k row is reduced to its sorted groups
- * by the kernel's resolver warp once per (query, slice) unit, which costs a
- * CTA a few microseconds per unit: for large batches with top-k rows the
- * separate spa_build_kv_sets is the cheaper place.
+ * by the kernel's resolver warp once per (query, slice) unit.
  *
  * Arguments as for spa_sparse_sink_attn_fwd, without indptr/indices, plus:
  * pos        int32 [n_queries], 0 <= pos < 2^30 (else SPA_DEV_BAD_INDEX and
@@ -333,6 +331,25 @@ int spa_sparse_sink_attn_fwd_fp8(
     const float* v_cmp_scale, int64_t cmp_num_pages, int32_t cmp_page_size,
     const int32_t* pt_cmp, int32_t pt_cmp_cols, int32_t fp8_format,
     const int32_t* req, int32_t n_requests, const int32_t* indptr, const int32_t* indices,
+    const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
+    void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
+
+/* spa_sparse_sink_attn_fwd_fp8_inline_sets -- spa_sparse_sink_attn_fwd_fp8
+ * over the sets of section 3a, built inside the kernel: the arguments of
+ * spa_sparse_sink_attn_fwd_fp8 with indptr/indices replaced by pos, topk,
+ * topk_width, window and ratio (meaning, limits and errors as in 3a). O and
+ * LSE are bit-identical to spa_build_kv_sets followed by
+ * spa_sparse_sink_attn_fwd_fp8 with the same num_splits. */
+int spa_sparse_sink_attn_fwd_fp8_inline_sets(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries,
+    int32_t num_heads, int32_t head_dim,
+    const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+    const int32_t* pt_raw, int32_t pt_raw_cols,
+    const uint8_t* k_cmp_fp8, const uint8_t* v_cmp_fp8, const float* k_cmp_scale,
+    const float* v_cmp_scale, int64_t cmp_num_pages, int32_t cmp_page_size,
+    const int32_t* pt_cmp, int32_t pt_cmp_cols, int32_t fp8_format,
+    const int32_t* req, int32_t n_requests, const int32_t* pos,
+    const int32_t* topk, int32_t topk_width, int32_t window, int32_t ratio,
     const float* sink, float scale, uint16_t* out, float* lse, int32_t num_splits,
     void* workspace, size_t workspace_bytes, uint32_t* dev_status, spa_stream_t stream);
 

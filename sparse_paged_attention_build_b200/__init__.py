@@ -81,6 +81,12 @@ def _load():
         P, P, P, P, i64, i32, P, i32, i32,
         P, i32, P, P, P, ctypes.c_float, P, P, i32, P, sz, P, P]
     L.spa_sparse_sink_attn_fwd_fp8.restype = ctypes.c_int
+    L.spa_sparse_sink_attn_fwd_fp8_inline_sets.argtypes = [
+        P, i64, i64, i32, i32, i32,
+        P, P, i64, i32, P, i32,
+        P, P, P, P, i64, i32, P, i32, i32,
+        P, i32, P, P, i32, i32, i32, P, ctypes.c_float, P, P, i32, P, sz, P, P]
+    L.spa_sparse_sink_attn_fwd_fp8_inline_sets.restype = ctypes.c_int
     L.spa_paged_kv_write.argtypes = [P, P, i32, i32, P, P, P, i32, i32, i32, i64, P, P, P, P]
     L.spa_paged_kv_write.restype = ctypes.c_int
     L.spa_unpack_d512_pages.argtypes = [P, i64, i32, P, i32, P, P, P]
@@ -291,19 +297,14 @@ def sparse_sink_attn_fwd_inline_sets(q, k_raw, v_raw, pt_raw, req, pos, topk, wi
     return out, lse
 
 
-def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale,
-                             k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale, pt_cmp, out=None, lse=None,
-                             num_splits=0, workspace=None, dev_status=None, stream=None, fp8_format=0):
-    """Like sparse_sink_attn_fwd, with the compressed pool in FP8 (OCP E4M3
-    codes uint8 [pages, page_size, d], FP32 scales [pages, page_size, d/64])
-    decoded inside the attention gather; bit-identical to decoding the pages
-    with dequant_fp8_pages first."""
+def _fp8_attn_buffers(q, k_raw, v_raw, pt_raw, req, ints, sink, k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale,
+                      pt_cmp, out, lse, num_splits, workspace):
+    """Checks and output/workspace buffers shared by the two FP8 calls."""
     _need(q, "q", torch.bfloat16)
     for name, t in (("k_raw", k_raw), ("v_raw", v_raw)):
         _need(t, name, torch.bfloat16)
         assert t.is_contiguous(), name
-    for name, t in (("pt_raw", pt_raw), ("req", req), ("indptr", indptr), ("indices", indices),
-                    ("pt_cmp", pt_cmp)):
+    for name, t in (("pt_raw", pt_raw), ("req", req), ("pt_cmp", pt_cmp)) + tuple(ints):
         _need(t, name, torch.int32)
     for name, t in (("k_cmp_fp8", k_cmp_fp8), ("v_cmp_fp8", v_cmp_fp8)):
         _need(t, name, torch.uint8)
@@ -323,6 +324,20 @@ def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink
     ws_bytes = attn_workspace_size(N, H, d, num_splits)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    return out, lse, workspace
+
+
+def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink, scale,
+                             k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale, pt_cmp, out=None, lse=None,
+                             num_splits=0, workspace=None, dev_status=None, stream=None, fp8_format=0):
+    """Like sparse_sink_attn_fwd, with the compressed pool in FP8 (OCP E4M3
+    codes uint8 [pages, page_size, d], FP32 scales [pages, page_size, d/64])
+    decoded inside the attention gather; bit-identical to decoding the pages
+    with dequant_fp8_pages first."""
+    out, lse, workspace = _fp8_attn_buffers(q, k_raw, v_raw, pt_raw, req, (("indptr", indptr), ("indices", indices)),
+                                            sink, k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale, pt_cmp, out, lse,
+                                            num_splits, workspace)
+    N, H, d = q.shape
     pt_raw = pt_raw.contiguous()
     _check("spa_sparse_sink_attn_fwd_fp8", lib.spa_sparse_sink_attn_fwd_fp8(
         _p(q), q.stride(0), q.stride(1), N, H, d,
@@ -330,6 +345,31 @@ def sparse_sink_attn_fwd_fp8(q, k_raw, v_raw, pt_raw, req, indptr, indices, sink
         _p(k_cmp_fp8), _p(v_cmp_fp8), _p(k_cmp_scale), _p(v_cmp_scale), k_cmp_fp8.shape[0], k_cmp_fp8.shape[1],
         _p(pt_cmp.contiguous()), pt_cmp.shape[1], int(fp8_format),
         _p(req.contiguous()), pt_raw.shape[0], _p(indptr.contiguous()), _p(indices.contiguous()),
+        _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
+        _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
+    return out, lse
+
+
+def sparse_sink_attn_fwd_fp8_inline_sets(q, k_raw, v_raw, pt_raw, req, pos, topk, window, ratio, sink, scale,
+                                         k_cmp_fp8, v_cmp_fp8, k_cmp_scale, v_cmp_scale, pt_cmp, out=None,
+                                         lse=None, num_splits=0, workspace=None, dev_status=None, stream=None,
+                                         fp8_format=0):
+    """sparse_sink_attn_fwd_fp8 over the sets built inside the kernel from
+    pos, topk (int32 [N, K] with K <= 512, or None), window and ratio, as in
+    sparse_sink_attn_fwd_inline_sets."""
+    ints = (("pos", pos),) + ((("topk", topk),) if topk is not None else ())
+    out, lse, workspace = _fp8_attn_buffers(q, k_raw, v_raw, pt_raw, req, ints, sink, k_cmp_fp8, v_cmp_fp8,
+                                            k_cmp_scale, v_cmp_scale, pt_cmp, out, lse, num_splits, workspace)
+    N, H, d = q.shape
+    pt_raw = pt_raw.contiguous()
+    topk = None if topk is None else topk.contiguous()
+    _check("spa_sparse_sink_attn_fwd_fp8_inline_sets", lib.spa_sparse_sink_attn_fwd_fp8_inline_sets(
+        _p(q), q.stride(0), q.stride(1), N, H, d,
+        _p(k_raw), _p(v_raw), k_raw.shape[0], k_raw.shape[1], _p(pt_raw), pt_raw.shape[1],
+        _p(k_cmp_fp8), _p(v_cmp_fp8), _p(k_cmp_scale), _p(v_cmp_scale), k_cmp_fp8.shape[0], k_cmp_fp8.shape[1],
+        _p(pt_cmp.contiguous()), pt_cmp.shape[1], int(fp8_format),
+        _p(req.contiguous()), pt_raw.shape[0], _p(pos.contiguous()), _p(topk),
+        0 if topk is None else topk.shape[1], int(window), int(ratio),
         _p(None if sink is None else sink.contiguous()), float(scale), _p(out), _p(lse), num_splits,
         _p(workspace), 0 if workspace is None else workspace.numel(), _p(dev_status), _stream(stream)))
     return out, lse

@@ -396,6 +396,26 @@ spa::AttnArgs attn_args(const uint16_t* q, int64_t q_stride_tok, int64_t q_strid
   return a;
 }
 
+// The inline-set arguments of the *_inline_sets entries (checks that need
+// no device data), copied into `a`.
+int inline_sets_args(spa::AttnArgs& a, const int32_t* pos, const int32_t* topk, int32_t topk_width,
+                     int32_t window, int32_t ratio) {
+  if (window < 1) return fail(SPA_ERR_INVALID_ARG, "window must be >= 1");
+  if (ratio != 0 && ratio != 4 && ratio != 128) return fail(SPA_ERR_UNSUPPORTED, "ratio must be 0, 4 or 128");
+  if (topk_width < 0) return fail(SPA_ERR_INVALID_ARG, "topk_width < 0");
+  if (ratio > 0 && topk != nullptr && topk_width > spa::kInlineTopkMaxWidth)
+    return fail(SPA_ERR_UNSUPPORTED, "topk_width > %d (sets built in the kernel)", spa::kInlineTopkMaxWidth);
+  if (pos == nullptr && a.n_queries > 0) return fail(SPA_ERR_INVALID_ARG, "pos must be non-NULL");
+  if (!aligned(topk, 4)) return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
+  a.set_pos = pos;
+  a.set_window = window;
+  a.set_ratio = ratio;
+  // with ratio 0 the row picks nothing: the set is the window alone
+  a.set_topk = ratio > 0 ? topk : nullptr;
+  a.set_topk_width = ratio > 0 && topk != nullptr ? topk_width : 0;
+  return SPA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -431,29 +451,18 @@ int spa_sparse_sink_attn_fwd_inline_sets(const uint16_t* q, int64_t q_stride_tok
                                          const float* sink, float scale, uint16_t* out, float* lse,
                                          int32_t num_splits, void* workspace, size_t workspace_bytes,
                                          uint32_t* dev_status, spa_stream_t stream) {
-  if (window < 1) return fail(SPA_ERR_INVALID_ARG, "window must be >= 1");
-  if (ratio != 0 && ratio != 4 && ratio != 128) return fail(SPA_ERR_UNSUPPORTED, "ratio must be 0, 4 or 128");
-  if (topk_width < 0) return fail(SPA_ERR_INVALID_ARG, "topk_width < 0");
-  if (ratio > 0 && topk != nullptr && topk_width > spa::kInlineTopkMaxWidth)
-    return fail(SPA_ERR_UNSUPPORTED, "topk_width > %d (sets built in the kernel)", spa::kInlineTopkMaxWidth);
-  if (ratio > 0 && n_queries > 0 && (pt_cmp == nullptr || k_cmp == nullptr || v_cmp == nullptr))
-    return fail(SPA_ERR_INVALID_ARG, "ratio > 0 needs the compressed pool (k_cmp, v_cmp, pt_cmp)");
-  if (pt_cmp != nullptr && n_queries > 0 && (k_cmp == nullptr || v_cmp == nullptr))
-    return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
-  if (pos == nullptr && n_queries > 0) return fail(SPA_ERR_INVALID_ARG, "pos must be non-NULL");
-  if (!aligned(topk, 4)) return fail(SPA_ERR_ALIGNMENT, "32-bit arrays must be 4-byte aligned");
   spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
                               raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
                               pt_cmp_cols, req, n_requests, nullptr, nullptr, sink, scale, out, lse, workspace,
                               dev_status);
+  const int st = inline_sets_args(a, pos, topk, topk_width, window, ratio);
+  if (st != SPA_OK) return st;
+  if (ratio > 0 && n_queries > 0 && (pt_cmp == nullptr || k_cmp == nullptr || v_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "ratio > 0 needs the compressed pool (k_cmp, v_cmp, pt_cmp)");
+  if (pt_cmp != nullptr && n_queries > 0 && (k_cmp == nullptr || v_cmp == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "k_cmp/v_cmp NULL with pt_cmp set");
   a.k_cmp = k_cmp;
   a.v_cmp = v_cmp;
-  a.set_pos = pos;
-  a.set_window = window;
-  a.set_ratio = ratio;
-  // with ratio 0 the row picks nothing: the set is the window alone
-  a.set_topk = ratio > 0 ? topk : nullptr;
-  a.set_topk_width = ratio > 0 && topk != nullptr ? topk_width : 0;
   return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -477,6 +486,35 @@ int spa_sparse_sink_attn_fwd_fp8(const uint16_t* q, int64_t q_stride_tok, int64_
                               raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
                               pt_cmp_cols, req, n_requests, indptr, indices, sink, scale, out, lse, workspace,
                               dev_status);
+  a.k_cmp_fp8 = k_cmp_fp8;
+  a.v_cmp_fp8 = v_cmp_fp8;
+  a.k_cmp_scale = k_cmp_scale;
+  a.v_cmp_scale = v_cmp_scale;
+  a.fp8_fnuz = fp8_format == 1;
+  return attn_run(a, num_splits, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int spa_sparse_sink_attn_fwd_fp8_inline_sets(
+    const uint16_t* q, int64_t q_stride_tok, int64_t q_stride_head, int32_t n_queries, int32_t num_heads,
+    int32_t head_dim, const uint16_t* k_raw, const uint16_t* v_raw, int64_t raw_num_pages, int32_t raw_page_size,
+    const int32_t* pt_raw, int32_t pt_raw_cols, const uint8_t* k_cmp_fp8, const uint8_t* v_cmp_fp8,
+    const float* k_cmp_scale, const float* v_cmp_scale, int64_t cmp_num_pages, int32_t cmp_page_size,
+    const int32_t* pt_cmp, int32_t pt_cmp_cols, int32_t fp8_format, const int32_t* req, int32_t n_requests,
+    const int32_t* pos, const int32_t* topk, int32_t topk_width, int32_t window, int32_t ratio, const float* sink,
+    float scale, uint16_t* out, float* lse, int32_t num_splits, void* workspace, size_t workspace_bytes,
+    uint32_t* dev_status, spa_stream_t stream) {
+  spa::AttnArgs a = attn_args(q, q_stride_tok, q_stride_head, n_queries, num_heads, head_dim, k_raw, v_raw,
+                              raw_num_pages, raw_page_size, pt_raw, pt_raw_cols, cmp_num_pages, cmp_page_size, pt_cmp,
+                              pt_cmp_cols, req, n_requests, nullptr, nullptr, sink, scale, out, lse, workspace,
+                              dev_status);
+  const int st = inline_sets_args(a, pos, topk, topk_width, window, ratio);
+  if (st != SPA_OK) return st;
+  if (fp8_format != 0 && fp8_format != 1)
+    return fail(SPA_ERR_INVALID_ARG, "fp8_format must be 0 (OCP E4M3) or 1 (E4M3 FNUZ)");
+  if (pt_cmp == nullptr) return fail(SPA_ERR_INVALID_ARG, "pt_cmp must be non-NULL on the FP8 path");
+  if (n_queries > 0 &&
+      (k_cmp_fp8 == nullptr || v_cmp_fp8 == nullptr || k_cmp_scale == nullptr || v_cmp_scale == nullptr))
+    return fail(SPA_ERR_INVALID_ARG, "FP8 codes and scales must be non-NULL");
   a.k_cmp_fp8 = k_cmp_fp8;
   a.v_cmp_fp8 = v_cmp_fp8;
   a.k_cmp_scale = k_cmp_scale;

@@ -121,41 +121,39 @@ __device__ __forceinline__ void load_topk_row(const int32_t* row, int width, int
 
 // Through bitmaps rather than a sort (a sort of 512 entries costs about ten
 // times the instructions, and the resolver shares its issue slots with a
-// softmax warp): a window [w0, hi) of groups gets one bit per group in the
-// free part of `area` after the `total` groups listed so far; every entry
-// in the window sets its bit (repeats fall together); the words come back
-// into registers (word 32 r + lane in register r) and the set bits'
-// indices are appended, ascending, over the bitmap. One window covers up to
-// 32 * (kWords - total) >= 32 * (kWords - kInlineTopkMax) groups, so sets
-// with up to 32 * kWords complete groups take one pass; past that the next
-// window starts at the smallest entry not yet listed, so there are at most
-// as many passes as windows holding an entry.
+// softmax warp). `area` holds the list in its first kInlineTopkMax words and
+// a bitmap in the kWords - kInlineTopkMax after them: a window [w0, hi) of
+// up to 32 * (kWords - kInlineTopkMax) groups gets one bit per group, every
+// entry in the window sets its bit (repeats fall together), and the set
+// bits' indices are appended to the list in ascending order, 32 words per
+// step. The next window starts at the smallest entry not yet listed, so
+// there are at most as many passes as windows holding an entry (one for the
+// usual contexts: 8192 groups per window). The loops stay rolled: this code
+// runs once per unit, and its size, not its speed, is what costs (the
+// caller keeps it out of line for the same reason).
 template <int kWords>
 __device__ __forceinline__ int32_t pick_groups(const int32_t (&g)[kTopkRegs], int32_t n_complete, int lane,
                                                int32_t* area) {
-  constexpr int kR = kWords / 32;
-  static_assert(kWords % 32 == 0 && kWords > kInlineTopkMax, "room for a window after the longest list");
+  constexpr int kBitmapWords = kWords - kInlineTopkMax;
+  static_assert(kBitmapWords >= 32 && kBitmapWords % 32 == 0, "room for a bitmap after the longest list");
+  uint32_t* bits = reinterpret_cast<uint32_t*>(area + kInlineTopkMax);
   int32_t total = 0;
   int32_t w0 = 0;
   while (w0 < n_complete) {
-    const int64_t span_end = w0 + 32LL * (kWords - total);
+    const int64_t span_end = w0 + 32LL * kBitmapWords;
     const int32_t hi = span_end < n_complete ? static_cast<int32_t>(span_end) : n_complete;
-    uint32_t* bits = reinterpret_cast<uint32_t*>(area + total);
-    const int words = (hi - w0 + 31) >> 5;   // <= kWords - total
+    const int words = (hi - w0 + 31) >> 5;
+#pragma unroll 1
     for (int w = lane; w < words; w += 32) bits[w] = 0u;
     __syncwarp();
 #pragma unroll
     for (int r = 0; r < kTopkRegs; ++r)
       if (g[r] >= w0 && g[r] < hi) atomicOr(bits + ((g[r] - w0) >> 5), 1u << ((g[r] - w0) & 31));
     __syncwarp();
-    uint32_t m[kR];
-#pragma unroll
-    for (int r = 0; r < kR; ++r) m[r] = 32 * r + lane < words ? bits[32 * r + lane] : 0u;
-    __syncwarp();   // every word is read before the list overwrites them
-#pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      if (32 * r >= words) continue;   // uniform across the warp
-      const int32_t c = __popc(m[r]);
+#pragma unroll 1
+    for (int b0 = 0; b0 < words; b0 += 32) {
+      uint32_t m = b0 + lane < words ? bits[b0 + lane] : 0u;
+      const int32_t c = __popc(m);
       int32_t incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -163,8 +161,9 @@ __device__ __forceinline__ int32_t pick_groups(const int32_t (&g)[kTopkRegs], in
         if (lane >= o) incl += t;
       }
       int32_t at = total + incl - c;
-      const int32_t base = w0 + (32 * r + lane) * 32;
-      for (uint32_t bm = m[r]; bm != 0u; bm &= bm - 1u) area[at++] = base + (__ffs(bm) - 1);
+      const int32_t base = w0 + (b0 + lane) * 32;
+#pragma unroll 1
+      for (; m != 0u; m &= m - 1u) area[at++] = base + (__ffs(m) - 1);
       total += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncwarp();

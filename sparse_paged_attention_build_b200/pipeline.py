@@ -12,7 +12,8 @@ import numpy as np
 import torch
 
 from . import (build_kv_sets, dequant_fp8_pages, kv_sets_capacity, sparse_sink_attn_fwd, sparse_sink_attn_fwd_fp8,
-               sparse_sink_attn_fwd_inline_sets, attn_workspace_size, new_status, read_status)
+               sparse_sink_attn_fwd_inline_sets, sparse_sink_attn_fwd_fp8_inline_sets, attn_workspace_size,
+               new_status, read_status)
 from . import lib
 
 
@@ -28,12 +29,10 @@ def _dev(a, dtype=None, device="cuda"):
 INLINE_TOPK_MAX = 512   # widest top-k row the attention kernel sorts itself
 
 
-def inline_sets_supported(w, fp8_path="decode") -> bool:
+def inline_sets_supported(w) -> bool:
     """Whether the attention kernel can build this workload's sets itself:
-    top-k rows of at most INLINE_TOPK_MAX entries (or none), and the BF16
-    attention (a mixed cache decoded to BF16 first, not inside the gather)."""
-    fused = w.k_cmp_fp8 is not None and fp8_path == "fused"
-    return not fused and (w.topk is None or w.topk.shape[1] <= INLINE_TOPK_MAX)
+    top-k rows of at most INLINE_TOPK_MAX entries (or none)."""
+    return w.topk is None or w.topk.shape[1] <= INLINE_TOPK_MAX
 
 
 def splits_for(w, num_splits=0) -> int:
@@ -46,22 +45,6 @@ def splits_for(w, num_splits=0) -> int:
     return int(lib.spa_sparse_sink_attn_choose_splits(w.N, w.H, 0))
 
 
-def prefer_inline_sets(w, fp8_path="decode", num_splits=0, sm_count=148) -> bool:
-    """Where the sets are cheaper to build: inside the attention kernel
-    without a top-k list (a closed form, no extra launch) or for small
-    batches with one; a separate build kernel for large batches with top-k
-    rows. Measured on B200: picking a unit's groups from its row costs the
-    CTA about 3 us of its critical path (its resolver shares issue slots
-    with a softmax warp), 16k ratio-4 prefill queries lost 0.17 ms that way
-    against a 0.02 ms build launch, while 64 to 1024 queries gained 2-6 us
-    per step."""
-    if not inline_sets_supported(w, fp8_path):
-        return False
-    if w.topk is None:
-        return True
-    return w.N * splits_for(w, num_splits) <= 8 * sm_count
-
-
 class DeviceBatch:
     """A workload resident in device memory, with its outputs."""
 
@@ -69,14 +52,13 @@ class DeviceBatch:
         self.w = w
         # "csr": the sets are built by spa_build_kv_sets, then read by the
         # attention; "inline": the sets are built inside the attention kernel
-        # (spa_sparse_sink_attn_fwd_inline_sets), from the same inputs
+        # (the *_inline_sets calls), from the same inputs
         if sets not in ("csr", "inline"):
             raise ValueError("sets is 'csr' or 'inline'")
         if fp8_path not in ("fused", "decode"):
             raise ValueError("fp8_path is 'fused' or 'decode'")
-        if sets == "inline" and not inline_sets_supported(w, fp8_path):
-            raise ValueError("sets built inside the kernel need top-k rows of at most 512 entries and no FP8 "
-                             "decode inside the gather")
+        if sets == "inline" and not inline_sets_supported(w):
+            raise ValueError("sets built inside the kernel need top-k rows of at most 512 entries")
         self.inline_sets = sets == "inline"
         self.device = device
         bf16 = torch.bfloat16
@@ -134,6 +116,14 @@ class DeviceBatch:
 
     def attend(self, stream=None):
         w = self.w
+        if self.fused and self.inline_sets:
+            sparse_sink_attn_fwd_fp8_inline_sets(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.pos,
+                                                 self.topk, w.W, w.ratio, self.sink, w.scale, self.k_cmp_fp8,
+                                                 self.v_cmp_fp8, self.k_cmp_scale, self.v_cmp_scale, self.pt_cmp,
+                                                 out=self.out, lse=self.lse, num_splits=self.num_splits,
+                                                 workspace=self.attn_ws, dev_status=self.status, stream=stream,
+                                                 fp8_format=self.w.fp8_format)
+            return
         if self.fused:
             sparse_sink_attn_fwd_fp8(self.q, self.k_raw, self.v_raw, self.pt_raw, self.req, self.indptr,
                                      self.indices, self.sink, w.scale, self.k_cmp_fp8, self.v_cmp_fp8,

@@ -203,6 +203,35 @@ def test_attention_inline_sets_window_only_needs_no_compressed_pool(L):
     assert attn_inline_call(L, ratio=0, ptc=None, kc=None, vc=None, n=0, q=None, out=None, lse=None) == 0
 
 
+def attn8_inline_call(L, **kw):
+    a = dict(q=FAKE, sq=16384, sh=128, n=4, H=128, d=128, kr=FAKE, vr=FAKE, rp=10, rps=64, ptr=FAKE,
+             ptrc=4, k8=FAKE, v8=FAKE, ks=FAKE, vs=FAKE, cp=10, cps=128, ptc=FAKE, ptcc=4, fmt=0,
+             req=FAKE, B=1, pos=FAKE, topk=FAKE, K=512, W=128, ratio=4, sink=FAKE, scale=0.088, out=FAKE,
+             lse=FAKE, splits=1, ws=None, wsb=0)
+    a.update(kw)
+    return L.spa_sparse_sink_attn_fwd_fp8_inline_sets(
+        a["q"], a["sq"], a["sh"], a["n"], a["H"], a["d"], a["kr"], a["vr"], a["rp"], a["rps"], a["ptr"],
+        a["ptrc"], a["k8"], a["v8"], a["ks"], a["vs"], a["cp"], a["cps"], a["ptc"], a["ptcc"], a["fmt"],
+        a["req"], a["B"], a["pos"], a["topk"], a["K"], a["W"], a["ratio"], a["sink"], a["scale"], a["out"],
+        a["lse"], a["splits"], a["ws"], a["wsb"], None, None)
+
+
+@pytest.mark.parametrize("kw,status,clause", [
+    (dict(W=0), 1, "window must be >= 1"),
+    (dict(ratio=5), 2, "ratio must be 0, 4 or 128"),
+    (dict(K=513), 2, "topk_width > 512"),
+    (dict(pos=None), 1, "pos must be non-NULL"),
+    (dict(fmt=2), 1, "fp8_format must be 0"),
+    (dict(ptc=None), 1, "pt_cmp must be non-NULL on the FP8 path"),
+    (dict(ks=None), 1, "FP8 codes and scales must be non-NULL"),
+    (dict(d=512), 2, "head_dim 512: the FP8 gather takes 64 or 128"),
+    (dict(splits=12), 4, "workspace needs"),
+])
+def test_guard_matrix_attention_fp8_inline_sets(L, kw, status, clause):
+    assert attn8_inline_call(L, **kw) == status
+    assert clause in L.spa_last_error_detail().decode()
+
+
 def test_attention_inline_sets_ignores_topk_width_at_ratio_0(L):
     # ratio 0 picks no group, so a row of any width is accepted (and unread)
     assert attn_inline_call(L, ratio=0, topk=FAKE, K=4096, ptc=None, kc=None, vc=None, n=0, q=None, out=None,

@@ -26,11 +26,11 @@ def spa():
     return m
 
 
-def _both(w, splits):
+def _both(w, splits, fp8_path="decode"):
     from sparse_paged_attention_build_b200.pipeline import DeviceBatch
     res = []
     for sets in ("csr", "inline"):
-        b = DeviceBatch(w, num_splits=splits, sets=sets)
+        b = DeviceBatch(w, num_splits=splits, sets=sets, fp8_path=fp8_path)
         b.step()
         torch.cuda.synchronize()
         res.append(b)
@@ -87,6 +87,19 @@ def test_inline_sets_from_topk_rows(spa, name, shrink, splits):
     _assert_identical(csr, inl, f"{name}/{shrink} splits={splits}")
 
 
+@pytest.mark.parametrize("shrink,splits,fmt", [(8, 0, 0), (8, 4, 0), (1, 0, 0), (8, 2, 1)])
+def test_inline_sets_fp8_gather(spa, shrink, splits, fmt):
+    """The mixed cache with its FP8 pages decoded inside the gather
+    (spa_sparse_sink_attn_fwd_fp8_inline_sets against build + the FP8 call),
+    OCP E4M3 and E4M3 FNUZ codes."""
+    from sparse_paged_attention_build_b200 import workloads
+    w = workloads.make("c5", shrink=shrink, fp8_format=fmt)
+    csr, inl = _both(w, splits, fp8_path="fused")
+    assert csr.fused and inl.fused
+    assert csr.status_word() == 0
+    _assert_identical(csr, inl, f"c5/{shrink} fused, splits={splits}, format {fmt}")
+
+
 def _planted_topk(w, width, seed):
     """Top-k rows of `width` entries with repeats, padding (-1, -7), groups
     that are not complete yet and values past 2^30 planted in them."""
@@ -116,13 +129,13 @@ def test_inline_sets_planted_topk_rows(spa, width):
 
 
 @pytest.mark.parametrize("splits", [0, 3])
-def test_inline_sets_past_16384_groups(spa, splits):
-    """Contexts whose complete groups outnumber 16384 (the resolver's bitmap)
-    take its sorting network instead; one request stays below."""
+def test_inline_sets_past_one_bitmap_window(spa, splits):
+    """Contexts whose complete groups outnumber one window of the resolver's
+    bitmap (8192 groups) take several windows; one request stays below."""
     from sparse_paged_attention_build_b200 import workloads
     w = workloads._decode("long", 11, 4, np.array([70000, 65541, 100000, 16000]), 8, 64, 128, 4, 512, 64,
                           fp8=False)
-    assert ((w.pos.astype(np.int64) + 1) // 4 > 16384).sum() == 3
+    assert ((w.pos.astype(np.int64) + 1) // 4 > 8192).sum() == 3
     csr, inl = _both(w, splits)
     assert csr.status_word() == 0
     _assert_identical(csr, inl, f"long contexts, splits={splits}")
