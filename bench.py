@@ -314,7 +314,8 @@ def main():
                "device_status": dres["status"], "config": config_of(wd, world, dres["nnz"], args.fp8_path),
                "sets": SETS_TEXT[dres["sets"]], "e2e": dres["e2e"]}
         if dres["e2e"] is not None:
-            dec["e2e"]["tok_per_s"] = dres["total_queries"] * dres["e2e"]["value"] / max(dres["value"], 1e-30)
+            # the same tokens per step, at the end-to-end rate of pairs
+            dec["e2e"]["tok_per_s"] = dec["tok_per_s"] * dres["e2e"]["value"] / max(dres["value"], 1e-30)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -333,6 +334,8 @@ def main():
         }
         if w.kind == "decode":
             line["tok_per_s"] = res["total_queries"] / (res["elapsed_ms"] / 1e3)
+            if res["e2e"] is not None:
+                line["e2e"]["tok_per_s"] = line["tok_per_s"] * res["e2e"]["value"] / max(res["value"], 1e-30)
         if dec is not None:
             line["decode"] = dec
         if cpu is not None:
