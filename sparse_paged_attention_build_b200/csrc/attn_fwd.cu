@@ -56,6 +56,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <type_traits>
 
 #include "attn_common.cuh"
 
@@ -362,11 +363,16 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
         // into the same 128-byte swizzled BF16 layout. The tile is complete
         // once the TMA bytes have landed and lane 0 has arrived after every
         // lane's shared-memory writes. (Staging the codes through cp.async
-        // to overlap the next tile's fetch measured slower on B200.)
+        // in the destination stage, and issuing the next tile's loads before
+        // this tile's decode, both measured slower on B200.)
         constexpr int kPieces = D / 16;   // 16 codes per piece
         constexpr int kPerLane = kT * kPieces / 32;
+        static_assert(kPieces * 16 == D && (D == 64 || D == 128), "16 codes per piece, one or two halves");
         const uint8_t* pool8 = is_k ? P.k_cmp8 : P.v_cmp8;
         const float* psc = is_k ? P.k_cmp_sc : P.v_cmp_sc;
+        // Lane l always handles piece l % kPieces (16 codes) of rows
+        // (l + 32 j) / kPieces.
+        const int piece = lane % kPieces;
         for (int t = 0; ok && t < ntiles; ++t, ++g) {
           const int stage = g % nst;
           if (!mbar_wait(empty + stage, ((g / nst) & 1) ^ 1, abort_flag, P.dev_status, P.wait_ns)) { ok = false; break; }
@@ -403,11 +409,22 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
             }
           }
           uint8_t* tile = smem + (is_k ? L::kKOff : L::kVOff) + stage * L::kTileBytes;
+          // Every load first (one round trip), then the codes and scales are
+          // staged in the FP8 rows' own bytes of the destination tile
+          // (d = 128: the codes over the row's second half, the scales at the
+          // start of its first half; d = 64: the codes in the row's last 64
+          // bytes, the scale in its first 4), bytes no TMA row and no other
+          // row touches, and a rolled loop decodes 32 / kPieces rows per
+          // step, reading a step's staged bytes before any lane overwrites
+          // them. The rolled loop keeps the decode's code small: unrolled,
+          // it was fetched anew for every tile and took most of the tile's
+          // time.
+          auto code_off = [](int r, int pc) { return (D == 128 ? kT * 128 : 64) + r * 128 + pc * 16; };
           uint4 raw[kPerLane];
           float sc[kPerLane];
 #pragma unroll
           for (int j = 0; j < kPerLane; ++j) {   // every load first
-            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
+            const int r = (lane + 32 * j) / kPieces;
             const uint32_t er = r < nv ? trow[r] : kInvalidRow;
             raw[j] = make_uint4(0u, 0u, 0u, 0u);
             sc[j] = 0.f;
@@ -419,17 +436,38 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           }
 #pragma unroll
           for (int j = 0; j < kPerLane; ++j) {
-            const int cidx = lane + 32 * j, r = cidx / kPieces, piece = cidx % kPieces;
+            const int r = (lane + 32 * j) / kPieces;
             const uint32_t er = r < nv ? trow[r] : kInvalidRow;
             if (er == kInvalidRow || (er & kRawBit)) continue;
-            uint32_t o[8];
-            if (P.fp8_fnuz) decode_e4m3x16<true>(raw[j], sc[j], o);
-            else decode_e4m3x16<false>(raw[j], sc[j], o);
-            const int hf = (piece * 16) / 64, ch0 = ((piece * 16) % 64) / 8;
-            uint8_t* row_ptr = tile + hf * (kT * 128) + r * 128;
-            *reinterpret_cast<uint4*>(row_ptr + ((ch0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(row_ptr + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+            *reinterpret_cast<uint4*>(tile + code_off(r, piece)) = raw[j];
+            if (piece % 4 == 0) *reinterpret_cast<float*>(tile + r * 128 + (piece / 4) * 4) = sc[j];
           }
+          __syncwarp();
+          auto decode_all = [&](auto fnuz) {
+#pragma unroll 1
+            for (int j = 0; j < kPerLane; ++j) {
+              const int r = (lane + 32 * j) / kPieces;
+              const uint32_t er = r < nv ? trow[r] : kInvalidRow;
+              const bool mine = er != kInvalidRow && !(er & kRawBit);
+              uint4 code = make_uint4(0u, 0u, 0u, 0u);
+              float scale = 0.f;
+              if (mine) {
+                code = *reinterpret_cast<const uint4*>(tile + code_off(r, piece));
+                scale = *reinterpret_cast<const float*>(tile + r * 128 + (piece / 4) * 4);
+              }
+              __syncwarp();   // this step's rows are read before any lane writes them
+              if (mine) {
+                uint32_t o[8];
+                decode_e4m3x16<decltype(fnuz)::value>(code, scale, o);
+                const int hf = (piece * 16) / 64, ch0 = ((piece * 16) % 64) / 8;
+                uint8_t* row_ptr = tile + hf * (kT * 128) + r * 128;
+                *reinterpret_cast<uint4*>(row_ptr + ((ch0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(row_ptr + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+              }
+            }
+          };
+          if (P.fp8_fnuz) decode_all(std::true_type{});
+          else decode_all(std::false_type{});
           fence_proxy_async_smem();   // generic-proxy writes -> the UMMA's reads
           __syncwarp();
           if (lane == 0) mbar_arrive(full + stage);

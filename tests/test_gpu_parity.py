@@ -333,6 +333,30 @@ def test_fused_fp8_gather_bit_identical_to_page_decode(spa, shrink, splits):
     check_attn(fus.out, fus.lse, O, L, f"fused c5/{shrink}")
 
 
+@pytest.mark.parametrize("fmt,splits", [(0, 0), (1, 2)])
+def test_fused_fp8_gather_head_dim_64(spa, fmt, splits):
+    """The FP8 gather at d = 64 (one 64-code piece group per row, one scale):
+    bit-identical to decoding the pages first, and within tolerance of the
+    oracle on every element."""
+    import oracle
+    from sparse_paged_attention_build_b200 import workloads
+    from sparse_paged_attention_build_b200.pipeline import DeviceBatch
+    w = workloads._decode("fp8-d64", 23, 16, np.full(16, 4096), 16, 64, 64, 4, 128, 64, fp8=True, fmt=fmt)
+    dec = DeviceBatch(w, num_splits=splits, fp8_path="decode")
+    fus = DeviceBatch(w, num_splits=splits, fp8_path="fused")
+    dec.step()
+    fus.step()
+    torch.cuda.synchronize()
+    assert dec.status_word() == 0 and fus.status_word() == 0
+    assert_bit_identical(dec.out, dec.lse, fus.out, fus.lse, f"d64 FP8 format {fmt} splits={splits}")
+    k = oracle.dequant_fp8_pages(w.k_cmp_fp8, w.k_cmp_scale, w.cmp_page_ids, fmt=fmt)
+    v = oracle.dequant_fp8_pages(w.v_cmp_fp8, w.v_cmp_scale, w.cmp_page_ids, fmt=fmt)
+    ip, idx = oracle.build_kv_sets(w.pos, w.W, w.ratio, w.topk)
+    O, L = oracle.sparse_sink_attn(w.q, w.k_raw, w.v_raw, w.pt_raw, w.req, ip, idx, w.sink, w.scale,
+                                   k_cmp=k, v_cmp=v, pt_cmp=w.pt_cmp)
+    check_attn(fus.out, fus.lse, O, L, f"fused d64 format {fmt}")
+
+
 def test_fused_fp8_full_size_against_oracle(spa):
     from sparse_paged_attention_build_b200.pipeline import DeviceBatch
     w = workload("c5")
