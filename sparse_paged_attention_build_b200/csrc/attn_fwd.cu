@@ -153,7 +153,9 @@ struct Layout {
   // s_full, p_ready, o_done, mma_done, soft_sync[2]
   static constexpr int kNumBars = 2 + 2 + 3 + 2 * kStagesK + 2 * kStagesV + 1 + 1 + 1 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kUsed = kMiscOff + 32;   // + the testing stall barrier at kMiscOff + 16
+  // misc: TMEM slot, abort flag, ticket, have_o, the testing stall barrier
+  // at +16 and the cluster merge's receive barrier at +24
+  static constexpr int kUsed = kMiscOff + 32;
   // + alignment slack; at least 80 KB so that no more than two CTAs share an
   // SM (TMEM holds two 256-column allocations)
   static constexpr int kBytes = (kUsed + 1024) < 80 * 1024 ? 80 * 1024 : (kUsed + 1024);
@@ -245,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     mbar_init(B.mma_done, 1);
     *abort_flag = 0;
     mbar_init(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 16), 1);   // never arrived at
+    mbar_init(reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 24), 1);   // cluster merge: rows received
     mbar_init_fence();
   }
   if (warp == kMmaWarp) {
@@ -894,18 +897,22 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
     // `rank`: LSE = M + log2(L), O = sum_s w_s O_s with w_s = 2^(m_s - M)/L
     // (page "[WS2] Add CP-aware Attention contract and dispatch metadata",
     // Summary: the deterministic (out, lse) merge). CTA r owns rows
-    // [r*per, (r+1)*per) of the output. After the first cluster barrier
-    // every CTA has all slices' (m, l) of its rows (each slice stored its
-    // own into every CTA before the barrier), scales its O rows by its weight and
-    // stores each row as FP16 straight into its owner's idle K/V ring
-    // (posted remote stores, slot = the sender's rank; its own rows with
-    // local stores); after the second barrier each owner sums its slots in
-    // FP32 and writes BF16 O. A weighted row is at most max|v| in magnitude
-    // and FP16 keeps 11 bits, more than the BF16 output; the remote stores
-    // (about 12 bytes per clock per SM on B200) move half the bytes of FP32
-    // rows. No shared memory is read or written remotely after the second
-    // barrier, so no third one is needed. Every thread of every CTA reaches
-    // both barriers: every earlier wait in the kernel is bounded.
+    // [r*per, (r+1)*per) of the output. After the cluster barrier every CTA
+    // has all slices' (m, l) of its rows (each slice stored its own into
+    // every CTA before the barrier), scales its O rows by its weight and
+    // writes each as FP16: its own rows into its receive slot, the others
+    // into a staging block per owner, laid out as that owner's slot; one
+    // thread then sends each block with one bulk copy into the owner's idle
+    // K/V ring (slot = the sender's rank), completing the owner's receive
+    // barrier, armed before the cluster barrier for the rows of all other
+    // slices. Each owner waits on its barrier, sums its slots in FP32 and
+    // writes BF16 O; a sender leaves only once its copies have read their
+    // rows. (Posted remote stores from every thread, about 12 bytes per
+    // clock per SM on B200, and a second cluster barrier took 3.8 us of a
+    // 25 us decode launch.) A weighted row is at most max|v| in magnitude and
+    // FP16 keeps 11 bits, more than the BF16 output, at half the bytes of
+    // FP32 rows. Every thread of every CTA reaches the cluster barrier: every
+    // earlier wait in the kernel is bounded.
     const int rank = static_cast<int>(cluster_ctarank());
     const int i = static_cast<int>(blockIdx.x / S);
     const float2* ml_all = reinterpret_cast<const float2*>(smem + L::kMergeOff);   // [S][128] (m, l)
@@ -918,6 +925,15 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
                   "receive slots fit the idle rings");
     static_assert(L::kTabOff == L::kVOff + kStagesV * L::kTileBytes && L::kVOff == L::kKOff + kStagesK * L::kTileBytes,
                   "rings and tables are contiguous");
+    // the rows of this CTA's own slot come by local stores, the others by
+    // one bulk copy per sender, staged in the sender's idle rings after the
+    // receive slots
+    uint64_t* rx_bar = reinterpret_cast<uint64_t*>(smem + L::kMiscOff + 24);
+    const int my_rows = min(per, 128 - rank * per);
+    if (tid == 0) mbar_arrive_expect_tx(rx_bar, static_cast<uint32_t>((S - 1) * my_rows * D * 2));
+    constexpr int kRxMaxBytes = (128 + kAttnMaxClusterSplits - 1) * D * 2;
+    const uint32_t stage_addr = rx_addr + kRxMaxBytes;       // [S][per][D] FP16, as the receive slots
+    static_assert(2 * kRxMaxBytes <= L::kDescOff - L::kKOff, "receive slots and send staging fit the idle rings");
     __syncwarp();
     cluster_sync_all();                                      // every slice's (m, l) is in place; rings idle
     if (tid < kSoftThreads) {
@@ -944,9 +960,11 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       const bool have_o = *reinterpret_cast<const int*>(smem + L::kMiscOff + 12) != 0;
       const uint32_t o_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16) + L::kOCol;
       const int owner = row / per, rr = row - owner * per;
-      const uint32_t slot = rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 2);
-      const uint32_t dst = dsmem_addr(slot, owner);
       const bool local = owner == rank;
+      // own rows: straight into this CTA's slot; the others: into the
+      // staging block of their owner, laid out as the owner's slot
+      const uint32_t slot = local ? rx_addr + static_cast<uint32_t>(((rank * per + rr) * D) * 2)
+                                  : stage_addr + static_cast<uint32_t>(((owner * per + rr) * D) * 2);
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -966,17 +984,26 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
           for (int k = 0; k < 4; ++k)
             h[k] = pack_f16x2(__uint_as_float(o[8 * v + 2 * k]) * scale_own,
                               __uint_as_float(o[8 * v + 2 * k + 1]) * scale_own);
-          if (local)
-            *reinterpret_cast<uint4*>(smem + (slot - sbase) + phys * 16) = make_uint4(h[0], h[1], h[2], h[3]);
-          else
-            st_dsmem_f4(dst + phys * 16, make_float4(__uint_as_float(h[0]), __uint_as_float(h[1]),
-                                                     __uint_as_float(h[2]), __uint_as_float(h[3])));
+          *reinterpret_cast<uint4*>(smem + (slot - sbase) + phys * 16) = make_uint4(h[0], h[1], h[2], h[3]);
         }
       }
     }
-    __syncwarp();
-    cluster_sync_all();                                      // every slice's weighted rows have arrived
-    if (tid < kSoftThreads) {
+    fence_proxy_async_smem();   // the staged rows (generic writes) -> the bulk copies' reads
+    __syncthreads();
+    if (tid == 0) {
+      for (int o = 0; o < S; ++o) {
+        if (o == rank) continue;
+        const int rows = min(per, 128 - o * per);
+        bulk_copy_to_cluster(dsmem_addr(rx_addr + static_cast<uint32_t>((rank * per * D) * 2), o),
+                             stage_addr + static_cast<uint32_t>((o * per * D) * 2),
+                             static_cast<uint32_t>(rows * D * 2), dsmem_addr(smem_u32(rx_bar), o));
+      }
+      bulk_commit_group();
+    }
+    // every other slice's rows for this CTA have landed (a wait that gives
+    // up leaves the status word set and the rows unwritten)
+    const bool rx_ok = tid >= kSoftThreads || mbar_wait(rx_bar, 0, abort_flag, P.dev_status, P.wait_ns);
+    if (tid < kSoftThreads && rx_ok) {
       const int r0 = min(rank * per, heads_here), r1 = min(r0 + per, heads_here);
       const uint8_t* rx = smem + L::kKOff;
       uint16_t* obase = P.out + (static_cast<int64_t>(i) * P.num_heads + head0) * D;
@@ -1001,6 +1028,7 @@ __global__ void __launch_bounds__(kThreads, 2) sparse_sink_attn_kernel(const __g
       }
     }
   }
+  if (P.cluster_merge && tid == 0) bulk_wait_read_all();   // the outgoing copies have read their rows
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
