@@ -57,9 +57,16 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
                               const int32_t* inl_list = nullptr) {
   constexpr int kPer = kChunkKeys / kParts / 32;
   const int k0 = part * (kChunkKeys / kParts);
+  // Rows of lanes past the chunk's keys are skipped with a warp-uniform
+  // branch, and faults are gathered into one status report at the end: a
+  // short chunk (decode) then runs a few iterations of a short body, which
+  // matters because the code is fetched cold on the first chunk of a launch.
+  uint32_t err = 0;
   int32_t key[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
+    key[e] = -2;
+    if (k0 + 32 * e >= nkeys) continue;   // warp-uniform
     const int k = k0 + lane + 32 * e;
     const int32_t at = key_base + k;
     key[e] = k >= nkeys ? -2
@@ -72,19 +79,21 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     page[e] = -1;
+    if (k0 + 32 * e >= nkeys) continue;   // warp-uniform
     const int32_t kk = key[e];
     if (kk == -2) continue;
-    if (kk < 0) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
+    if (kk < 0) { err |= SPA_DEV_BAD_INDEX; key[e] = -3; continue; }
     const bool raw = (kk & SPA_WINDOW_TAG) != 0;
     const int32_t t = kk & (SPA_WINDOW_TAG - 1);
     const int32_t* pt = raw ? P.pt_raw : P.pt_cmp;
     const int32_t cols = raw ? P.pt_raw_cols : P.pt_cmp_cols;
     const int32_t lp = t >> (raw ? P.raw_ps_log2 : P.cmp_ps_log2);
-    if (pt == nullptr || lp >= cols) { report(P.dev_status, SPA_DEV_BAD_INDEX); key[e] = -3; continue; }
+    if (pt == nullptr || lp >= cols) { err |= SPA_DEV_BAD_INDEX; key[e] = -3; continue; }
     page[e] = __ldg(pt + static_cast<int64_t>(b) * cols + lp);
   }
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
+    if (k0 + 32 * e >= nkeys) continue;   // warp-uniform
     const int k = k0 + lane + 32 * e;
     const int32_t kk = key[e];
     uint32_t row = kInvalidRow;
@@ -95,13 +104,14 @@ __device__ void resolve_chunk(const Prm& P, int32_t b, int32_t key_base, int32_t
       const int64_t pages = raw ? P.raw_pages : P.cmp_pages;
       const int64_t pg = page[e];
       if (pg < 0 || pg >= pages) {
-        report(P.dev_status, SPA_DEV_BAD_PAGE);
+        err |= SPA_DEV_BAD_PAGE;
       } else {
         row = static_cast<uint32_t>((pg << ps_log2) + (t & ((1 << ps_log2) - 1))) | (raw ? kRawBit : 0u);
       }
     }
     if (k < nkeys) tab[k] = row;
   }
+  if (err != 0) report(P.dev_status, err);
 }
 
 // ---- the complete groups a query's top-k row picks (sets built here)
