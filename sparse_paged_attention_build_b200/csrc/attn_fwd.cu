@@ -28,7 +28,7 @@
 //   warps 0-3  softmax + epilogue; thread t owns head row t = TMEM lane t.
 //              They also move each unit's Q from shared memory into TMEM.
 //   warp  4    TMEM allocation; lane 0 issues every UMMA and commit
-//   warp  5    resolver: for a chunk of up to 768 keys of a unit it loads
+//   warp  5    resolver: for a chunk of up to 640 keys of a unit it loads
 //              the keys, looks their pages up and writes the physical row
 //              of every key (bit 31 = raw pool) to a double-buffered table,
 //              plus a chunk descriptor that every other role follows. All

@@ -131,11 +131,11 @@ def test_inline_sets_planted_topk_rows(spa, width):
 @pytest.mark.parametrize("splits", [0, 3])
 def test_inline_sets_past_one_bitmap_window(spa, splits):
     """Contexts whose complete groups outnumber one window of the resolver's
-    bitmap (8192 groups) take several windows; one request stays below."""
+    bitmap (4096 groups) take several windows; one request stays below."""
     from sparse_paged_attention_build_b200 import workloads
     w = workloads._decode("long", 11, 4, np.array([70000, 65541, 100000, 16000]), 8, 64, 128, 4, 512, 64,
                           fp8=False)
-    assert ((w.pos.astype(np.int64) + 1) // 4 > 8192).sum() == 3
+    assert ((w.pos.astype(np.int64) + 1) // 4 > 4096).sum() == 3
     csr, inl = _both(w, splits)
     assert csr.status_word() == 0
     _assert_identical(csr, inl, f"long contexts, splits={splits}")
