@@ -217,7 +217,7 @@ def test_attention_full_size_sampled(spa, name):
                O, L, name)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 5, 16])
+@pytest.mark.parametrize("splits", [1, 2, 3, 4, 5, 6, 7, 8, 9, 16])
 def test_attention_split_counts(spa, splits):
     b = batch(spa, "c4", 8, num_splits=splits)
     b.step()
