@@ -138,9 +138,9 @@ __device__ __forceinline__ void load_topk_row(const int32_t* row, int width, int
 // bits' indices are appended to the list in ascending order, 32 words per
 // step. The next window starts at the smallest entry not yet listed, so
 // there are at most as many passes as windows holding an entry (one up to
-// 4096 complete groups). The loops stay rolled: this code
-// runs once per unit, and its size, not its speed, is what costs (the
-// caller keeps it out of line for the same reason).
+// 4096 complete groups). The loops stay rolled: this code runs once per
+// unit, and its size, not its speed, is what costs (the caller keeps it
+// out of line for the same reason).
 template <int kWords>
 __device__ __forceinline__ int32_t pick_groups(const int32_t (&g)[kTopkRegs], int32_t n_complete, int lane,
                                                int32_t* area) {
